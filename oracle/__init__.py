@@ -1,0 +1,101 @@
+"""CPU oracle for the Gated DeltaNet-2 token mixer (double precision).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the package's ``smoke()`` check and the
+benchmark's CPU-baseline leg are the only callers.  The CUDA path never imports
+this package, and this package imports nothing from the CUDA path.
+
+* ``forward`` / ``decode_step`` call ``gdn2_oracle.c``: the recurrence of the
+  Gated Delta Rule-2 written out token by token (snilld.dk article, the compact
+  update; readout after the update as in the guide's PyTorch loop).
+* ``chunkwise.forward`` re-derives the chunkwise WY form in numpy; it is a
+  second, independent route to the same numbers, used to pin chunk invariance.
+
+Every function takes float64 numpy arrays in the layouts of the C ABI:
+tokens [B, T, H, D], states [B, H, d_k, d_v].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn2_oracle.c")
+LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(src: str = _SRC, out: str = LIB_PATH, extra=()) -> str:
+    """Compile the C oracle into a shared library with gcc; returns its path."""
+    cmd = ["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-pthread", *extra, src, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _bind(lib):
+    D = ctypes.POINTER(ctypes.c_double)
+    L = ctypes.c_long
+    lib.gdn2_oracle_forward.argtypes = [D] * 9 + [L] * 5 + [ctypes.c_int]
+    lib.gdn2_oracle_forward.restype = ctypes.c_int
+    lib.gdn2_oracle_decode_step.argtypes = [D] * 8 + [L] * 4 + [ctypes.c_int]
+    lib.gdn2_oracle_decode_step.restype = ctypes.c_int
+    return lib
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) the C oracle.  ``path`` loads another build."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        if not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(_SRC):
+            build()
+        _lib = _bind(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def forward(q, k, v, log_alpha, b, w, S0=None, nthreads=None, lib=None):
+    """Returns (o [B,T,H,dv], S_T [B,H,dk,dv]) for tokens [B,T,H,D]."""
+    q, k, v, log_alpha, b, w, S0 = map(_f64, (q, k, v, log_alpha, b, w, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    S_T = np.zeros((B, H, dk, dv))
+    lib = lib or load()
+    rc = lib.gdn2_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                 _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv,
+                                 nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle forward failed: {rc}")
+    return o, S_T
+
+
+def decode_step(q, k, v, log_alpha, b, w, S, nthreads=None, lib=None):
+    """One token per unit: tokens [B,H,D], S [B,H,dk,dv].  Returns (o, S_new)."""
+    q, k, v, log_alpha, b, w = map(_f64, (q, k, v, log_alpha, b, w))
+    S = np.array(S, dtype=np.float64, copy=True, order="C")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, H, dv))
+    lib = lib or load()
+    rc = lib.gdn2_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                     _ptr(S), _ptr(o), B, H, dk, dv, nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle decode failed: {rc}")
+    return o, S
