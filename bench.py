@@ -1,0 +1,374 @@
+"""Benchmark of the Gated DeltaNet-2 token mixer on B200.
+
+Primary line: prefill tokens/s per layer of the chunkwise forward on the 1.3B
+layer shape (B=8, H=16, T=4096, d_k=d_v=128, bf16 q/k/v/b/w, fp32 log-alpha,
+state and output).  Alongside it, in the same JSON line: decode steps/s on
+B=256 sequences x H=16 heads (1000 steps, fresh tokens per step), each with its
+roofline against the measured HBM copy bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own copy of the
+workload (independent (batch, head) units need no exchange), the timed region is
+bracketed by barriers, and the slowest rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gdn2_inputs as gi  # noqa: E402
+
+PREFILL = gi.WORKLOADS["prefill_b8_h16_t4096"]
+DECODE = gi.WORKLOADS["decode_b256_h16"]
+METRIC = "GDN-2 prefill tokens/s per layer"
+UNIT = "tokens/s"
+# algorithmic HBM bytes per token-head: q,k,v,b,w bf16 + log-alpha fp32 in, o fp32 out
+PREFILL_BYTES_PER_TOKEN_HEAD = 5 * 128 * 2 + 128 * 4 + 128 * 4
+# dense-tile tensor FLOPs per token-head at C=64, d=128: 2C(3dk + 2dv) + 6 dk dv
+PREFILL_FLOP_PER_TOKEN_HEAD = 2 * 64 * (3 * 128 + 2 * 128) + 6 * 128 * 128
+# state read + write per (sequence, head) and step, fp32 128x128
+DECODE_STATE_BYTES = 2 * 128 * 128 * 4
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"], "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "src": "fallback"}
+
+
+def profile_traffic(kernel):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.md), or None."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 3 and cells[0] == kernel:
+                try:
+                    return float(cells[2])
+                except ValueError:
+                    return None
+    return None
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            c = [x.strip() for x in ln.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                sm.append(float(c[1]))
+                mx = float(c[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, c[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != n:
+        raise SystemExit(f"--gpus {n} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(x, world, device):
+    """Largest value of x over all ranks (x on every rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def time_prefill(args, rank, world, dev):
+    import torch
+    import gated_delta_rule_95_b200 as g
+    d = gi.prefill_inputs(PREFILL)
+    x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    B, T, H = PREFILL.B, PREFILL.T, PREFILL.H
+    o = torch.empty((B, T, H, PREFILL.dv), dtype=torch.float32, device=dev)
+    S_T = torch.empty((B, H, PREFILL.dk, PREFILL.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], None, o=o, S_T=S_T)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(st)
+        for i in range(args.steps):
+            ev[i][0].record(st)
+            step()
+            ev[i][1].record(st)
+        t1.record(st)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    kernel_ms = [a.elapsed_time(b) for a, b in ev]
+    ok = g.gdn2_device_status() == 0
+    return dict(total_ms=total_ms, kernel_ms=float(np.mean(kernel_ms)), clocks=clk.summary(), ok=ok,
+                tokens=B * T, token_heads=B * T * H)
+
+
+def time_prefill_e2e(args, dev):
+    """Same step through the public API with pinned host buffers, copies included."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    d = gi.prefill_inputs(PREFILL)
+    host = {k: v.pin_memory() for k, v in d.items() if v is not None}
+    B, T, H = PREFILL.B, PREFILL.T, PREFILL.H
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    o_host = torch.empty((B, T, H, PREFILL.dv), dtype=torch.float32).pin_memory()
+    s_host = torch.empty((B, H, PREFILL.dk, PREFILL.dv), dtype=torch.float32).pin_memory()
+    d2h = o_host.numel() * 4 + s_host.numel() * 4
+
+    def step():
+        x = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+        o, S = g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], None)
+        o_host.copy_(o, non_blocking=True)
+        s_host.copy_(S, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 5))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(n):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n
+    return {"value": B * T / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+def time_decode(dev, n_steps):
+    import torch
+    import gated_delta_rule_95_b200 as g
+    S = gi.decode_state(DECODE).to(dev)
+    toks = gi.decode_tokens_many(DECODE, range(n_steps))
+    td = [{k: v.to(dev) for k, v in t.items()} for t in toks]
+    del toks
+    o = torch.empty((DECODE.B, DECODE.H, DECODE.dv), dtype=torch.float32, device=dev)
+
+    def run(j):
+        t = td[j]
+        g.gdn2_decode_step(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], S, o=o)
+
+    for j in range(3):
+        run(j)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(st)
+        for j in range(n_steps):
+            run(j)
+        t1.record(st)
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n_steps
+    return dict(ms_per_step=ms, clocks=clk.summary(), ok=g.gdn2_device_status() == 0)
+
+
+def cpu_baseline(seconds_target=15.0):
+    """The oracle, as it stands, on a bounded sample of the prefill workload."""
+    import oracle
+    cores = os.cpu_count() or 1
+    d = gi.prefill_inputs(PREFILL, B=1, H=PREFILL.H)
+    f = {k: gi.as_f64(d[k]) for k in ("q", "k", "v", "log_alpha", "b", "w")}
+    # calibrate on one head, then size the sample to about seconds_target
+    one = {k: v[:, :, :1] for k, v in f.items()}
+    t = time.perf_counter()
+    oracle.forward(**one, nthreads=1)
+    per_unit = time.perf_counter() - t
+    units = int(max(1, min(PREFILL.H, round(seconds_target * cores / max(per_unit, 1e-3) / 2))))
+    units = max(1, min(units, PREFILL.H))
+    sample = {k: v[:, :, :units] for k, v in f.items()}
+    threads = min(cores, units)
+    t = time.perf_counter()
+    oracle.forward(**sample, nthreads=threads)
+    dt = time.perf_counter() - t
+    # tokens/s per layer equivalent: units of one head over T tokens are units/H layers-worth
+    value = units * PREFILL.T / PREFILL.H / dt
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{units} of the {PREFILL.B * PREFILL.H} (batch, head) units, full T={PREFILL.T}, "
+                      f"fp64 token-by-token recurrence, {dt:.1f} s wall; value scaled to tokens/s per layer "
+                      f"(units x T / H / time)"}
+
+
+def config_dict():
+    return {"workload": "prefill_b8_h16_t4096: B=8 H=16 T=4096 d_k=d_v=128 C=64, bf16 q,k,v,b,w; "
+                        "fp32 log-alpha, state and output",
+            "global_batch": PREFILL.B, "seq_len": PREFILL.T, "heads": PREFILL.H, "d_k": 128, "d_v": 128,
+            "chunk": 64, "l2": "inputs larger than L2 (1.2 GB read per step)", "parallelism": "replicas"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    vals = []
+    cb = None
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(seconds_target=5.0)
+        if i >= args.warmup:
+            vals.append(cb["value"])
+    value = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": PREFILL.B * PREFILL.T / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(),
+            "cpu_baseline": dict(cb, value=value),
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=DECODE.steps)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import torch
+    rank, world, local = dist_init(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pk = peaks()
+
+    pre = time_prefill(args, rank, world, dev)
+    ms = pre["total_ms"] / args.steps
+    value = world * pre["tokens"] / (ms * 1e-3)
+    achieved = pre["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (pre["kernel_ms"] * 1e-3) / 1e9
+    tflops = pre["token_heads"] * PREFILL_FLOP_PER_TOKEN_HEAD / (pre["kernel_ms"] * 1e-3) / 1e12
+    traffic = profile_traffic("chunk_fwd_tc_kernel")
+
+    dec = time_decode(dev, args.decode_steps)
+    dec_units = DECODE.B * DECODE.H
+    dec_gbs = dec_units * DECODE_STATE_BYTES / (dec["ms_per_step"] * 1e-3) / 1e9
+    barrier(world)
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, see DESIGN.md)",
+        "config": config_dict(),
+        "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel", "achieved": achieved,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                     "traffic": traffic, "peak_src": pk["src"],
+                     "bytes_per_token_head": PREFILL_BYTES_PER_TOKEN_HEAD,
+                     "tensor": {"achieved_tflops": tflops, "peak_tflops": pk["bf16_tflops"],
+                                "frac": tflops / pk["bf16_tflops"],
+                                "flop_per_token_head": PREFILL_FLOP_PER_TOKEN_HEAD}},
+        "decode": {"metric": "GDN-2 decode steps/s", "value": 1e3 / dec["ms_per_step"], "unit": "steps/s",
+                   "ms_per_step": dec["ms_per_step"], "steps": args.decode_steps,
+                   "workload": "decode_b256_h16: B=256 H=16 d_k=d_v=128, bf16 tokens, fp32 state",
+                   "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": dec_gbs,
+                                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],
+                                "traffic": profile_traffic("decode_step_kernel")},
+                   "clocks": dec["clocks"]},
+        "gpu_launches": args.steps,
+        "clocks": pre["clocks"],
+        "device_status_ok": bool(pre["ok"] and dec["ok"]),
+    }
+    if not args.no_e2e:
+        line["e2e"] = time_prefill_e2e(args, dev)
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

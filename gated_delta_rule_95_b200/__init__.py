@@ -1,0 +1,135 @@
+"""Gated DeltaNet-2 token mixer for NVIDIA B200 (sm_100a).
+
+Python binding of ``libgdn2.so`` (the C ABI declared in ``include/gdn2.h``).
+It only marshals arguments: every step of the computation runs in the
+library's CUDA kernels.  PyTorch provides device memory and streams.  There is
+no CPU fallback: without the built library every call raises.
+
+    o, S_T = gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None)   # prefill, C = 64
+    o      = gdn2_decode_step(q, k, v, log_alpha, b, w, S)       # S updated in place
+
+Shapes: prefill tokens [B, T, H, D], decode tokens [B, H, D], states
+[B, H, d_k, d_v] float32; q, k, v, b, w in bfloat16 or float32 (one dtype);
+log_alpha float32 (log of the channel-wise decay, <= 0); o is always float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+GDN2_F32, GDN2_BF16 = 0, 1
+_DT = {torch.float32: GDN2_F32, torch.bfloat16: GDN2_BF16}
+
+
+class GDN2Error(RuntimeError):
+    """A gdn2_* call returned a non-zero status."""
+
+    def __init__(self, fn, status):
+        msg = lib().gdn2_status_string(status).decode()
+        if status == 5:
+            msg += " (" + lib().gdn2_last_cuda_error().decode() + ")"
+        super().__init__(f"{fn}: status {status}: {msg}")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libgdn2.so")
+
+
+def lib():
+    """The loaded C library (ctypes).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m gated_delta_rule_95_b200.build` "
+                               "(or __graft_entry__.build()); there is no fallback path")
+        L = ctypes.CDLL(path)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        L.gdn2_chunk_fwd.argtypes = [P] * 9 + [I] * 6 + [P]
+        L.gdn2_chunk_fwd.restype = I
+        L.gdn2_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
+        L.gdn2_decode_step.restype = I
+        L.gdn2_device_status.argtypes = []
+        L.gdn2_device_status.restype = I
+        L.gdn2_status_string.argtypes = [I]
+        L.gdn2_status_string.restype = ctypes.c_char_p
+        L.gdn2_last_cuda_error.argtypes = []
+        L.gdn2_last_cuda_error.restype = ctypes.c_char_p
+        L.gdn2_version.argtypes = []
+        L.gdn2_version.restype = I
+        _LIB = L
+    return _LIB
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check_tokens(name, tensors, dtype, device):
+    for n, t in tensors.items():
+        if not t.is_cuda or t.device != device:
+            raise ValueError(f"{name}: {n} must be a CUDA tensor on {device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: {n} must be contiguous")
+        want = torch.float32 if n in ("log_alpha", "S0", "S", "S_T", "o") else dtype
+        if t.dtype != want:
+            raise ValueError(f"{name}: {n} must be {want}, got {t.dtype}")
+
+
+def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_state=True, stream=None):
+    """Chunkwise prefill forward.  Returns (o [B,T,H,d_v], S_T [B,H,d_k,d_v] or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DT:
+        raise ValueError(f"gdn2_chunk_fwd: unsupported dtype {q.dtype}")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ts = dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, o=o)
+    if S0 is not None:
+        ts["S0"] = S0
+    if S_T is not None:
+        ts["S_T"] = S_T
+    _check_tokens("gdn2_chunk_fwd", ts, q.dtype, q.device)
+    rc = lib().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                              _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_chunk_fwd", rc)
+    return o, S_T
+
+
+def gdn2_decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
+    """One decode step; S [B,H,d_k,d_v] fp32 is updated in place.  Returns o [B,H,d_v]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DT:
+        raise ValueError(f"gdn2_decode_step: unsupported dtype {q.dtype}")
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=torch.float32, device=q.device)
+    _check_tokens("gdn2_decode_step", dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, S=S, o=o), q.dtype,
+                  q.device)
+    rc = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
+                                B, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_decode_step", rc)
+    return o
+
+
+def gdn2_device_status() -> int:
+    """Synchronises the device and returns (then clears) the library's device status."""
+    return lib().gdn2_device_status()

@@ -1,0 +1,124 @@
+// C ABI of the Gated DeltaNet-2 token mixer: argument checks, dispatch, status.
+// Every entry point validates before touching CUDA, so argument errors come
+// back synchronously and without a device.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/gdn2.h"
+#include "gdn2_internal.h"
+
+namespace gdn2 {
+
+__device__ unsigned g_error_word = 0;
+
+// Address of the error word on the current device (looked up once per device).
+unsigned* device_error_word() {
+  constexpr int kMaxDev = 64;
+  static unsigned* ptrs[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) ptrs[dev] = static_cast<unsigned*>(p);
+  }
+  return ptrs[dev];
+}
+
+namespace {
+
+thread_local char g_last_cuda[256] = "";
+
+gdn2_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda, sizeof(g_last_cuda), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return GDN2_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+// Largest element count of any tensor must fit comfortably in 63 bits and in
+// the 32-bit grid/tensor-map limits used by the kernels.
+bool sizes_ok(long long B, long long T, long long H, long long dk, long long dv) {
+  if (B < 0 || T < 0 || H < 0) return false;
+  if (!head_dim_ok((int)dk) || !head_dim_ok((int)dv)) return false;
+  if (B * H > 0x7fffffffLL) return false;
+  if (T > (1LL << 31) - 64) return false;
+  const long long tok = B * T * H;
+  return tok <= (1LL << 46) / 128;
+}
+
+}  // namespace
+}  // namespace gdn2
+
+using namespace gdn2;
+
+extern "C" gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                                      const void* b, const void* w, const float* S0, float* o, float* S_T, int B,
+                                      int T, int H, int d_k, int d_v, gdn2_dtype dt, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (!sizes_ok(B, T, H, d_k, d_v)) return GDN2_ERR_SHAPE;
+  const bool tokens = (long long)B * T * H > 0;
+  if (tokens && (!q || !k || !v || !log_alpha || !b || !w || !o)) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, b, w, S0, o, S_T};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if ((long long)B * H == 0) return GDN2_OK;
+
+  ChunkArgs a{q, k, v, b, w, log_alpha, S0, o, S_T, B, T, H, d_k, d_v, dt == GDN2_BF16};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (T == 0)
+    e = launch_state_copy(a, st);
+  else
+    e = a.bf16 ? launch_chunk_fwd_tc(a, st) : launch_chunk_fwd_f32(a, st);
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
+extern "C" gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
+                                        const void* b, const void* w, float* S, float* o, int B, int H, int d_k,
+                                        int d_v, gdn2_dtype dt, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (!sizes_ok(B, 1, H, d_k, d_v)) return GDN2_ERR_SHAPE;
+  if ((long long)B * H == 0) return GDN2_OK;
+  if (!q || !k || !v || !log_alpha || !b || !w || !S || !o) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, b, w, S, o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN2_ERR_ALIGN;
+  DecodeArgs a{q, k, v, b, w, log_alpha, S, o, B, H, d_k, d_v, dt == GDN2_BF16};
+  cudaError_t e = launch_decode_step(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
+extern "C" gdn2_status gdn2_device_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (word) {
+    e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN2_ERR_TIMEOUT;
+  }
+  return GDN2_OK;
+}
+
+extern "C" const char* gdn2_status_string(int status) {
+  switch (status) {
+    case GDN2_OK: return "ok";
+    case GDN2_ERR_NULL: return "a required pointer is NULL";
+    case GDN2_ERR_SHAPE: return "bad shape (negative size, d_k/d_v not 64 or 128, or too large)";
+    case GDN2_ERR_DTYPE: return "unknown dtype";
+    case GDN2_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case GDN2_ERR_CUDA: return "CUDA error";
+    case GDN2_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+extern "C" const char* gdn2_last_cuda_error(void) { return g_last_cuda; }
+
+extern "C" int gdn2_version(void) { return 100; }

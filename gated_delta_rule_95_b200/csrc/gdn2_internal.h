@@ -1,0 +1,37 @@
+// Internal interface between the C ABI (api.cu) and the kernel launchers.
+#pragma once
+#include <cuda_runtime.h>
+
+namespace gdn2 {
+
+struct DecodeArgs {
+  const void *q, *k, *v, *b, *w;
+  const float* log_alpha;
+  float* S;
+  float* o;
+  int B, H, dk, dv;
+  bool bf16;
+};
+
+struct ChunkArgs {
+  const void *q, *k, *v, *b, *w;
+  const float* log_alpha;
+  const float* S0;
+  float* o;
+  float* S_T;
+  int B, T, H, dk, dv;
+  bool bf16;
+};
+
+// Device error word of this library (bit set = a bounded wait gave up).
+unsigned* device_error_word();
+
+cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
+// bf16 inputs: tcgen05/TMEM kernel fed by TMA.
+cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st);
+// fp32 inputs: fp32 CUDA-core kernel of the same chunkwise algorithm.
+cudaError_t launch_chunk_fwd_f32(const ChunkArgs& a, cudaStream_t st);
+// T = 0: S_T = S0 (or zeros).
+cudaError_t launch_state_copy(const ChunkArgs& a, cudaStream_t st);
+
+}  // namespace gdn2

@@ -1,0 +1,117 @@
+/*
+ * gdn2.h — C ABI of the Gated DeltaNet-2 token mixer for NVIDIA B200 (sm_100a).
+ *
+ * The operation (snilld.dk, "Gated DeltaNet-2 fra NVIDIA kan gore dekodning
+ * billigere...", section "Hvad Gated DeltaNet-2 aendrer", the compact update),
+ * per batch element b and head h, with a d_k x d_v fp32 state S:
+ *
+ *     S_t = (I - k_t (b_t * k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t * v_t)^T
+ *     o_t = S_t^T q_t
+ *
+ * alpha_t in (0,1]^{d_k} is the channel-wise decay (applied before the edit),
+ * b_t in [0,1]^{d_k} the erase gate on the key axis, w_t in [0,1]^{d_v} the write
+ * gate on the value axis.  The readout uses the updated state (Gated DeltaNet-2
+ * guide, "End-to-End PyTorch Implementation").  There is no query scaling.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory and keeps no pointer after the call returns.
+ *   - Tensors are dense, row-major (C order), and 16-byte aligned.
+ *   - The decay gate is passed as log(alpha), fp32, finite and <= 0.  Within one
+ *     chunk of 64 tokens the cumulative log decay of a channel must stay above
+ *     about -80 (the chunk form scales keys by exp(-sum log alpha)); beyond that
+ *     the result is undefined.
+ *   - dt selects the type of q, k, v, b and w: GDN2_BF16 or GDN2_F32.  The
+ *     output o and the state (S0, S_T, S) are always fp32, and accumulation is
+ *     fp32.  (o is stored in fp32 because its values are heavy-tailed: rounding
+ *     it to bf16 alone would cost over half of a 2e-2 max-error/RMS budget.)
+ *   - d_k and d_v are each 64 or 128.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it.  Argument errors are returned synchronously before any
+ *     work is queued; launch failures return GDN2_ERR_CUDA.  A device-side wait
+ *     that runs out of time sets a device error word that gdn2_device_status()
+ *     reports as GDN2_ERR_TIMEOUT; it never traps or hangs the GPU.
+ *   - No exception crosses this boundary.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#if defined(__GNUC__)
+#define GDN2_API __attribute__((visibility("default")))
+#else
+#define GDN2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN2_OK = 0,
+  GDN2_ERR_NULL = 1,    /* a required pointer is NULL */
+  GDN2_ERR_SHAPE = 2,   /* negative size, or d_k / d_v not 64 or 128, or sizes overflow */
+  GDN2_ERR_DTYPE = 3,   /* dt is not a gdn2_dtype value */
+  GDN2_ERR_ALIGN = 4,   /* a pointer is not 16-byte aligned */
+  GDN2_ERR_CUDA = 5,    /* a CUDA runtime/driver call failed (see gdn2_last_cuda_error) */
+  GDN2_ERR_TIMEOUT = 6  /* a bounded device-side wait gave up (device error word set) */
+} gdn2_status;
+
+typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
+
+/*
+ * Chunkwise-parallel prefill forward, chunk size C = 64.
+ *
+ * Follows the chunkwise decomposition of the Gated DeltaNet-2 guide ("Chunkwise
+ * Parallel Algorithm for GPU Training": chunks of C tokens, intra-chunk work as
+ * tensor-core products, the state handed across chunks) in the WY form with the
+ * cumulative channel-wise decay folded into the factors of each rank-one erase
+ * (snilld.dk, "Hvad betyder det for traening og inferens").  The result equals
+ * the token-by-token recurrence above up to rounding.
+ *
+ *   q, k, b      : [B, T, H, d_k]  dt
+ *   v, w         : [B, T, H, d_v]  dt
+ *   log_alpha    : [B, T, H, d_k]  fp32
+ *   S0           : [B, H, d_k, d_v] fp32, read only; NULL means a zero state
+ *   o            : [B, T, H, d_v]  fp32, written
+ *   S_T          : [B, H, d_k, d_v] fp32, the state after token T-1, written;
+ *                  NULL means "do not write"; may alias S0
+ *   B, T, H      : >= 0; T need not be a multiple of 64 (the last chunk may be
+ *                  partial); T = 0 copies S0 (or zeros) to S_T
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const void* b, const void* w, const float* S0, float* o, float* S_T,
+                           int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
+
+/*
+ * One recurrent decode step: the update above for a single token per
+ * (sequence, head), with the state updated in place (Gated DeltaNet-2 guide,
+ * "4.5x Higher Decoding Throughput with Zero KV Cache": a fixed-size state
+ * streamed once per generated token).
+ *
+ *   q, k, b      : [B, H, d_k]  dt
+ *   v, w         : [B, H, d_v]  dt
+ *   log_alpha    : [B, H, d_k]  fp32
+ *   S            : [B, H, d_k, d_v] fp32, read and overwritten with S'
+ *   o            : [B, H, d_v]  fp32, written
+ */
+GDN2_API gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
+                             const void* b, const void* w, float* S, float* o,
+                             int B, int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
+
+/* Synchronises the current device, then reports and clears the device error
+ * word: GDN2_OK, GDN2_ERR_TIMEOUT, or GDN2_ERR_CUDA if the sync itself failed. */
+GDN2_API gdn2_status gdn2_device_status(void);
+
+/* Static description of a status code. */
+GDN2_API const char* gdn2_status_string(int status);
+
+/* Text of the last CUDA error seen by this library on the calling thread. */
+GDN2_API const char* gdn2_last_cuda_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GDN2_API int gdn2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN2_H */

@@ -1,0 +1,76 @@
+"""The C ABI library on the host: it loads, exports every symbol the header
+declares, and rejects bad arguments before touching CUDA (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_95_b200 as g
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            with open(os.path.join(ROOT, "include", fn)) as f:
+                names += re.findall(r"GDN2_API[^;(]*?\b(gdn2_\w+)\s*\(", f.read())
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = header_symbols()
+    assert "gdn2_chunk_fwd" in names and "gdn2_decode_step" in names
+
+
+@pytest.mark.parametrize("name", header_symbols())
+def test_library_exports(name):
+    assert hasattr(g.lib(), name)
+
+
+def test_version_and_status_strings():
+    L = g.lib()
+    assert L.gdn2_version() >= 100
+    for s in range(7):
+        assert L.gdn2_status_string(s)
+
+
+P = ctypes.c_void_p
+A = P(0x10000)   # aligned, never dereferenced: validation fails before any use
+M = P(0x10008)   # misaligned
+
+
+def chunk(q=A, k=A, v=A, la=A, b=A, w=A, S0=None, o=A, ST=None, B=1, T=64, H=1, dk=128, dv=128, dt=1):
+    return g.lib().gdn2_chunk_fwd(q, k, v, la, b, w, S0, o, ST, B, T, H, dk, dv, dt, None)
+
+
+def decode(q=A, k=A, v=A, la=A, b=A, w=A, S=A, o=A, B=1, H=1, dk=128, dv=128, dt=1):
+    return g.lib().gdn2_decode_step(q, k, v, la, b, w, S, o, B, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=96), 2), (dict(dv=32), 2), (dict(B=-1), 2), (dict(T=-5), 2), (dict(H=-1), 2),
+    (dict(dt=7), 3), (dict(q=None), 1), (dict(o=None), 1), (dict(la=None), 1),
+    (dict(k=M), 4), (dict(S0=M), 4), (dict(ST=M), 4),
+    (dict(B=0), 0), (dict(H=0), 0),
+])
+def test_chunk_fwd_validation(kw, status):
+    assert chunk(**kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=80), 2), (dict(B=-2), 2), (dict(dt=2), 3), (dict(S=None), 1), (dict(w=None), 1),
+    (dict(v=M), 4), (dict(S=M), 4), (dict(B=0), 0),
+])
+def test_decode_step_validation(kw, status):
+    assert decode(**kw) == status
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
+    la = torch.zeros(1, 64, 1, 128)
+    with pytest.raises(ValueError):
+        g.gdn2_chunk_fwd(x, x, x, la, x, x, o=x, S_T=torch.zeros(1, 1, 128, 128))
