@@ -7,7 +7,7 @@
 #include <cstdio>
 #include <cstring>
 
-#include "../../include/gdn2.h"
+#include "gdn2.h"
 #include "gdn2_internal.h"
 
 namespace gdn2 {

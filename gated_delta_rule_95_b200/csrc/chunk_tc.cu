@@ -54,7 +54,7 @@ constexpr uint32_t OFF_W = OFF_V + 2 * P64;     // w -> Vw lo
 constexpr uint32_t OFF_LA = OFF_W + 2 * P64;    // 2 x 32 KB: log-alpha of a chunk, then its [Kb; Qh] lo tile
 constexpr uint32_t OFF_KNLO = OFF_LA + 2 * 32768;  // Kn lo (2 x 64 rows)
 constexpr uint32_t OFF_S = OFF_KNLO + 2 * P64;  // S bf16: 2 panels (value channels) x 128 rows (key channels)
-constexpr uint32_t OFF_SCR = OFF_S + 2 * P128;  // solve scratch (fp32 64x64 + 3x16x16), then P hi / P lo
+constexpr uint32_t OFF_SCR = OFF_S + 2 * P128;  // solve scratch (fp32 64x68 + 16x48), then P hi / P lo
 constexpr uint32_t OFF_T = OFF_SCR + 20480;     // T bf16 [t][s]
 constexpr uint32_t TILES = OFF_T + P64;         // 220 KB
 
@@ -63,7 +63,8 @@ struct Misc {
   uint64_t bar_la[2];
   uint32_t tmem_base;
   int abort;
-  float gC[128];  // Gamma at the chunk end, per key channel
+  float gC[128];     // Gamma at the chunk end, per key channel
+  float half0[128];  // sum of log alpha over the first 32 tokens, per key channel
 };
 constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 
@@ -83,19 +84,6 @@ constexpr uint32_t ID_SQ = idesc_bf16(128, 64, 1, 0, 0);   // S^T (MN-major) x Q
 constexpr uint32_t ID_UP = idesc_bf16(128, 64, 0, 0, 0);   // U~^T (K-major) x P (K-major)
 constexpr uint32_t ID_KU = idesc_bf16(128, 128, 1, 0, 0);  // Kn^T (MN-major) x U~^T (K-major)
 
-// Element (row, col) of a bf16 tile made of 64-column panels of `rows` rows.
-__device__ __forceinline__ uint32_t bf_off(int row, int col, uint32_t panel_bytes) {
-  return (uint32_t)(col >> 6) * panel_bytes + sw128_off(row, (col & 63) >> 3) + (uint32_t)((col & 7) << 1);
-}
-__device__ __forceinline__ float ld_bf(const unsigned char* base, uint32_t off) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
-}
-// Stores x as hi = bf16(x) at hi_base and lo = bf16(x - hi) at lo_base.
-__device__ __forceinline__ void st_split(unsigned char* hi_base, unsigned char* lo_base, uint32_t off, float x) {
-  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-  *reinterpret_cast<__nv_bfloat16*>(hi_base + off) = hi;
-  *reinterpret_cast<__nv_bfloat16*>(lo_base + off) = __float2bfloat16_rn(x - __bfloat162float(hi));
-}
 // 8 fp32 values -> hi and lo bf16 16-byte chunks.
 __device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
   uint32_t* h = &hi.x;
@@ -116,41 +104,11 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return u;
 }
 
-// fp32 64x64 scratch for the solve: A in the lower triangle, T (transposed) in the
-// upper one; column index XOR-swizzled by row so that row-per-thread writes
-// spread over the banks.
-__device__ __forceinline__ int midx(int r, int c) { return r * 64 + (c ^ ((r & 7) << 2)); }
-
-// T(r, c) of the unit lower-triangular inverse, read from the scratch.
-__device__ __forceinline__ float t_get(const float* M, int r, int c) {
-  return r == c ? 1.f : (r > c ? M[midx(c, r)] : 0.f);
-}
-
-// Off-diagonal 16x16 blocks (J + lev, J) of T = (I + A)^-1:
-//     T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ
-// Blocks of one level depend only on lower levels.
-__device__ void solve_level(float* M, float* X, int lev, int tid) {
-  const int nblk = 4 - lev;
-  for (int e = tid; e < nblk * 256; e += NT) {
-    const int J = e >> 8, r = (e >> 4) & 15, c = e & 15, I = J + lev;
-    float z = 0.f;
-    for (int K = J; K < I; ++K) {
-#pragma unroll
-      for (int s = 0; s < 16; ++s) z = fmaf(M[midx(16 * I + r, 16 * K + s)], t_get(M, 16 * K + s, 16 * J + c), z);
-    }
-    X[e] = z;
-  }
-  __syncthreads();
-  for (int e = tid; e < nblk * 256; e += NT) {
-    const int J = e >> 8, r = (e >> 4) & 15, c = e & 15, I = J + lev;
-    float t = 0.f;
-#pragma unroll
-    for (int s = 0; s < 16; ++s)
-      if (s <= r) t = fmaf(t_get(M, 16 * I + r, 16 * I + s), X[(J << 8) + (s << 4) + c], t);
-    M[midx(16 * J + c, 16 * I + r)] = -t;
-  }
-  __syncthreads();
-}
+// fp32 scratch of the triangular solve: a 64 x 64 matrix with rows padded to 68
+// floats (16-byte aligned rows that start 4 banks apart).  It first holds A
+// (strictly lower, zero elsewhere) and is overwritten block-row by block-row
+// with T = (I + A)^-1 (unit lower triangular, explicit zeros above).
+constexpr int LDM = 68;
 
 struct TcParams {
   const float* S0;
@@ -199,7 +157,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
 
   // ---- TMA issue (thread 0) and the bookkeeping of what is in flight ----------------
-  int pend_qkb = 0, pend_v = 0, pend_w = 0, pend_mma = 0, pend_la[2] = {0, 0};
+  int pend_qkb = 0, pend_v = 0, pend_w = 0, pend_mma = 0, pend_la0 = 0, pend_la1 = 0;
   auto issue_qkb = [&](int c) {
     mbar_arrive_expect_tx(&ms.bar_qkb, (uint32_t)(3 * (dk >> 6)) * P64);
     for (int pn = 0; pn < (dk >> 6); ++pn) {
@@ -223,7 +181,7 @@ __global__ void __launch_bounds__(NT, 1)
     const int buf = c & 1;
     mbar_arrive_expect_tx(&ms.bar_la[buf], (uint32_t)(C * dk * 4));
     tma_load_4d(sm + OFF_LA + buf * 32768, &tmLA, &ms.bar_la[buf], 0, h, C * c, bb);
-    pend_la[buf] = 1;
+    if (buf) pend_la1 = 1; else pend_la0 = 1;
   };
   if (tid == 0 && p.nchunks > 0) {
     issue_qkb(0);
@@ -253,9 +211,9 @@ __global__ void __launch_bounds__(NT, 1)
   };
   store_S_bf16();
 
-  uint32_t ph_qkb = 0, ph_v = 0, ph_w = 0, ph_mma = 0, ph_la[2] = {0, 0};
-  float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);           // solve scratch 64x64 fp32
-  float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 16384);   // level products 3x16x16 fp32
+  uint32_t ph_qkb = 0, ph_v = 0, ph_w = 0, ph_mma = 0, ph_la0 = 0, ph_la1 = 0;
+  float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);                  // solve matrix, 64 x LDM fp32
+  float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);   // block-row product, 16 x 48 fp32
 
   auto wait_on = [&](uint64_t* bar, uint32_t& ph, int& pend) -> bool {
     const bool ok = mbar_wait_bounded(bar, ph, &ms.abort, p.err, WAIT_LIMIT);
@@ -281,50 +239,98 @@ __global__ void __launch_bounds__(NT, 1)
       bool ok = wait_on(&ms.bar_qkb, ph_qkb, pend_qkb);
       ok = ok && wait_on(&ms.bar_v, ph_v, pend_v);
       ok = ok && wait_on(&ms.bar_w, ph_w, pend_w);
-      ok = ok && wait_on(&ms.bar_la[lb], ph_la[lb], pend_la[lb]);
+      ok = ok && (lb ? wait_on(&ms.bar_la[1], ph_la1, pend_la1) : wait_on(&ms.bar_la[0], ph_la0, pend_la0));
       if (__syncthreads_or(!ok)) break;
     }
     // ===== prep: decay cumsum and the folded operands, in place ========================
+    float* la = reinterpret_cast<float*>(LO);
     {
-      // Thread (ch, half): key channel ch (also value channel ch), tokens [32 half, 32 half + 32).
+      // in-chunk cumsum of log alpha, in place in the fp32 staging [t][d_k]:
+      // thread (ch, half) owns key channel ch and tokens [32 half, 32 half + 32)
       const int ch = tid & 127, half = tid >> 7;
-      const bool kval = ch < dk, vval = ch < dv;
-      const float* la = reinterpret_cast<const float*>(LO);
-      float gs[32];
-      float g = 0.f;
-      if (kval) {
-        if (half == 1) {
+      if (ch < dk && half == 0) {
+        float tot = 0.f;
 #pragma unroll 8
-          for (int t = 0; t < 32; ++t) g += la[t * dk + ch];
-        }
-#pragma unroll
-        for (int tt = 0; tt < 32; ++tt) {
-          g += la[(32 * half + tt) * dk + ch];
-          gs[tt] = g;
-        }
-      } else {
-#pragma unroll
-        for (int tt = 0; tt < 32; ++tt) gs[tt] = 0.f;
+        for (int t = 0; t < 32; ++t) tot += la[t * dk + ch];
+        ms.half0[ch] = tot;
       }
-      if (half == 1) ms.gC[ch] = kval ? __expf(gs[31]) : 0.f;
-      __syncthreads();  // every log-alpha value is read before the buffer becomes the lo tile
-#pragma unroll
-      for (int tt = 0; tt < 32; ++tt) {
-        const int t = 32 * half + tt;
-        const uint32_t o64 = bf_off(t, ch, P64), oKb = bf_off(t, ch, P128), oQh = bf_off(64 + t, ch, P128);
-        float kb = 0.f, qh = 0.f, kn = 0.f, vw = 0.f;
-        if (kval) {
-          const float G = __expf(gs[tt]), Gi = __expf(-gs[tt]);
-          const float kk = ld_bf(sm + OFF_KN, o64);
-          kb = kk * ld_bf(sm + OFF_H, oKb) * G;
-          qh = ld_bf(sm + OFF_H, oQh) * G;
-          kn = kk * Gi;
+      __syncthreads();
+      float g = 0.f;
+      if (ch < dk) {
+        g = half ? ms.half0[ch] : 0.f;
+#pragma unroll 8
+        for (int tt = 0; tt < 32; ++tt) {
+          const int idx = (32 * half + tt) * dk + ch;
+          g += la[idx];
+          la[idx] = g;
         }
-        if (vval) vw = ld_bf(sm + OFF_W, o64) * ld_bf(sm + OFF_V, o64);
-        st_split(sm + OFF_H, LO, oKb, kb);
-        st_split(sm + OFF_H, LO, oQh, qh);
-        st_split(sm + OFF_KN, sm + OFF_KNLO, o64, kn);
-        st_split(sm + OFF_V, sm + OFF_W, o64, vw);
+      }
+      if (half == 1) ms.gC[ch] = ch < dk ? __expf(g) : 0.f;
+    }
+    __syncthreads();
+    {
+      // thread (cg, tg): channels [8 cg, 8 cg + 8) (one 16-byte chunk), tokens tg + 16 r
+      const int cg = tid & 15, tg = tid >> 4, c0 = 8 * cg;
+      const bool kval = c0 < dk, vval = c0 < dv;
+      const uint32_t pn = (uint32_t)(cg >> 3);
+      const int chk = cg & 7;
+      float gv[4][8];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (kval) {
+          const float4 a = *reinterpret_cast<const float4*>(la + (tg + 16 * r) * dk + c0);
+          const float4 b = *reinterpret_cast<const float4*>(la + (tg + 16 * r) * dk + c0 + 4);
+          gv[r][0] = a.x; gv[r][1] = a.y; gv[r][2] = a.z; gv[r][3] = a.w;
+          gv[r][4] = b.x; gv[r][5] = b.y; gv[r][6] = b.z; gv[r][7] = b.w;
+        }
+      }
+      __syncthreads();  // every cumsum value is read before the buffer becomes the lo tile
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int t = tg + 16 * r;
+        const uint32_t o64 = pn * P64 + sw128_off(t, chk);
+        const uint32_t oKb = pn * P128 + sw128_off(t, chk);
+        const uint32_t oQh = pn * P128 + sw128_off(64 + t, chk);
+        float kb[8], qh[8], kn[8], vw[8];
+        if (kval) {
+          float kk[8], bg[8], qq[8];
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + OFF_KN + o64), kk);
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + OFF_H + oKb), bg);
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + OFF_H + oQh), qq);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float G = __expf(gv[r][m]), Gi = __expf(-gv[r][m]);
+            kb[m] = kk[m] * bg[m] * G;
+            qh[m] = qq[m] * G;
+            kn[m] = kk[m] * Gi;
+          }
+        } else {
+#pragma unroll
+          for (int m = 0; m < 8; ++m) kb[m] = qh[m] = kn[m] = 0.f;
+        }
+        if (vval) {
+          float vv[8], ww[8];
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + OFF_V + o64), vv);
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + OFF_W + o64), ww);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) vw[m] = ww[m] * vv[m];
+        } else {
+#pragma unroll
+          for (int m = 0; m < 8; ++m) vw[m] = 0.f;
+        }
+        uint4 hi, lo;
+        split8(kb, hi, lo);
+        *reinterpret_cast<uint4*>(sm + OFF_H + oKb) = hi;
+        *reinterpret_cast<uint4*>(LO + oKb) = lo;
+        split8(qh, hi, lo);
+        *reinterpret_cast<uint4*>(sm + OFF_H + oQh) = hi;
+        *reinterpret_cast<uint4*>(LO + oQh) = lo;
+        split8(kn, hi, lo);
+        *reinterpret_cast<uint4*>(sm + OFF_KN + o64) = hi;
+        *reinterpret_cast<uint4*>(sm + OFF_KNLO + o64) = lo;
+        split8(vw, hi, lo);
+        *reinterpret_cast<uint4*>(sm + OFF_V + o64) = hi;
+        *reinterpret_cast<uint4*>(sm + OFF_W + o64) = lo;
       }
     }
     fence_proxy_async_smem();
@@ -361,37 +367,87 @@ __global__ void __launch_bounds__(NT, 1)
         f.y = (s + 1 < t) ? v[x + 1] : 0.f;
         f.z = (s + 2 < t) ? v[x + 2] : 0.f;
         f.w = (s + 3 < t) ? v[x + 3] : 0.f;
-        *reinterpret_cast<float4*>(Msc + midx(t, s)) = f;
+        *reinterpret_cast<float4*>(Msc + t * LDM + s) = f;
       }
     }
     __syncthreads();
-    // ===== T = (I + A)^-1, blocked: 16x16 diagonal blocks, then three levels ===========
-    if (tid < 64) {
-      const int I = tid >> 4, cc = tid & 15;
+    // ===== T = (I + A)^-1 by 16-row blocks ==============================================
+    // Diagonal blocks T_II = (I + A_II)^-1 by forward substitution, one column per thread.
+    {
       float x[16];
+      const int I = tid >> 4, cc = tid & 15;
+      if (tid < 64) {
+        const float* Ab = Msc + 16 * I * LDM + 16 * I;
 #pragma unroll
-      for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-      for (int r = 1; r < 16; ++r) {
-        float acc = 0.f;
+        for (int r = 1; r < 16; ++r) {
+          float acc = 0.f;
 #pragma unroll
-        for (int s = 0; s < r; ++s) acc = fmaf(Msc[midx(16 * I + r, 16 * I + s)], x[s], acc);
-        x[r] = (r > cc) ? -acc : x[r];
+          for (int s4 = 0; s4 < r; s4 += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(Ab + r * LDM + s4);
+            acc = fmaf(a.x, x[s4], acc);
+            if (s4 + 1 < r) acc = fmaf(a.y, x[s4 + 1], acc);
+            if (s4 + 2 < r) acc = fmaf(a.z, x[s4 + 2], acc);
+            if (s4 + 3 < r) acc = fmaf(a.w, x[s4 + 3], acc);
+          }
+          x[r] = (r > cc) ? -acc : x[r];
+        }
+      }
+      __syncthreads();
+      if (tid < 64) {
+        float* Tb = Msc + 16 * I * LDM + 16 * I;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tb[r * LDM + cc] = x[r];
+      }
+      __syncthreads();
+    }
+    // Block rows I = 1..3:  T_I,<I = -T_II (A_I,<I T_<I,<I); every entry above the
+    // diagonal is an explicit zero, so the products run over full ranges.
+#pragma unroll
+    for (int I = 1; I < 4; ++I) {
+      const int r = tid >> 4, c = tid & 15;
+      const float* Arow = Msc + (16 * I + r) * LDM;
+      float z[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k4 = 0; k4 < 16 * I; k4 += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(Arow + k4);
+#pragma unroll
+        for (int u = 0; u < I; ++u) {
+          const float* Tc = Msc + k4 * LDM + c + 16 * u;
+          z[u] = fmaf(a.x, Tc[0], z[u]);
+          z[u] = fmaf(a.y, Tc[LDM], z[u]);
+          z[u] = fmaf(a.z, Tc[2 * LDM], z[u]);
+          z[u] = fmaf(a.w, Tc[3 * LDM], z[u]);
+        }
       }
 #pragma unroll
-      for (int r = 0; r < 16; ++r)
-        if (r > cc) Msc[midx(16 * I + cc, 16 * I + r)] = x[r];
+      for (int u = 0; u < I; ++u) Xsc[r * 48 + c + 16 * u] = z[u];
+      __syncthreads();
+      const float* Trow = Msc + (16 * I + r) * LDM + 16 * I;
+      float y[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 tr = *reinterpret_cast<const float4*>(Trow + s4);
+#pragma unroll
+        for (int u = 0; u < I; ++u) {
+          const float* Xc = Xsc + s4 * 48 + c + 16 * u;
+          y[u] = fmaf(tr.x, Xc[0], y[u]);
+          y[u] = fmaf(tr.y, Xc[48], y[u]);
+          y[u] = fmaf(tr.z, Xc[96], y[u]);
+          y[u] = fmaf(tr.w, Xc[144], y[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < I; ++u) Msc[(16 * I + r) * LDM + c + 16 * u] = -y[u];
+      __syncthreads();
     }
-    __syncthreads();
-    solve_level(Msc, Xsc, 1, tid);
-    solve_level(Msc, Xsc, 2, tid);
-    solve_level(Msc, Xsc, 3, tid);
     // T as a bf16 K-major operand [t][s]
     for (int e = tid; e < 512; e += NT) {
       const int t = e >> 3, q8 = e & 7;
-      float f[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) f[m] = t_get(Msc, t, 8 * q8 + m);
+      const float4 a = *reinterpret_cast<const float4*>(Msc + t * LDM + 8 * q8);
+      const float4 b = *reinterpret_cast<const float4*>(Msc + t * LDM + 8 * q8 + 4);
+      const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       *reinterpret_cast<uint4*>(sm + OFF_T + sw128_off(t, q8)) = pack8(f);
     }
     __syncthreads();  // the scratch is free: P hi / lo go there
@@ -548,8 +604,8 @@ __global__ void __launch_bounds__(NT, 1)
     if (pend_qkb) mbar_wait_bounded(&ms.bar_qkb, ph_qkb, &never, nullptr, WAIT_LIMIT);
     if (pend_v) mbar_wait_bounded(&ms.bar_v, ph_v, &never, nullptr, WAIT_LIMIT);
     if (pend_w) mbar_wait_bounded(&ms.bar_w, ph_w, &never, nullptr, WAIT_LIMIT);
-    for (int b2 = 0; b2 < 2; ++b2)
-      if (pend_la[b2]) mbar_wait_bounded(&ms.bar_la[b2], ph_la[b2], &never, nullptr, WAIT_LIMIT);
+    if (pend_la0) mbar_wait_bounded(&ms.bar_la[0], ph_la0, &never, nullptr, WAIT_LIMIT);
+    if (pend_la1) mbar_wait_bounded(&ms.bar_la[1], ph_la1, &never, nullptr, WAIT_LIMIT);
     if (pend_mma) mbar_wait_bounded(&ms.bar_mma, ph_mma, &never, nullptr, WAIT_LIMIT);
   }
   tc_fence_before();

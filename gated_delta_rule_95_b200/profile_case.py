@@ -1,0 +1,56 @@
+"""Runs one kernel of the library on a seeded workload a few times, for profilers.
+
+    python -m gated_delta_rule_95_b200.profile_case --kind prefill --B 8 --H 16 --T 1024 --reps 2
+    python -m gated_delta_rule_95_b200.profile_case --kind decode --B 256 --H 16 --reps 4
+
+Inputs follow the recipe of the named workload (gdn2_inputs) with the given
+sizes; it exits 0 after a device synchronisation and a clean device status.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kind", choices=["prefill", "decode"], required=True)
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--B", type=int, default=None)
+    ap.add_argument("--H", type=int, default=None)
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--reps", type=int, default=2)
+    a = ap.parse_args()
+
+    import torch
+
+    import gdn2_inputs as gi
+    import gated_delta_rule_95_b200 as g
+
+    dev = torch.device("cuda", 0)
+    if a.kind == "prefill":
+        wl = gi.WORKLOADS[a.workload or "prefill_b8_h16_t4096"]
+        d = gi.prefill_inputs(wl, B=a.B, T=a.T, H=a.H)
+        x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+        for _ in range(a.reps):
+            g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
+    else:
+        wl = gi.WORKLOADS[a.workload or "decode_b256_h16"]
+        S = gi.decode_state(wl, B=a.B, H=a.H).to(dev)
+        for j in range(a.reps):
+            t = {k: v.to(dev) for k, v in gi.decode_tokens(wl, j, B=a.B, H=a.H).items()}
+            g.gdn2_decode_step(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], S)
+    torch.cuda.synchronize()
+    status = g.gdn2_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status}")
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
