@@ -66,54 +66,66 @@ def profile_traffic(kernel):
 
 
 class Clocks:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clock and clock-event (throttle) reasons through NVML on a
+    background thread while the timed region runs (reading only)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
+    def __init__(self, index, period_s=0.002):
+        self.index, self.period = index, period_s
+        self.sm, self.reasons, self.mx = [], set(), None
+
+    def _handle(self):
+        """NVML handle of the CUDA device (matched by UUID: NVML and CUDA indices can differ)."""
+        import pynvml as N
+        import torch
+        try:
+            u = str(torch.cuda.get_device_properties(self.index).uuid)
+            return N.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ids = [x for x in vis.split(",") if x.strip()]
+            idx = int(ids[self.index]) if ids and ids[self.index].strip().isdigit() else self.index
+            return N.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        import pynvml as N
+        h = self._handle()
+        self.mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+        getr = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            N.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop:
+            self.sm.append(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+            r = getr(h)
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+            time.sleep(self.period)
 
     def __enter__(self):
+        import threading
+        self.stop = False
+        self.thread = None
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as N
+            N.nvmlInit()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
         return self
 
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        self.stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            c = [x.strip() for x in ln.split(",")]
-            if len(c) < 9:
-                continue
-            try:
-                sm.append(float(c[1]))
-                mx = float(c[2])
-            except ValueError:
-                continue
-            for n, val in zip(names, c[5:9]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.sm:
+            return {"sm_mhz": None, "sm_max_mhz": self.mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(self.sm)), "sm_max_mhz": self.mx, "reasons": sorted(self.reasons),
+                "samples": len(self.sm), "source": "NVML during the timed region"}
 
 
 def dist_init(n):
@@ -216,7 +228,7 @@ def time_prefill_e2e(args, dev):
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 
 
-def time_decode(dev, n_steps):
+def time_decode(dev, n_steps, world=1):
     import torch
     import gated_delta_rule_95_b200 as g
     S = gi.decode_state(DECODE).to(dev)
@@ -232,6 +244,7 @@ def time_decode(dev, n_steps):
     for j in range(3):
         run(j)
     torch.cuda.synchronize()
+    barrier(world)
     st = torch.cuda.current_stream()
     with Clocks(dev.index if dev.index is not None else 0) as clk:
         t0 = torch.cuda.Event(enable_timing=True)
@@ -241,34 +254,39 @@ def time_decode(dev, n_steps):
             run(j)
         t1.record(st)
         torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / n_steps
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / n_steps
     return dict(ms_per_step=ms, clocks=clk.summary(), ok=g.gdn2_device_status() == 0)
 
 
 def cpu_baseline(seconds_target=15.0):
-    """The oracle, as it stands, on a bounded sample of the prefill workload."""
+    """The oracle, as it stands, on a bounded sample of the prefill workload:
+    whole (batch, head) units over the full sequence, as many as fit in about
+    seconds_target of wall time on the host's cores."""
     import oracle
     cores = os.cpu_count() or 1
-    d = gi.prefill_inputs(PREFILL, B=1, H=PREFILL.H)
+    d = gi.prefill_inputs(PREFILL)
     f = {k: gi.as_f64(d[k]) for k in ("q", "k", "v", "log_alpha", "b", "w")}
-    # calibrate on one head, then size the sample to about seconds_target
-    one = {k: v[:, :, :1] for k, v in f.items()}
+    del d
+    one = {k: v[:1, :, :1] for k, v in f.items()}
     t = time.perf_counter()
     oracle.forward(**one, nthreads=1)
     per_unit = time.perf_counter() - t
-    units = int(max(1, min(PREFILL.H, round(seconds_target * cores / max(per_unit, 1e-3) / 2))))
-    units = max(1, min(units, PREFILL.H))
-    sample = {k: v[:, :, :units] for k, v in f.items()}
+    total = PREFILL.B * PREFILL.H
+    units = int(max(1, min(total, seconds_target * cores / max(per_unit, 1e-3))))
+    nb = max(1, min(PREFILL.B, units // PREFILL.H)) if units >= PREFILL.H else 1
+    nh = PREFILL.H if units >= PREFILL.H else units
+    units = nb * nh
+    sample = {k: np.ascontiguousarray(v[:nb, :, :nh]) for k, v in f.items()}
+    del f
     threads = min(cores, units)
     t = time.perf_counter()
     oracle.forward(**sample, nthreads=threads)
     dt = time.perf_counter() - t
-    # tokens/s per layer equivalent: units of one head over T tokens are units/H layers-worth
     value = units * PREFILL.T / PREFILL.H / dt
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{units} of the {PREFILL.B * PREFILL.H} (batch, head) units, full T={PREFILL.T}, "
-                      f"fp64 token-by-token recurrence, {dt:.1f} s wall; value scaled to tokens/s per layer "
-                      f"(units x T / H / time)"}
+            "sample": f"{units} of the {total} (batch, head) units ({nb} sequences x {nh} heads), full T="
+                      f"{PREFILL.T}, fp64 token-by-token recurrence, {dt:.1f} s wall on {threads} threads; "
+                      f"value = units x T / H / time (tokens/s per layer)"}
 
 
 def config_dict():
@@ -285,7 +303,7 @@ def run_reference(args):
     vals = []
     cb = None
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(seconds_target=5.0)
+        cb = cpu_baseline(seconds_target=8.0)
         if i >= args.warmup:
             vals.append(cb["value"])
     value = float(np.mean(vals))
@@ -327,7 +345,7 @@ def main():
     tflops = pre["token_heads"] * PREFILL_FLOP_PER_TOKEN_HEAD / (pre["kernel_ms"] * 1e-3) / 1e12
     traffic = profile_traffic("chunk_fwd_tc_kernel")
 
-    dec = time_decode(dev, args.decode_steps)
+    dec = time_decode(dev, args.decode_steps, world)
     dec_units = DECODE.B * DECODE.H
     dec_gbs = dec_units * DECODE_STATE_BYTES / (dec["ms_per_step"] * 1e-3) / 1e9
     barrier(world)
