@@ -10,7 +10,7 @@
 //
 //     Kb = K*B*Gamma    Qh = Q*Gamma    Kn = K/Gamma    Vw = W*V
 //     [A; P]  = [Kb; Qh] Kn^T           A strictly lower, P lower incl. diagonal
-//     T       = (I + A)^-1              blocked triangular inverse, fp32
+//     T       = (I + A)^-1              recursive 2x2 block inverse, fp32
 //     U^T     = Vw^T T^T                W^T = Kb^T T^T
 //     U~^T    = U^T - S^T W^T           (= (U - W S)^T, the erase-corrected writes)
 //     O^T     = S^T Qh^T + U~^T P^T
@@ -26,10 +26,14 @@
 // Shared-memory and written tensor-memory operands are rounded to tf32 (nearest);
 // the accumulators S^T and U~^T are read by the tensor core at tf32 precision.
 //
-// One CTA (256 threads, 8 warps) owns one (batch, head) and walks its chunks.
-// Thread 0 issues TMA and MMAs; all warps do the elementwise work.  The raw bf16
-// inputs of chunk c+1 are prefetched into L2 while chunk c runs, and its
-// log-alpha tile is loaded by TMA into shared memory.
+// One CTA (512 threads, 16 warps) owns one (batch, head) and walks its chunks.
+// Thread 0 issues TMA and MMAs; all warps do the elementwise work.  Latency is
+// hidden across chunks: the raw bf16 inputs of chunk c+1 are prefetched into L2
+// while chunk c starts and copied by TMA into tiles that chunk c no longer needs
+// once its second product is done; the log-alpha tile of chunk c+1 is loaded by
+// TMA while chunk c runs; and the output store and state decay of chunk c-1 run
+// while chunk c's first product is on the tensor cores (the output accumulator
+// is double-buffered in tensor memory).
 // d_k or d_v = 64 run the same code with the upper half of each operand zero.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -43,28 +47,34 @@ namespace gdn2 {
 namespace {
 
 constexpr int C = 64;
-constexpr int NT = 256;
+constexpr int NT = 512;
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
 
 // ---- shared memory map (byte offsets from a 1024-byte aligned base) ----------------
 // fp32 operand tiles with the 128B swizzle, in panels of 32 columns (128 B rows).
 constexpr uint32_t R64 = 64 * 128;    // a panel of 64 rows  (8 KB)
 constexpr uint32_t R128 = 128 * 128;  // a panel of 128 rows (16 KB)
-constexpr uint32_t OFF_KQ = 0;                  // [Kb; Qh] [t][i]: 4 panels x 128 rows
+constexpr uint32_t OFF_KQ = 0;                  // [Kb; Qh] [t][i]: 4 panels x 128 rows (first: raw q, k, b, v)
 constexpr uint32_t OFF_KN = OFF_KQ + 4 * R128;  // Kn [s][i]: 4 panels x 64 rows; later W [t][i]
 constexpr uint32_t OFF_KNT = OFF_KN + 4 * R64;  // Kn^T [i][s]: 2 panels x 128 rows
 constexpr uint32_t OFF_T = OFF_KNT + 2 * R128;  // T [t][s]: 2 panels x 64 rows (first: Vw [t][j], 32 KB over T and P)
 constexpr uint32_t OFF_P = OFF_T + 2 * R64;     // P [t][s]: 2 panels x 64 rows
-constexpr uint32_t OFF_LA = OFF_P + 2 * R64;    // log alpha [64][d_k] fp32 (TMA), cumsum in place
-constexpr uint32_t OFF_SCR = OFF_LA + 32768;    // solve scratch: fp32 64 x LDM, then 16 x 48
-constexpr uint32_t TILES = OFF_SCR + 20480;     // 212 KB
+constexpr uint32_t OFF_LA = OFF_P + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows
+constexpr uint32_t OFF_SCR = OFF_LA + 4 * R64;  // solve scratch: fp32 64 x LDM, then 32 x LDX (first: raw w)
+// raw bf16 staging (TMA, 128B swizzle): a [64 tokens][128 channels] tile = 2 panels of
+// 64 channels x 64 rows
+constexpr uint32_t B16 = 2 * R64;
+constexpr uint32_t RAW_Q = OFF_KQ, RAW_K = OFF_KQ + B16, RAW_B = OFF_KQ + 2 * B16, RAW_V = OFF_KQ + 3 * B16;
+constexpr uint32_t RAW_W = OFF_SCR;
+constexpr int LDM = 68;                         // padded row (floats) of the 64 x 64 solve matrix
+constexpr int LDX = 36;                         // padded row of the 32 x 32 block product
+constexpr uint32_t TILES = OFF_SCR + 22528;     // 214 KB
 
 struct Misc {
-  uint64_t bar_la, bar_mma;
+  uint64_t bar_la, bar_mma, bar_raw;
   uint32_t tmem_base;
   int abort;
-  float gC[128];     // Gamma at the chunk end, per key channel
-  float half0[128];  // sum of log alpha over the first 32 tokens, per key channel
+  float gC[2][128];  // Gamma at the chunk end, per key channel (chunk parity)
 };
 constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 
@@ -72,22 +82,16 @@ constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 constexpr uint32_t TM_AP = 0;     // [A; P], later W^T   lanes: tokens of Kb | Qh (key channel for W^T)
 constexpr uint32_t TM_W = 0;
 constexpr uint32_t TM_U = 64;     // U^T, then U~^T      lanes: value channel, columns: s
-constexpr uint32_t TM_O = 128;    // O^T                 lanes: value channel, columns: t
-constexpr uint32_t TM_S = 192;    // S^T (the state)     lanes: value channel, columns: key channel
-constexpr uint32_t TM_KBT = 320;  // Kb^T                lanes: key channel,   columns: s
-constexpr uint32_t TM_VWT = 384;  // Vw^T                lanes: value channel, columns: s
+constexpr uint32_t TM_O = 128;    // O^T, two buffers    lanes: value channel, columns: t
+constexpr uint32_t TM_S = 256;    // S^T (the state)     lanes: value channel, columns: key channel
+constexpr uint32_t TM_KBT = 384;  // Kb^T                lanes: key channel,   columns: s
+constexpr uint32_t TM_VWT = 448;  // Vw^T                lanes: value channel, columns: s
 constexpr uint32_t TM_COLS = 512;
 
 // instruction descriptors (M = 128, both operands K-major)
 constexpr uint32_t ID_64 = idesc_tf32(128, 64, 0, 0, 0, 0);
 constexpr uint32_t ID_64NEG = idesc_tf32(128, 64, 0, 0, 0, 1);  // B negated
 constexpr uint32_t ID_128 = idesc_tf32(128, 128, 0, 0, 0, 0);
-
-// fp32 scratch of the triangular solve: a 64 x 64 matrix with rows padded to 68
-// floats (16-byte aligned rows that start 4 banks apart).  It first holds A
-// (strictly lower, zero elsewhere) and is overwritten block-row by block-row
-// with T = (I + A)^-1 (unit lower triangular, explicit zeros above).
-constexpr int LDM = 68;
 
 struct TcParams {
   const __nv_bfloat16 *q, *k, *v, *b, *w;
@@ -98,8 +102,20 @@ struct TcParams {
   unsigned* err;
 };
 
+// fp32 -> tf32, round to nearest with ties away from zero on the magnitude (add half an
+// ulp of the 10-bit mantissa, clear the 13 dropped bits); two integer instructions.
+__device__ __forceinline__ float rna_tf32(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
 __device__ __forceinline__ void st4_tf32(unsigned char* p, const float* f) {
-  *reinterpret_cast<float4*>(p) = make_float4(to_tf32(f[0]), to_tf32(f[1]), to_tf32(f[2]), to_tf32(f[3]));
+  *reinterpret_cast<float4*>(p) = make_float4(rna_tf32(f[0]), rna_tf32(f[1]), rna_tf32(f[2]), rna_tf32(f[3]));
+}
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void fma4(float4& z, float a, const float4& x) {
+  z.x = fmaf(a, x.x, z.x);
+  z.y = fmaf(a, x.y, z.y);
+  z.z = fmaf(a, x.z, z.z);
+  z.w = fmaf(a, x.w, z.w);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -114,13 +130,16 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t sbase = smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, hf = warp >> 2;  // TMEM lane quadrant, column half
+  const int qd = warp & 3, cq = warp >> 2;  // TMEM lane quadrant, column quarter
   const int unit = blockIdx.x, bb = unit / p.H, h = unit % p.H;
   const int dk = p.dk, dv = p.dv;
+  const int jrow = 32 * qd + lane;  // this thread's TMEM lane
+  const int c0 = 8 * warp;          // prep: this warp's 8 channels
 
   if (tid == 0) {
     mbar_init(&ms.bar_la, 1);
     mbar_init(&ms.bar_mma, 1);
+    mbar_init(&ms.bar_raw, 1);
     fence_mbar_init();
     ms.abort = 0;
     tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
@@ -137,7 +156,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
 
   // ---- async copies (thread 0) ---------------------------------------------------------
-  int pend_la = 0, pend_mma = 0;
+  int pend_la = 0, pend_mma = 0, pend_raw = 0;
   auto prefetch_raw = [&](int c) {  // raw bf16 inputs of chunk c into L2
     for (int pn = 0; pn < (dk >> 6); ++pn) {
       tma_prefetch_l2_4d(&tmQ, 64 * pn, h, C * c, bb);
@@ -149,39 +168,50 @@ __global__ void __launch_bounds__(NT, 1)
       tma_prefetch_l2_4d(&tmW, 64 * pn, h, C * c, bb);
     }
   };
-  auto issue_la = [&](int c) {
+  auto issue_la = [&](int c) {  // log alpha of chunk c: dk/32 boxes of 32 channels x 64 tokens
     mbar_arrive_expect_tx(&ms.bar_la, (uint32_t)(C * dk * 4));
-    tma_load_4d(sm + OFF_LA, &tmLA, &ms.bar_la, 0, h, C * c, bb);
+    for (int pn = 0; pn < (dk >> 5); ++pn)
+      tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, C * c, bb);
     pend_la = 1;
   };
+  auto issue_raw = [&](int c) {  // raw bf16 inputs of chunk c into the staging tiles
+    mbar_arrive_expect_tx(&ms.bar_raw, (uint32_t)(3 * (dk >> 6) + 2 * (dv >> 6)) * R64);
+    for (int pn = 0; pn < (dk >> 6); ++pn) {
+      tma_load_4d(sm + RAW_Q + pn * R64, &tmQ, &ms.bar_raw, 64 * pn, h, C * c, bb);
+      tma_load_4d(sm + RAW_K + pn * R64, &tmK, &ms.bar_raw, 64 * pn, h, C * c, bb);
+      tma_load_4d(sm + RAW_B + pn * R64, &tmB, &ms.bar_raw, 64 * pn, h, C * c, bb);
+    }
+    for (int pn = 0; pn < (dv >> 6); ++pn) {
+      tma_load_4d(sm + RAW_V + pn * R64, &tmV, &ms.bar_raw, 64 * pn, h, C * c, bb);
+      tma_load_4d(sm + RAW_W + pn * R64, &tmW, &ms.bar_raw, 64 * pn, h, C * c, bb);
+    }
+    pend_raw = 1;
+  };
   if (tid == 0 && p.nchunks > 0) {
-    prefetch_raw(0);
+    issue_raw(0);
     issue_la(0);
+    if (p.nchunks > 1) prefetch_raw(1);
   }
 
   // ---- entering state S0 -> S^T in tensor memory -----------------------------------------
-  // Thread (qd, hf, lane) owns lane j = 32 qd + lane (a value channel) and the key-channel
-  // columns [64 hf, 64 hf + 64) of S^T.
-  const int jrow = 32 * qd + lane;
+  // Thread (qd, cq, lane) owns lane j = 32 qd + lane (a value channel) and the key-channel
+  // columns [32 cq, 32 cq + 32) of S^T.
   {
+    float v[32];
     const bool ok = p.S0 && jrow < dv;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float v[32];
-#pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const int i = 64 * hf + 32 * half + x;
-        v[x] = (ok && i < dk) ? p.S0[((size_t)unit * dk + i) * dv + jrow] : 0.f;
-      }
-      tmem_st32(tlane + TM_S + 64 * hf + 32 * half, v);
+    for (int x = 0; x < 32; ++x) {
+      const int i = 32 * cq + x;
+      v[x] = (ok && i < dk) ? p.S0[((size_t)unit * dk + i) * dv + jrow] : 0.f;
     }
+    tmem_st32(tlane + TM_S + 32 * cq, v);
     tmem_st_wait();
   }
 
-  uint32_t ph_la = 0, ph_mma = 0;
+  uint32_t ph_la = 0, ph_mma = 0, ph_raw = 0;
   float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);                  // solve matrix, 64 x LDM fp32
-  float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);   // block-row product, 16 x 48 fp32
-  float* la = reinterpret_cast<float*>(sm + OFF_LA);
+  float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);   // block product, 32 x LDX fp32
+  const float* la = reinterpret_cast<const float*>(sm + OFF_LA);
 
   auto wait_on = [&](uint64_t* bar, uint32_t& ph, int& pend) -> bool {
     const bool ok = mbar_wait_bounded(bar, ph, &ms.abort, p.err, WAIT_LIMIT);
@@ -196,105 +226,122 @@ __global__ void __launch_bounds__(NT, 1)
     umma_commit(&ms.bar_mma);
     pend_mma = 1;
   };
+  // Output of chunk cc (O^T in tensor-memory buffer cc & 1) to global memory.
+  auto store_o = [&](int cc) {
+    float v[16];
+    tmem_ld16(tlane + TM_O + 64 * (cc & 1) + 16 * cq, v);
+    tmem_ld_wait();
+    const int tb = C * cc, nn = min(C, p.T - tb);
+    if (jrow < dv) {
+      float* op = p.o + (((size_t)bb * p.T + tb + 16 * cq) * p.H + h) * dv + jrow;
+      const size_t tstride = (size_t)p.H * dv;
+#pragma unroll
+      for (int x = 0; x < 16; ++x)
+        if (16 * cq + x < nn) op[x * tstride] = v[x];
+    }
+  };
+  // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory.
+  auto decay_state = [&](int gb) {
+    float v[32];
+    tmem_ld32(tlane + TM_S + 32 * cq, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int x = 0; x < 32; ++x) v[x] *= ms.gC[gb][32 * cq + x];
+    tmem_st32(tlane + TM_S + 32 * cq, v);
+  };
   tc_fence_before();
   __syncthreads();
 
+  bool dead = false;
   for (int c = 0; c < p.nchunks; ++c) {
-    const int t0 = C * c, n = min(C, p.T - t0);
-    if (tid == 0 && c + 1 < p.nchunks) prefetch_raw(c + 1);
-    // ===== raw inputs of this chunk: issue the global loads first ==========================
-    // Thread (cg, tg): channels [8 cg, 8 cg + 8) (16 bytes of bf16), tokens tg + 16 r.
-    const int cg = tid & 15, tg = tid >> 4, c0 = 8 * cg;
-    const bool kval = c0 < dk, vval = c0 < dv;
-    uint4 rq[4], rk[4], rb[4], rv[4], rw[4];
+    const int ob = c & 1;
+    if (tid == 0 && c + 2 < p.nchunks) prefetch_raw(c + 2);
+    // ===== decay cumsum by warp scan, then the folded operands in registers ============
+    // Warp w owns channels [8 w, 8 w + 8); lane l owns tokens 2 l and 2 l + 1.
+    {
+      bool ok = wait_on(&ms.bar_la, ph_la, pend_la);
+      ok = ok && wait_on(&ms.bar_raw, ph_raw, pend_raw);
+      if (__syncthreads_or(!ok)) { dead = true; break; }
+    }
+    const bool kval = c0 < dk;
+    float kb[2][8], qh[2][8], kn[2][8], vw[2][8];
+    {
+      float a[2][8];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int t = tg + 16 * r;
-      const bool in = t < n;
-      const size_t tok = ((size_t)bb * p.T + t0 + t) * p.H + h;
-      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-      rq[r] = (in && kval) ? __ldg(reinterpret_cast<const uint4*>(p.q + tok * dk + c0)) : z;
-      rk[r] = (in && kval) ? __ldg(reinterpret_cast<const uint4*>(p.k + tok * dk + c0)) : z;
-      rb[r] = (in && kval) ? __ldg(reinterpret_cast<const uint4*>(p.b + tok * dk + c0)) : z;
-      rv[r] = (in && vval) ? __ldg(reinterpret_cast<const uint4*>(p.v + tok * dv + c0)) : z;
-      rw[r] = (in && vval) ? __ldg(reinterpret_cast<const uint4*>(p.w + tok * dv + c0)) : z;
-    }
-    // ===== decay cumsum, in place in the log-alpha tile ======================================
-    {
-      const bool ok = wait_on(&ms.bar_la, ph_la, pend_la);
-      if (__syncthreads_or(!ok)) break;
-    }
-    {
-      // thread (ch, half) owns key channel ch and tokens [32 half, 32 half + 32)
-      const int ch = tid & 127, half = tid >> 7;
-      if (ch < dk && half == 0) {
-        float tot = 0.f;
-#pragma unroll 8
-        for (int t = 0; t < 32; ++t) tot += la[t * dk + ch];
-        ms.half0[ch] = tot;
-      }
-      __syncthreads();
-      float g = 0.f;
-      if (ch < dk) {
-        g = half ? ms.half0[ch] : 0.f;
-#pragma unroll 8
-        for (int tt = 0; tt < 32; ++tt) {
-          const int idx = (32 * half + tt) * dk + ch;
-          g += la[idx];
-          la[idx] = g;
-        }
-      }
-      if (half == 1) ms.gC[ch] = ch < dk ? __expf(g) : 0.f;
-    }
-    __syncthreads();
-    // ===== folded operands: Kb, Qh, Kn, Vw (fp32, rounded to tf32) ===========================
-    {
-      float gv[4][8];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int t = tg + 16 * r;
+      for (int m = 0; m < 2; ++m) {
         if (kval) {
-          const float4 a = *reinterpret_cast<const float4*>(la + t * dk + c0);
-          const float4 e = *reinterpret_cast<const float4*>(la + t * dk + c0 + 4);
-          gv[r][0] = a.x; gv[r][1] = a.y; gv[r][2] = a.z; gv[r][3] = a.w;
-          gv[r][4] = e.x; gv[r][5] = e.y; gv[r][6] = e.z; gv[r][7] = e.w;
+          const float* row = la;  // element (t, i) at f32_off(t, i, R64)
+          const float4 x0 = ld4(reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(row) +
+                                                               f32_off(2 * lane + m, c0, R64)));
+          const float4 x1 = ld4(reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(row) +
+                                                               f32_off(2 * lane + m, c0 + 4, R64)));
+          a[m][0] = x0.x; a[m][1] = x0.y; a[m][2] = x0.z; a[m][3] = x0.w;
+          a[m][4] = x1.x; a[m][5] = x1.y; a[m][6] = x1.z; a[m][7] = x1.w;
         } else {
 #pragma unroll
-          for (int m = 0; m < 8; ++m) gv[r][m] = 0.f;
+          for (int e = 0; e < 8; ++e) a[m][e] = 0.f;
         }
       }
+      float gtot[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float tot = a[0][e] + a[1][e];
+        float inc = tot;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, inc, off);
+          if (lane >= off) inc += y;
+        }
+        const float exc = inc - tot;
+        a[0][e] = exc + a[0][e];  // g at token 2 l
+        a[1][e] = inc;            // g at token 2 l + 1
+        gtot[e] = __shfl_sync(0xffffffffu, inc, 31);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ms.gC[ob][c0 + e] = kval ? __expf(gtot[e]) : 0.f;
+      }
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint32_t ro = (uint32_t)(c0 >> 6) * R64 + sw128_off(2 * lane + m, (c0 & 63) >> 3);
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        const bool vval = c0 < dv;
+        float kk[8], bgt[8], qq[8], vv[8], ww[8];
+        unpack_bf16x8(kval ? *reinterpret_cast<const uint4*>(sm + RAW_K + ro) : z4, kk);
+        unpack_bf16x8(kval ? *reinterpret_cast<const uint4*>(sm + RAW_B + ro) : z4, bgt);
+        unpack_bf16x8(kval ? *reinterpret_cast<const uint4*>(sm + RAW_Q + ro) : z4, qq);
+        unpack_bf16x8(vval ? *reinterpret_cast<const uint4*>(sm + RAW_V + ro) : z4, vv);
+        unpack_bf16x8(vval ? *reinterpret_cast<const uint4*>(sm + RAW_W + ro) : z4, ww);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float G = __expf(a[m][e]), Gi = __expf(-a[m][e]);
+          kb[m][e] = kk[e] * bgt[e] * G;
+          qh[m][e] = qq[e] * G;
+          kn[m][e] = kk[e] * Gi;
+          vw[m][e] = ww[e] * vv[e];
+        }
+      }
+    }
+    // the previous chunk's last products must be done before its tiles are overwritten
+    {
+      bool ok = true;
+      if (c > 0) ok = wait_mma();
       fence_proxy_async_smem();
-      __syncthreads();  // the log-alpha tile is free: load the next chunk's
-      if (tid == 0 && c + 1 < p.nchunks) issue_la(c + 1);
+      if (__syncthreads_or(!ok)) { dead = true; break; }
+    }
+    if (tid == 0 && c + 1 < p.nchunks) issue_la(c + 1);  // the log-alpha tile has been read
+    tc_fence_after();
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int t = tg + 16 * r;
-        float kb[8], qh[8], kn[8], vw[8];
-        {
-          float kk[8], bgt[8], qq[8], vv[8], ww[8];
-          unpack_bf16x8(rk[r], kk);
-          unpack_bf16x8(rb[r], bgt);
-          unpack_bf16x8(rq[r], qq);
-          unpack_bf16x8(rv[r], vv);
-          unpack_bf16x8(rw[r], ww);
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float G = __expf(gv[r][m]), Gi = __expf(-gv[r][m]);
-            kb[m] = kk[m] * bgt[m] * G;
-            qh[m] = qq[m] * G;
-            kn[m] = kk[m] * Gi;
-            vw[m] = ww[m] * vv[m];
-          }
-        }
-        st4_tf32(sm + OFF_KQ + f32_off(t, c0, R128), kb);
-        st4_tf32(sm + OFF_KQ + f32_off(t, c0 + 4, R128), kb + 4);
-        st4_tf32(sm + OFF_KQ + f32_off(64 + t, c0, R128), qh);
-        st4_tf32(sm + OFF_KQ + f32_off(64 + t, c0 + 4, R128), qh + 4);
-        st4_tf32(sm + OFF_KN + f32_off(t, c0, R64), kn);
-        st4_tf32(sm + OFF_KN + f32_off(t, c0 + 4, R64), kn + 4);
-        st4_tf32(sm + OFF_T + f32_off(t, c0, R64), vw);
-        st4_tf32(sm + OFF_T + f32_off(t, c0 + 4, R64), vw + 4);
-      }
+    for (int m = 0; m < 2; ++m) {
+      const int t = 2 * lane + m;
+      st4_tf32(sm + OFF_KQ + f32_off(t, c0, R128), kb[m]);
+      st4_tf32(sm + OFF_KQ + f32_off(t, c0 + 4, R128), kb[m] + 4);
+      st4_tf32(sm + OFF_KQ + f32_off(64 + t, c0, R128), qh[m]);
+      st4_tf32(sm + OFF_KQ + f32_off(64 + t, c0 + 4, R128), qh[m] + 4);
+      st4_tf32(sm + OFF_KN + f32_off(t, c0, R64), kn[m]);
+      st4_tf32(sm + OFF_KN + f32_off(t, c0 + 4, R64), kn[m] + 4);
+      st4_tf32(sm + OFF_T + f32_off(t, c0, R64), vw[m]);
+      st4_tf32(sm + OFF_T + f32_off(t, c0 + 4, R64), vw[m] + 4);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -302,7 +349,6 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) {
       tc_fence_after();
       // [A; P] = [Kb; Qh] Kn^T : M=128 (tokens of both halves), N=64 (s), K=128 (key channels)
-      // O^T    = S^T Qh^T      : A = S^T from tensor memory, B = Qh rows of the KQ tile
 #pragma unroll
       for (int ks = 0; ks < 16; ++ks) {
         const uint32_t ko = (uint32_t)((ks & 3) * 32);
@@ -310,53 +356,63 @@ __global__ void __launch_bounds__(NT, 1)
         const uint64_t bKN = sdesc_sw128(sbase + OFF_KN + (ks >> 2) * R64 + ko, 16, 1024);
         umma_tf32_ss(tmem + TM_AP, aKQ, bKN, ID_64, ks > 0);
       }
-#pragma unroll
-      for (int ks = 0; ks < 16; ++ks) {
-        const uint32_t ko = (uint32_t)((ks & 3) * 32);
-        const uint64_t bQH = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + R64 + ko, 16, 1024);
-        umma_tf32_ts(tmem + TM_O, tmem + TM_S + 8 * ks, bQH, ID_64, ks > 0);
-      }
       commit_mma();
     }
-    // ===== transposed operands while the tensor cores run: Kb^T, Vw^T into tensor
-    // memory (lane = channel), Kn^T into shared memory (row = key channel) ============
+    // ===== while the tensor cores run: transposed operands, the next chunk's raw inputs,
+    // and the output store and state decay of the previous chunk ==========================
     {
-      const int ch = tid & 127;  // also this thread's tensor-memory lane (warp quadrant)
+      const int ch = tid & 127, part = tid >> 7;  // ch is also this thread's TMEM lane
+      float v[32];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        float v[32];
-        if (tid < 128) {
+        if (part == 0) {  // Kb^T -> tensor memory
 #pragma unroll
           for (int x = 0; x < 32; ++x) v[x] = *reinterpret_cast<const float*>(sm + OFF_KQ + f32_off(32 * hh + x, ch, R128));
           tmem_st32(tlane + TM_KBT + 32 * hh, v);
+        } else if (part == 1) {  // Vw^T -> tensor memory
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = *reinterpret_cast<const float*>(sm + OFF_T + f32_off(32 * hh + x, ch, R64));
+          tmem_st32(tlane + TM_VWT + 32 * hh, v);
+        } else if (part - 2 == hh) {  // Kn^T rows, tokens [32 hh, 32 hh + 32)
 #pragma unroll
           for (int x = 0; x < 32; ++x) v[x] = *reinterpret_cast<const float*>(sm + OFF_KN + f32_off(32 * hh + x, ch, R64));
 #pragma unroll
           for (int x = 0; x < 32; x += 4)
             *reinterpret_cast<float4*>(sm + OFF_KNT + f32_off(ch, 32 * hh + x, R128)) =
                 make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
-        } else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) v[x] = *reinterpret_cast<const float*>(sm + OFF_T + f32_off(32 * hh + x, ch, R64));
-          tmem_st32(tlane + TM_VWT + 32 * hh, v);
         }
       }
-      tmem_st_wait();
     }
+    if (c > 0) {
+      store_o(c - 1);
+      decay_state(ob ^ 1);
+    }
+    tmem_st_wait();
     fence_proxy_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(!wait_mma())) break;
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      // O^T = S^T Qh^T : A = S^T from tensor memory, B = Qh rows of the KQ tile
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        const uint32_t ko = (uint32_t)((ks & 3) * 32);
+        const uint64_t bQH = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + R64 + ko, 16, 1024);
+        umma_tf32_ts(tmem + TM_O + 64 * ob, tmem + TM_S + 8 * ks, bQH, ID_64, ks > 0);
+      }
+    }
+    if (__syncthreads_or(!wait_mma())) { dead = true; break; }
     tc_fence_after();
     // ===== A to the solve scratch, P to its operand tile =====================================
     {
-      float v[32];
-      tmem_ld32(tlane + TM_AP + 32 * hf, v);
+      float v[16];
+      tmem_ld16(tlane + TM_AP + 16 * cq, v);
       tmem_ld_wait();
       if (qd < 2) {
         const int t = 32 * qd + lane;
 #pragma unroll
-        for (int x = 0; x < 32; x += 4) {
-          const int s = 32 * hf + x;
+        for (int x = 0; x < 16; x += 4) {
+          const int s = 16 * cq + x;
           float4 f;
           f.x = (s + 0 < t) ? v[x + 0] : 0.f;
           f.y = (s + 1 < t) ? v[x + 1] : 0.f;
@@ -367,17 +423,17 @@ __global__ void __launch_bounds__(NT, 1)
       } else {
         const int t = 32 * (qd - 2) + lane;  // P row, causal incl. diagonal
 #pragma unroll
-        for (int x = 0; x < 32; x += 4) {
+        for (int x = 0; x < 16; x += 4) {
           float f[4];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) f[m] = (32 * hf + x + m <= t) ? v[x + m] : 0.f;
-          st4_tf32(sm + OFF_P + f32_off(t, 32 * hf + x, R64), f);
+          for (int m = 0; m < 4; ++m) f[m] = (16 * cq + x + m <= t) ? v[x + m] : 0.f;
+          st4_tf32(sm + OFF_P + f32_off(t, 16 * cq + x, R64), f);
         }
       }
     }
     __syncthreads();
-    // ===== T = (I + A)^-1 by 16-row blocks ==============================================
-    // Diagonal blocks T_II = (I + A_II)^-1 by forward substitution, one column per thread.
+    // ===== T = (I + A)^-1: 16x16 diagonal blocks, then 32x32, then 64x64 ===================
+    // Every entry above the diagonal is an explicit zero, so block products run dense.
     {
       float x[16];
       const int I = tid >> 4, cc = tid & 15;
@@ -390,7 +446,7 @@ __global__ void __launch_bounds__(NT, 1)
           float acc = 0.f;
 #pragma unroll
           for (int s4 = 0; s4 < r; s4 += 4) {
-            const float4 a = *reinterpret_cast<const float4*>(Ab + r * LDM + s4);
+            const float4 a = ld4(Ab + r * LDM + s4);
             acc = fmaf(a.x, x[s4], acc);
             if (s4 + 1 < r) acc = fmaf(a.y, x[s4 + 1], acc);
             if (s4 + 2 < r) acc = fmaf(a.z, x[s4 + 2], acc);
@@ -407,55 +463,67 @@ __global__ void __launch_bounds__(NT, 1)
       }
       __syncthreads();
     }
-    // Block rows I = 1..3:  T_I,<I = -T_II (A_I,<I T_<I,<I); every entry above the
-    // diagonal is an explicit zero, so the products run over full ranges.  Thread
-    // (r, c4) computes four adjacent columns of a row.
+    {
+      // 32x32 blocks: T_{2p+1,2p} = -T_{2p+1,2p+1} A_{2p+1,2p} T_{2p,2p}, p = 0, 1
+      const int pp = tid >> 8, r = (tid >> 4) & 15, cc = tid & 15;
+      const int I = 2 * pp + 1, J = 2 * pp;
+      const float* Arow = Msc + (16 * I + r) * LDM + 16 * J;
+      float z = 0.f;
 #pragma unroll
-    for (int I = 1; I < 4; ++I) {
-      const int nq = 4 * I;  // float4 columns in the block row
-      for (int e = tid; e < 16 * nq; e += NT) {
-        const int r = e / nq, c4 = e % nq;
-        const float* Arow = Msc + (16 * I + r) * LDM;
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 a = ld4(Arow + s4);
+        const float* Tc = Msc + (16 * J + s4) * LDM + 16 * J + cc;
+        z = fmaf(a.x, Tc[0], fmaf(a.y, Tc[LDM], fmaf(a.z, Tc[2 * LDM], fmaf(a.w, Tc[3 * LDM], z))));
+      }
+      Xsc[pp * 256 + r * 16 + cc] = z;
+      __syncthreads();
+      const float* Trow = Msc + (16 * I + r) * LDM + 16 * I;
+      float y = 0.f;
+#pragma unroll
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 t4 = ld4(Trow + s4);
+        const float* Xc = Xsc + pp * 256 + s4 * 16 + cc;
+        y = fmaf(t4.x, Xc[0], fmaf(t4.y, Xc[16], fmaf(t4.z, Xc[32], fmaf(t4.w, Xc[48], y))));
+      }
+      Msc[(16 * I + r) * LDM + 16 * J + cc] = -y;
+      __syncthreads();
+    }
+    {
+      // 64x64: T_21 = -T_22 (A_21 T_11) with 32x32 blocks; thread (r, c4) owns 4 columns
+      const int r = (tid >> 3) & 31, c4 = tid & 7;
+      if (tid < 256) {
+        const float* Arow = Msc + (32 + r) * LDM;
         float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int k4 = 0; k4 < 16 * I; k4 += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(Arow + k4);
-          const float4 t0v = *reinterpret_cast<const float4*>(Msc + (k4 + 0) * LDM + 4 * c4);
-          const float4 t1v = *reinterpret_cast<const float4*>(Msc + (k4 + 1) * LDM + 4 * c4);
-          const float4 t2v = *reinterpret_cast<const float4*>(Msc + (k4 + 2) * LDM + 4 * c4);
-          const float4 t3v = *reinterpret_cast<const float4*>(Msc + (k4 + 3) * LDM + 4 * c4);
-          z.x = fmaf(a.x, t0v.x, fmaf(a.y, t1v.x, fmaf(a.z, t2v.x, fmaf(a.w, t3v.x, z.x))));
-          z.y = fmaf(a.x, t0v.y, fmaf(a.y, t1v.y, fmaf(a.z, t2v.y, fmaf(a.w, t3v.y, z.y))));
-          z.z = fmaf(a.x, t0v.z, fmaf(a.y, t1v.z, fmaf(a.z, t2v.z, fmaf(a.w, t3v.z, z.z))));
-          z.w = fmaf(a.x, t0v.w, fmaf(a.y, t1v.w, fmaf(a.z, t2v.w, fmaf(a.w, t3v.w, z.w))));
+#pragma unroll
+        for (int k4 = 0; k4 < 32; k4 += 4) {
+          const float4 a = ld4(Arow + k4);
+          fma4(z, a.x, ld4(Msc + (k4 + 0) * LDM + 4 * c4));
+          fma4(z, a.y, ld4(Msc + (k4 + 1) * LDM + 4 * c4));
+          fma4(z, a.z, ld4(Msc + (k4 + 2) * LDM + 4 * c4));
+          fma4(z, a.w, ld4(Msc + (k4 + 3) * LDM + 4 * c4));
         }
-        *reinterpret_cast<float4*>(Xsc + r * 48 + 4 * c4) = z;
+        *reinterpret_cast<float4*>(Xsc + r * LDX + 4 * c4) = z;
       }
       __syncthreads();
-      for (int e = tid; e < 16 * nq; e += NT) {
-        const int r = e / nq, c4 = e % nq;
-        const float* Trow = Msc + (16 * I + r) * LDM + 16 * I;
+      if (tid < 256) {
+        const float* Trow = Msc + (32 + r) * LDM + 32;
         float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int s4 = 0; s4 < 16; s4 += 4) {
-          const float4 tr = *reinterpret_cast<const float4*>(Trow + s4);
-          const float4 x0 = *reinterpret_cast<const float4*>(Xsc + (s4 + 0) * 48 + 4 * c4);
-          const float4 x1 = *reinterpret_cast<const float4*>(Xsc + (s4 + 1) * 48 + 4 * c4);
-          const float4 x2 = *reinterpret_cast<const float4*>(Xsc + (s4 + 2) * 48 + 4 * c4);
-          const float4 x3 = *reinterpret_cast<const float4*>(Xsc + (s4 + 3) * 48 + 4 * c4);
-          y.x = fmaf(tr.x, x0.x, fmaf(tr.y, x1.x, fmaf(tr.z, x2.x, fmaf(tr.w, x3.x, y.x))));
-          y.y = fmaf(tr.x, x0.y, fmaf(tr.y, x1.y, fmaf(tr.z, x2.y, fmaf(tr.w, x3.y, y.y))));
-          y.z = fmaf(tr.x, x0.z, fmaf(tr.y, x1.z, fmaf(tr.z, x2.z, fmaf(tr.w, x3.z, y.z))));
-          y.w = fmaf(tr.x, x0.w, fmaf(tr.y, x1.w, fmaf(tr.z, x2.w, fmaf(tr.w, x3.w, y.w))));
+        for (int s4 = 0; s4 < 32; s4 += 4) {
+          const float4 t4 = ld4(Trow + s4);
+          fma4(y, t4.x, ld4(Xsc + (s4 + 0) * LDX + 4 * c4));
+          fma4(y, t4.y, ld4(Xsc + (s4 + 1) * LDX + 4 * c4));
+          fma4(y, t4.z, ld4(Xsc + (s4 + 2) * LDX + 4 * c4));
+          fma4(y, t4.w, ld4(Xsc + (s4 + 3) * LDX + 4 * c4));
         }
-        *reinterpret_cast<float4*>(Msc + (16 * I + r) * LDM + 4 * c4) = make_float4(-y.x, -y.y, -y.z, -y.w);
+        *reinterpret_cast<float4*>(Msc + (32 + r) * LDM + 4 * c4) = make_float4(-y.x, -y.y, -y.z, -y.w);
       }
       __syncthreads();
     }
     // T as a tf32 K-major operand [t][s]
     for (int e = tid; e < 64 * 16; e += NT) {
       const int t = e >> 4, s4 = e & 15;
-      const float4 a = *reinterpret_cast<const float4*>(Msc + t * LDM + 4 * s4);
+      const float4 a = ld4(Msc + t * LDM + 4 * s4);
       const float f[4] = {a.x, a.y, a.z, a.w};
       st4_tf32(sm + OFF_T + f32_off(t, 4 * s4, R64), f);
     }
@@ -474,17 +542,17 @@ __global__ void __launch_bounds__(NT, 1)
       }
       commit_mma();
     }
-    if (__syncthreads_or(!wait_mma())) break;
+    if (__syncthreads_or(!wait_mma())) { dead = true; break; }
     tc_fence_after();
+    if (tid == 0 && c + 1 < p.nchunks) issue_raw(c + 1);  // the KQ tile and the scratch are free
     // ===== W (token rows) to shared memory: thread = key channel i, one column ==========
     {
-      float v[32];
-      tmem_ld32(tlane + TM_W + 32 * hf, v);
+      float v[16];
+      tmem_ld16(tlane + TM_W + 16 * cq, v);
       tmem_ld_wait();
-      const int i = 32 * qd + lane;
 #pragma unroll
-      for (int x = 0; x < 32; ++x)
-        *reinterpret_cast<float*>(sm + OFF_KN + f32_off(32 * hf + x, i, R64)) = to_tf32(v[x]);
+      for (int x = 0; x < 16; ++x)
+        *reinterpret_cast<float*>(sm + OFF_KN + f32_off(16 * cq + x, jrow, R64)) = rna_tf32(v[x]);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -499,7 +567,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       commit_mma();
     }
-    if (__syncthreads_or(!wait_mma())) break;
+    if (__syncthreads_or(!wait_mma())) { dead = true; break; }
     tc_fence_after();
     if (tid == 0) {
       // O^T += U~^T P^T : A = U~^T from tensor memory, B = P (N = t), K = s
@@ -508,52 +576,32 @@ __global__ void __launch_bounds__(NT, 1)
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t bP = sdesc_sw128(sbase + OFF_P + (ks >> 2) * R64 + (ks & 3) * 32, 16, 1024);
         const uint64_t bK = sdesc_sw128(sbase + OFF_KNT + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
-        umma_tf32_ts(tmem + TM_O, tmem + TM_U + 8 * ks, bP, ID_64, 1);
+        umma_tf32_ts(tmem + TM_O + 64 * ob, tmem + TM_U + 8 * ks, bP, ID_64, 1);
         umma_tf32_ts(tmem + TM_S, tmem + TM_U + 8 * ks, bK, ID_128, 1);
       }
-      commit_mma();
+      commit_mma();  // waited on at the start of the next chunk (or below)
     }
-    if (__syncthreads_or(!wait_mma())) break;
-    tc_fence_after();
-    // ===== outputs of the chunk, and the state decay ======================================
-    {
-      float v[32];
-      tmem_ld32(tlane + TM_O + 32 * hf, v);  // O^T: lane = value channel j, columns = tokens
-      tmem_ld_wait();
-      if (jrow < dv) {
-        float* op = p.o + (((size_t)bb * p.T + t0 + 32 * hf) * p.H + h) * dv + jrow;
-        const size_t tstride = (size_t)p.H * dv;
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if (32 * hf + x < n) op[x * tstride] = v[x];
-      }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int i0 = 64 * hf + 32 * half;
-        tmem_ld32(tlane + TM_S + i0, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) v[x] *= ms.gC[i0 + x];
-        tmem_st32(tlane + TM_S + i0, v);
-      }
-      tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
   }
 
-  // ---- final state ----------------------------------------------------------------------
-  tc_fence_after();
-  if (!ms.abort && p.S_T && jrow < dv) {
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
+  // ---- last chunk's output and decay, then the final state -------------------------------
+  if (!dead && p.nchunks > 0) {
+    if (__syncthreads_or(!wait_mma())) dead = true;
+  }
+  if (!dead && p.nchunks > 0) {
+    tc_fence_after();
+    store_o(p.nchunks - 1);
+    decay_state((p.nchunks - 1) & 1);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (p.S_T && jrow < dv) {
       float v[32];
-      const int i0 = 64 * hf + 32 * half;
-      tmem_ld32(tlane + TM_S + i0, v);
+      tmem_ld32(tlane + TM_S + 32 * cq, v);
       tmem_ld_wait();
 #pragma unroll
       for (int x = 0; x < 32; ++x)
-        if (i0 + x < dk) p.S_T[((size_t)unit * dk + i0 + x) * dv + jrow] = v[x];
+        if (32 * cq + x < dk) p.S_T[((size_t)unit * dk + 32 * cq + x) * dv + jrow] = v[x];
     }
   }
   // ---- teardown: after a give-up, let outstanding async work drain (bounded) ------------
@@ -561,6 +609,7 @@ __global__ void __launch_bounds__(NT, 1)
     volatile int never = 0;
     if (pend_la) mbar_wait_bounded(&ms.bar_la, ph_la, &never, nullptr, WAIT_LIMIT);
     if (pend_mma) mbar_wait_bounded(&ms.bar_mma, ph_mma, &never, nullptr, WAIT_LIMIT);
+    if (pend_raw) mbar_wait_bounded(&ms.bar_raw, ph_raw, &never, nullptr, WAIT_LIMIT);
   }
   tc_fence_before();
   __syncthreads();
@@ -608,8 +657,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
             make_map(&mb, a.b, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
             make_map(&mv, a.v, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
             make_map(&mw, a.w, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
-            make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dk, a.dk,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
+            make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dk, 32, SW);
   if (!ok) return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
