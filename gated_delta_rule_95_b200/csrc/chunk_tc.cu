@@ -10,7 +10,7 @@
 //
 //     Kb = K*B*Gamma    Qh = Q*Gamma    Kn = K/Gamma    Vw = W*V
 //     [A; P]  = [Kb; Qh] Kn^T           A strictly lower, P lower incl. diagonal
-//     T       = (I + A)^-1              recursive 2x2 block inverse, fp32
+//     T       = (I + A)^-1              recursive 2x2 block inverse (fp32 diagonal blocks)
 //     U^T     = Vw^T T^T                W^T = Kb^T T^T
 //     U~^T    = U^T - S^T W^T           (= (U - W S)^T, the erase-corrected writes)
 //     O^T     = S^T Qh^T + U~^T P^T
@@ -111,12 +111,6 @@ __device__ __forceinline__ void st4_tf32(unsigned char* p, const float* f) {
   *reinterpret_cast<float4*>(p) = make_float4(rna_tf32(f[0]), rna_tf32(f[1]), rna_tf32(f[2]), rna_tf32(f[3]));
 }
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ void fma4(float4& z, float a, const float4& x) {
-  z.x = fmaf(a, x.x, z.x);
-  z.y = fmaf(a, x.y, z.y);
-  z.z = fmaf(a, x.z, z.z);
-  z.w = fmaf(a, x.w, z.w);
-}
 
 __global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -443,16 +437,16 @@ __global__ void __launch_bounds__(NT, 1)
         for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
 #pragma unroll
         for (int r = 1; r < 16; ++r) {
-          float acc = 0.f;
+          float acc0 = 0.f, acc1 = 0.f;  // two chains: even and odd columns
 #pragma unroll
           for (int s4 = 0; s4 < r; s4 += 4) {
             const float4 a = ld4(Ab + r * LDM + s4);
-            acc = fmaf(a.x, x[s4], acc);
-            if (s4 + 1 < r) acc = fmaf(a.y, x[s4 + 1], acc);
-            if (s4 + 2 < r) acc = fmaf(a.z, x[s4 + 2], acc);
-            if (s4 + 3 < r) acc = fmaf(a.w, x[s4 + 3], acc);
+            acc0 = fmaf(a.x, x[s4], acc0);
+            if (s4 + 1 < r) acc1 = fmaf(a.y, x[s4 + 1], acc1);
+            if (s4 + 2 < r) acc0 = fmaf(a.z, x[s4 + 2], acc0);
+            if (s4 + 3 < r) acc1 = fmaf(a.w, x[s4 + 3], acc1);
           }
-          x[r] = (r > cc) ? -acc : x[r];
+          x[r] = (r > cc) ? -(acc0 + acc1) : x[r];
         }
       }
       __syncthreads();
@@ -463,60 +457,81 @@ __global__ void __launch_bounds__(NT, 1)
       }
       __syncthreads();
     }
+    // The block products of the next two levels run as warp-level tf32 MMAs
+    // (m16n8k8) on fragments read straight from the scratch matrices.
     {
-      // 32x32 blocks: T_{2p+1,2p} = -T_{2p+1,2p+1} A_{2p+1,2p} T_{2p,2p}, p = 0, 1
-      const int pp = tid >> 8, r = (tid >> 4) & 15, cc = tid & 15;
+      // 32x32 blocks: T_{2p+1,2p} = -T_{2p+1,2p+1} (A_{2p+1,2p} T_{2p,2p}), p = 0, 1;
+      // warp 2 p + nt computes the 16 x 8 output columns [8 nt, 8 nt + 8) of block p.
+      const int g = lane >> 2, t = lane & 3;
+      const int pp = warp >> 1, nt = warp & 1;
       const int I = 2 * pp + 1, J = 2 * pp;
-      const float* Arow = Msc + (16 * I + r) * LDM + 16 * J;
-      float z = 0.f;
+      float* Xp = Xsc + 16 * pp * LDX;
+      if (warp < 4) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int s4 = 0; s4 < 16; s4 += 4) {
-        const float4 a = ld4(Arow + s4);
-        const float* Tc = Msc + (16 * J + s4) * LDM + 16 * J + cc;
-        z = fmaf(a.x, Tc[0], fmaf(a.y, Tc[LDM], fmaf(a.z, Tc[2 * LDM], fmaf(a.w, Tc[3 * LDM], z))));
+        for (int ks = 0; ks < 2; ++ks) {
+          const float* Ar = Msc + (16 * I + g) * LDM + 16 * J + 8 * ks + t;
+          const float* Bc = Msc + (16 * J + 8 * ks + t) * LDM + 16 * J + 8 * nt + g;
+          const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                 __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+          const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
+          mma_16x8x8_tf32(d, a, b);
+        }
+        *reinterpret_cast<float2*>(Xp + g * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(Xp + (g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
       }
-      Xsc[pp * 256 + r * 16 + cc] = z;
       __syncthreads();
-      const float* Trow = Msc + (16 * I + r) * LDM + 16 * I;
-      float y = 0.f;
+      if (warp < 4) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int s4 = 0; s4 < 16; s4 += 4) {
-        const float4 t4 = ld4(Trow + s4);
-        const float* Xc = Xsc + pp * 256 + s4 * 16 + cc;
-        y = fmaf(t4.x, Xc[0], fmaf(t4.y, Xc[16], fmaf(t4.z, Xc[32], fmaf(t4.w, Xc[48], y))));
+        for (int ks = 0; ks < 2; ++ks) {
+          const float* Ar = Msc + (16 * I + g) * LDM + 16 * I + 8 * ks + t;
+          const float* Bc = Xp + (8 * ks + t) * LDX + 8 * nt + g;
+          const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                 __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+          const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
+          mma_16x8x8_tf32(d, a, b);
+        }
+        float* Tr = Msc + (16 * I + g) * LDM + 16 * J + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
+        *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
       }
-      Msc[(16 * I + r) * LDM + 16 * J + cc] = -y;
       __syncthreads();
     }
     {
-      // 64x64: T_21 = -T_22 (A_21 T_11) with 32x32 blocks; thread (r, c4) owns 4 columns
-      const int r = (tid >> 3) & 31, c4 = tid & 7;
-      if (tid < 256) {
-        const float* Arow = Msc + (32 + r) * LDM;
-        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      // 64x64: T_21 = -T_22 (A_21 T_11) with 32x32 blocks; warp 4 mt + nt (8 warps)
+      // computes the 16 x 8 output tile (rows [16 mt, +16), columns [8 nt, +8)).
+      const int g = lane >> 2, t = lane & 3;
+      const int mt = (warp >> 2) & 1, nt = warp & 3;
+      if (warp < 8) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k4 = 0; k4 < 32; k4 += 4) {
-          const float4 a = ld4(Arow + k4);
-          fma4(z, a.x, ld4(Msc + (k4 + 0) * LDM + 4 * c4));
-          fma4(z, a.y, ld4(Msc + (k4 + 1) * LDM + 4 * c4));
-          fma4(z, a.z, ld4(Msc + (k4 + 2) * LDM + 4 * c4));
-          fma4(z, a.w, ld4(Msc + (k4 + 3) * LDM + 4 * c4));
+        for (int ks = 0; ks < 4; ++ks) {
+          const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 8 * ks + t;
+          const float* Bc = Msc + (8 * ks + t) * LDM + 8 * nt + g;
+          const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                 __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+          const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
+          mma_16x8x8_tf32(d, a, b);
         }
-        *reinterpret_cast<float4*>(Xsc + r * LDX + 4 * c4) = z;
+        *reinterpret_cast<float2*>(Xsc + (16 * mt + g) * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(Xsc + (16 * mt + g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
       }
       __syncthreads();
-      if (tid < 256) {
-        const float* Trow = Msc + (32 + r) * LDM + 32;
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (warp < 8) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int s4 = 0; s4 < 32; s4 += 4) {
-          const float4 t4 = ld4(Trow + s4);
-          fma4(y, t4.x, ld4(Xsc + (s4 + 0) * LDX + 4 * c4));
-          fma4(y, t4.y, ld4(Xsc + (s4 + 1) * LDX + 4 * c4));
-          fma4(y, t4.z, ld4(Xsc + (s4 + 2) * LDX + 4 * c4));
-          fma4(y, t4.w, ld4(Xsc + (s4 + 3) * LDX + 4 * c4));
+        for (int ks = 0; ks < 4; ++ks) {
+          const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 32 + 8 * ks + t;
+          const float* Bc = Xsc + (8 * ks + t) * LDX + 8 * nt + g;
+          const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                 __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+          const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
+          mma_16x8x8_tf32(d, a, b);
         }
-        *reinterpret_cast<float4*>(Msc + (32 + r) * LDM + 4 * c4) = make_float4(-y.x, -y.y, -y.z, -y.w);
+        float* Tr = Msc + (32 + 16 * mt + g) * LDM + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
+        *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
       }
       __syncthreads();
     }

@@ -238,4 +238,16 @@ __device__ __forceinline__ uint32_t f32_off(int row, int col, uint32_t panel_byt
   return (uint32_t)(col >> 5) * panel_bytes + sw128_off(row, (col & 31) >> 2) + (uint32_t)((col & 3) << 2);
 }
 
+
+// Warp-level tensor-core product D += A B with A 16x8 (row-major), B 8x8 (column-major),
+// tf32 inputs (fp32 bit patterns whose low 13 bits are ignored), fp32 accumulate.
+// Fragments, with g = lane / 4 and t = lane % 4: a = {A[g][t], A[g+8][t], A[g][t+4],
+// A[g+8][t+4]}, b = {B[t][g], B[t+4][g]}, d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 }  // namespace gdn2
