@@ -74,7 +74,7 @@ struct Misc {
   uint64_t bar_la, bar_mma, bar_raw;
   uint32_t tmem_base;
   int abort;
-  float gC[2][128];  // Gamma at the chunk end, per key channel (chunk parity)
+  alignas(16) float gC[2][128];  // Gamma at the chunk end, per key channel (chunk parity)
 };
 constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 
@@ -149,7 +149,8 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tmem = ms.tmem_base;
   const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
 
-  // ---- async copies (thread 0) ---------------------------------------------------------
+  // ---- async copies (issued by thread TMA_TID, so that thread 0 only issues MMAs) ----------
+  constexpr int TMA_TID = 32;
   int pend_la = 0, pend_mma = 0, pend_raw = 0;
   auto prefetch_raw = [&](int c) {  // raw bf16 inputs of chunk c into L2
     for (int pn = 0; pn < (dk >> 6); ++pn) {
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     pend_raw = 1;
   };
-  if (tid == 0 && p.nchunks > 0) {
+  if (tid == TMA_TID && p.nchunks > 0) {
     issue_raw(0);
     issue_la(0);
     if (p.nchunks > 1) prefetch_raw(1);
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(NT, 1)
     const bool ok = mbar_wait_bounded(bar, ph, &ms.abort, p.err, WAIT_LIMIT);
     if (ok) {
       ph ^= 1;
-      if (tid == 0) pend = 0;
+      pend = 0;
     }
     return ok;
   };
@@ -240,7 +241,13 @@ __global__ void __launch_bounds__(NT, 1)
     tmem_ld32(tlane + TM_S + 32 * cq, v);
     tmem_ld_wait();
 #pragma unroll
-    for (int x = 0; x < 32; ++x) v[x] *= ms.gC[gb][32 * cq + x];
+    for (int x = 0; x < 32; x += 4) {
+      const float4 gq = *reinterpret_cast<const float4*>(&ms.gC[gb][32 * cq + x]);
+      v[x] *= gq.x;
+      v[x + 1] *= gq.y;
+      v[x + 2] *= gq.z;
+      v[x + 3] *= gq.w;
+    }
     tmem_st32(tlane + TM_S + 32 * cq, v);
   };
   tc_fence_before();
@@ -249,9 +256,10 @@ __global__ void __launch_bounds__(NT, 1)
   bool dead = false;
   for (int c = 0; c < p.nchunks; ++c) {
     const int ob = c & 1;
-    if (tid == 0 && c + 2 < p.nchunks) prefetch_raw(c + 2);
+    if (tid == TMA_TID && c + 2 < p.nchunks) prefetch_raw(c + 2);
     // ===== decay cumsum by warp scan, then the folded operands in registers ============
-    // Warp w owns channels [8 w, 8 w + 8); lane l owns tokens 2 l and 2 l + 1.
+    // Warp w owns channels [8 w, 8 w + 8); lane l owns tokens l and l + 32 (rows that
+    // differ in their low bits, so the swizzled tile accesses are conflict-free).
     {
       bool ok = wait_on(&ms.bar_la, ph_la, pend_la);
       ok = ok && wait_on(&ms.bar_raw, ph_raw, pend_raw);
@@ -266,9 +274,9 @@ __global__ void __launch_bounds__(NT, 1)
         if (kval) {
           const float* row = la;  // element (t, i) at f32_off(t, i, R64)
           const float4 x0 = ld4(reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(row) +
-                                                               f32_off(2 * lane + m, c0, R64)));
+                                                               f32_off(lane + 32 * m, c0, R64)));
           const float4 x1 = ld4(reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(row) +
-                                                               f32_off(2 * lane + m, c0 + 4, R64)));
+                                                               f32_off(lane + 32 * m, c0 + 4, R64)));
           a[m][0] = x0.x; a[m][1] = x0.y; a[m][2] = x0.z; a[m][3] = x0.w;
           a[m][4] = x1.x; a[m][5] = x1.y; a[m][6] = x1.z; a[m][7] = x1.w;
         } else {
@@ -279,17 +287,20 @@ __global__ void __launch_bounds__(NT, 1)
       float gtot[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float tot = a[0][e] + a[1][e];
-        float inc = tot;
+        float i0 = a[0][e], i1 = a[1][e];  // inclusive scans over tokens 0..31 and 32..63
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, inc, off);
-          if (lane >= off) inc += y;
+          const float y0 = __shfl_up_sync(0xffffffffu, i0, off);
+          const float y1 = __shfl_up_sync(0xffffffffu, i1, off);
+          if (lane >= off) {
+            i0 += y0;
+            i1 += y1;
+          }
         }
-        const float exc = inc - tot;
-        a[0][e] = exc + a[0][e];  // g at token 2 l
-        a[1][e] = inc;            // g at token 2 l + 1
-        gtot[e] = __shfl_sync(0xffffffffu, inc, 31);
+        const float half = __shfl_sync(0xffffffffu, i0, 31);
+        a[0][e] = i0;         // g at token l
+        a[1][e] = i1 + half;  // g at token l + 32
+        gtot[e] = __shfl_sync(0xffffffffu, a[1][e], 31);
       }
       if (lane == 0) {
 #pragma unroll
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
-        const uint32_t ro = (uint32_t)(c0 >> 6) * R64 + sw128_off(2 * lane + m, (c0 & 63) >> 3);
+        const uint32_t ro = (uint32_t)(c0 >> 6) * R64 + sw128_off(lane + 32 * m, (c0 & 63) >> 3);
         const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
         const bool vval = c0 < dv;
         float kk[8], bgt[8], qq[8], vv[8], ww[8];
@@ -323,11 +334,11 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       if (__syncthreads_or(!ok)) { dead = true; break; }
     }
-    if (tid == 0 && c + 1 < p.nchunks) issue_la(c + 1);  // the log-alpha tile has been read
+    if (tid == TMA_TID && c + 1 < p.nchunks) issue_la(c + 1);  // the log-alpha tile has been read
     tc_fence_after();
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      const int t = 2 * lane + m;
+      const int t = lane + 32 * m;
       st4_tf32(sm + OFF_KQ + f32_off(t, c0, R128), kb[m]);
       st4_tf32(sm + OFF_KQ + f32_off(t, c0 + 4, R128), kb[m] + 4);
       st4_tf32(sm + OFF_KQ + f32_off(64 + t, c0, R128), qh[m]);
@@ -395,7 +406,8 @@ __global__ void __launch_bounds__(NT, 1)
         umma_tf32_ts(tmem + TM_O + 64 * ob, tmem + TM_S + 8 * ks, bQH, ID_64, ks > 0);
       }
     }
-    if (__syncthreads_or(!wait_mma())) { dead = true; break; }
+    // the other threads read A and P out while thread 0 is still issuing
+    const bool ok_ap = wait_mma();
     tc_fence_after();
     // ===== A to the solve scratch, P to its operand tile =====================================
     {
@@ -425,7 +437,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
     }
-    __syncthreads();
+    if (__syncthreads_or(!ok_ap)) { dead = true; break; }
     // ===== T = (I + A)^-1: 16x16 diagonal blocks, then 32x32, then 64x64 ===================
     // Every entry above the diagonal is an explicit zero, so block products run dense.
     {
@@ -559,7 +571,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     if (__syncthreads_or(!wait_mma())) { dead = true; break; }
     tc_fence_after();
-    if (tid == 0 && c + 1 < p.nchunks) issue_raw(c + 1);  // the KQ tile and the scratch are free
+    if (tid == TMA_TID && c + 1 < p.nchunks) issue_raw(c + 1);  // the KQ tile and the scratch are free
     // ===== W (token rows) to shared memory: thread = key channel i, one column ==========
     {
       float v[16];
@@ -620,7 +632,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
   }
   // ---- teardown: after a give-up, let outstanding async work drain (bounded) ------------
-  if (tid == 0 && ms.abort) {
+  if ((tid == 0 || tid == TMA_TID) && ms.abort) {
     volatile int never = 0;
     if (pend_la) mbar_wait_bounded(&ms.bar_la, ph_la, &never, nullptr, WAIT_LIMIT);
     if (pend_mma) mbar_wait_bounded(&ms.bar_mma, ph_mma, &never, nullptr, WAIT_LIMIT);
