@@ -59,7 +59,8 @@ constexpr uint32_t OFF_KN = OFF_KQ + 4 * R128;  // Kn [s][i]: 4 panels x 64 rows
 constexpr uint32_t OFF_KNT = OFF_KN + 4 * R64;  // Kn^T [i][s]: 2 panels x 128 rows
 constexpr uint32_t OFF_T = OFF_KNT + 2 * R128;  // T [t][s]: 2 panels x 64 rows (first: Vw [t][j], 32 KB over T and P)
 constexpr uint32_t OFF_P = OFF_T + 2 * R64;     // P [t][s]: 2 panels x 64 rows
-constexpr uint32_t OFF_LA = OFF_P + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows
+constexpr uint32_t OFF_LA = OFF_P + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows;
+                                                // between uses: the output tile [t][j] fp32 of a TMA store
 constexpr uint32_t OFF_SCR = OFF_LA + 4 * R64;  // solve scratch: fp32 64 x LDM, then 32 x LDX (first: raw w)
 // raw bf16 staging (TMA, 128B swizzle): a [64 tokens][128 channels] tile = 2 panels of
 // 64 channels x 64 rows
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmLA,
-                        const TcParams p) {
+                        const __grid_constant__ CUtensorMap tmO, const TcParams p) {
   extern __shared__ unsigned char smem_raw[];
   // 128B-swizzled tiles need 1024-byte aligned shared addresses
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(NT, 1)
     ms.abort = 0;
     tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmB); tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmLA);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 0) {
     tmem_alloc(&ms.tmem_base, TM_COLS);
@@ -221,19 +223,21 @@ __global__ void __launch_bounds__(NT, 1)
     umma_commit(&ms.bar_mma);
     pend_mma = 1;
   };
-  // Output of chunk cc (O^T in tensor-memory buffer cc & 1) to global memory.
-  auto store_o = [&](int cc) {
+  // Output of chunk cc (O^T in tensor-memory buffer cc & 1) into the shared-memory
+  // tile [t][j] (rows of d_v floats) that a TMA store then writes out.
+  auto stage_o = [&](int cc) {
     float v[16];
     tmem_ld16(tlane + TM_O + 64 * (cc & 1) + 16 * cq, v);
     tmem_ld_wait();
-    const int tb = C * cc, nn = min(C, p.T - tb);
     if (jrow < dv) {
-      float* op = p.o + (((size_t)bb * p.T + tb + 16 * cq) * p.H + h) * dv + jrow;
-      const size_t tstride = (size_t)p.H * dv;
+      float* st = reinterpret_cast<float*>(sm + OFF_LA) + jrow;
 #pragma unroll
-      for (int x = 0; x < 16; ++x)
-        if (16 * cq + x < nn) op[x * tstride] = v[x];
+      for (int x = 0; x < 16; ++x) st[(16 * cq + x) * dv] = v[x];
     }
+  };
+  auto store_o = [&](int cc) {  // thread TMA_TID, after the staging is visible
+    tma_store_4d(&tmO, sm + OFF_LA, 0, h, C * cc, bb);
+    bulk_commit();
   };
   // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory.
   auto decay_state = [&](int gb) {
@@ -334,7 +338,6 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       if (__syncthreads_or(!ok)) { dead = true; break; }
     }
-    if (tid == TMA_TID && c + 1 < p.nchunks) issue_la(c + 1);  // the log-alpha tile has been read
     tc_fence_after();
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
@@ -389,13 +392,14 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
     if (c > 0) {
-      store_o(c - 1);
+      stage_o(c - 1);  // the log-alpha tile is free until the next chunk's copy
       decay_state(ob ^ 1);
     }
     tmem_st_wait();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == TMA_TID && c > 0) store_o(c - 1);
     if (tid == 0) {
       tc_fence_after();
       // O^T = S^T Qh^T : A = S^T from tensor memory, B = Qh rows of the KQ tile
@@ -557,6 +561,10 @@ __global__ void __launch_bounds__(NT, 1)
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == TMA_TID && c + 1 < p.nchunks) {
+      bulk_wait_read_all();  // the output staging has been read
+      issue_la(c + 1);
+    }
     if (tid == 0) {
       tc_fence_after();
       // U^T = Vw^T T^T : A = Vw^T (tensor memory), B = T (N = t), K = s
@@ -612,16 +620,19 @@ __global__ void __launch_bounds__(NT, 1)
 
   // ---- last chunk's output and decay, then the final state -------------------------------
   if (!dead && p.nchunks > 0) {
+    if (tid == TMA_TID) bulk_wait_read_all();  // the staging tile is about to be rewritten
     if (__syncthreads_or(!wait_mma())) dead = true;
   }
   if (!dead && p.nchunks > 0) {
     tc_fence_after();
-    store_o(p.nchunks - 1);
+    stage_o(p.nchunks - 1);
     decay_state((p.nchunks - 1) & 1);
     tmem_st_wait();
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid == TMA_TID) store_o(p.nchunks - 1);
     if (p.S_T && jrow < dv) {
       float v[32];
       tmem_ld32(tlane + TM_S + 32 * cq, v);
@@ -638,6 +649,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (pend_mma) mbar_wait_bounded(&ms.bar_mma, ph_mma, &never, nullptr, WAIT_LIMIT);
     if (pend_raw) mbar_wait_bounded(&ms.bar_raw, ph_raw, &never, nullptr, WAIT_LIMIT);
   }
+  if (tid == TMA_TID) bulk_wait_all();  // output stores complete before the block exits
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -676,7 +688,7 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
 
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   if (a.B * a.H == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv, mb, mw, mla;
+  CUtensorMap mq, mk, mv, mb, mw, mla, mo;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
   bool ok = make_map(&mq, a.q, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
@@ -684,7 +696,9 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
             make_map(&mb, a.b, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
             make_map(&mv, a.v, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
             make_map(&mw, a.w, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
-            make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dk, 32, SW);
+            make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dk, 32, SW) &&
+            make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dv, a.dv,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
@@ -708,7 +722,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   p.dv = a.dv;
   p.nchunks = (a.T + C - 1) / C;
   p.err = device_error_word();
-  chunk_fwd_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, p);
+  chunk_fwd_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
   return cudaGetLastError();
 }
 
