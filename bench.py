@@ -89,18 +89,17 @@ class Clocks:
             idx = int(ids[self.index]) if ids and ids[self.index].strip().isdigit() else self.index
             return N.nvmlDeviceGetHandleByIndex(idx)
 
+    def _sample(self, N):
+        self.sm.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+        r = self.getr(self.h)
+        for name, bit in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
     def _run(self):
         import pynvml as N
-        h = self._handle()
-        self.mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
-        getr = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-            N.nvmlDeviceGetCurrentClocksThrottleReasons
         while not self.stop:
-            self.sm.append(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
-            r = getr(h)
-            for name, bit in self.REASONS.items():
-                if r & bit:
-                    self.reasons.add(name)
+            self._sample(N)
             time.sleep(self.period)
 
     def __enter__(self):
@@ -110,6 +109,11 @@ class Clocks:
         try:
             import pynvml as N
             N.nvmlInit()
+            self.h = self._handle()
+            self.mx = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.getr = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                N.nvmlDeviceGetCurrentClocksThrottleReasons
+            self._sample(N)
             self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
         except Exception:
@@ -120,6 +124,11 @@ class Clocks:
         self.stop = True
         if self.thread is not None:
             self.thread.join(timeout=2)
+            try:
+                import pynvml as N
+                self._sample(N)
+            except Exception:
+                pass
 
     def summary(self):
         if not self.sm:
@@ -128,7 +137,8 @@ class Clocks:
                 "samples": len(self.sm), "source": "NVML during the timed region"}
 
 
-def dist_init(n):
+def dist_init(n, backend="nccl"):
+    """One process per GPU: reads RANK / WORLD_SIZE / LOCAL_RANK from the environment."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world != n:
@@ -136,8 +146,13 @@ def dist_init(n):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return rank, world, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def job_throughput(world, units_per_rank, ms_max):
+    """Whole-job rate: every rank processes units_per_rank in the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 def max_over_ranks(x, world, device):
@@ -340,7 +355,7 @@ def main():
 
     pre = time_prefill(args, rank, world, dev)
     ms = pre["total_ms"] / args.steps
-    value = world * pre["tokens"] / (ms * 1e-3)
+    value = job_throughput(world, pre["tokens"], ms)
     achieved = pre["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (pre["kernel_ms"] * 1e-3) / 1e9
     tflops = pre["token_heads"] * PREFILL_FLOP_PER_TOKEN_HEAD / (pre["kernel_ms"] * 1e-3) / 1e12
     traffic = profile_traffic("chunk_fwd_tc_kernel")
