@@ -38,6 +38,8 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 5 * 128 * 2 + 128 * 4 + 128 * 4
 PREFILL_FLOP_PER_TOKEN_HEAD = 2 * 64 * (3 * 128 + 2 * 128) + 6 * 128 * 128
 # state read + write per (sequence, head) and step, fp32 128x128
 DECODE_STATE_BYTES = 2 * 128 * 128 * 4
+# nominal dense tf32 : bf16 tensor throughput on B200 (1.1 : 2.25 PFLOP/s); the products run in tf32
+TF32_PER_BF16 = 1.1 / 2.25
 
 
 def peaks():
@@ -373,7 +375,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, see DESIGN.md)",
+        "vs_baseline": None, "dtype": "tf32", "data": "synthetic (seeded, see DESIGN.md)",
         "config": config_dict(),
         "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel", "achieved": achieved,
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
@@ -381,6 +383,8 @@ def main():
                      "bytes_per_token_head": PREFILL_BYTES_PER_TOKEN_HEAD,
                      "tensor": {"achieved_tflops": tflops, "peak_tflops": pk["bf16_tflops"],
                                 "frac": tflops / pk["bf16_tflops"],
+                                "peak_tflops_tf32": pk["bf16_tflops"] * TF32_PER_BF16,
+                                "frac_tf32": tflops / (pk["bf16_tflops"] * TF32_PER_BF16),
                                 "flop_per_token_head": PREFILL_FLOP_PER_TOKEN_HEAD}},
         "decode": {"metric": "GDN-2 decode steps/s", "value": 1e3 / dec["ms_per_step"], "unit": "steps/s",
                    "ms_per_step": dec["ms_per_step"], "steps": args.decode_steps,
