@@ -23,16 +23,19 @@
 // the A operand of the next products; so are R^T and U~^T, which are rounded to tf32
 // in place first.  Shared-memory operands are rounded to tf32 (nearest).
 //
-// One CTA (512 threads, 16 warps) owns one (batch, head) and walks its chunks.
-// Thread t owns channel ch = t mod 128 (a key channel and a value channel, and the
-// tensor-memory lane of the same index) over the 16 tokens [16 sg, 16 sg + 16),
-// sg = t / 128: the decay cumsum runs along its own tokens, and the operand tiles,
-// Kn^T and the Vw^T accumulator preload are written without any transposition.
-// Thread 0 issues the MMAs, thread 256 every TMA copy.  While [A; P] is on the tensor
-// cores the previous chunk's output is staged for a TMA store and its state decay is
-// applied; the state product runs while warps 0-7 invert (I + A), and warps 8-15
-// round R^T and start the next chunk's copies.  The next chunk's raw inputs are
-// prefetched into L2 two chunks ahead.
+// One CTA owns one (batch, head) and walks its chunks.  Warps 0-15 (512 threads) do the
+// elementwise work: thread t owns channel ch = t mod 128 (a key channel and a value
+// channel, and the tensor-memory lane of the same index) over the 16 tokens
+// [16 sg, 16 sg + 16), sg = t / 128, so the decay cumsum runs along its own tokens and
+// the operand tiles, Kn^T and the Vw^T accumulator preload are written without any
+// transposition.  Warp 16 is the control warp: its first thread issues every MMA and
+// every TMA copy, so that an issue that stalls on a full tensor-core queue never holds
+// up the elementwise warps.  The two sides hand over through mbarriers only (every wait
+// bounded).  While [A; P] is on the tensor cores the previous chunk's output is staged
+// for a TMA store and its state decay is applied; the state product runs while warps
+// 0-7 invert (I + A), and warps 8-15 round R^T; the next chunk's raw inputs are copied
+// as soon as the state product has released their tiles, and prefetched into L2 two
+// chunks ahead.
 // d_k or d_v = 64 run the same code with the upper half of each operand zero.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -46,9 +49,11 @@ namespace gdn2 {
 namespace {
 
 constexpr int C = 64;
-constexpr int NT = 512;
+constexpr int NCOMP = 512;                      // warps 0-15: elementwise work
+constexpr int NT = NCOMP + 32;                  // + the control warp
+constexpr int CTL = NCOMP;                      // the thread that issues MMAs and TMA copies
 constexpr int NSOLVE = 256;                     // warps 0-7 run the triangular solve
-constexpr int TMA_TID = 256;                    // first thread of warp 8 issues every TMA copy
+constexpr int BAR_COMP = 1, BAR_SOLVE = 2;      // named barriers: all compute warps; solve warps
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -56,12 +61,12 @@ constexpr float LOG2E = 1.4426950408889634f;
 // fp32 operand tiles with the 128B swizzle, in panels of 32 columns (128 B rows).
 constexpr uint32_t R64 = 64 * 128;    // a panel of 64 rows  (8 KB)
 constexpr uint32_t R128 = 128 * 128;  // a panel of 128 rows (16 KB)
+constexpr uint32_t R192 = 192 * 128;  // a panel of 192 rows (24 KB)
 constexpr uint32_t OFF_KQ = 0;                  // [-Kb; Qh] [t][i]: 4 panels x 128 rows (first: raw q, k, b, v)
 constexpr uint32_t OFF_KN = OFF_KQ + 4 * R128;  // Kn [s][i]: 4 panels x 64 rows (first: raw w)
-constexpr uint32_t OFF_KNT = OFF_KN + 4 * R64;  // Kn^T [i][s]: 2 panels x 128 rows
-constexpr uint32_t OFF_T = OFF_KNT + 2 * R128;  // T [t][s]: 2 panels x 64 rows
-constexpr uint32_t OFF_P = OFF_T + 2 * R64;     // P [t][s]: 2 panels x 64 rows
-constexpr uint32_t OFF_LA = OFF_P + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows;
+constexpr uint32_t OFF_PK = OFF_KN + 4 * R64;   // [P; Kn^T] [t | i][s]: 2 panels x 192 rows
+constexpr uint32_t OFF_T = OFF_PK + 2 * R192;   // T [t][s]: 2 panels x 64 rows
+constexpr uint32_t OFF_LA = OFF_T + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows;
                                                 // between uses: the output tile [t][j] fp32 of a TMA store
 constexpr uint32_t OFF_SCR = OFF_LA + 4 * R64;  // solve scratch: fp32 64 x LDM, then 32 x LDX
 // raw bf16 staging (TMA, 128B swizzle): a [64 tokens][128 channels] tile = 2 panels of
@@ -74,7 +79,9 @@ constexpr int LDX = 36;                         // padded row of the 32 x 32 blo
 constexpr uint32_t TILES = OFF_SCR + 22528;     // 214 KB
 
 struct Misc {
-  uint64_t bar_la, bar_mma, bar_raw, bar_s, bar_drain;
+  uint64_t bar_la, bar_raw;                            // TMA loads landed
+  uint64_t bar_mma, bar_s, bar_drain;                  // tensor-core products done
+  uint64_t bar_ops, bar_stage, bar_solved, bar_uround;  // compute warps -> control warp (16 arrivals)
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[2][128];    // Gamma at the chunk end, per key channel (chunk parity)
@@ -84,15 +91,16 @@ constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 
 // ---- tensor memory columns (fp32, 128 lanes) -------------------------------------------
 constexpr uint32_t TM_AP = 0;    // [-A; P]      lanes: tokens of Kb | Qh, columns: s
-constexpr uint32_t TM_R = 64;    // R^T          lanes: value channel, columns: t
-constexpr uint32_t TM_O = 128;   // O^T          lanes: value channel, columns: t (adjacent to R^T)
-constexpr uint32_t TM_U = 192;   // U~^T         lanes: value channel, columns: s
+constexpr uint32_t TM_U = 64;    // U~^T         lanes: value channel, columns: s
+constexpr uint32_t TM_R = 128;   // R^T          lanes: value channel, columns: t
+constexpr uint32_t TM_O = 192;   // O^T          lanes: value channel, columns: t (after R^T, before S^T)
 constexpr uint32_t TM_S = 256;   // S^T (state)  lanes: value channel, columns: key channel
 constexpr uint32_t TM_COLS = 512;
 
 // instruction descriptors (M = 128, both operands K-major)
 constexpr uint32_t ID_64 = idesc_tf32(128, 64, 0, 0, 0, 0);
 constexpr uint32_t ID_128 = idesc_tf32(128, 128, 0, 0, 0, 0);
+constexpr uint32_t ID_192 = idesc_tf32(128, 192, 0, 0, 0, 0);
 
 struct TcParams {
   const __nv_bfloat16 *q, *k, *v, *b, *w;
@@ -128,7 +136,7 @@ __global__ void __launch_bounds__(NT, 1)
   Misc& ms = *reinterpret_cast<Misc*>(sm + TILES);
   const uint32_t sbase = smem_u32(sm);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int ch = tid & 127;  // channel (key i and value j) and tensor-memory lane
   const int sg = tid >> 7;   // token segment [16 sg, 16 sg + 16); column group of TMEM accesses
   const int unit = blockIdx.x, bb = unit / p.H, h = unit % p.H;
@@ -141,6 +149,10 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(&ms.bar_raw, 1);
     mbar_init(&ms.bar_s, 1);
     mbar_init(&ms.bar_drain, 1);
+    mbar_init(&ms.bar_ops, NCOMP / 32);
+    mbar_init(&ms.bar_stage, NCOMP / 32);
+    mbar_init(&ms.bar_solved, NCOMP / 32);
+    mbar_init(&ms.bar_uround, NCOMP / 32);
     fence_mbar_init();
     ms.abort = 0;
     tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
@@ -157,466 +169,464 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tmem = ms.tmem_base;
   const uint32_t tlane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // lanes [32 (warp mod 4), +32)
 
-  // ---- async copies (thread TMA_TID) ------------------------------------------------------
-  int pend_la = 0, pend_mma = 0, pend_raw = 0, pend_s = 0;
-  auto prefetch_raw = [&](int c) {  // raw bf16 inputs of chunk c into L2
-    for (int pn = 0; pn < (dk >> 6); ++pn) {
-      tma_prefetch_l2_4d(&tmQ, 64 * pn, h, C * c, bb);
-      tma_prefetch_l2_4d(&tmK, 64 * pn, h, C * c, bb);
-      tma_prefetch_l2_4d(&tmB, 64 * pn, h, C * c, bb);
-    }
-    for (int pn = 0; pn < (dv >> 6); ++pn) {
-      tma_prefetch_l2_4d(&tmV, 64 * pn, h, C * c, bb);
-      tma_prefetch_l2_4d(&tmW, 64 * pn, h, C * c, bb);
-    }
-  };
-  auto issue_la = [&](int c) {  // log alpha of chunk c: dk/32 boxes of 32 channels x 64 tokens
-    mbar_arrive_expect_tx(&ms.bar_la, (uint32_t)(C * dk * 4));
-    for (int pn = 0; pn < (dk >> 5); ++pn)
-      tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, C * c, bb);
-    pend_la = 1;
-  };
-  auto issue_raw = [&](int c) {  // raw bf16 inputs of chunk c into the staging tiles
-    mbar_arrive_expect_tx(&ms.bar_raw, (uint32_t)(3 * (dk >> 6) + 2 * (dv >> 6)) * R64);
-    for (int pn = 0; pn < (dk >> 6); ++pn) {
-      tma_load_4d(sm + RAW_Q + pn * R64, &tmQ, &ms.bar_raw, 64 * pn, h, C * c, bb);
-      tma_load_4d(sm + RAW_K + pn * R64, &tmK, &ms.bar_raw, 64 * pn, h, C * c, bb);
-      tma_load_4d(sm + RAW_B + pn * R64, &tmB, &ms.bar_raw, 64 * pn, h, C * c, bb);
-    }
-    for (int pn = 0; pn < (dv >> 6); ++pn) {
-      tma_load_4d(sm + RAW_V + pn * R64, &tmV, &ms.bar_raw, 64 * pn, h, C * c, bb);
-      tma_load_4d(sm + RAW_W + pn * R64, &tmW, &ms.bar_raw, 64 * pn, h, C * c, bb);
-    }
-    pend_raw = 1;
-  };
-  if (tid == TMA_TID && p.nchunks > 0) {
-    issue_raw(0);
-    issue_la(0);
-    if (p.nchunks > 1) prefetch_raw(1);
-  }
 
-  // ---- entering state S0 -> S^T in tensor memory -----------------------------------------
-  // Thread (ch, sg) owns lane j = ch (a value channel) and the key-channel columns
-  // [32 sg, 32 sg + 32) of S^T.
-  {
-    float v[32];
-    const bool ok = p.S0 && vval;
-#pragma unroll
-    for (int x = 0; x < 32; ++x) {
-      const int i = 32 * sg + x;
-      v[x] = (ok && i < dk) ? p.S0[((size_t)unit * dk + i) * dv + ch] : 0.f;
-    }
-    tmem_st32(tlane + TM_S + 32 * sg, v);
-    tmem_st_wait();
-  }
-
-  uint32_t ph_la = 0, ph_mma = 0, ph_raw = 0, ph_s = 0;
-  float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);                  // solve matrix, 64 x LDM fp32
-  float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);   // block product, 32 x LDX fp32
-  const unsigned char* la_t = sm + OFF_LA;
-
-  auto wait_on = [&](uint64_t* bar, uint32_t& ph, int& pend) -> bool {
+  auto wait_on = [&](uint64_t* bar, uint32_t& ph) -> bool {
     const bool ok = mbar_wait_bounded(bar, ph, &ms.abort, p.err, WAIT_LIMIT);
-    if (ok) {
-      ph ^= 1;
-      pend = 0;
-    }
+    if (ok) ph ^= 1;
     return ok;
   };
-  auto wait_mma = [&]() -> bool { return wait_on(&ms.bar_mma, ph_mma, pend_mma); };
-  auto commit_mma = [&]() {
-    umma_commit(&ms.bar_mma);
-    pend_mma = 1;
+  auto warp_arrive = [&](uint64_t* bar) {  // one arrival per warp, after all its lanes
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(bar);
   };
-  // Output of the last finished chunk (O^T in tensor memory) into the shared-memory
-  // tile [t][j] (rows of d_v floats) that a TMA store then writes out.
-  auto stage_o = [&]() {
-    float v[16];
-    tmem_ld16(tlane + TM_O + 16 * sg, v);
-    tmem_ld_wait();
-    if (vval) {
-      float* st = reinterpret_cast<float*>(sm + OFF_LA) + ch;
-#pragma unroll
-      for (int x = 0; x < 16; ++x) st[(16 * sg + x) * dv] = v[x];
-    }
-  };
-  auto store_o = [&](int cc) {  // thread TMA_TID, after the staging is visible
-    tma_store_4d(&tmO, sm + OFF_LA, 0, h, C * cc, bb);
-    bulk_commit();
-  };
-  // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory.
-  auto decay_state = [&](int gb) {
-    float v[32];
-    tmem_ld32(tlane + TM_S + 32 * sg, v);
-    tmem_ld_wait();
-#pragma unroll
-    for (int x = 0; x < 32; x += 4) {
-      const float4 gq = *reinterpret_cast<const float4*>(&ms.gC[gb][32 * sg + x]);
-      v[x] *= gq.x;
-      v[x + 1] *= gq.y;
-      v[x + 2] *= gq.z;
-      v[x + 3] *= gq.w;
-    }
-    tmem_st32(tlane + TM_S + 32 * sg, v);
-  };
-  tc_fence_before();
-  __syncthreads();
 
-  bool dead = false;
-  for (int c = 0; c < p.nchunks; ++c) {
-    const int ob = c & 1;
-    if (tid == TMA_TID && c + 2 < p.nchunks) prefetch_raw(c + 2);
-    // ===== in-chunk cumulative log decay (base 2) along this thread's 16 tokens ==============
-    float g[16];
+  if (warp == NCOMP / 32) {
+    // ========================= control warp: MMAs and TMA copies =========================
+    if (tid == CTL) {
+      int n_la = 0, n_raw = 0;
+      auto prefetch_raw = [&](int c) {  // raw bf16 inputs of chunk c into L2
+        for (int pn = 0; pn < (dk >> 6); ++pn) {
+          tma_prefetch_l2_4d(&tmQ, 64 * pn, h, C * c, bb);
+          tma_prefetch_l2_4d(&tmK, 64 * pn, h, C * c, bb);
+          tma_prefetch_l2_4d(&tmB, 64 * pn, h, C * c, bb);
+        }
+        for (int pn = 0; pn < (dv >> 6); ++pn) {
+          tma_prefetch_l2_4d(&tmV, 64 * pn, h, C * c, bb);
+          tma_prefetch_l2_4d(&tmW, 64 * pn, h, C * c, bb);
+        }
+      };
+      auto issue_la = [&](int c) {  // log alpha of chunk c: dk/32 boxes of 32 channels x 64 tokens
+        mbar_arrive_expect_tx(&ms.bar_la, (uint32_t)(C * dk * 4));
+        for (int pn = 0; pn < (dk >> 5); ++pn)
+          tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, C * c, bb);
+        ++n_la;
+      };
+      auto issue_raw = [&](int c) {  // raw bf16 inputs of chunk c into the staging tiles
+        mbar_arrive_expect_tx(&ms.bar_raw, (uint32_t)(3 * (dk >> 6) + 2 * (dv >> 6)) * R64);
+        for (int pn = 0; pn < (dk >> 6); ++pn) {
+          tma_load_4d(sm + RAW_Q + pn * R64, &tmQ, &ms.bar_raw, 64 * pn, h, C * c, bb);
+          tma_load_4d(sm + RAW_K + pn * R64, &tmK, &ms.bar_raw, 64 * pn, h, C * c, bb);
+          tma_load_4d(sm + RAW_B + pn * R64, &tmB, &ms.bar_raw, 64 * pn, h, C * c, bb);
+        }
+        for (int pn = 0; pn < (dv >> 6); ++pn) {
+          tma_load_4d(sm + RAW_V + pn * R64, &tmV, &ms.bar_raw, 64 * pn, h, C * c, bb);
+          tma_load_4d(sm + RAW_W + pn * R64, &tmW, &ms.bar_raw, 64 * pn, h, C * c, bb);
+        }
+        ++n_raw;
+      };
+      auto store_o = [&](int cc) {  // the staged output tile of chunk cc
+        tma_store_4d(&tmO, sm + OFF_LA, 0, h, C * cc, bb);
+        bulk_commit();
+      };
+      uint32_t ph_ops = 0, ph_stage = 0, ph_solved = 0, ph_uround = 0, ph_s = 0;
+      bool alive = true;
+      if (p.nchunks > 0) {
+        issue_raw(0);
+        issue_la(0);
+        if (p.nchunks > 1) prefetch_raw(1);
+      }
+      for (int c = 0; c < p.nchunks; ++c) {
+        if (c + 2 < p.nchunks) prefetch_raw(c + 2);
+        // [-A; P] = [-Kb; Qh] Kn^T : M=128 (tokens of both halves), N=64 (s), K=128 (key channels)
+        if (!(alive = wait_on(&ms.bar_ops, ph_ops))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks) {
+          const uint32_t ko = (uint32_t)((ks & 3) * 32);
+          const uint64_t aKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + ko, 16, 1024);
+          const uint64_t bKN = sdesc_sw128(sbase + OFF_KN + (ks >> 2) * R64 + ko, 16, 1024);
+          umma_tf32_ss(tmem + TM_AP, aKQ, bKN, ID_64, ks > 0);
+        }
+        umma_commit(&ms.bar_mma);
+        // [R^T | O^T] += S^T [-Kb; Qh]^T : A = S^T (tensor memory), B = the KQ tile (N = 128)
+        if (!(alive = wait_on(&ms.bar_stage, ph_stage))) break;
+        tc_fence_after();
+        if (c > 0) store_o(c - 1);
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks) {
+          const uint64_t bKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
+          umma_tf32_ts(tmem + TM_R, tmem + TM_S + 8 * ks, bKQ, ID_128, 1);
+        }
+        umma_commit(&ms.bar_s);
+        // both products have read the KQ and Kn tiles: the next chunk's copies
+        if (!(alive = wait_on(&ms.bar_s, ph_s))) break;
+        if (c + 1 < p.nchunks) {
+          issue_raw(c + 1);
+          bulk_wait_read_all();  // the output staging has been read
+          issue_la(c + 1);
+        }
+        // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t
+        if (!(alive = wait_on(&ms.bar_solved, ph_solved))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t bT = sdesc_sw128(sbase + OFF_T + (ks >> 2) * R64 + (ks & 3) * 32, 16, 1024);
+          umma_tf32_ts(tmem + TM_U, tmem + TM_R + 8 * ks, bT, ID_64, ks > 0);
+        }
+        umma_commit(&ms.bar_mma);
+        // [O^T | S^T] += U~^T [P; Kn^T]^T : O^T += U~^T P^T and S^T += U~^T Kn in one N = 192 product
+        if (!(alive = wait_on(&ms.bar_uround, ph_uround))) break;
+        tc_fence_after();
+        if (c + 1 == p.nchunks) bulk_wait_read_all();  // the last staging may be rewritten after this
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t bPK = sdesc_sw128(sbase + OFF_PK + (ks >> 2) * R192 + (ks & 3) * 32, 16, 1024);
+          umma_tf32_ts(tmem + TM_O, tmem + TM_U + 8 * ks, bPK, ID_192, 1);
+        }
+        umma_commit(&ms.bar_mma);
+      }
+      // the last chunk's output, staged by the compute warps
+      if (alive && p.nchunks > 0 && wait_on(&ms.bar_stage, ph_stage)) store_o(p.nchunks - 1);
+      // after a give-up: every MMA issued so far (a fresh commit tracks all of them) and
+      // the last copies must land before the block releases its memory
+      if (ms.abort) {
+        volatile int never = 0;
+        umma_commit(&ms.bar_drain);
+        mbar_wait_bounded(&ms.bar_drain, 0, &never, nullptr, WAIT_LIMIT);
+        if (n_la > 0) mbar_wait_bounded(&ms.bar_la, (uint32_t)((n_la - 1) & 1), &never, nullptr, WAIT_LIMIT);
+        if (n_raw > 0) mbar_wait_bounded(&ms.bar_raw, (uint32_t)((n_raw - 1) & 1), &never, nullptr, WAIT_LIMIT);
+      }
+      bulk_wait_all();  // output stores complete before the block exits
+    }
+    __syncwarp();  // the warp reconverges before the block-wide barrier
+  } else {
+    // ========================= compute warps 0-15 =========================================
+    // entering state S0 -> S^T in tensor memory: lane j = ch (a value channel), key-channel
+    // columns [32 sg, 32 sg + 32)
     {
-      bool ok = wait_on(&ms.bar_la, ph_la, pend_la);
-      ok = ok && wait_on(&ms.bar_raw, ph_raw, pend_raw);
-      float acc = 0.f;
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const float x = kval ? *reinterpret_cast<const float*>(la_t + f32_off(16 * sg + r, ch, R64)) : 0.f;
-        acc = fmaf(x, LOG2E, acc);
-        g[r] = acc;
-      }
-      ms.segtot[sg][ch] = acc;
-      if (__syncthreads_or(!ok)) { dead = true; break; }
-    }
-    tc_fence_after();
-    // ===== folded operands of this thread's channel; Vw^T preloads the R^T accumulator ========
-    float nkb[16], qh[16], kn[16];
-    {
-      float off = 0.f;
-      for (int s2 = 0; s2 < sg; ++s2) off += ms.segtot[s2][ch];
-      if (sg == 3) ms.gC[ob][ch] = kval ? ex2_approx(off + g[15]) : 0.f;
-      float vw[16];
-      const uint32_t pnl = (uint32_t)(ch >> 6) * R64;  // raw tiles: panels of 64 channels
-      const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const uint32_t ro = pnl + sw128_off(16 * sg + r, chk) + byt;
-        const float gg = g[r] + off;
-        const float G = ex2_approx(gg), Gi = ex2_approx(-gg);
-        float kk = 0.f, bg = 0.f, qq = 0.f, vv = 0.f, ww = 0.f;
-        if (kval) {
-          kk = bf16_at(sm + RAW_K + ro);
-          bg = bf16_at(sm + RAW_B + ro);
-          qq = bf16_at(sm + RAW_Q + ro);
-        }
-        if (vval) {
-          vv = bf16_at(sm + RAW_V + ro);
-          ww = bf16_at(sm + RAW_W + ro);
-        }
-        nkb[r] = -(kk * bg) * G;
-        qh[r] = qq * G;
-        kn[r] = kk * Gi;
-        vw[r] = ww * vv;
-      }
-      // the R^T columns are free: the previous chunk's U~ product has completed
-      tmem_st16(tlane + TM_R + 16 * sg, vw);
-    }
-    // the previous chunk's last products must be done before Kn^T, O and S are touched,
-    // and every raw read before the operand tiles overwrite the staging
-    {
-      bool ok = true;
-      if (c > 0) ok = wait_mma();
-      if (__syncthreads_or(!ok)) { dead = true; break; }
-    }
-    tc_fence_after();
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int t = 16 * sg + r;
-      *reinterpret_cast<float*>(sm + OFF_KQ + f32_off(t, ch, R128)) = rna_tf32(nkb[r]);
-      *reinterpret_cast<float*>(sm + OFF_KQ + f32_off(64 + t, ch, R128)) = rna_tf32(qh[r]);
-      *reinterpret_cast<float*>(sm + OFF_KN + f32_off(t, ch, R64)) = rna_tf32(kn[r]);
-    }
-#pragma unroll
-    for (int r = 0; r < 16; r += 4) st4_tf32(sm + OFF_KNT + f32_off(ch, 16 * sg + r, R128), kn + r);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      // [-A; P] = [-Kb; Qh] Kn^T : M=128 (tokens of both halves), N=64 (s), K=128 (key channels)
-#pragma unroll
-      for (int ks = 0; ks < 16; ++ks) {
-        const uint32_t ko = (uint32_t)((ks & 3) * 32);
-        const uint64_t aKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + ko, 16, 1024);
-        const uint64_t bKN = sdesc_sw128(sbase + OFF_KN + (ks >> 2) * R64 + ko, 16, 1024);
-        umma_tf32_ss(tmem + TM_AP, aKQ, bKN, ID_64, ks > 0);
-      }
-      commit_mma();
-    }
-    // ===== while the tensor cores run: the previous chunk's output and state decay, and the
-    // output accumulator cleared ===============================================================
-    {
-      if (c > 0) stage_o();  // the log-alpha tile is free until the next chunk's copy
-      float z[16];
-#pragma unroll
-      for (int x = 0; x < 16; ++x) z[x] = 0.f;
-      tmem_st16(tlane + TM_O + 16 * sg, z);
-      if (c > 0) decay_state(ob ^ 1);
-    }
-    tmem_st_wait();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == TMA_TID && c > 0) store_o(c - 1);
-    if (tid == 0) {
-      tc_fence_after();
-      // [R^T | O^T] += S^T [-Kb; Qh]^T : A = S^T (tensor memory), B = the KQ tile (N = 128)
-#pragma unroll
-      for (int ks = 0; ks < 16; ++ks) {
-        const uint64_t bKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
-        umma_tf32_ts(tmem + TM_R, tmem + TM_S + 8 * ks, bKQ, ID_128, 1);
-      }
-      umma_commit(&ms.bar_s);
-    }
-    // ===== A (sign restored) to the solve scratch, P to its operand tile ========================
-    {
-      const bool ok_ap = wait_mma();
-      tc_fence_after();
-      float v[16];
-      tmem_ld16(tlane + TM_AP + 16 * sg, v);
-      tmem_ld_wait();
-      if (ch < 64) {
-        const int t = ch;
-#pragma unroll
-        for (int x = 0; x < 16; x += 4) {
-          const int s = 16 * sg + x;
-          float4 f;
-          f.x = (s + 0 < t) ? -v[x + 0] : 0.f;
-          f.y = (s + 1 < t) ? -v[x + 1] : 0.f;
-          f.z = (s + 2 < t) ? -v[x + 2] : 0.f;
-          f.w = (s + 3 < t) ? -v[x + 3] : 0.f;
-          *reinterpret_cast<float4*>(Msc + t * LDM + s) = f;
-        }
-      } else {
-        const int t = ch - 64;  // P row, causal incl. diagonal
-#pragma unroll
-        for (int x = 0; x < 16; x += 4) {
-          float f[4];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) f[m] = (16 * sg + x + m <= t) ? v[x + m] : 0.f;
-          st4_tf32(sm + OFF_P + f32_off(t, 16 * sg + x, R64), f);
-        }
-      }
-      if (__syncthreads_or(!ok_ap)) { dead = true; break; }
-    }
-    // ===== T = (I + A)^-1 on warps 0-7 (16x16 diagonal blocks, then 32x32, then 64x64; every
-    // entry above the diagonal is an explicit zero, so block products run dense).  Warps 8-15
-    // meanwhile round R^T in tensor memory once the state product is done, and thread
-    // TMA_TID starts the next chunk's copies into the tiles that product has released. ======
-    bool ok_s = true;
-    if (warp < 8) {
-      {
-        float x[16];
-        const int I = tid >> 4, cc = tid & 15;
-        if (tid < 64) {
-          const float* Ab = Msc + 16 * I * LDM + 16 * I;
-#pragma unroll
-          for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-          for (int r = 1; r < 16; ++r) {
-            float acc0 = 0.f, acc1 = 0.f;  // two chains: even and odd columns
-#pragma unroll
-            for (int s4 = 0; s4 < r; s4 += 4) {
-              const float4 a = ld4(Ab + r * LDM + s4);
-              acc0 = fmaf(a.x, x[s4], acc0);
-              if (s4 + 1 < r) acc1 = fmaf(a.y, x[s4 + 1], acc1);
-              if (s4 + 2 < r) acc0 = fmaf(a.z, x[s4 + 2], acc0);
-              if (s4 + 3 < r) acc1 = fmaf(a.w, x[s4 + 3], acc1);
-            }
-            x[r] = (r > cc) ? -(acc0 + acc1) : x[r];
-          }
-        }
-        named_bar_sync(1, NSOLVE);
-        if (tid < 64) {
-          float* Tb = Msc + 16 * I * LDM + 16 * I;
-#pragma unroll
-          for (int r = 0; r < 16; ++r) Tb[r * LDM + cc] = x[r];
-        }
-        named_bar_sync(1, NSOLVE);
-      }
-      // The block products of the next two levels run as warp-level tf32 MMAs
-      // (m16n8k8) on fragments read straight from the scratch matrices.
-      {
-        // 32x32 blocks: T_{2p+1,2p} = -T_{2p+1,2p+1} (A_{2p+1,2p} T_{2p,2p}), p = 0, 1;
-        // warp 2 p + nt computes the 16 x 8 output columns [8 nt, 8 nt + 8) of block p.
-        const int g = lane >> 2, t = lane & 3;
-        const int pp = warp >> 1, nt = warp & 1;
-        const int I = 2 * pp + 1, J = 2 * pp;
-        float* Xp = Xsc + 16 * pp * LDX;
-        if (warp < 4) {
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const float* Ar = Msc + (16 * I + g) * LDM + 16 * J + 8 * ks + t;
-            const float* Bc = Msc + (16 * J + 8 * ks + t) * LDM + 16 * J + 8 * nt + g;
-            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
-            mma_16x8x8_tf32(d, a, b);
-          }
-          *reinterpret_cast<float2*>(Xp + g * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
-          *reinterpret_cast<float2*>(Xp + (g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
-        }
-        named_bar_sync(1, NSOLVE);
-        if (warp < 4) {
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const float* Ar = Msc + (16 * I + g) * LDM + 16 * I + 8 * ks + t;
-            const float* Bc = Xp + (8 * ks + t) * LDX + 8 * nt + g;
-            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
-            mma_16x8x8_tf32(d, a, b);
-          }
-          float* Tr = Msc + (16 * I + g) * LDM + 16 * J + 8 * nt + 2 * t;
-          *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
-          *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
-        }
-        named_bar_sync(1, NSOLVE);
-      }
-      {
-        // 64x64: T_21 = -T_22 (A_21 T_11) with 32x32 blocks; warp 4 mt + nt (8 warps)
-        // computes the 16 x 8 output tile (rows [16 mt, +16), columns [8 nt, +8)).
-        const int g = lane >> 2, t = lane & 3;
-        const int mt = (warp >> 2) & 1, nt = warp & 3;
-        if (warp < 8) {
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 8 * ks + t;
-            const float* Bc = Msc + (8 * ks + t) * LDM + 8 * nt + g;
-            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
-            mma_16x8x8_tf32(d, a, b);
-          }
-          *reinterpret_cast<float2*>(Xsc + (16 * mt + g) * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
-          *reinterpret_cast<float2*>(Xsc + (16 * mt + g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
-        }
-        named_bar_sync(1, NSOLVE);
-        if (warp < 8) {
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 32 + 8 * ks + t;
-            const float* Bc = Xsc + (8 * ks + t) * LDX + 8 * nt + g;
-            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
-            mma_16x8x8_tf32(d, a, b);
-          }
-          float* Tr = Msc + (32 + 16 * mt + g) * LDM + 8 * nt + 2 * t;
-          *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
-          *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
-        }
-        named_bar_sync(1, NSOLVE);
-      }
-      // T as a tf32 K-major operand [t][s]
-      for (int e = tid; e < 64 * 16; e += NSOLVE) {
-        const int t = e >> 4, s4 = e & 15;
-        const float4 a = ld4(Msc + t * LDM + 4 * s4);
-        const float f[4] = {a.x, a.y, a.z, a.w};
-        st4_tf32(sm + OFF_T + f32_off(t, 4 * s4, R64), f);
-      }
-    } else {
-      ok_s = wait_on(&ms.bar_s, ph_s, pend_s);
-      tc_fence_after();
       float v[32];
-      tmem_ld32(tlane + TM_R + 32 * (sg - 2), v);
-      tmem_ld_wait();
+      const bool ok = p.S0 && vval;
 #pragma unroll
-      for (int x = 0; x < 32; ++x) v[x] = rna_tf32(v[x]);
-      tmem_st32(tlane + TM_R + 32 * (sg - 2), v);
-      tmem_st_wait();
-      if (tid == TMA_TID && ok_s && c + 1 < p.nchunks) {
-        issue_raw(c + 1);      // the KQ and Kn tiles have been read by both products
-        bulk_wait_read_all();  // the output staging has been read
-        issue_la(c + 1);
+      for (int x = 0; x < 32; ++x) {
+        const int i = 32 * sg + x;
+        v[x] = (ok && i < dk) ? p.S0[((size_t)unit * dk + i) * dv + ch] : 0.f;
       }
+      tmem_st32(tlane + TM_S + 32 * sg, v);
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (__syncthreads_or(!ok_s)) { dead = true; break; }
-    if (tid == 0) {
-      tc_fence_after();
-      // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t bT = sdesc_sw128(sbase + OFF_T + (ks >> 2) * R64 + (ks & 3) * 32, 16, 1024);
-        umma_tf32_ts(tmem + TM_U, tmem + TM_R + 8 * ks, bT, ID_64, ks > 0);
-      }
-      commit_mma();
-    }
-    // ===== U~^T rounded to tf32 in place: the A operand of the chunk's last products ==========
-    {
-      const bool ok_u = wait_mma();
-      tc_fence_after();
-      float v[16];
-      tmem_ld16(tlane + TM_U + 16 * sg, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int x = 0; x < 16; ++x) v[x] = rna_tf32(v[x]);
-      tmem_st16(tlane + TM_U + 16 * sg, v);
-      tmem_st_wait();
-      tc_fence_before();
-      if (__syncthreads_or(!ok_u)) { dead = true; break; }
-    }
-    if (tid == 0) {
-      tc_fence_after();
-      // O^T += U~^T P^T : A = U~^T from tensor memory, B = P (N = t), K = s
-      // S^T += U~^T Kn  : B = Kn^T rows (N = key channels)
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t bP = sdesc_sw128(sbase + OFF_P + (ks >> 2) * R64 + (ks & 3) * 32, 16, 1024);
-        const uint64_t bK = sdesc_sw128(sbase + OFF_KNT + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
-        umma_tf32_ts(tmem + TM_O, tmem + TM_U + 8 * ks, bP, ID_64, 1);
-        umma_tf32_ts(tmem + TM_S, tmem + TM_U + 8 * ks, bK, ID_128, 1);
-      }
-      commit_mma();  // waited on at the start of the next chunk (or below)
-    }
-  }
-
-  // ---- last chunk's output and decay, then the final state -------------------------------
-  if (!dead && p.nchunks > 0) {
-    if (tid == TMA_TID) bulk_wait_read_all();  // the staging tile is about to be rewritten
-    if (__syncthreads_or(!wait_mma())) dead = true;
-  }
-  if (!dead && p.nchunks > 0) {
-    tc_fence_after();
-    stage_o();
-    decay_state((p.nchunks - 1) & 1);
-    tmem_st_wait();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (tid == TMA_TID) store_o(p.nchunks - 1);
-    if (p.S_T && vval) {
+    uint32_t ph_la = 0, ph_mma = 0, ph_raw = 0, ph_s = 0;
+    float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);                 // solve matrix, 64 x LDM fp32
+    float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);  // block product, 32 x LDX fp32
+    const unsigned char* la_t = sm + OFF_LA;
+    const int lane = tid & 31;
+    auto wait_mma = [&]() -> bool { return wait_on(&ms.bar_mma, ph_mma); };
+    // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory.
+    auto decay_state = [&](int gb) {
       float v[32];
       tmem_ld32(tlane + TM_S + 32 * sg, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int x = 0; x < 32; ++x)
-        if (32 * sg + x < dk) p.S_T[((size_t)unit * dk + 32 * sg + x) * dv + ch] = v[x];
+      for (int x = 0; x < 32; x += 4) {
+        const float4 gq = *reinterpret_cast<const float4*>(&ms.gC[gb][32 * sg + x]);
+        v[x] *= gq.x;
+        v[x + 1] *= gq.y;
+        v[x + 2] *= gq.z;
+        v[x + 3] *= gq.w;
+      }
+      tmem_st32(tlane + TM_S + 32 * sg, v);
+    };
+    // Output of the last finished chunk (O^T in tensor memory) into the shared-memory tile
+    // [t][j] (rows of d_v floats) that the control warp's TMA store writes out.
+    auto stage_o = [&]() {
+      float v[16];
+      tmem_ld16(tlane + TM_O + 16 * sg, v);
+      tmem_ld_wait();
+      if (vval) {
+        float* st = reinterpret_cast<float*>(sm + OFF_LA) + ch;
+#pragma unroll
+        for (int x = 0; x < 16; ++x) st[(16 * sg + x) * dv] = v[x];
+      }
+    };
+
+    bool dead = false;
+    bool ok_prev = true;  // failed waits of the previous chunk's tail, voted at the next barrier
+    for (int c = 0; c < p.nchunks; ++c) {
+      const int ob = c & 1;
+      // ===== in-chunk cumulative log decay (base 2) along this thread's 16 tokens ============
+      float g[16];
+      {
+        bool ok = ok_prev && wait_on(&ms.bar_la, ph_la);
+        ok = ok && wait_on(&ms.bar_raw, ph_raw);
+        float acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const float x = kval ? *reinterpret_cast<const float*>(la_t + f32_off(16 * sg + r, ch, R64)) : 0.f;
+          acc = fmaf(x, LOG2E, acc);
+          g[r] = acc;
+        }
+        ms.segtot[sg][ch] = acc;
+        if (named_bar_or(BAR_COMP, NCOMP, !ok)) { dead = true; break; }
+      }
+      tc_fence_after();
+      // ===== folded operands of this thread's channel; Vw^T preloads the R^T accumulator ======
+      float nkb[16], qh[16], kn[16];
+      {
+        float off = 0.f;
+        for (int s2 = 0; s2 < sg; ++s2) off += ms.segtot[s2][ch];
+        if (sg == 3) ms.gC[ob][ch] = kval ? ex2_approx(off + g[15]) : 0.f;
+        float vw[16];
+        const uint32_t pnl = (uint32_t)(ch >> 6) * R64;  // raw tiles: panels of 64 channels
+        const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const uint32_t ro = pnl + sw128_off(16 * sg + r, chk) + byt;
+          const float gg = g[r] + off;
+          const float G = ex2_approx(gg), Gi = ex2_approx(-gg);
+          float kk = 0.f, bg = 0.f, qq = 0.f, vv = 0.f, ww = 0.f;
+          if (kval) {
+            kk = bf16_at(sm + RAW_K + ro);
+            bg = bf16_at(sm + RAW_B + ro);
+            qq = bf16_at(sm + RAW_Q + ro);
+          }
+          if (vval) {
+            vv = bf16_at(sm + RAW_V + ro);
+            ww = bf16_at(sm + RAW_W + ro);
+          }
+          nkb[r] = -(kk * bg) * G;
+          qh[r] = qq * G;
+          kn[r] = kk * Gi;
+          vw[r] = ww * vv;
+        }
+        // the R^T columns are free: the previous chunk's U~ product has completed
+        tmem_st16(tlane + TM_R + 16 * sg, vw);
+      }
+      // the previous chunk's last product must be done before Kn^T, O and S are touched,
+      // and every raw read before the operand tiles overwrite the staging
+      {
+        const bool ok = (c == 0) || wait_mma();
+        if (named_bar_or(BAR_COMP, NCOMP, !ok)) { dead = true; break; }
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const int t = 16 * sg + r;
+        *reinterpret_cast<float*>(sm + OFF_KQ + f32_off(t, ch, R128)) = rna_tf32(nkb[r]);
+        *reinterpret_cast<float*>(sm + OFF_KQ + f32_off(64 + t, ch, R128)) = rna_tf32(qh[r]);
+        *reinterpret_cast<float*>(sm + OFF_KN + f32_off(t, ch, R64)) = rna_tf32(kn[r]);
+      }
+#pragma unroll
+      for (int r = 0; r < 16; r += 4) st4_tf32(sm + OFF_PK + f32_off(64 + ch, 16 * sg + r, R192), kn + r);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(&ms.bar_ops);
+      // ===== while [A; P] is on the tensor cores: the previous chunk's output and state
+      // decay, and the output accumulator cleared ==============================================
+      {
+        if (c > 0) stage_o();  // the log-alpha tile is free until the next chunk's copy
+        float z[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) z[x] = 0.f;
+        tmem_st16(tlane + TM_O + 16 * sg, z);
+        if (c > 0) decay_state(ob ^ 1);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(&ms.bar_stage);
+      // ===== A (sign restored) to the solve scratch, P to its operand tile =====================
+      {
+        const bool ok_ap = wait_mma();
+        tc_fence_after();
+        float v[16];
+        tmem_ld16(tlane + TM_AP + 16 * sg, v);
+        tmem_ld_wait();
+        if (ch < 64) {
+          const int t = ch;
+#pragma unroll
+          for (int x = 0; x < 16; x += 4) {
+            const int s = 16 * sg + x;
+            float4 f;
+            f.x = (s + 0 < t) ? -v[x + 0] : 0.f;
+            f.y = (s + 1 < t) ? -v[x + 1] : 0.f;
+            f.z = (s + 2 < t) ? -v[x + 2] : 0.f;
+            f.w = (s + 3 < t) ? -v[x + 3] : 0.f;
+            *reinterpret_cast<float4*>(Msc + t * LDM + s) = f;
+          }
+        } else {
+          const int t = ch - 64;  // P row, causal incl. diagonal
+#pragma unroll
+          for (int x = 0; x < 16; x += 4) {
+            float f[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) f[m] = (16 * sg + x + m <= t) ? v[x + m] : 0.f;
+            st4_tf32(sm + OFF_PK + f32_off(t, 16 * sg + x, R192), f);
+          }
+        }
+        if (named_bar_or(BAR_COMP, NCOMP, !ok_ap)) { dead = true; break; }
+      }
+      // ===== T = (I + A)^-1 on warps 0-7 (16x16 diagonal blocks, then 32x32, then 64x64; every
+      // entry above the diagonal is an explicit zero, so block products run dense).  Warps
+      // 8-15 meanwhile round R^T in tensor memory once the state product is done. ===========
+      bool ok_s = true;
+      if (warp < 8) {
+        {
+          float x[16];
+          const int I = tid >> 4, cc = tid & 15;
+          if (tid < 64) {
+            const float* Ab = Msc + 16 * I * LDM + 16 * I;
+    #pragma unroll
+            for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+    #pragma unroll
+            for (int r = 1; r < 16; ++r) {
+              float acc0 = 0.f, acc1 = 0.f;  // two chains: even and odd columns
+    #pragma unroll
+              for (int s4 = 0; s4 < r; s4 += 4) {
+                const float4 a = ld4(Ab + r * LDM + s4);
+                acc0 = fmaf(a.x, x[s4], acc0);
+                if (s4 + 1 < r) acc1 = fmaf(a.y, x[s4 + 1], acc1);
+                if (s4 + 2 < r) acc0 = fmaf(a.z, x[s4 + 2], acc0);
+                if (s4 + 3 < r) acc1 = fmaf(a.w, x[s4 + 3], acc1);
+              }
+              x[r] = (r > cc) ? -(acc0 + acc1) : x[r];
+            }
+          }
+          named_bar_sync(BAR_SOLVE, NSOLVE);
+          if (tid < 64) {
+            float* Tb = Msc + 16 * I * LDM + 16 * I;
+    #pragma unroll
+            for (int r = 0; r < 16; ++r) Tb[r * LDM + cc] = x[r];
+          }
+          named_bar_sync(BAR_SOLVE, NSOLVE);
+        }
+        // The block products of the next two levels run as warp-level tf32 MMAs
+        // (m16n8k8) on fragments read straight from the scratch matrices.
+        {
+          // 32x32 blocks: T_{2p+1,2p} = -T_{2p+1,2p+1} (A_{2p+1,2p} T_{2p,2p}), p = 0, 1;
+          // warp 2 p + nt computes the 16 x 8 output columns [8 nt, 8 nt + 8) of block p.
+          const int g = lane >> 2, t = lane & 3;
+          const int pp = warp >> 1, nt = warp & 1;
+          const int I = 2 * pp + 1, J = 2 * pp;
+          float* Xp = Xsc + 16 * pp * LDX;
+          if (warp < 4) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+              const float* Ar = Msc + (16 * I + g) * LDM + 16 * J + 8 * ks + t;
+              const float* Bc = Msc + (16 * J + 8 * ks + t) * LDM + 16 * J + 8 * nt + g;
+              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
+              mma_16x8x8_tf32(d, a, b);
+            }
+            *reinterpret_cast<float2*>(Xp + g * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(Xp + (g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
+          }
+          named_bar_sync(BAR_SOLVE, NSOLVE);
+          if (warp < 4) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+              const float* Ar = Msc + (16 * I + g) * LDM + 16 * I + 8 * ks + t;
+              const float* Bc = Xp + (8 * ks + t) * LDX + 8 * nt + g;
+              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
+              mma_16x8x8_tf32(d, a, b);
+            }
+            float* Tr = Msc + (16 * I + g) * LDM + 16 * J + 8 * nt + 2 * t;
+            *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
+            *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
+          }
+          named_bar_sync(BAR_SOLVE, NSOLVE);
+        }
+        {
+          // 64x64: T_21 = -T_22 (A_21 T_11) with 32x32 blocks; warp 4 mt + nt (8 warps)
+          // computes the 16 x 8 output tile (rows [16 mt, +16), columns [8 nt, +8)).
+          const int g = lane >> 2, t = lane & 3;
+          const int mt = (warp >> 2) & 1, nt = warp & 3;
+          if (warp < 8) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 8 * ks + t;
+              const float* Bc = Msc + (8 * ks + t) * LDM + 8 * nt + g;
+              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
+              mma_16x8x8_tf32(d, a, b);
+            }
+            *reinterpret_cast<float2*>(Xsc + (16 * mt + g) * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(Xsc + (16 * mt + g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
+          }
+          named_bar_sync(BAR_SOLVE, NSOLVE);
+          if (warp < 8) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 32 + 8 * ks + t;
+              const float* Bc = Xsc + (8 * ks + t) * LDX + 8 * nt + g;
+              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
+              mma_16x8x8_tf32(d, a, b);
+            }
+            float* Tr = Msc + (32 + 16 * mt + g) * LDM + 8 * nt + 2 * t;
+            *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
+            *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
+          }
+          named_bar_sync(BAR_SOLVE, NSOLVE);
+        }
+        // T as a tf32 K-major operand [t][s]
+        for (int e = tid; e < 64 * 16; e += NSOLVE) {
+          const int t = e >> 4, s4 = e & 15;
+          const float4 a = ld4(Msc + t * LDM + 4 * s4);
+          const float f[4] = {a.x, a.y, a.z, a.w};
+          st4_tf32(sm + OFF_T + f32_off(t, 4 * s4, R64), f);
+        }
+      } else {
+        ok_s = wait_on(&ms.bar_s, ph_s);
+        tc_fence_after();
+        float v[32];
+        tmem_ld32(tlane + TM_R + 32 * (sg - 2), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) v[x] = rna_tf32(v[x]);
+        tmem_st32(tlane + TM_R + 32 * (sg - 2), v);
+        tmem_st_wait();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(&ms.bar_solved);
+      // ===== U~^T rounded to tf32 in place: the A operand of the chunk's last product =========
+      {
+        const bool ok_u = wait_mma();
+        tc_fence_after();
+        float v[16];
+        tmem_ld16(tlane + TM_U + 16 * sg, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[x] = rna_tf32(v[x]);
+        tmem_st16(tlane + TM_U + 16 * sg, v);
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(&ms.bar_uround);
+        ok_prev = ok_s && ok_u;
+      }
+    }
+
+    // ---- last chunk's output and decay, then the final state -----------------------------
+    if (!dead && p.nchunks > 0) {
+      const bool ok = ok_prev && wait_mma();
+      if (named_bar_or(BAR_COMP, NCOMP, !ok)) dead = true;
+    }
+    if (!dead && p.nchunks > 0) {
+      tc_fence_after();
+      stage_o();
+      decay_state((p.nchunks - 1) & 1);
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(&ms.bar_stage);
+      if (p.S_T && vval) {
+        float v[32];
+        tmem_ld32(tlane + TM_S + 32 * sg, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          if (32 * sg + x < dk) p.S_T[((size_t)unit * dk + 32 * sg + x) * dv + ch] = v[x];
+      }
     }
   }
-  // ---- teardown: after a give-up, let outstanding async work drain (bounded) ------------
-  if (ms.abort) {
-    volatile int never = 0;
-    if (tid == 0) {  // every MMA this thread issued: a fresh commit tracks all of them
-      umma_commit(&ms.bar_drain);
-      mbar_wait_bounded(&ms.bar_drain, 0, &never, nullptr, WAIT_LIMIT);
-    }
-    if (tid == TMA_TID) {
-      if (pend_la) mbar_wait_bounded(&ms.bar_la, ph_la, &never, nullptr, WAIT_LIMIT);
-      if (pend_raw) mbar_wait_bounded(&ms.bar_raw, ph_raw, &never, nullptr, WAIT_LIMIT);
-    }
-  }
-  if (tid == TMA_TID) bulk_wait_all();  // output stores complete before the block exits
+  // ---- teardown ---------------------------------------------------------------------------
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
