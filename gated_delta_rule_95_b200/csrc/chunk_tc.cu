@@ -56,6 +56,7 @@ constexpr int NSOLVE = 256;                     // warps 0-7 run the triangular 
 constexpr int BAR_COMP = 1, BAR_SOLVE = 2;      // named barriers: all compute warps; solve warps
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr int PF_AHEAD = 3;                     // chunks of input prefetched into L2 ahead of use
 
 // ---- shared memory map (byte offsets from a 1024-byte aligned base) ----------------
 // fp32 operand tiles with the 128B swizzle, in panels of 32 columns (128 B rows).
@@ -125,6 +126,9 @@ __device__ __forceinline__ float bf16_at(const unsigned char* p) {
   return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short*>(p)) << 16);
 }
 
+// DK, DV: key and value head dimensions (64 or 128), fixed at compile time so that each
+// launch runs straight-line code for its own shape.
+template <int DK, int DV>
 __global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
@@ -140,7 +144,7 @@ __global__ void __launch_bounds__(NT, 1)
   const int ch = tid & 127;  // channel (key i and value j) and tensor-memory lane
   const int sg = tid >> 7;   // token segment [16 sg, 16 sg + 16); column group of TMEM accesses
   const int unit = blockIdx.x, bb = unit / p.H, h = unit % p.H;
-  const int dk = p.dk, dv = p.dv;
+  constexpr int dk = DK, dv = DV;
   const bool kval = ch < dk, vval = ch < dv;
 
   if (tid == 0) {
@@ -184,7 +188,8 @@ __global__ void __launch_bounds__(NT, 1)
     // ========================= control warp: MMAs and TMA copies =========================
     if (tid == CTL) {
       int n_la = 0, n_raw = 0;
-      auto prefetch_raw = [&](int c) {  // raw bf16 inputs of chunk c into L2
+      auto prefetch_raw = [&](int c) {  // every input tile of chunk c into L2
+        for (int pn = 0; pn < (dk >> 5); ++pn) tma_prefetch_l2_4d(&tmLA, 32 * pn, h, C * c, bb);
         for (int pn = 0; pn < (dk >> 6); ++pn) {
           tma_prefetch_l2_4d(&tmQ, 64 * pn, h, C * c, bb);
           tma_prefetch_l2_4d(&tmK, 64 * pn, h, C * c, bb);
@@ -223,14 +228,14 @@ __global__ void __launch_bounds__(NT, 1)
       if (p.nchunks > 0) {
         issue_raw(0);
         issue_la(0);
-        if (p.nchunks > 1) prefetch_raw(1);
+        for (int cc = 1; cc <= PF_AHEAD && cc < p.nchunks; ++cc) prefetch_raw(cc);
       }
       for (int c = 0; c < p.nchunks; ++c) {
-        if (c + 2 < p.nchunks) prefetch_raw(c + 2);
+        if (c + PF_AHEAD < p.nchunks) prefetch_raw(c + PF_AHEAD);
         // [-A; P] = [-Kb; Qh] Kn^T : M=128 (tokens of both halves), N=64 (s), K=128 (key channels)
         if (!(alive = wait_on(&ms.bar_ops, ph_ops))) break;
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 16; ++ks) {
           const uint32_t ko = (uint32_t)((ks & 3) * 32);
           const uint64_t aKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + ko, 16, 1024);
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (!(alive = wait_on(&ms.bar_stage, ph_stage))) break;
         tc_fence_after();
         if (c > 0) store_o(c - 1);
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 16; ++ks) {
           const uint64_t bKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
           umma_tf32_ts(tmem + TM_R, tmem + TM_S + 8 * ks, bKQ, ID_128, 1);
@@ -258,7 +263,7 @@ __global__ void __launch_bounds__(NT, 1)
         // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t
         if (!(alive = wait_on(&ms.bar_solved, ph_solved))) break;
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bT = sdesc_sw128(sbase + OFF_T + (ks >> 2) * R64 + (ks & 3) * 32, 16, 1024);
           umma_tf32_ts(tmem + TM_U, tmem + TM_R + 8 * ks, bT, ID_64, ks > 0);
@@ -268,7 +273,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (!(alive = wait_on(&ms.bar_uround, ph_uround))) break;
         tc_fence_after();
         if (c + 1 == p.nchunks) bulk_wait_read_all();  // the last staging may be rewritten after this
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bPK = sdesc_sw128(sbase + OFF_PK + (ks >> 2) * R192 + (ks & 3) * 32, 16, 1024);
           umma_tf32_ts(tmem + TM_O, tmem + TM_U + 8 * ks, bPK, ID_192, 1);
@@ -303,6 +308,9 @@ __global__ void __launch_bounds__(NT, 1)
       }
       tmem_st32(tlane + TM_S + 32 * sg, v);
     }
+    // the T operand tile: blocks above the 8x8 block diagonal stay zero for good
+    for (int e = tid; e < 2 * (int)R64 / 16; e += NCOMP)
+      *reinterpret_cast<float4*>(sm + OFF_T + 16 * e) = make_float4(0.f, 0.f, 0.f, 0.f);
     uint32_t ph_la = 0, ph_mma = 0, ph_raw = 0, ph_s = 0;
     float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);                 // solve matrix, 64 x LDM fp32
     float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);  // block product, 32 x LDX fp32
@@ -453,37 +461,65 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (named_bar_or(BAR_COMP, NCOMP, !ok_ap)) { dead = true; break; }
       }
-      // ===== T = (I + A)^-1 on warps 0-7 (16x16 diagonal blocks, then 32x32, then 64x64; every
-      // entry above the diagonal is an explicit zero, so block products run dense).  Warps
-      // 8-15 meanwhile round R^T in tensor memory once the state product is done. ===========
+      // ===== T = (I + A)^-1 on warps 0-7: 8x8 diagonal blocks by forward substitution (fp32),
+      // then 2x2 block merges T21 = -T22 (A21 T11) at 16, 32 and 64 (every entry above the
+      // diagonal is an explicit zero, so block products run dense).  Each level writes its
+      // blocks to the fp32 scratch (read by the next level) and, rounded, to the T operand
+      // tile.  Warps 8-15 meanwhile round R^T in tensor memory once the state product is done.
       bool ok_s = true;
       if (warp < 8) {
+        auto put_t = [&](int row, int col, float x) {  // one element of the T operand tile
+          *reinterpret_cast<float*>(sm + OFF_T + f32_off(row, col, R64)) = rna_tf32(x);
+        };
+        auto put_t2 = [&](int row, int col, float x0, float x1) {  // col even
+          *reinterpret_cast<float2*>(sm + OFF_T + f32_off(row, col, R64)) = make_float2(rna_tf32(x0), rna_tf32(x1));
+        };
+        if (tid < 64) {
+          // thread (blk, cc): column cc of the inverse of diagonal block blk (rows 8 blk ..)
+          const int r0 = 8 * (tid >> 3), cc = tid & 7;
+          const float* Ab = Msc + r0 * LDM + r0;
+          float x[8];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+          for (int r = 1; r < 8; ++r) {
+            const float4 a0 = ld4(Ab + r * LDM), a1 = ld4(Ab + r * LDM + 4);
+            const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            float acc = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < r; ++s2) acc = fmaf(ar[s2], x[s2], acc);
+            x[r] = (r > cc) ? -acc : x[r];
+          }
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            Msc[(r0 + r) * LDM + r0 + cc] = x[r];
+            put_t(r0 + r, r0 + cc, x[r]);
+          }
+        }
+        named_bar_sync(BAR_SOLVE, NSOLVE);
         {
-          float x[16];
-          const int I = tid >> 4, cc = tid & 15;
-          if (tid < 64) {
-            const float* Ab = Msc + 16 * I * LDM + 16 * I;
-    #pragma unroll
-            for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
-    #pragma unroll
-            for (int r = 1; r < 16; ++r) {
-              float acc0 = 0.f, acc1 = 0.f;  // two chains: even and odd columns
-    #pragma unroll
-              for (int s4 = 0; s4 < r; s4 += 4) {
-                const float4 a = ld4(Ab + r * LDM + s4);
-                acc0 = fmaf(a.x, x[s4], acc0);
-                if (s4 + 1 < r) acc1 = fmaf(a.y, x[s4 + 1], acc1);
-                if (s4 + 2 < r) acc0 = fmaf(a.z, x[s4 + 2], acc0);
-                if (s4 + 3 < r) acc1 = fmaf(a.w, x[s4 + 3], acc1);
-              }
-              x[r] = (r > cc) ? -(acc0 + acc1) : x[r];
-            }
+          // 16x16 blocks q = 0..3: T_21 = -T_22 (A_21 T_11) with 8x8 blocks; thread (q, r, cc)
+          // computes one entry of each product.
+          const int q = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7;
+          const int i0 = 16 * q + 8, j0 = 16 * q;
+          float* Xq = Xsc + 64 * q;
+          {
+            const float4 a0 = ld4(Msc + (i0 + r) * LDM + j0), a1 = ld4(Msc + (i0 + r) * LDM + j0 + 4);
+            const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            float z = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) z = fmaf(ar[s2], Msc[(j0 + s2) * LDM + j0 + cc], z);
+            Xq[8 * r + cc] = z;
           }
           named_bar_sync(BAR_SOLVE, NSOLVE);
-          if (tid < 64) {
-            float* Tb = Msc + 16 * I * LDM + 16 * I;
-    #pragma unroll
-            for (int r = 0; r < 16; ++r) Tb[r * LDM + cc] = x[r];
+          {
+            const float4 t0 = ld4(Msc + (i0 + r) * LDM + i0), t1 = ld4(Msc + (i0 + r) * LDM + i0 + 4);
+            const float tr[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            float y = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) y = fmaf(tr[s2], Xq[8 * s2 + cc], y);
+            Msc[(i0 + r) * LDM + j0 + cc] = -y;
+            put_t(i0 + r, j0 + cc, -y);
           }
           named_bar_sync(BAR_SOLVE, NSOLVE);
         }
@@ -498,7 +534,7 @@ __global__ void __launch_bounds__(NT, 1)
           float* Xp = Xsc + 16 * pp * LDX;
           if (warp < 4) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
+#pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
               const float* Ar = Msc + (16 * I + g) * LDM + 16 * J + 8 * ks + t;
               const float* Bc = Msc + (16 * J + 8 * ks + t) * LDM + 16 * J + 8 * nt + g;
@@ -513,7 +549,7 @@ __global__ void __launch_bounds__(NT, 1)
           named_bar_sync(BAR_SOLVE, NSOLVE);
           if (warp < 4) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
+#pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
               const float* Ar = Msc + (16 * I + g) * LDM + 16 * I + 8 * ks + t;
               const float* Bc = Xp + (8 * ks + t) * LDX + 8 * nt + g;
@@ -522,9 +558,11 @@ __global__ void __launch_bounds__(NT, 1)
               const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
               mma_16x8x8_tf32(d, a, b);
             }
-            float* Tr = Msc + (16 * I + g) * LDM + 16 * J + 8 * nt + 2 * t;
-            *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
-            *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
+            const int row = 16 * I + g, col = 16 * J + 8 * nt + 2 * t;
+            *reinterpret_cast<float2*>(Msc + row * LDM + col) = make_float2(-d[0], -d[1]);
+            *reinterpret_cast<float2*>(Msc + (row + 8) * LDM + col) = make_float2(-d[2], -d[3]);
+            put_t2(row, col, -d[0], -d[1]);
+            put_t2(row + 8, col, -d[2], -d[3]);
           }
           named_bar_sync(BAR_SOLVE, NSOLVE);
         }
@@ -533,44 +571,32 @@ __global__ void __launch_bounds__(NT, 1)
           // computes the 16 x 8 output tile (rows [16 mt, +16), columns [8 nt, +8)).
           const int g = lane >> 2, t = lane & 3;
           const int mt = (warp >> 2) & 1, nt = warp & 3;
-          if (warp < 8) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 8 * ks + t;
-              const float* Bc = Msc + (8 * ks + t) * LDM + 8 * nt + g;
-              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
-              mma_16x8x8_tf32(d, a, b);
-            }
-            *reinterpret_cast<float2*>(Xsc + (16 * mt + g) * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(Xsc + (16 * mt + g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 8 * ks + t;
+            const float* Bc = Msc + (8 * ks + t) * LDM + 8 * nt + g;
+            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
+            mma_16x8x8_tf32(d, a, b);
           }
+          *reinterpret_cast<float2*>(Xsc + (16 * mt + g) * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
+          *reinterpret_cast<float2*>(Xsc + (16 * mt + g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
           named_bar_sync(BAR_SOLVE, NSOLVE);
-          if (warp < 8) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 32 + 8 * ks + t;
-              const float* Bc = Xsc + (8 * ks + t) * LDX + 8 * nt + g;
-              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
-              mma_16x8x8_tf32(d, a, b);
-            }
-            float* Tr = Msc + (32 + 16 * mt + g) * LDM + 8 * nt + 2 * t;
-            *reinterpret_cast<float2*>(Tr) = make_float2(-d[0], -d[1]);
-            *reinterpret_cast<float2*>(Tr + 8 * LDM) = make_float2(-d[2], -d[3]);
+          d[0] = d[1] = d[2] = d[3] = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 32 + 8 * ks + t;
+            const float* Bc = Xsc + (8 * ks + t) * LDX + 8 * nt + g;
+            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
+                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
+            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
+            mma_16x8x8_tf32(d, a, b);
           }
-          named_bar_sync(BAR_SOLVE, NSOLVE);
-        }
-        // T as a tf32 K-major operand [t][s]
-        for (int e = tid; e < 64 * 16; e += NSOLVE) {
-          const int t = e >> 4, s4 = e & 15;
-          const float4 a = ld4(Msc + t * LDM + 4 * s4);
-          const float f[4] = {a.x, a.y, a.z, a.w};
-          st4_tf32(sm + OFF_T + f32_off(t, 4 * s4, R64), f);
+          const int row = 32 + 16 * mt + g, col = 8 * nt + 2 * t;
+          put_t2(row, col, -d[0], -d[1]);
+          put_t2(row + 8, col, -d[2], -d[3]);
         }
       } else {
         ok_s = wait_on(&ms.bar_s, ph_s);
@@ -661,6 +687,21 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
   return r == CUDA_SUCCESS;
 }
 
+template <int DK, int DV>
+cudaError_t launch_shape(int grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw, const CUtensorMap& mla,
+                         const CUtensorMap& mo, const TcParams& p) {
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  chunk_fwd_tc_kernel<DK, DV><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
@@ -677,13 +718,6 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
             make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dv, a.dv,
                      CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   TcParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k = static_cast<const __nv_bfloat16*>(a.k);
@@ -699,7 +733,12 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   p.dv = a.dv;
   p.nchunks = (a.T + C - 1) / C;
   p.err = device_error_word();
-  chunk_fwd_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
+  cudaError_t e = cudaErrorInvalidValue;
+  if (a.dk == 128 && a.dv == 128) e = launch_shape<128, 128>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
+  else if (a.dk == 128 && a.dv == 64) e = launch_shape<128, 64>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
+  else if (a.dk == 64 && a.dv == 128) e = launch_shape<64, 128>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
+  else if (a.dk == 64 && a.dv == 64) e = launch_shape<64, 64>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
