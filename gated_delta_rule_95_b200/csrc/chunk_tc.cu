@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(NT, 1)
         // [-A; P] = [-Kb; Qh] Kn^T : M=128 (tokens of both halves), N=64 (s), K=128 (key channels)
         if (!(alive = wait_on(&ms.bar_ops, ph_ops))) break;
         tc_fence_after();
-#pragma unroll 1
+#pragma unroll
         for (int ks = 0; ks < 16; ++ks) {
           const uint32_t ko = (uint32_t)((ks & 3) * 32);
           const uint64_t aKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + ko, 16, 1024);
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(NT, 1)
         // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t
         if (!(alive = wait_on(&ms.bar_solved, ph_solved))) break;
         tc_fence_after();
-#pragma unroll 1
+#pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bT = sdesc_sw128(sbase + OFF_T + (ks >> 2) * R64 + (ks & 3) * 32, 16, 1024);
           umma_tf32_ts(tmem + TM_U, tmem + TM_R + 8 * ks, bT, ID_64, ks > 0);
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (!(alive = wait_on(&ms.bar_uround, ph_uround))) break;
         tc_fence_after();
         if (c + 1 == p.nchunks) bulk_wait_read_all();  // the last staging may be rewritten after this
-#pragma unroll 1
+#pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bPK = sdesc_sw128(sbase + OFF_PK + (ks >> 2) * R192 + (ks & 3) * 32, 16, 1024);
           umma_tf32_ts(tmem + TM_O, tmem + TM_U + 8 * ks, bPK, ID_192, 1);
