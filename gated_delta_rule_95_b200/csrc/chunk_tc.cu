@@ -53,7 +53,7 @@ constexpr int NCOMP = 512;                      // warps 0-15: elementwise work
 constexpr int NT = NCOMP + 32;                  // + the control warp
 constexpr int CTL = NCOMP;                      // the thread that issues MMAs and TMA copies
 constexpr int NSOLVE = 256;                     // warps 0-7 run the triangular solve
-constexpr int BAR_COMP = 1, BAR_SOLVE = 2;      // named barriers: all compute warps; solve warps
+constexpr int BAR_COMP = 1, BAR_SOLVE = 2, BAR_AUX = 3;  // named barriers: compute warps; warps 0-7; 8-15
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int PF_AHEAD = 3;                     // chunks of input prefetched into L2 ahead of use
@@ -67,26 +67,27 @@ constexpr uint32_t OFF_KQ = 0;                  // [-Kb; Qh] [t][i]: 4 panels x 
 constexpr uint32_t OFF_KN = OFF_KQ + 4 * R128;  // Kn [s][i]: 4 panels x 64 rows (first: raw w)
 constexpr uint32_t OFF_PK = OFF_KN + 4 * R64;   // [P; Kn^T] [t | i][s]: 2 panels x 192 rows
 constexpr uint32_t OFF_T = OFF_PK + 2 * R192;   // T [t][s]: 2 panels x 64 rows
-constexpr uint32_t OFF_LA = OFF_T + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows;
+constexpr uint32_t OFF_LA = OFF_T + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows,
+                                                // turned in place into the in-chunk cumulative log2 decay;
                                                 // between uses: the output tile [t][j] fp32 of a TMA store
 constexpr uint32_t OFF_SCR = OFF_LA + 4 * R64;  // solve scratch: fp32 64 x LDM, then 32 x LDX
 // raw bf16 staging (TMA, 128B swizzle): a [64 tokens][128 channels] tile = 2 panels of
 // 64 channels x 64 rows
 constexpr uint32_t B16 = 2 * R64;
-constexpr uint32_t RAW_Q = OFF_KQ, RAW_K = OFF_KQ + B16, RAW_B = OFF_KQ + 2 * B16, RAW_V = OFF_KQ + 3 * B16;
-constexpr uint32_t RAW_W = OFF_KN;
+constexpr uint32_t RAW_Q = OFF_KQ, RAW_K = OFF_KQ + B16, RAW_B = OFF_KQ + 2 * B16;  // free once the
+constexpr uint32_t RAW_V = OFF_KN, RAW_W = OFF_KN + B16;  // state product (KQ) / [A; P] (Kn) has read them
 constexpr int LDM = 68;                         // padded row (floats) of the 64 x 64 solve matrix
 constexpr int LDX = 36;                         // padded row of the 32 x 32 block product
 constexpr uint32_t TILES = OFF_SCR + 22528;     // 214 KB
 
 struct Misc {
-  uint64_t bar_la, bar_raw;                            // TMA loads landed
+  uint64_t bar_la, bar_raw, bar_vw;                    // TMA loads landed: log alpha; q, k, b; v, w
   uint64_t bar_mma, bar_s, bar_drain;                  // tensor-core products done
   uint64_t bar_ops, bar_stage, bar_solved, bar_uround;  // compute warps -> control warp (16 arrivals)
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[2][128];    // Gamma at the chunk end, per key channel (chunk parity)
-  alignas(16) float segtot[4][128];  // per token segment: sum of log2 alpha, per key channel
+  alignas(16) float segtot[2][128];  // per half chunk: sum of log2 alpha, per key channel
 };
 constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 
@@ -96,6 +97,7 @@ constexpr uint32_t TM_U = 64;    // U~^T         lanes: value channel, columns: 
 constexpr uint32_t TM_R = 128;   // R^T          lanes: value channel, columns: t
 constexpr uint32_t TM_O = 192;   // O^T          lanes: value channel, columns: t (after R^T, before S^T)
 constexpr uint32_t TM_S = 256;   // S^T (state)  lanes: value channel, columns: key channel
+constexpr uint32_t TM_VW = 384;  // Vw^T of the next chunk   lanes: value channel, columns: t
 constexpr uint32_t TM_COLS = 512;
 
 // instruction descriptors (M = 128, both operands K-major)
@@ -151,12 +153,13 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(&ms.bar_la, 1);
     mbar_init(&ms.bar_mma, 1);
     mbar_init(&ms.bar_raw, 1);
+    mbar_init(&ms.bar_vw, 1);
     mbar_init(&ms.bar_s, 1);
     mbar_init(&ms.bar_drain, 1);
     mbar_init(&ms.bar_ops, NCOMP / 32);
     mbar_init(&ms.bar_stage, NCOMP / 32);
     mbar_init(&ms.bar_solved, NCOMP / 32);
-    mbar_init(&ms.bar_uround, NCOMP / 32);
+    mbar_init(&ms.bar_uround, NSOLVE / 32);
     fence_mbar_init();
     ms.abort = 0;
     tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (warp == NCOMP / 32) {
     // ========================= control warp: MMAs and TMA copies =========================
     if (tid == CTL) {
-      int n_la = 0, n_raw = 0;
+      int n_la = 0, n_raw = 0, n_vw = 0;
       auto prefetch_raw = [&](int c) {  // every input tile of chunk c into L2
         for (int pn = 0; pn < (dk >> 5); ++pn) tma_prefetch_l2_4d(&tmLA, 32 * pn, h, C * c, bb);
         for (int pn = 0; pn < (dk >> 6); ++pn) {
@@ -206,27 +209,32 @@ __global__ void __launch_bounds__(NT, 1)
           tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, C * c, bb);
         ++n_la;
       };
-      auto issue_raw = [&](int c) {  // raw bf16 inputs of chunk c into the staging tiles
-        mbar_arrive_expect_tx(&ms.bar_raw, (uint32_t)(3 * (dk >> 6) + 2 * (dv >> 6)) * R64);
+      auto issue_qkb = [&](int c) {  // raw q, k, b of chunk c into the KQ tile
+        mbar_arrive_expect_tx(&ms.bar_raw, (uint32_t)(3 * (dk >> 6)) * R64);
         for (int pn = 0; pn < (dk >> 6); ++pn) {
           tma_load_4d(sm + RAW_Q + pn * R64, &tmQ, &ms.bar_raw, 64 * pn, h, C * c, bb);
           tma_load_4d(sm + RAW_K + pn * R64, &tmK, &ms.bar_raw, 64 * pn, h, C * c, bb);
           tma_load_4d(sm + RAW_B + pn * R64, &tmB, &ms.bar_raw, 64 * pn, h, C * c, bb);
         }
-        for (int pn = 0; pn < (dv >> 6); ++pn) {
-          tma_load_4d(sm + RAW_V + pn * R64, &tmV, &ms.bar_raw, 64 * pn, h, C * c, bb);
-          tma_load_4d(sm + RAW_W + pn * R64, &tmW, &ms.bar_raw, 64 * pn, h, C * c, bb);
-        }
         ++n_raw;
       };
-      auto store_o = [&](int cc) {  // the staged output tile of chunk cc
+      auto issue_vw = [&](int c) {  // raw v, w of chunk c into the Kn tile
+        mbar_arrive_expect_tx(&ms.bar_vw, (uint32_t)(2 * (dv >> 6)) * R64);
+        for (int pn = 0; pn < (dv >> 6); ++pn) {
+          tma_load_4d(sm + RAW_V + pn * R64, &tmV, &ms.bar_vw, 64 * pn, h, C * c, bb);
+          tma_load_4d(sm + RAW_W + pn * R64, &tmW, &ms.bar_vw, 64 * pn, h, C * c, bb);
+        }
+        ++n_vw;
+      };
+      auto store_o = [&](int cc) {  // the staged output tile of chunk cc (rows past T are clipped)
         tma_store_4d(&tmO, sm + OFF_LA, 0, h, C * cc, bb);
         bulk_commit();
       };
       uint32_t ph_ops = 0, ph_stage = 0, ph_solved = 0, ph_uround = 0, ph_s = 0;
       bool alive = true;
       if (p.nchunks > 0) {
-        issue_raw(0);
+        issue_qkb(0);
+        issue_vw(0);
         issue_la(0);
         for (int cc = 1; cc <= PF_AHEAD && cc < p.nchunks; ++cc) prefetch_raw(cc);
       }
@@ -243,23 +251,29 @@ __global__ void __launch_bounds__(NT, 1)
           umma_tf32_ss(tmem + TM_AP, aKQ, bKN, ID_64, ks > 0);
         }
         umma_commit(&ms.bar_mma);
-        // [R^T | O^T] += S^T [-Kb; Qh]^T : A = S^T (tensor memory), B = the KQ tile (N = 128)
+        // [X^T | O^T] = S^T [-Kb; Qh]^T : A = S^T (tensor memory), B = the KQ tile (N = 128);
+        // X^T = -S^T Kb^T becomes R^T = Vw^T + X^T when warps 8-15 round it
         if (!(alive = wait_on(&ms.bar_stage, ph_stage))) break;
         tc_fence_after();
         if (c > 0) store_o(c - 1);
+        // [A; P] has read the Kn tile: the next chunk's v, w.  (Its completion is this
+        // barrier's phase 3c; no later phase can complete before this thread issues again.)
+        if (!(alive = mbar_wait_bounded(&ms.bar_mma, (uint32_t)((3 * c) & 1), &ms.abort, p.err, WAIT_LIMIT))) break;
+        if (c + 1 < p.nchunks) issue_vw(c + 1);
 #pragma unroll 1
         for (int ks = 0; ks < 16; ++ks) {
           const uint64_t bKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
-          umma_tf32_ts(tmem + TM_R, tmem + TM_S + 8 * ks, bKQ, ID_128, 1);
+          umma_tf32_ts(tmem + TM_R, tmem + TM_S + 8 * ks, bKQ, ID_128, ks > 0);
         }
         umma_commit(&ms.bar_s);
-        // both products have read the KQ and Kn tiles: the next chunk's copies
-        if (!(alive = wait_on(&ms.bar_s, ph_s))) break;
+        // the next chunk's log alpha once the output staging has been read
         if (c + 1 < p.nchunks) {
-          issue_raw(c + 1);
-          bulk_wait_read_all();  // the output staging has been read
+          bulk_wait_read_all();
           issue_la(c + 1);
         }
+        // the state product has read the KQ tile: the next chunk's q, k, b
+        if (!(alive = wait_on(&ms.bar_s, ph_s))) break;
+        if (c + 1 < p.nchunks) issue_qkb(c + 1);
         // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t
         if (!(alive = wait_on(&ms.bar_solved, ph_solved))) break;
         tc_fence_after();
@@ -290,6 +304,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_wait_bounded(&ms.bar_drain, 0, &never, nullptr, WAIT_LIMIT);
         if (n_la > 0) mbar_wait_bounded(&ms.bar_la, (uint32_t)((n_la - 1) & 1), &never, nullptr, WAIT_LIMIT);
         if (n_raw > 0) mbar_wait_bounded(&ms.bar_raw, (uint32_t)((n_raw - 1) & 1), &never, nullptr, WAIT_LIMIT);
+        if (n_vw > 0) mbar_wait_bounded(&ms.bar_vw, (uint32_t)((n_vw - 1) & 1), &never, nullptr, WAIT_LIMIT);
       }
       bulk_wait_all();  // output stores complete before the block exits
     }
@@ -311,10 +326,9 @@ __global__ void __launch_bounds__(NT, 1)
     // the T operand tile: blocks above the 8x8 block diagonal stay zero for good
     for (int e = tid; e < 2 * (int)R64 / 16; e += NCOMP)
       *reinterpret_cast<float4*>(sm + OFF_T + 16 * e) = make_float4(0.f, 0.f, 0.f, 0.f);
-    uint32_t ph_la = 0, ph_mma = 0, ph_raw = 0, ph_s = 0;
+    uint32_t ph_mma = 0, ph_s = 0;
     float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);                 // solve matrix, 64 x LDM fp32
     float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);  // block product, 32 x LDX fp32
-    const unsigned char* la_t = sm + OFF_LA;
     const int lane = tid & 31;
     auto wait_mma = [&]() -> bool { return wait_on(&ms.bar_mma, ph_mma); };
     // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory.
@@ -333,7 +347,8 @@ __global__ void __launch_bounds__(NT, 1)
       tmem_st32(tlane + TM_S + 32 * sg, v);
     };
     // Output of the last finished chunk (O^T in tensor memory) into the shared-memory tile
-    // [t][j] (rows of d_v floats) that the control warp's TMA store writes out.
+    // [t][j] (rows of d_v floats, over the log-decay tile, whose reads are done) that the
+    // control warp's TMA store writes out.
     auto stage_o = [&]() {
       float v[16];
       tmem_ld16(tlane + TM_O + 16 * sg, v);
@@ -345,62 +360,89 @@ __global__ void __launch_bounds__(NT, 1)
       }
     };
 
-    bool dead = false;
-    bool ok_prev = true;  // failed waits of the previous chunk's tail, voted at the next barrier
-    for (int c = 0; c < p.nchunks; ++c) {
-      const int ob = c & 1;
-      // ===== in-chunk cumulative log decay (base 2) along this thread's 16 tokens ============
-      float g[16];
+    // Warps 8-15, one chunk ahead (chunk cc): the in-chunk cumulative log decay (base 2),
+    // written back in place over the log-alpha tile; the end-of-chunk decay per key channel;
+    // and Vw^T = (W * V)^T into the tensor-memory columns TM_VW.  Thread (ch, hf) owns the
+    // 32 tokens [32 hf, 32 hf + 32) of channel ch.
+    uint32_t ph_la = 0, ph_raw = 0, ph_vw = 0;
+    auto prep_ahead = [&](int cc, bool ok) -> bool {
+      const int hf = sg - 2;
+      // Vw^T: v and w arrive first (copied as soon as [A; P] has read the Kn tile)
+      ok = ok && wait_on(&ms.bar_vw, ph_vw);
       {
-        bool ok = ok_prev && wait_on(&ms.bar_la, ph_la);
-        ok = ok && wait_on(&ms.bar_raw, ph_raw);
+        float vw[32];
+        const uint32_t pnl = (uint32_t)(ch >> 6) * R64;
+        const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          const uint32_t ro = pnl + sw128_off(32 * hf + r, chk) + byt;
+          vw[r] = vval ? bf16_at(sm + RAW_V + ro) * bf16_at(sm + RAW_W + ro) : 0.f;
+        }
+        tmem_st32(tlane + TM_VW + 32 * hf, vw);
+      }
+      // the cumulative log2 decay, in place
+      unsigned char* la_w = sm + OFF_LA;
+      ok = ok && wait_on(&ms.bar_la, ph_la);
+      {
+        float x[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+          x[r] = kval ? *reinterpret_cast<const float*>(la_w + f32_off(32 * hf + r, ch, R64)) : 0.f;
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const float x = kval ? *reinterpret_cast<const float*>(la_t + f32_off(16 * sg + r, ch, R64)) : 0.f;
-          acc = fmaf(x, LOG2E, acc);
-          g[r] = acc;
+        for (int r = 0; r < 32; ++r) {
+          acc = fmaf(x[r], LOG2E, acc);
+          x[r] = acc;
         }
-        ms.segtot[sg][ch] = acc;
-        if (named_bar_or(BAR_COMP, NCOMP, !ok)) { dead = true; break; }
+        ms.segtot[hf][ch] = acc;
+        named_bar_sync(BAR_AUX, NCOMP - NSOLVE);
+        const float off = hf ? ms.segtot[0][ch] : 0.f;
+        if (kval) {
+#pragma unroll
+          for (int r = 0; r < 32; ++r) *reinterpret_cast<float*>(la_w + f32_off(32 * hf + r, ch, R64)) = x[r] + off;
+        }
+        if (hf == 1) ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
       }
-      tc_fence_after();
-      // ===== folded operands of this thread's channel; Vw^T preloads the R^T accumulator ======
+      tmem_st_wait();
+      return ok;
+    };
+
+    bool dead = false;
+    bool ok_prev = true;  // failed waits of the previous chunk's tail, voted at the next barrier
+    if (p.nchunks > 0 && warp >= NSOLVE / 32) ok_prev = prep_ahead(0, true);
+    tc_fence_before();
+    if (named_bar_or(BAR_COMP, NCOMP, !ok_prev)) dead = true;
+    tc_fence_after();
+    for (int c = 0; c < p.nchunks && !dead; ++c) {
+      const int ob = c & 1;
+      // ===== folded operands of this thread's channel over its 16 tokens (the cumulative decay
+      // was computed one chunk ahead, in place over the log-alpha tile) =========================
       float nkb[16], qh[16], kn[16];
+      bool ok_raw = wait_on(&ms.bar_raw, ph_raw);
       {
-        float off = 0.f;
-        for (int s2 = 0; s2 < sg; ++s2) off += ms.segtot[s2][ch];
-        if (sg == 3) ms.gC[ob][ch] = kval ? ex2_approx(off + g[15]) : 0.f;
-        float vw[16];
+        const unsigned char* la_t = sm + OFF_LA;
         const uint32_t pnl = (uint32_t)(ch >> 6) * R64;  // raw tiles: panels of 64 channels
         const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
           const uint32_t ro = pnl + sw128_off(16 * sg + r, chk) + byt;
-          const float gg = g[r] + off;
+          const float gg = kval ? *reinterpret_cast<const float*>(la_t + f32_off(16 * sg + r, ch, R64)) : 0.f;
           const float G = ex2_approx(gg), Gi = ex2_approx(-gg);
-          float kk = 0.f, bg = 0.f, qq = 0.f, vv = 0.f, ww = 0.f;
+          float kk = 0.f, bg = 0.f, qq = 0.f;
           if (kval) {
             kk = bf16_at(sm + RAW_K + ro);
             bg = bf16_at(sm + RAW_B + ro);
             qq = bf16_at(sm + RAW_Q + ro);
           }
-          if (vval) {
-            vv = bf16_at(sm + RAW_V + ro);
-            ww = bf16_at(sm + RAW_W + ro);
-          }
           nkb[r] = -(kk * bg) * G;
           qh[r] = qq * G;
           kn[r] = kk * Gi;
-          vw[r] = ww * vv;
         }
-        // the R^T columns are free: the previous chunk's U~ product has completed
-        tmem_st16(tlane + TM_R + 16 * sg, vw);
       }
       // the previous chunk's last product must be done before Kn^T, O and S are touched,
       // and every raw read before the operand tiles overwrite the staging
       {
-        const bool ok = (c == 0) || wait_mma();
+        const bool ok = ok_raw && ((c == 0) || wait_mma());
         if (named_bar_or(BAR_COMP, NCOMP, !ok)) { dead = true; break; }
       }
       tc_fence_after();
@@ -417,14 +459,10 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_before();
       warp_arrive(&ms.bar_ops);
       // ===== while [A; P] is on the tensor cores: the previous chunk's output and state
-      // decay, and the output accumulator cleared ==============================================
-      {
-        if (c > 0) stage_o();  // the log-alpha tile is free until the next chunk's copy
-        float z[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) z[x] = 0.f;
-        tmem_st16(tlane + TM_O + 16 * sg, z);
-        if (c > 0) decay_state(ob ^ 1);
+      // decay ==================================================================================
+      if (c > 0) {
+        stage_o();
+        decay_state(ob ^ 1);
       }
       tmem_st_wait();
       fence_proxy_async_smem();
@@ -598,35 +636,52 @@ __global__ void __launch_bounds__(NT, 1)
           put_t2(row, col, -d[0], -d[1]);
           put_t2(row + 8, col, -d[2], -d[3]);
         }
-      } else {
-        ok_s = wait_on(&ms.bar_s, ph_s);
+        fence_proxy_async_smem();  // the T operand tile
+        tc_fence_before();
+        warp_arrive(&ms.bar_solved);
+        // ===== U~^T rounded to tf32 in place: the A operand of the chunk's last product =======
+        const bool ok_u = wait_mma();
         tc_fence_after();
         float v[32];
-        tmem_ld32(tlane + TM_R + 32 * (sg - 2), v);
+        tmem_ld32(tlane + TM_U + 32 * sg, v);
         tmem_ld_wait();
 #pragma unroll
         for (int x = 0; x < 32; ++x) v[x] = rna_tf32(v[x]);
-        tmem_st32(tlane + TM_R + 32 * (sg - 2), v);
-        tmem_st_wait();
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      warp_arrive(&ms.bar_solved);
-      // ===== U~^T rounded to tf32 in place: the A operand of the chunk's last product =========
-      {
-        const bool ok_u = wait_mma();
-        tc_fence_after();
-        float v[16];
-        tmem_ld16(tlane + TM_U + 16 * sg, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 16; ++x) v[x] = rna_tf32(v[x]);
-        tmem_st16(tlane + TM_U + 16 * sg, v);
+        tmem_st32(tlane + TM_U + 32 * sg, v);
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(&ms.bar_uround);
-        ok_prev = ok_s && ok_u;
+        ok_prev = ok_u;
+      } else {
+        // ===== R^T = Vw^T + X^T rounded to tf32 in place once the state product is done ======
+        ok_s = wait_on(&ms.bar_s, ph_s);
+        tc_fence_after();
+        {
+          float v[32], w[32];
+          tmem_ld32(tlane + TM_R + 32 * (sg - 2), v);
+          tmem_ld32(tlane + TM_VW + 32 * (sg - 2), w);
+          tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = rna_tf32(v[x] + w[x]);
+          tmem_st32(tlane + TM_R + 32 * (sg - 2), v);
+          tmem_st_wait();
+        }
+        fence_proxy_async_smem();  // this warp's rows of the P operand tile
+        tc_fence_before();
+        warp_arrive(&ms.bar_solved);
+        // ===== then one chunk ahead: cumulative decay and Vw^T of the next chunk =============
+        if (c + 1 < p.nchunks) ok_s = prep_ahead(c + 1, ok_s);
+        // These warps do not use U~; they step their phase bit past its product without
+        // waiting (by now the chunk's last product may have completed as well, and a parity
+        // wait must never trail its barrier by two phases).  Their next wait, on that last
+        // product, cannot be overtaken: the barrier's following phase needs these warps.
+        ph_mma ^= 1;
+        ok_prev = ok_s;
+        tc_fence_before();
       }
+      // the next chunk reads what warps 8-15 prepared
+      if (named_bar_or(BAR_COMP, NCOMP, !ok_prev)) { dead = true; break; }
+      tc_fence_after();
     }
 
     // ---- last chunk's output and decay, then the final state -----------------------------
@@ -673,14 +728,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B, T, H, D] tensor; one box = 64 tokens x box_d channels of one (b, h).
+// [B, T, H, D] tensor; one box = box_t tokens x box_d channels of one (b, h).
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int B, int T, int H, int D,
-              int box_d, CUtensorMapSwizzle swz) {
+              int box_d, CUtensorMapSwizzle swz, int box_t = C) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)D * esize, (cuuint64_t)H * D * esize, (cuuint64_t)T * H * D * esize};
-  cuuint32_t box[4] = {(cuuint32_t)box_d, 1, (cuuint32_t)C, 1};
+  cuuint32_t box[4] = {(cuuint32_t)box_d, 1, (cuuint32_t)box_t, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
