@@ -56,7 +56,7 @@ constexpr int NSOLVE = 256;                     // warps 0-7 run the triangular 
 constexpr int BAR_COMP = 1, BAR_SOLVE = 2, BAR_AUX = 3;  // named barriers: compute warps; warps 0-7; 8-15
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
 constexpr float LOG2E = 1.4426950408889634f;
-constexpr int PF_AHEAD = 3;                     // chunks of input prefetched into L2 ahead of use
+constexpr int PF_AHEAD = 2;                     // chunks of input prefetched into L2 ahead of use
 
 // ---- shared memory map (byte offsets from a 1024-byte aligned base) ----------------
 // fp32 operand tiles with the 128B swizzle, in panels of 32 columns (128 B rows).
