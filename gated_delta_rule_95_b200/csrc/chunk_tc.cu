@@ -127,6 +127,14 @@ __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast
 __device__ __forceinline__ float bf16_at(const unsigned char* p) {
   return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short*>(p)) << 16);
 }
+// two adjacent bf16 elements (4-byte aligned) of shared memory as fp32
+__device__ __forceinline__ float2 bf16x2_at(const unsigned char* p) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+__device__ __forceinline__ void st2_tf32(unsigned char* p, const float2& f) {
+  *reinterpret_cast<float2*>(p) = make_float2(rna_tf32(f.x), rna_tf32(f.y));
+}
 
 // DK, DV: key and value head dimensions (64 or 128), fixed at compile time so that each
 // launch runs straight-line code for its own shape.
@@ -380,7 +388,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
         tmem_st32(tlane + TM_VW + 32 * hf, vw);
       }
-      // the cumulative log2 decay, in place
+      // the cumulative decay Gamma = 2^g, in place
       unsigned char* la_w = sm + OFF_LA;
       ok = ok && wait_on(&ms.bar_la, ph_la);
       {
@@ -399,7 +407,8 @@ __global__ void __launch_bounds__(NT, 1)
         const float off = hf ? ms.segtot[0][ch] : 0.f;
         if (kval) {
 #pragma unroll
-          for (int r = 0; r < 32; ++r) *reinterpret_cast<float*>(la_w + f32_off(32 * hf + r, ch, R64)) = x[r] + off;
+          for (int r = 0; r < 32; ++r)
+            *reinterpret_cast<float*>(la_w + f32_off(32 * hf + r, ch, R64)) = ex2_approx(x[r] + off);
         }
         if (hf == 1) ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
       }
@@ -415,28 +424,33 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_after();
     for (int c = 0; c < p.nchunks && !dead; ++c) {
       const int ob = c & 1;
-      // ===== folded operands of this thread's channel over its 16 tokens (the cumulative decay
-      // was computed one chunk ahead, in place over the log-alpha tile) =========================
-      float nkb[16], qh[16], kn[16];
+      // ===== folded operands.  For this step thread t owns the key-channel pair
+      // (2 cp, 2 cp + 1), cp = t mod 64, over the 8 tokens [8 ts, 8 ts + 8), ts = t / 64, so
+      // that every raw load and tile store moves both channels at once.  Gamma = 2^g was
+      // computed one chunk ahead, in place over the log-alpha tile. ==========================
+      const int cp = tid & 63, ts = tid >> 6, c2 = 2 * cp;
+      const bool kv2 = c2 < dk;
+      float2 nkb[8], qh[8], kn[8];
       bool ok_raw = wait_on(&ms.bar_raw, ph_raw);
       {
         const unsigned char* la_t = sm + OFF_LA;
-        const uint32_t pnl = (uint32_t)(ch >> 6) * R64;  // raw tiles: panels of 64 channels
-        const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
+        const uint32_t pnl = (uint32_t)(c2 >> 6) * R64;  // raw tiles: panels of 64 channels
+        const int chk = (c2 & 63) >> 3, byt = (c2 & 7) * 2;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const uint32_t ro = pnl + sw128_off(16 * sg + r, chk) + byt;
-          const float gg = kval ? *reinterpret_cast<const float*>(la_t + f32_off(16 * sg + r, ch, R64)) : 0.f;
-          const float G = ex2_approx(gg), Gi = ex2_approx(-gg);
-          float kk = 0.f, bg = 0.f, qq = 0.f;
-          if (kval) {
-            kk = bf16_at(sm + RAW_K + ro);
-            bg = bf16_at(sm + RAW_B + ro);
-            qq = bf16_at(sm + RAW_Q + ro);
+        for (int r = 0; r < 8; ++r) {
+          const int t = 8 * ts + r;
+          const uint32_t ro = pnl + sw128_off(t, chk) + byt;
+          float2 G = make_float2(1.f, 1.f), kk = make_float2(0.f, 0.f), bg = kk, qq = kk;
+          if (kv2) {
+            G = *reinterpret_cast<const float2*>(la_t + f32_off(t, c2, R64));
+            kk = bf16x2_at(sm + RAW_K + ro);
+            bg = bf16x2_at(sm + RAW_B + ro);
+            qq = bf16x2_at(sm + RAW_Q + ro);
           }
-          nkb[r] = -(kk * bg) * G;
-          qh[r] = qq * G;
-          kn[r] = kk * Gi;
+          const float2 Gi = make_float2(rcp_approx(G.x), rcp_approx(G.y));
+          nkb[r] = make_float2(-(kk.x * bg.x) * G.x, -(kk.y * bg.y) * G.y);
+          qh[r] = make_float2(qq.x * G.x, qq.y * G.y);
+          kn[r] = make_float2(kk.x * Gi.x, kk.y * Gi.y);
         }
       }
       // the previous chunk's last product must be done before Kn^T, O and S are touched,
@@ -447,14 +461,27 @@ __global__ void __launch_bounds__(NT, 1)
       }
       tc_fence_after();
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const int t = 16 * sg + r;
-        *reinterpret_cast<float*>(sm + OFF_KQ + f32_off(t, ch, R128)) = rna_tf32(nkb[r]);
-        *reinterpret_cast<float*>(sm + OFF_KQ + f32_off(64 + t, ch, R128)) = rna_tf32(qh[r]);
-        *reinterpret_cast<float*>(sm + OFF_KN + f32_off(t, ch, R64)) = rna_tf32(kn[r]);
+      for (int r = 0; r < 8; ++r) {
+        const int t = 8 * ts + r;
+        st2_tf32(sm + OFF_KQ + f32_off(t, c2, R128), nkb[r]);
+        st2_tf32(sm + OFF_KQ + f32_off(64 + t, c2, R128), qh[r]);
+        st2_tf32(sm + OFF_KN + f32_off(t, c2, R64), kn[r]);
       }
+      {
+        // Kn^T rows 2 cp and 2 cp + 1, tokens [8 ts, 8 ts + 8).  The first store of each
+        // thread goes to row 2 cp + ((cp >> 2) & 1), so that the 8 threads sharing a
+        // 128-byte wavefront hit 8 different swizzle phases.
+        const int sw = (cp >> 2) & 1;
 #pragma unroll
-      for (int r = 0; r < 16; r += 4) st4_tf32(sm + OFF_PK + f32_off(64 + ch, 16 * sg + r, R192), kn + r);
+        for (int e = 0; e < 2; ++e) {
+          const int rsel = e ^ sw;  // 0: channel 2 cp, 1: channel 2 cp + 1
+          float f[8];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) f[r] = rsel ? kn[r].y : kn[r].x;
+          st4_tf32(sm + OFF_PK + f32_off(64 + c2 + rsel, 8 * ts, R192), f);
+          st4_tf32(sm + OFF_PK + f32_off(64 + c2 + rsel, 8 * ts + 4, R192), f + 4);
+        }
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       warp_arrive(&ms.bar_ops);

@@ -311,6 +311,12 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
       : "memory");
   return r != 0;
 }
+// 1/x by the special-function unit (PTX rcp.approx.ftz.f32).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // 2^x by the special-function unit (PTX ex2.approx.ftz.f32; a few ulp, flushes subnormals).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
