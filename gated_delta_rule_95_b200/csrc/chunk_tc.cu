@@ -83,7 +83,7 @@ constexpr uint32_t TILES = OFF_SCR + 22528;     // 214 KB
 struct Misc {
   uint64_t bar_la, bar_raw, bar_vw;                    // TMA loads landed: log alpha; q, k, b; v, w
   uint64_t bar_mma, bar_s, bar_drain;                  // tensor-core products done
-  uint64_t bar_ops, bar_stage, bar_solved, bar_uround;  // compute warps -> control warp (16 arrivals)
+  uint64_t bar_ops, bar_stage, bar_tdiag, bar_solved, bar_uround;  // compute warps -> control warp
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[2][128];    // Gamma at the chunk end, per key channel (chunk parity)
@@ -97,10 +97,11 @@ constexpr uint32_t TM_U = 64;    // U~^T         lanes: value channel, columns: 
 constexpr uint32_t TM_R = 128;   // R^T          lanes: value channel, columns: t
 constexpr uint32_t TM_O = 192;   // O^T          lanes: value channel, columns: t (after R^T, before S^T)
 constexpr uint32_t TM_S = 256;   // S^T (state)  lanes: value channel, columns: key channel
-constexpr uint32_t TM_VW = 384;  // Vw^T of the next chunk   lanes: value channel, columns: t
+constexpr uint32_t TM_VW = 384;  // Vw^T, two buffers (chunk parity)   lanes: value channel, columns: t
 constexpr uint32_t TM_COLS = 512;
 
 // instruction descriptors (M = 128, both operands K-major)
+constexpr uint32_t ID_32 = idesc_tf32(128, 32, 0, 0, 0, 0);
 constexpr uint32_t ID_64 = idesc_tf32(128, 64, 0, 0, 0, 0);
 constexpr uint32_t ID_128 = idesc_tf32(128, 128, 0, 0, 0, 0);
 constexpr uint32_t ID_192 = idesc_tf32(128, 192, 0, 0, 0, 0);
@@ -166,7 +167,8 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(&ms.bar_drain, 1);
     mbar_init(&ms.bar_ops, NCOMP / 32);
     mbar_init(&ms.bar_stage, NCOMP / 32);
-    mbar_init(&ms.bar_solved, NCOMP / 32);
+    mbar_init(&ms.bar_tdiag, NCOMP / 32);   // R^T rounded, diagonal 32x32 blocks of T written
+    mbar_init(&ms.bar_solved, NSOLVE / 32);  // the T_21 block written
     mbar_init(&ms.bar_uround, NSOLVE / 32);
     fence_mbar_init();
     ms.abort = 0;
@@ -238,7 +240,7 @@ __global__ void __launch_bounds__(NT, 1)
         tma_store_4d(&tmO, sm + OFF_LA, 0, h, C * cc, bb);
         bulk_commit();
       };
-      uint32_t ph_ops = 0, ph_stage = 0, ph_solved = 0, ph_uround = 0, ph_s = 0;
+      uint32_t ph_ops = 0, ph_stage = 0, ph_tdiag = 0, ph_solved = 0, ph_uround = 0, ph_s = 0;
       bool alive = true;
       if (p.nchunks > 0) {
         issue_qkb(0);
@@ -282,13 +284,28 @@ __global__ void __launch_bounds__(NT, 1)
         // the state product has read the KQ tile: the next chunk's q, k, b
         if (!(alive = wait_on(&ms.bar_s, ph_s))) break;
         if (c + 1 < p.nchunks) issue_qkb(c + 1);
-        // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t
+        // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t, in 32-column halves
+        // of s.  With T = [T11 0; T21 T22] (32 x 32 blocks): U~^T[:, :32] = R1^T T11^T and
+        // U~^T[:, 32:] = R2^T T22^T + R1^T T21^T; everything but the T21 term is issued as soon
+        // as the diagonal blocks exist, overlapping the last level of the solve.
+        if (!(alive = wait_on(&ms.bar_tdiag, ph_tdiag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {  // s in [0, 32), t in [0, 32)
+          const uint64_t bT = sdesc_sw128(sbase + OFF_T + ks * 32, 16, 1024);
+          umma_tf32_ts(tmem + TM_U, tmem + TM_R + 8 * ks, bT, ID_32, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 4; ks < 8; ++ks) {  // s in [32, 64), t in [32, 64)
+          const uint64_t bT = sdesc_sw128(sbase + OFF_T + R64 + 32 * 128 + (ks & 3) * 32, 16, 1024);
+          umma_tf32_ts(tmem + TM_U + 32, tmem + TM_R + 8 * ks, bT, ID_32, ks > 4);
+        }
         if (!(alive = wait_on(&ms.bar_solved, ph_solved))) break;
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bT = sdesc_sw128(sbase + OFF_T + (ks >> 2) * R64 + (ks & 3) * 32, 16, 1024);
-          umma_tf32_ts(tmem + TM_U, tmem + TM_R + 8 * ks, bT, ID_64, ks > 0);
+        for (int ks = 0; ks < 4; ++ks) {  // s in [32, 64), t in [0, 32): the T21 block
+          const uint64_t bT = sdesc_sw128(sbase + OFF_T + 32 * 128 + ks * 32, 16, 1024);
+          umma_tf32_ts(tmem + TM_U + 32, tmem + TM_R + 8 * ks, bT, ID_32, 1);
         }
         umma_commit(&ms.bar_mma);
         // [O^T | S^T] += U~^T [P; Kn^T]^T : O^T += U~^T P^T and S^T += U~^T Kn in one N = 192 product
@@ -368,57 +385,57 @@ __global__ void __launch_bounds__(NT, 1)
       }
     };
 
-    // Warps 8-15, one chunk ahead (chunk cc): the in-chunk cumulative log decay (base 2),
-    // written back in place over the log-alpha tile; the end-of-chunk decay per key channel;
-    // and Vw^T = (W * V)^T into the tensor-memory columns TM_VW.  Thread (ch, hf) owns the
-    // 32 tokens [32 hf, 32 hf + 32) of channel ch.
+    // Warps 8-15, one chunk ahead (chunk cc).  Thread (ch, hf) owns the 32 tokens
+    // [32 hf, 32 hf + 32) of channel ch.
     uint32_t ph_la = 0, ph_raw = 0, ph_vw = 0;
-    auto prep_ahead = [&](int cc, bool ok) -> bool {
+    // Vw^T = (W * V)^T into the tensor-memory buffer of chunk cc's parity (v and w are copied
+    // as soon as [A; P] has read the Kn tile).
+    auto vw_ahead = [&](int cc, bool ok) -> bool {
       const int hf = sg - 2;
-      // Vw^T: v and w arrive first (copied as soon as [A; P] has read the Kn tile)
       ok = ok && wait_on(&ms.bar_vw, ph_vw);
-      {
-        float vw[32];
-        const uint32_t pnl = (uint32_t)(ch >> 6) * R64;
-        const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
+      float vw[32];
+      const uint32_t pnl = (uint32_t)(ch >> 6) * R64;
+      const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
-          const uint32_t ro = pnl + sw128_off(32 * hf + r, chk) + byt;
-          vw[r] = vval ? bf16_at(sm + RAW_V + ro) * bf16_at(sm + RAW_W + ro) : 0.f;
-        }
-        tmem_st32(tlane + TM_VW + 32 * hf, vw);
+      for (int r = 0; r < 32; ++r) {
+        const uint32_t ro = pnl + sw128_off(32 * hf + r, chk) + byt;
+        vw[r] = vval ? bf16_at(sm + RAW_V + ro) * bf16_at(sm + RAW_W + ro) : 0.f;
       }
-      // the cumulative decay Gamma = 2^g, in place
+      tmem_st32(tlane + TM_VW + 64 * (cc & 1) + 32 * hf, vw);
+      tmem_st_wait();
+      return ok;
+    };
+    // The in-chunk cumulative decay Gamma = 2^g (base-2 cumsum of log alpha), written back
+    // in place over the log-alpha tile, and the end-of-chunk decay per key channel.
+    auto decay_ahead = [&](int cc, bool ok) -> bool {
+      const int hf = sg - 2;
       unsigned char* la_w = sm + OFF_LA;
       ok = ok && wait_on(&ms.bar_la, ph_la);
-      {
-        float x[32];
+      float x[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        x[r] = kval ? *reinterpret_cast<const float*>(la_w + f32_off(32 * hf + r, ch, R64)) : 0.f;
+      float acc = 0.f;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        acc = fmaf(x[r], LOG2E, acc);
+        x[r] = acc;
+      }
+      ms.segtot[hf][ch] = acc;
+      named_bar_sync(BAR_AUX, NCOMP - NSOLVE);
+      const float off = hf ? ms.segtot[0][ch] : 0.f;
+      if (kval) {
 #pragma unroll
         for (int r = 0; r < 32; ++r)
-          x[r] = kval ? *reinterpret_cast<const float*>(la_w + f32_off(32 * hf + r, ch, R64)) : 0.f;
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < 32; ++r) {
-          acc = fmaf(x[r], LOG2E, acc);
-          x[r] = acc;
-        }
-        ms.segtot[hf][ch] = acc;
-        named_bar_sync(BAR_AUX, NCOMP - NSOLVE);
-        const float off = hf ? ms.segtot[0][ch] : 0.f;
-        if (kval) {
-#pragma unroll
-          for (int r = 0; r < 32; ++r)
-            *reinterpret_cast<float*>(la_w + f32_off(32 * hf + r, ch, R64)) = ex2_approx(x[r] + off);
-        }
-        if (hf == 1) ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
+          *reinterpret_cast<float*>(la_w + f32_off(32 * hf + r, ch, R64)) = ex2_approx(x[r] + off);
       }
-      tmem_st_wait();
+      if (hf == 1) ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
       return ok;
     };
 
     bool dead = false;
     bool ok_prev = true;  // failed waits of the previous chunk's tail, voted at the next barrier
-    if (p.nchunks > 0 && warp >= NSOLVE / 32) ok_prev = prep_ahead(0, true);
+    if (p.nchunks > 0 && warp >= NSOLVE / 32) ok_prev = decay_ahead(0, vw_ahead(0, true));
     tc_fence_before();
     if (named_bar_or(BAR_COMP, NCOMP, !ok_prev)) dead = true;
     tc_fence_after();
@@ -631,6 +648,10 @@ __global__ void __launch_bounds__(NT, 1)
           }
           named_bar_sync(BAR_SOLVE, NSOLVE);
         }
+        // the diagonal 32x32 blocks of T are in the operand tile: most of the U~ product can go
+        fence_proxy_async_smem();
+        tc_fence_before();
+        warp_arrive(&ms.bar_tdiag);
         {
           // 64x64: T_21 = -T_22 (A_21 T_11) with 32x32 blocks; warp 4 mt + nt (8 warps)
           // computes the 16 x 8 output tile (rows [16 mt, +16), columns [8 nt, +8)).
@@ -681,12 +702,12 @@ __global__ void __launch_bounds__(NT, 1)
         ok_prev = ok_u;
       } else {
         // ===== R^T = Vw^T + X^T rounded to tf32 in place once the state product is done ======
-        ok_s = wait_on(&ms.bar_s, ph_s);
+        ok_s = ok_s && wait_on(&ms.bar_s, ph_s);
         tc_fence_after();
         {
           float v[32], w[32];
           tmem_ld32(tlane + TM_R + 32 * (sg - 2), v);
-          tmem_ld32(tlane + TM_VW + 32 * (sg - 2), w);
+          tmem_ld32(tlane + TM_VW + 64 * (c & 1) + 32 * (sg - 2), w);
           tmem_ld_wait();
 #pragma unroll
           for (int x = 0; x < 32; ++x) v[x] = rna_tf32(v[x] + w[x]);
@@ -695,9 +716,9 @@ __global__ void __launch_bounds__(NT, 1)
         }
         fence_proxy_async_smem();  // this warp's rows of the P operand tile
         tc_fence_before();
-        warp_arrive(&ms.bar_solved);
-        // ===== then one chunk ahead: cumulative decay and Vw^T of the next chunk =============
-        if (c + 1 < p.nchunks) ok_s = prep_ahead(c + 1, ok_s);
+        warp_arrive(&ms.bar_tdiag);
+        // ===== then one chunk ahead: Vw^T and the cumulative decay of the next chunk =========
+        if (c + 1 < p.nchunks) ok_s = decay_ahead(c + 1, vw_ahead(c + 1, ok_s));
         // These warps do not use U~; they step their phase bit past its product without
         // waiting (by now the chunk's last product may have completed as well, and a parity
         // wait must never trail its barrier by two phases).  Their next wait, on that last
