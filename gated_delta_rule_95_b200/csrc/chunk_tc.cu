@@ -11,7 +11,8 @@
 //     Kb = K*B*Gamma    Qh = Q*Gamma    Kn = K/Gamma    Vw = W*V
 //     [A; P]  = [Kb; Qh] Kn^T           A strictly lower, P lower incl. diagonal
 //     T       = (I + A)^-1              recursive 2x2 block inverse (fp32 diagonal blocks)
-//     R^T     = Vw^T - S^T Kb^T         O^T = S^T Qh^T        (one product over [Kb; Qh])
+//     X^T     = -S^T Kb^T               O^T = S^T Qh^T        (one product over [-Kb; Qh])
+//     R^T     = Vw^T + X^T
 //     U~^T    = R^T T^T                 (= ((I + A)^-1 (Vw - Kb S))^T, the erase-corrected writes)
 //     O^T    += U~^T P^T
 //     S^T    <- (S^T + U~^T Kn) Diag(Gamma_C)
@@ -26,16 +27,19 @@
 // One CTA owns one (batch, head) and walks its chunks.  Warps 0-15 (512 threads) do the
 // elementwise work: thread t owns channel ch = t mod 128 (a key channel and a value
 // channel, and the tensor-memory lane of the same index) over the 16 tokens
-// [16 sg, 16 sg + 16), sg = t / 128, so the decay cumsum runs along its own tokens and
-// the operand tiles, Kn^T and the Vw^T accumulator preload are written without any
-// transposition.  Warp 16 is the control warp: its first thread issues every MMA and
-// every TMA copy, so that an issue that stalls on a full tensor-core queue never holds
-// up the elementwise warps.  The two sides hand over through mbarriers only (every wait
-// bounded).  While [A; P] is on the tensor cores the previous chunk's output is staged
-// for a TMA store and its state decay is applied; the state product runs while warps
-// 0-7 invert (I + A), and warps 8-15 round R^T; the next chunk's raw inputs are copied
-// as soon as the state product has released their tiles, and prefetched into L2 two
-// chunks ahead.
+// [16 sg, 16 sg + 16), sg = t / 128; for the operand build it owns the key-channel pair
+// (2 (t mod 64), +1) over the 8 tokens [8 (t / 64), +8).  Warp 16 is the control warp:
+// its first thread issues every MMA and every TMA copy, so that an issue that stalls on a
+// full tensor-core queue never holds up the elementwise warps.  The two sides hand over
+// through mbarriers only (every wait bounded).  Per chunk: the operand tiles are built,
+// [A; P] runs while the previous chunk's output is staged for a TMA store and its state
+// decay applied; then warps 0-7 read A out and invert (I + A) while the state product
+// runs and warps 8-15 round R^T and prepare the next chunk (its Vw^T, and its cumulative
+// decay Gamma written in place over the log-alpha tile); the U~ product is issued in two
+// parts so that only its T21 term waits for the last level of the solve.  The next
+// chunk's v, w are copied once [A; P] has read the Kn tile, q, k, b once the state
+// product has read the KQ tile, log alpha once the output staging has been read; every
+// input is prefetched into L2 two chunks ahead.
 // d_k or d_v = 64 run the same code with the upper half of each operand zero.
 #include <cuda.h>
 #include <cuda_bf16.h>
