@@ -30,6 +30,7 @@ import gdn2_inputs as gi  # noqa: E402
 
 PREFILL = gi.WORKLOADS["prefill_b8_h16_t4096"]
 DECODE = gi.WORKLOADS["decode_b256_h16"]
+PACKED = gi.WORKLOADS["packed_n64_h16"]
 METRIC = "GDN-2 prefill tokens/s per layer"
 UNIT = "tokens/s"
 # algorithmic HBM bytes per token-head: q,k,v,b,w bf16 + log-alpha fp32 in, o fp32 out
@@ -211,6 +212,36 @@ def time_prefill(args, rank, world, dev):
                 tokens=B * T, token_heads=B * T * H)
 
 
+def time_packed(args, dev):
+    """The packed serving batch (variable-length sequences with entering states)."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    lengths = gi.packed_lengths(PACKED.B, 16, PACKED.T, PACKED.seed)
+    d = gi.packed_inputs(PACKED, lengths)
+    x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    T, H = x["q"].shape[0], PACKED.H
+    o = torch.empty((T, H, PACKED.dv), dtype=torch.float32, device=dev)
+    S_T = torch.empty((PACKED.B, H, PACKED.dk, PACKED.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        g.gdn2_chunk_fwd_varlen(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["cu_seqlens"], x["S0"],
+                                o=o, S_T=S_T)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for _ in range(args.steps):
+        step()
+    t1.record(st)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    return dict(ms=ms, tokens=T, token_heads=T * H, units=PACKED.B * H, n_seq=PACKED.B,
+                ok=g.gdn2_device_status() == 0)
+
+
 def time_prefill_e2e(args, dev):
     """Same step through the public API with pinned host buffers, copies included."""
     import torch
@@ -363,6 +394,10 @@ def main():
     traffic = profile_traffic("chunk_fwd_tc_kernel")
 
     dec = time_decode(dev, args.decode_steps, world)
+    pak = time_packed(args, dev)
+    # algorithmic bytes: the token streams plus each sequence's entering and final state
+    pak_bytes = pak["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD + pak["units"] * DECODE_STATE_BYTES
+    pak_gbs = pak_bytes / (pak["ms"] * 1e-3) / 1e9
     dec_units = DECODE.B * DECODE.H
     dec_gbs = dec_units * DECODE_STATE_BYTES / (dec["ms_per_step"] * 1e-3) / 1e9
     barrier(world)
@@ -393,9 +428,16 @@ def main():
                                 "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],
                                 "traffic": profile_traffic("decode_step_kernel")},
                    "clocks": dec["clocks"]},
+        "packed": {"metric": "GDN-2 packed prefill tokens/s per layer", "value": pak["tokens"] / (pak["ms"] * 1e-3),
+                   "unit": "tokens/s", "ms_per_step": pak["ms"], "steps": args.steps,
+                   "workload": f"packed_n64_h16: {pak['n_seq']} sequences, lengths log-uniform in [16, 8192] "
+                               f"({pak['tokens']} tokens), H=16 d_k=d_v=128, bf16, entering states N(0, 0.02)",
+                   "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (packed)", "achieved": pak_gbs,
+                                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": pak_gbs / pk["hbm_gbs"],
+                                "traffic": None}},
         "gpu_launches": args.steps,
         "clocks": pre["clocks"],
-        "device_status_ok": bool(pre["ok"] and dec["ok"]),
+        "device_status_ok": bool(pre["ok"] and dec["ok"] and pak["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)

@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -55,6 +55,8 @@ def lib():
         P, I = ctypes.c_void_p, ctypes.c_int
         L.gdn2_chunk_fwd.argtypes = [P] * 9 + [I] * 6 + [P]
         L.gdn2_chunk_fwd.restype = I
+        L.gdn2_chunk_fwd_varlen.argtypes = [P] * 10 + [I] * 6 + [P]
+        L.gdn2_chunk_fwd_varlen.restype = I
         L.gdn2_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
         L.gdn2_decode_step.restype = I
         L.gdn2_device_status.argtypes = []
@@ -110,6 +112,39 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_
                               _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd", rc)
+    return o, S_T
+
+
+def gdn2_chunk_fwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, o=None, S_T=None, want_state=True,
+                          stream=None):
+    """Chunkwise prefill forward over packed variable-length sequences.
+
+    q, k, b: [T, H, d_k]; v, w: [T, H, d_v]; log_alpha: [T, H, d_k]; cu_seqlens: int32 [N + 1]
+    on the device.  Returns (o [T, H, d_v], S_T [N, H, d_k, d_v] or None)."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise ValueError("gdn2_chunk_fwd_varlen: bf16 inputs only")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise ValueError("gdn2_chunk_fwd_varlen: cu_seqlens must be a contiguous int32 vector")
+    if cu_seqlens.device != q.device:
+        raise ValueError("gdn2_chunk_fwd_varlen: cu_seqlens must be on the inputs' device")
+    N = cu_seqlens.numel() - 1
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=torch.float32, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    ts = dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, o=o)
+    if S0 is not None:
+        ts["S0"] = S0
+    if S_T is not None:
+        ts["S_T"] = S_T
+    _check_tokens("gdn2_chunk_fwd_varlen", ts, q.dtype, q.device)
+    rc = lib().gdn2_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(cu_seqlens),
+                                     _ptr(S0), _ptr(o), _ptr(S_T), N, T, H, dk, dv, _DT[q.dtype],
+                                     _stream(q.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_chunk_fwd_varlen", rc)
     return o, S_T
 
 

@@ -77,6 +77,28 @@ extern "C" gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* 
   return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
 }
 
+extern "C" gdn2_status gdn2_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* log_alpha,
+                                             const void* b, const void* w, const int* cu_seqlens, const float* S0,
+                                             float* o, float* S_T, int N, int T, int H, int d_k, int d_v,
+                                             gdn2_dtype dt, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (dt != GDN2_BF16) return GDN2_ERR_DTYPE;  // packed sequences: bf16 inputs only
+  if (!sizes_ok(1, T, H, d_k, d_v) || N < 0 || (long long)N * H > 0x7fffffffLL) return GDN2_ERR_SHAPE;
+  if ((long long)N * H == 0) return GDN2_OK;
+  if (!cu_seqlens) return GDN2_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !log_alpha || !b || !w || !o)) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, b, w, S0, o, S_T};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return GDN2_ERR_ALIGN;
+
+  ChunkArgs a{q, k, v, b, w, log_alpha, S0, o, S_T, N, T, H, d_k, d_v, true, cu_seqlens};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // no tokens at all: every sequence is empty and keeps its entering state
+  cudaError_t e = (T == 0) ? launch_state_copy(a, st) : launch_chunk_fwd_tc(a, st);
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
 extern "C" gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
                                         const void* b, const void* w, float* S, float* o, int B, int H, int d_k,
                                         int d_v, gdn2_dtype dt, void* stream) {
@@ -101,7 +123,7 @@ extern "C" gdn2_status gdn2_device_status(void) {
   if (word) {
     e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_fail(e);
-    return GDN2_ERR_TIMEOUT;
+    return (word & kErrBadSeqlens) ? GDN2_ERR_SHAPE : GDN2_ERR_TIMEOUT;
   }
   return GDN2_OK;
 }

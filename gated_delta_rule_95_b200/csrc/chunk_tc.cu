@@ -115,7 +115,8 @@ struct TcParams {
   const float* S0;
   float* S_T;
   float* o;
-  int T, H, dk, dv, nchunks;
+  int T, H, dk, dv;
+  const int* cu_seqlens;  // packed sequences: [N + 1] token offsets (device); NULL = fixed length T
   unsigned* err;
 };
 
@@ -142,8 +143,10 @@ __device__ __forceinline__ void st2_tf32(unsigned char* p, const float2& f) {
 }
 
 // DK, DV: key and value head dimensions (64 or 128), fixed at compile time so that each
-// launch runs straight-line code for its own shape.
-template <int DK, int DV>
+// launch runs straight-line code for its own shape.  VARLEN: the batch is a packed set of
+// sequences (a CTA per (sequence, head), token range from cu_seqlens); otherwise B
+// sequences of T tokens.
+template <int DK, int DV, bool VARLEN>
 __global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
@@ -158,7 +161,20 @@ __global__ void __launch_bounds__(NT, 1)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int ch = tid & 127;  // channel (key i and value j) and tensor-memory lane
   const int sg = tid >> 7;   // token segment [16 sg, 16 sg + 16); column group of TMEM accesses
-  const int unit = blockIdx.x, bb = unit / p.H, h = unit % p.H;
+  const int unit = blockIdx.x, h = unit % p.H;
+  // this CTA's sequence: batch coordinate bb, first token t0, length len, chunk count nch
+  int bb = unit / p.H, t0 = 0, len = p.T;
+  if constexpr (VARLEN) {
+    const int n = unit / p.H;
+    bb = 0;
+    t0 = p.cu_seqlens[n];
+    len = p.cu_seqlens[n + 1] - t0;
+    if (t0 < 0 || len < 0 || t0 + len > p.T) {  // offsets out of order or out of range
+      if (threadIdx.x == 0 && p.err) atomicOr(p.err, kErrBadSeqlens);
+      return;
+    }
+  }
+  const int nch = (len + C - 1) / C;
   constexpr int dk = DK, dv = DV;
   const bool kval = ch < dk, vval = ch < dv;
 
@@ -206,54 +222,54 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == CTL) {
       int n_la = 0, n_raw = 0, n_vw = 0;
       auto prefetch_raw = [&](int c) {  // every input tile of chunk c into L2
-        for (int pn = 0; pn < (dk >> 5); ++pn) tma_prefetch_l2_4d(&tmLA, 32 * pn, h, C * c, bb);
+        for (int pn = 0; pn < (dk >> 5); ++pn) tma_prefetch_l2_4d(&tmLA, 32 * pn, h, t0 + C * c, bb);
         for (int pn = 0; pn < (dk >> 6); ++pn) {
-          tma_prefetch_l2_4d(&tmQ, 64 * pn, h, C * c, bb);
-          tma_prefetch_l2_4d(&tmK, 64 * pn, h, C * c, bb);
-          tma_prefetch_l2_4d(&tmB, 64 * pn, h, C * c, bb);
+          tma_prefetch_l2_4d(&tmQ, 64 * pn, h, t0 + C * c, bb);
+          tma_prefetch_l2_4d(&tmK, 64 * pn, h, t0 + C * c, bb);
+          tma_prefetch_l2_4d(&tmB, 64 * pn, h, t0 + C * c, bb);
         }
         for (int pn = 0; pn < (dv >> 6); ++pn) {
-          tma_prefetch_l2_4d(&tmV, 64 * pn, h, C * c, bb);
-          tma_prefetch_l2_4d(&tmW, 64 * pn, h, C * c, bb);
+          tma_prefetch_l2_4d(&tmV, 64 * pn, h, t0 + C * c, bb);
+          tma_prefetch_l2_4d(&tmW, 64 * pn, h, t0 + C * c, bb);
         }
       };
       auto issue_la = [&](int c) {  // log alpha of chunk c: dk/32 boxes of 32 channels x 64 tokens
         mbar_arrive_expect_tx(&ms.bar_la, (uint32_t)(C * dk * 4));
         for (int pn = 0; pn < (dk >> 5); ++pn)
-          tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, C * c, bb);
+          tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, t0 + C * c, bb);
         ++n_la;
       };
       auto issue_qkb = [&](int c) {  // raw q, k, b of chunk c into the KQ tile
         mbar_arrive_expect_tx(&ms.bar_raw, (uint32_t)(3 * (dk >> 6)) * R64);
         for (int pn = 0; pn < (dk >> 6); ++pn) {
-          tma_load_4d(sm + RAW_Q + pn * R64, &tmQ, &ms.bar_raw, 64 * pn, h, C * c, bb);
-          tma_load_4d(sm + RAW_K + pn * R64, &tmK, &ms.bar_raw, 64 * pn, h, C * c, bb);
-          tma_load_4d(sm + RAW_B + pn * R64, &tmB, &ms.bar_raw, 64 * pn, h, C * c, bb);
+          tma_load_4d(sm + RAW_Q + pn * R64, &tmQ, &ms.bar_raw, 64 * pn, h, t0 + C * c, bb);
+          tma_load_4d(sm + RAW_K + pn * R64, &tmK, &ms.bar_raw, 64 * pn, h, t0 + C * c, bb);
+          tma_load_4d(sm + RAW_B + pn * R64, &tmB, &ms.bar_raw, 64 * pn, h, t0 + C * c, bb);
         }
         ++n_raw;
       };
       auto issue_vw = [&](int c) {  // raw v, w of chunk c into the Kn tile
         mbar_arrive_expect_tx(&ms.bar_vw, (uint32_t)(2 * (dv >> 6)) * R64);
         for (int pn = 0; pn < (dv >> 6); ++pn) {
-          tma_load_4d(sm + RAW_V + pn * R64, &tmV, &ms.bar_vw, 64 * pn, h, C * c, bb);
-          tma_load_4d(sm + RAW_W + pn * R64, &tmW, &ms.bar_vw, 64 * pn, h, C * c, bb);
+          tma_load_4d(sm + RAW_V + pn * R64, &tmV, &ms.bar_vw, 64 * pn, h, t0 + C * c, bb);
+          tma_load_4d(sm + RAW_W + pn * R64, &tmW, &ms.bar_vw, 64 * pn, h, t0 + C * c, bb);
         }
         ++n_vw;
       };
       auto store_o = [&](int cc) {  // the staged output tile of chunk cc (rows past T are clipped)
-        tma_store_4d(&tmO, sm + OFF_LA, 0, h, C * cc, bb);
+        tma_store_4d(&tmO, sm + OFF_LA, 0, h, t0 + C * cc, bb);
         bulk_commit();
       };
       uint32_t ph_ops = 0, ph_stage = 0, ph_tdiag = 0, ph_solved = 0, ph_uround = 0, ph_s = 0;
       bool alive = true;
-      if (p.nchunks > 0) {
+      if (nch > 0) {
         issue_qkb(0);
         issue_vw(0);
         issue_la(0);
-        for (int cc = 1; cc <= PF_AHEAD && cc < p.nchunks; ++cc) prefetch_raw(cc);
+        for (int cc = 1; cc <= PF_AHEAD && cc < nch; ++cc) prefetch_raw(cc);
       }
-      for (int c = 0; c < p.nchunks; ++c) {
-        if (c + PF_AHEAD < p.nchunks) prefetch_raw(c + PF_AHEAD);
+      for (int c = 0; c < nch; ++c) {
+        if (c + PF_AHEAD < nch) prefetch_raw(c + PF_AHEAD);
         // [-A; P] = [-Kb; Qh] Kn^T : M=128 (tokens of both halves), N=64 (s), K=128 (key channels)
         if (!(alive = wait_on(&ms.bar_ops, ph_ops))) break;
         tc_fence_after();
@@ -273,7 +289,7 @@ __global__ void __launch_bounds__(NT, 1)
         // [A; P] has read the Kn tile: the next chunk's v, w.  (Its completion is this
         // barrier's phase 3c; no later phase can complete before this thread issues again.)
         if (!(alive = mbar_wait_bounded(&ms.bar_mma, (uint32_t)((3 * c) & 1), &ms.abort, p.err, WAIT_LIMIT))) break;
-        if (c + 1 < p.nchunks) issue_vw(c + 1);
+        if (c + 1 < nch) issue_vw(c + 1);
 #pragma unroll 1
         for (int ks = 0; ks < 16; ++ks) {
           const uint64_t bKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
@@ -281,13 +297,13 @@ __global__ void __launch_bounds__(NT, 1)
         }
         umma_commit(&ms.bar_s);
         // the next chunk's log alpha once the output staging has been read
-        if (c + 1 < p.nchunks) {
+        if (c + 1 < nch) {
           bulk_wait_read_all();
           issue_la(c + 1);
         }
         // the state product has read the KQ tile: the next chunk's q, k, b
         if (!(alive = wait_on(&ms.bar_s, ph_s))) break;
-        if (c + 1 < p.nchunks) issue_qkb(c + 1);
+        if (c + 1 < nch) issue_qkb(c + 1);
         // U~^T = R^T T^T : A = R^T (tensor memory), B = T (N = s), K = t, in 32-column halves
         // of s.  With T = [T11 0; T21 T22] (32 x 32 blocks): U~^T[:, :32] = R1^T T11^T and
         // U~^T[:, 32:] = R2^T T22^T + R1^T T21^T; everything but the T21 term is issued as soon
@@ -315,7 +331,7 @@ __global__ void __launch_bounds__(NT, 1)
         // [O^T | S^T] += U~^T [P; Kn^T]^T : O^T += U~^T P^T and S^T += U~^T Kn in one N = 192 product
         if (!(alive = wait_on(&ms.bar_uround, ph_uround))) break;
         tc_fence_after();
-        if (c + 1 == p.nchunks) bulk_wait_read_all();  // the last staging may be rewritten after this
+        if (c + 1 == nch) bulk_wait_read_all();  // the last staging may be rewritten after this
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bPK = sdesc_sw128(sbase + OFF_PK + (ks >> 2) * R192 + (ks & 3) * 32, 16, 1024);
@@ -323,8 +339,10 @@ __global__ void __launch_bounds__(NT, 1)
         }
         umma_commit(&ms.bar_mma);
       }
-      // the last chunk's output, staged by the compute warps
-      if (alive && p.nchunks > 0 && wait_on(&ms.bar_stage, ph_stage)) store_o(p.nchunks - 1);
+      // the last chunk's output, staged by the compute warps (a packed sequence's partial last
+      // chunk is written by the compute warps themselves: its box would spill into the next
+      // sequence's rows)
+      if (alive && nch > 0 && wait_on(&ms.bar_stage, ph_stage) && !(VARLEN && len % C)) store_o(nch - 1);
       // after a give-up: every MMA issued so far (a fresh commit tracks all of them) and
       // the last copies must land before the block releases its memory
       if (ms.abort) {
@@ -351,6 +369,7 @@ __global__ void __launch_bounds__(NT, 1)
         v[x] = (ok && i < dk) ? p.S0[((size_t)unit * dk + i) * dv + ch] : 0.f;
       }
       tmem_st32(tlane + TM_S + 32 * sg, v);
+      tmem_st_wait();
     }
     // the T operand tile: blocks above the 8x8 block diagonal stay zero for good
     for (int e = tid; e < 2 * (int)R64 / 16; e += NCOMP)
@@ -403,7 +422,8 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int r = 0; r < 32; ++r) {
         const uint32_t ro = pnl + sw128_off(32 * hf + r, chk) + byt;
-        vw[r] = vval ? bf16_at(sm + RAW_V + ro) * bf16_at(sm + RAW_W + ro) : 0.f;
+        const bool tv = !VARLEN || C * cc + 32 * hf + r < len;
+        vw[r] = (vval && tv) ? bf16_at(sm + RAW_V + ro) * bf16_at(sm + RAW_W + ro) : 0.f;
       }
       tmem_st32(tlane + TM_VW + 64 * (cc & 1) + 32 * hf, vw);
       tmem_st_wait();
@@ -418,7 +438,8 @@ __global__ void __launch_bounds__(NT, 1)
       float x[32];
 #pragma unroll
       for (int r = 0; r < 32; ++r)
-        x[r] = kval ? *reinterpret_cast<const float*>(la_w + f32_off(32 * hf + r, ch, R64)) : 0.f;
+        x[r] = (kval && (!VARLEN || C * cc + 32 * hf + r < len))
+                   ? *reinterpret_cast<const float*>(la_w + f32_off(32 * hf + r, ch, R64)) : 0.f;
       float acc = 0.f;
 #pragma unroll
       for (int r = 0; r < 32; ++r) {
@@ -439,11 +460,11 @@ __global__ void __launch_bounds__(NT, 1)
 
     bool dead = false;
     bool ok_prev = true;  // failed waits of the previous chunk's tail, voted at the next barrier
-    if (p.nchunks > 0 && warp >= NSOLVE / 32) ok_prev = decay_ahead(0, vw_ahead(0, true));
+    if (nch > 0 && warp >= NSOLVE / 32) ok_prev = decay_ahead(0, vw_ahead(0, true));
     tc_fence_before();
     if (named_bar_or(BAR_COMP, NCOMP, !ok_prev)) dead = true;
     tc_fence_after();
-    for (int c = 0; c < p.nchunks && !dead; ++c) {
+    for (int c = 0; c < nch && !dead; ++c) {
       const int ob = c & 1;
       // ===== folded operands.  For this step thread t owns the key-channel pair
       // (2 cp, 2 cp + 1), cp = t mod 64, over the 8 tokens [8 ts, 8 ts + 8), ts = t / 64, so
@@ -462,7 +483,8 @@ __global__ void __launch_bounds__(NT, 1)
           const int t = 8 * ts + r;
           const uint32_t ro = pnl + sw128_off(t, chk) + byt;
           float2 G = make_float2(1.f, 1.f), kk = make_float2(0.f, 0.f), bg = kk, qq = kk;
-          if (kv2) {
+          // (packed sequences: the tile rows past this sequence's end hold the next one's tokens)
+          if (kv2 && (!VARLEN || C * c + t < len)) {
             G = *reinterpret_cast<const float2*>(la_t + f32_off(t, c2, R64));
             kk = bf16x2_at(sm + RAW_K + ro);
             bg = bf16x2_at(sm + RAW_B + ro);
@@ -722,7 +744,7 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         warp_arrive(&ms.bar_tdiag);
         // ===== then one chunk ahead: Vw^T and the cumulative decay of the next chunk =========
-        if (c + 1 < p.nchunks) ok_s = decay_ahead(c + 1, vw_ahead(c + 1, ok_s));
+        if (c + 1 < nch) ok_s = decay_ahead(c + 1, vw_ahead(c + 1, ok_s));
         // These warps do not use U~; they step their phase bit past its product without
         // waiting (by now the chunk's last product may have completed as well, and a parity
         // wait must never trail its barrier by two phases).  Their next wait, on that last
@@ -737,26 +759,42 @@ __global__ void __launch_bounds__(NT, 1)
     }
 
     // ---- last chunk's output and decay, then the final state -----------------------------
-    if (!dead && p.nchunks > 0) {
+    if (!dead && nch > 0) {
       const bool ok = ok_prev && wait_mma();
       if (named_bar_or(BAR_COMP, NCOMP, !ok)) dead = true;
     }
-    if (!dead && p.nchunks > 0) {
+    if (!dead && nch > 0) {
       tc_fence_after();
-      stage_o();
-      decay_state((p.nchunks - 1) & 1);
+      if (VARLEN && len % C) {
+        // partial last chunk of a packed sequence: rows straight to o, masked to the sequence
+        float v[16];
+        tmem_ld16(tlane + TM_O + 16 * sg, v);
+        tmem_ld_wait();
+        if (vval) {
+          const int tb = C * (nch - 1) + 16 * sg;  // token within the sequence
+          float* dst = p.o + ((size_t)(t0 + tb) * p.H + h) * dv + ch;
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            if (tb + x < len) dst[(size_t)x * p.H * dv] = v[x];
+        }
+      } else {
+        stage_o();
+      }
+      decay_state((nch - 1) & 1);
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       warp_arrive(&ms.bar_stage);
-      if (p.S_T && vval) {
-        float v[32];
-        tmem_ld32(tlane + TM_S + 32 * sg, v);
-        tmem_ld_wait();
+    }
+    // the final state (for an empty sequence: the entering one)
+    if (!dead && p.S_T && vval) {
+      tc_fence_after();
+      float v[32];
+      tmem_ld32(tlane + TM_S + 32 * sg, v);
+      tmem_ld_wait();
 #pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if (32 * sg + x < dk) p.S_T[((size_t)unit * dk + 32 * sg + x) * dv + ch] = v[x];
-      }
+      for (int x = 0; x < 32; ++x)
+        if (32 * sg + x < dk) p.S_T[((size_t)unit * dk + 32 * sg + x) * dv + ch] = v[x];
     }
   }
   // ---- teardown ---------------------------------------------------------------------------
@@ -794,35 +832,49 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
   return r == CUDA_SUCCESS;
 }
 
-template <int DK, int DV>
+template <int DK, int DV, bool VARLEN>
 cudaError_t launch_shape(int grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
                          const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw, const CUtensorMap& mla,
                          const CUtensorMap& mo, const TcParams& p) {
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV, VARLEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  chunk_fwd_tc_kernel<DK, DV><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
+  chunk_fwd_tc_kernel<DK, DV, VARLEN><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
   return cudaSuccess;
 }
 
 }  // namespace
 
+template <bool VARLEN>
+cudaError_t launch_dims(int grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
+                        const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw, const CUtensorMap& mla,
+                        const CUtensorMap& mo, const TcParams& p) {
+  if (p.dk == 128 && p.dv == 128) return launch_shape<128, 128, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (p.dk == 128 && p.dv == 64) return launch_shape<128, 64, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (p.dk == 64 && p.dv == 128) return launch_shape<64, 128, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (p.dk == 64 && p.dv == 64) return launch_shape<64, 64, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   if (a.B * a.H == 0) return cudaSuccess;
+  // packed sequences: one [1, total T, H, D] tensor, sequence n = tokens [cu[n], cu[n+1])
+  const bool varlen = a.cu_seqlens != nullptr;
+  const int Bm = varlen ? 1 : a.B;
   CUtensorMap mq, mk, mv, mb, mw, mla, mo;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
-  bool ok = make_map(&mq, a.q, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
-            make_map(&mk, a.k, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
-            make_map(&mb, a.b, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
-            make_map(&mv, a.v, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
-            make_map(&mw, a.w, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
-            make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dk, 32, SW) &&
-            make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dv, a.dv,
+  bool ok = make_map(&mq, a.q, BF, 2, Bm, a.T, a.H, a.dk, 64, SW) &&
+            make_map(&mk, a.k, BF, 2, Bm, a.T, a.H, a.dk, 64, SW) &&
+            make_map(&mb, a.b, BF, 2, Bm, a.T, a.H, a.dk, 64, SW) &&
+            make_map(&mv, a.v, BF, 2, Bm, a.T, a.H, a.dv, 64, SW) &&
+            make_map(&mw, a.w, BF, 2, Bm, a.T, a.H, a.dv, 64, SW) &&
+            make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, Bm, a.T, a.H, a.dk, 32, SW) &&
+            make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, Bm, a.T, a.H, a.dv, a.dv,
                      CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   TcParams p;
@@ -838,13 +890,11 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   p.H = a.H;
   p.dk = a.dk;
   p.dv = a.dv;
-  p.nchunks = (a.T + C - 1) / C;
+  p.cu_seqlens = a.cu_seqlens;
   p.err = device_error_word();
-  cudaError_t e = cudaErrorInvalidValue;
-  if (a.dk == 128 && a.dv == 128) e = launch_shape<128, 128>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
-  else if (a.dk == 128 && a.dv == 64) e = launch_shape<128, 64>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
-  else if (a.dk == 64 && a.dv == 128) e = launch_shape<64, 128>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
-  else if (a.dk == 64 && a.dv == 64) e = launch_shape<64, 64>(a.B * a.H, st, mq, mk, mv, mb, mw, mla, mo, p);
+  const int grid = a.B * a.H;
+  cudaError_t e = varlen ? launch_dims<true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
+                         : launch_dims<false>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

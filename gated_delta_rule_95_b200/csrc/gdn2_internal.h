@@ -19,11 +19,17 @@ struct ChunkArgs {
   const float* S0;
   float* o;
   float* S_T;
-  int B, T, H, dk, dv;
+  int B, T, H, dk, dv;  // packed sequences: B = number of sequences, T = total tokens
   bool bf16;
+  const int* cu_seqlens;  // packed sequences: [B + 1] device token offsets; NULL otherwise
 };
 
-// Device error word of this library (bit set = a bounded wait gave up).
+// Device error word of this library: bits set by kernels, read and cleared by
+// gdn2_device_status().
+enum : unsigned {
+  kErrWaitTimeout = 1u,  // a bounded wait gave up
+  kErrBadSeqlens = 2u    // packed-sequence offsets out of order or out of range
+};
 unsigned* device_error_word();
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);

@@ -6,10 +6,9 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-namespace gdn2 {
+#include "gdn2_internal.h"  // error word bits
 
-// Error word bits set on the device (read back by gdn2_device_status()).
-enum : unsigned { kErrWaitTimeout = 1u };
+namespace gdn2 {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

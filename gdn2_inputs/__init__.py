@@ -68,6 +68,10 @@ WORKLOADS = {
                                 steps=1000, state_std=0.02),
     "mixed_b4_h32_t8192": Workload("mixed_b4_h32_t8192", "prefill", 4, 32, 8192, 128, 128, "bf16", seed=4,
                                    regimes=True),
+    # packed serving batch: 64 sequences, lengths log-uniform in [16, 8192] (packed_lengths),
+    # each continuing from an entering state N(0, 0.02)
+    "packed_n64_h16": Workload("packed_n64_h16", "packed", 64, 16, 8192, 128, 128, "bf16", seed=5,
+                               state_std=0.02),
 }
 
 
@@ -161,6 +165,35 @@ def prefill_inputs(wl: Workload, B=None, T=None, H=None, seed=None):
                b=_round(b, wl.dtype), w=_round(w, wl.dtype),
                log_alpha=torch.from_numpy(la),
                S0=None if S0 is None else torch.from_numpy(S0))
+    return out
+
+
+def packed_lengths(n: int, lo: int, hi: int, seed: int):
+    """A seeded serving-like length mix: n lengths log-uniform in [lo, hi] (integers)."""
+    rng = np.random.default_rng([seed, 2000])
+    return [int(x) for x in np.exp(rng.uniform(np.log(lo), np.log(hi), size=n)).round()]
+
+
+def packed_inputs(wl: Workload, lengths, H=None, seed=None, state_std=None):
+    """Packed variable-length sequences drawn with a prefill workload's recipe.
+
+    Returns dict(q, k, v, b, w: dtype [T,H,D]; log_alpha: float32 [T,H,dk];
+    cu_seqlens: int32 [N+1]; S0: float32 [N,H,dk,dv] or None), T = sum(lengths).
+    """
+    import torch
+    H = wl.H if H is None else H
+    T = int(sum(lengths))
+    d = prefill_inputs(wl, B=1, T=max(T, 1), H=H, seed=seed)
+    out = {k: (None if v is None else v[0, :T]) for k, v in d.items() if k != "S0"}
+    cu = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lengths)
+    out["cu_seqlens"] = torch.from_numpy(cu)
+    std = wl.state_std if state_std is None else state_std
+    S0 = None
+    if std > 0:
+        key = [(wl.seed if seed is None else seed) + 7919]
+        S0 = torch.from_numpy(_draw(key, _TID["S"], (len(lengths), H, wl.dk, wl.dv), lambda x: std * x))
+    out["S0"] = S0
     return out
 
 

@@ -83,6 +83,34 @@ GDN2_API gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* v,
                            int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
 
 /*
+ * Chunkwise prefill forward over a packed batch of variable-length sequences, each
+ * with its own state: the serving case of many independent dialogues or documents
+ * whose states are carried between calls (DeltaNet-2 AI architecture guide: the
+ * inference endpoint accepts and returns the updated state; Gated DeltaNet-2 guide,
+ * "Enterprise Strategy": continuous dialogues and streaming documents).  Sequence n
+ * is the token range [cu_seqlens[n], cu_seqlens[n+1]) of the packed tensors; each
+ * sequence is computed exactly as gdn2_chunk_fwd computes one batch element.
+ *
+ *   q, k, b      : [T, H, d_k]  bf16 (T = total tokens of all sequences)
+ *   v, w         : [T, H, d_v]  bf16
+ *   log_alpha    : [T, H, d_k]  fp32
+ *   cu_seqlens   : [N + 1] int32 DEVICE array, cu_seqlens[0] = 0, non-decreasing,
+ *                  cu_seqlens[N] = T; a sequence may be empty.  Offsets out of order
+ *                  or out of range are detected on the device: that sequence is
+ *                  skipped and gdn2_device_status() reports GDN2_ERR_SHAPE.
+ *   S0           : [N, H, d_k, d_v] fp32, read only; NULL means zero states
+ *   o            : [T, H, d_v]  fp32, written
+ *   S_T          : [N, H, d_k, d_v] fp32, each sequence's final state, written;
+ *                  NULL means "do not write"; may alias S0
+ *   N, T, H      : >= 0
+ *   dt           : GDN2_BF16 (fp32 inputs return GDN2_ERR_DTYPE)
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* log_alpha,
+                                  const void* b, const void* w, const int* cu_seqlens, const float* S0,
+                                  float* o, float* S_T, int N, int T, int H, int d_k, int d_v, gdn2_dtype dt,
+                                  void* stream);
+
+/*
  * One recurrent decode step: the update above for a single token per
  * (sequence, head), with the state updated in place (Gated DeltaNet-2 guide,
  * "4.5x Higher Decoding Throughput with Zero KV Cache": a fixed-size state
@@ -99,7 +127,8 @@ GDN2_API gdn2_status gdn2_decode_step(const void* q, const void* k, const void* 
                              int B, int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
 
 /* Synchronises the current device, then reports and clears the device error
- * word: GDN2_OK, GDN2_ERR_TIMEOUT, or GDN2_ERR_CUDA if the sync itself failed. */
+ * word: GDN2_OK, GDN2_ERR_TIMEOUT (a bounded wait gave up), GDN2_ERR_SHAPE (bad
+ * cu_seqlens), or GDN2_ERR_CUDA if the sync itself failed. */
 GDN2_API gdn2_status gdn2_device_status(void);
 
 /* Static description of a status code. */

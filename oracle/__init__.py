@@ -86,6 +86,33 @@ def forward(q, k, v, log_alpha, b, w, S0=None, nthreads=None, lib=None):
     return o, S_T
 
 
+def forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, nthreads=None, lib=None):
+    """Packed variable-length sequences: tokens [T,H,D], sequence n = rows
+    [cu_seqlens[n], cu_seqlens[n+1]).  Each sequence is an independent run of the
+    recurrence from its own entering state (the stateful-serving reading of the
+    DeltaNet-2 AI architecture guide: the endpoint accepts and returns the state),
+    so this is `forward` on each slice.  Returns (o [T,H,dv], S_T [N,H,dk,dv])."""
+    q, k, v, log_alpha, b, w, S0 = map(_f64, (q, k, v, log_alpha, b, w, S0))
+    cu = [int(x) for x in np.asarray(cu_seqlens).ravel()]
+    N = len(cu) - 1
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((T, H, dv))
+    S_T = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        a, e = cu[n], cu[n + 1]
+        s0 = None if S0 is None else S0[n:n + 1]
+        if e == a:
+            if s0 is not None:
+                S_T[n] = s0[0]
+            continue
+        sl = [x[a:e][None] for x in (q, k, v, log_alpha, b, w)]
+        o_n, s_n = forward(*sl, S0=s0, nthreads=nthreads, lib=lib)
+        o[a:e] = o_n[0]
+        S_T[n] = s_n[0]
+    return o, S_T
+
+
 def decode_step(q, k, v, log_alpha, b, w, S, nthreads=None, lib=None):
     """One token per unit: tokens [B,H,D], S [B,H,dk,dv].  Returns (o, S_new)."""
     q, k, v, log_alpha, b, w = map(_f64, (q, k, v, log_alpha, b, w))

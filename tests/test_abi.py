@@ -68,6 +68,20 @@ def test_decode_step_validation(kw, status):
     assert decode(**kw) == status
 
 
+def varlen(q=A, k=A, v=A, la=A, b=A, w=A, cu=A, S0=None, o=A, ST=None, N=2, T=100, H=1, dk=128, dv=128, dt=1):
+    return g.lib().gdn2_chunk_fwd_varlen(q, k, v, la, b, w, cu, S0, o, ST, N, T, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=96), 2), (dict(N=-1), 2), (dict(T=-1), 2), (dict(dt=0), 3), (dict(dt=5), 3),
+    (dict(cu=None), 1), (dict(q=None), 1), (dict(o=None), 1),
+    (dict(cu=P(0x10002)), 4), (dict(v=M), 4), (dict(ST=M), 4),
+    (dict(N=0), 0), (dict(H=0), 0),
+])
+def test_chunk_fwd_varlen_validation(kw, status):
+    assert varlen(**kw) == status
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)

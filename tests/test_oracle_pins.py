@@ -38,3 +38,25 @@ def test_thread_count_does_not_change_result():
     o1, S1 = oracle.forward(**d, nthreads=1)
     o2, S2 = oracle.forward(**d, nthreads=7)
     assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+
+
+def test_packed_sequences_are_independent_runs():
+    """Packed variable-length sequences: the same tokens as equal-length batch rows give
+    the batch result exactly; an empty sequence hands its entering state through; a
+    sequence's result does not depend on its neighbours."""
+    import numpy as np
+    import gdn2_inputs as gi
+    import oracle
+    wl = gi.WORKLOADS["prefill_b8_h16_t4096"]
+    d = gi.prefill_inputs(wl, B=3, T=40, H=2)
+    f = {k: gi.as_f64(d[k]) for k in ("q", "k", "v", "log_alpha", "b", "w")}
+    S0 = np.random.default_rng(0).normal(0, 0.05, (3, 2, 128, 128))
+    o_ref, S_ref = oracle.forward(**f, S0=S0)
+    packed = {k: f[k].reshape(120, 2, -1) for k in f}
+    o, S = oracle.forward_varlen(**packed, cu_seqlens=np.array([0, 40, 80, 120]), S0=S0)
+    assert np.array_equal(o.reshape(3, 40, 2, -1), o_ref) and np.array_equal(S, S_ref)
+    # an empty sequence in the middle, and the neighbours unchanged
+    S0e = np.concatenate([S0[:1], S0[1:2] * 3, S0[1:]])
+    o2, S2 = oracle.forward_varlen(**packed, cu_seqlens=np.array([0, 40, 40, 80, 120]), S0=S0e)
+    assert np.array_equal(S2[1], S0e[1]) and np.array_equal(o2, o)
+    assert np.array_equal(S2[[0, 2, 3]], S)
