@@ -61,6 +61,7 @@ constexpr int BAR_COMP = 1, BAR_SOLVE = 2, BAR_AUX = 3;  // named barriers: comp
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int PF_AHEAD = 2;                     // chunks of input prefetched into L2 ahead of use
+constexpr int LPT_MAX_SEQ = 1024;               // packed batches up to this many sequences start longest first
 
 // ---- shared memory map (byte offsets from a 1024-byte aligned base) ----------------
 // fp32 operand tiles with the 128B swizzle, in panels of 32 columns (128 B rows).
@@ -117,6 +118,7 @@ struct TcParams {
   float* o;
   int T, H, dk, dv;
   const int* cu_seqlens;  // packed sequences: [N + 1] token offsets (device); NULL = fixed length T
+  int nseq;               // packed sequences: N
   unsigned* err;
 };
 
@@ -162,10 +164,29 @@ __global__ void __launch_bounds__(NT, 1)
   const int ch = tid & 127;  // channel (key i and value j) and tensor-memory lane
   const int sg = tid >> 7;   // token segment [16 sg, 16 sg + 16); column group of TMEM accesses
   const int unit = blockIdx.x, h = unit % p.H;
-  // this CTA's sequence: batch coordinate bb, first token t0, length len, chunk count nch
-  int bb = unit / p.H, t0 = 0, len = p.T;
+  // this CTA's sequence: batch coordinate bb, first token t0, length len, chunk count nch,
+  // and su, the (sequence, head) index of its entering and final state
+  int bb = unit / p.H, t0 = 0, len = p.T, su = unit;
   if constexpr (VARLEN) {
-    const int n = unit / p.H;
+    int n = unit / p.H;
+    if (p.nseq <= LPT_MAX_SEQ) {
+      // Launch order by length, longest first (ties by index), so that the longest
+      // sequences of an uneven batch do not start last: this CTA takes the sequence of
+      // rank unit / H.  The lengths are ranked in the (still unused) solve scratch.
+      __shared__ int picked;
+      int* lens = reinterpret_cast<int*>(sm + OFF_SCR);
+      for (int i = threadIdx.x; i < p.nseq; i += NT) lens[i] = p.cu_seqlens[i + 1] - p.cu_seqlens[i];
+      __syncthreads();
+      for (int i = threadIdx.x; i < p.nseq; i += NT) {
+        const int li = lens[i];
+        int rank = 0;
+        for (int m = 0; m < p.nseq; ++m) rank += (lens[m] > li) | (lens[m] == li && m < i);
+        if (rank == n) picked = i;
+      }
+      __syncthreads();
+      n = picked;
+    }
+    su = n * p.H + h;
     bb = 0;
     t0 = p.cu_seqlens[n];
     len = p.cu_seqlens[n + 1] - t0;
@@ -366,7 +387,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
         const int i = 32 * sg + x;
-        v[x] = (ok && i < dk) ? p.S0[((size_t)unit * dk + i) * dv + ch] : 0.f;
+        v[x] = (ok && i < dk) ? p.S0[((size_t)su * dk + i) * dv + ch] : 0.f;
       }
       tmem_st32(tlane + TM_S + 32 * sg, v);
       tmem_st_wait();
@@ -794,7 +815,7 @@ __global__ void __launch_bounds__(NT, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int x = 0; x < 32; ++x)
-        if (32 * sg + x < dk) p.S_T[((size_t)unit * dk + 32 * sg + x) * dv + ch] = v[x];
+        if (32 * sg + x < dk) p.S_T[((size_t)su * dk + 32 * sg + x) * dv + ch] = v[x];
     }
   }
   // ---- teardown ---------------------------------------------------------------------------
@@ -891,6 +912,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   p.dk = a.dk;
   p.dv = a.dv;
   p.cu_seqlens = a.cu_seqlens;
+  p.nseq = varlen ? a.B : 0;
   p.err = device_error_word();
   const int grid = a.B * a.H;
   cudaError_t e = varlen ? launch_dims<true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
