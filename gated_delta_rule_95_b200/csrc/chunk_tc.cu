@@ -29,9 +29,10 @@
 // channel, and the tensor-memory lane of the same index) over the 16 tokens
 // [16 sg, 16 sg + 16), sg = t / 128; for the operand build it owns the key-channel pair
 // (2 (t mod 64), +1) over the 8 tokens [8 (t / 64), +8).  Warp 16 is the control warp:
-// its first thread issues every MMA and every TMA copy, so that an issue that stalls on a
-// full tensor-core queue never holds up the elementwise warps.  The two sides hand over
-// through mbarriers only (every wait bounded).  Per chunk: the operand tiles are built,
+// its first thread issues every MMA and the input copies, so that an issue that stalls on a
+// full tensor-core queue never holds up the elementwise warps; the first thread of warp 17
+// issues the output stores and the log-alpha copies.  The sides hand over through
+// mbarriers only (every wait bounded).  Per chunk: the operand tiles are built,
 // [A; P] runs while the previous chunk's output is staged for a TMA store and its state
 // decay applied; then warps 0-7 read A out and invert (I + A) while the state product
 // runs and warps 8-15 round R^T and prepare the next chunk (its Vw^T, and its cumulative
@@ -54,8 +55,9 @@ namespace {
 
 constexpr int C = 64;
 constexpr int NCOMP = 512;                      // warps 0-15: elementwise work
-constexpr int NT = NCOMP + 32;                  // + the control warp
-constexpr int CTL = NCOMP;                      // the thread that issues MMAs and TMA copies
+constexpr int NT = NCOMP + 64;                  // + the control warp and the store warp
+constexpr int CTL = NCOMP;                      // the thread that issues MMAs and the input copies
+constexpr int STW = NCOMP + 32;                 // the thread that issues output stores and log-alpha copies
 constexpr int NSOLVE = 256;                     // warps 0-7 run the triangular solve
 constexpr int BAR_COMP = 1, BAR_SOLVE = 2, BAR_AUX = 3;  // named barriers: compute warps; warps 0-7; 8-15
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
@@ -89,6 +91,7 @@ struct Misc {
   uint64_t bar_la, bar_raw, bar_vw;                    // TMA loads landed: log alpha; q, k, b; v, w
   uint64_t bar_mma, bar_s, bar_drain;                  // tensor-core products done
   uint64_t bar_ops, bar_stage, bar_tdiag, bar_solved, bar_uround;  // compute warps -> control warp
+  uint64_t bar_lastread;  // store warp -> compute warps: the last staging tile may be rewritten
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[2][128];    // Gamma at the chunk end, per key channel (chunk parity)
@@ -211,6 +214,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(&ms.bar_tdiag, NCOMP / 32);   // R^T rounded, diagonal 32x32 blocks of T written
     mbar_init(&ms.bar_solved, NSOLVE / 32);  // the T_21 block written
     mbar_init(&ms.bar_uround, NSOLVE / 32);
+    mbar_init(&ms.bar_lastread, 1);
     fence_mbar_init();
     ms.abort = 0;
     tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
@@ -241,7 +245,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (warp == NCOMP / 32) {
     // ========================= control warp: MMAs and TMA copies =========================
     if (tid == CTL) {
-      int n_la = 0, n_raw = 0, n_vw = 0;
+      int n_raw = 0, n_vw = 0;
       auto prefetch_raw = [&](int c) {  // every input tile of chunk c into L2
         for (int pn = 0; pn < (dk >> 5); ++pn) tma_prefetch_l2_4d(&tmLA, 32 * pn, h, t0 + C * c, bb);
         for (int pn = 0; pn < (dk >> 6); ++pn) {
@@ -253,12 +257,6 @@ __global__ void __launch_bounds__(NT, 1)
           tma_prefetch_l2_4d(&tmV, 64 * pn, h, t0 + C * c, bb);
           tma_prefetch_l2_4d(&tmW, 64 * pn, h, t0 + C * c, bb);
         }
-      };
-      auto issue_la = [&](int c) {  // log alpha of chunk c: dk/32 boxes of 32 channels x 64 tokens
-        mbar_arrive_expect_tx(&ms.bar_la, (uint32_t)(C * dk * 4));
-        for (int pn = 0; pn < (dk >> 5); ++pn)
-          tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, t0 + C * c, bb);
-        ++n_la;
       };
       auto issue_qkb = [&](int c) {  // raw q, k, b of chunk c into the KQ tile
         mbar_arrive_expect_tx(&ms.bar_raw, (uint32_t)(3 * (dk >> 6)) * R64);
@@ -277,16 +275,11 @@ __global__ void __launch_bounds__(NT, 1)
         }
         ++n_vw;
       };
-      auto store_o = [&](int cc) {  // the staged output tile of chunk cc (rows past T are clipped)
-        tma_store_4d(&tmO, sm + OFF_LA, 0, h, t0 + C * cc, bb);
-        bulk_commit();
-      };
       uint32_t ph_ops = 0, ph_stage = 0, ph_tdiag = 0, ph_solved = 0, ph_uround = 0, ph_s = 0;
       bool alive = true;
       if (nch > 0) {
         issue_qkb(0);
         issue_vw(0);
-        issue_la(0);
         for (int cc = 1; cc <= PF_AHEAD && cc < nch; ++cc) prefetch_raw(cc);
       }
       for (int c = 0; c < nch; ++c) {
@@ -306,22 +299,16 @@ __global__ void __launch_bounds__(NT, 1)
         // X^T = -S^T Kb^T becomes R^T = Vw^T + X^T when warps 8-15 round it
         if (!(alive = wait_on(&ms.bar_stage, ph_stage))) break;
         tc_fence_after();
-        if (c > 0) store_o(c - 1);
         // [A; P] has read the Kn tile: the next chunk's v, w.  (Its completion is this
         // barrier's phase 3c; no later phase can complete before this thread issues again.)
         if (!(alive = mbar_wait_bounded(&ms.bar_mma, (uint32_t)((3 * c) & 1), &ms.abort, p.err, WAIT_LIMIT))) break;
         if (c + 1 < nch) issue_vw(c + 1);
-#pragma unroll 1
+#pragma unroll
         for (int ks = 0; ks < 16; ++ks) {
           const uint64_t bKQ = sdesc_sw128(sbase + OFF_KQ + (ks >> 2) * R128 + (ks & 3) * 32, 16, 1024);
           umma_tf32_ts(tmem + TM_R, tmem + TM_S + 8 * ks, bKQ, ID_128, ks > 0);
         }
         umma_commit(&ms.bar_s);
-        // the next chunk's log alpha once the output staging has been read
-        if (c + 1 < nch) {
-          bulk_wait_read_all();
-          issue_la(c + 1);
-        }
         // the state product has read the KQ tile: the next chunk's q, k, b
         if (!(alive = wait_on(&ms.bar_s, ph_s))) break;
         if (c + 1 < nch) issue_qkb(c + 1);
@@ -352,7 +339,6 @@ __global__ void __launch_bounds__(NT, 1)
         // [O^T | S^T] += U~^T [P; Kn^T]^T : O^T += U~^T P^T and S^T += U~^T Kn in one N = 192 product
         if (!(alive = wait_on(&ms.bar_uround, ph_uround))) break;
         tc_fence_after();
-        if (c + 1 == nch) bulk_wait_read_all();  // the last staging may be rewritten after this
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bPK = sdesc_sw128(sbase + OFF_PK + (ks >> 2) * R192 + (ks & 3) * 32, 16, 1024);
@@ -360,19 +346,54 @@ __global__ void __launch_bounds__(NT, 1)
         }
         umma_commit(&ms.bar_mma);
       }
-      // the last chunk's output, staged by the compute warps (a packed sequence's partial last
-      // chunk is written by the compute warps themselves: its box would spill into the next
-      // sequence's rows)
-      if (alive && nch > 0 && wait_on(&ms.bar_stage, ph_stage) && !(VARLEN && len % C)) store_o(nch - 1);
       // after a give-up: every MMA issued so far (a fresh commit tracks all of them) and
       // the last copies must land before the block releases its memory
       if (ms.abort) {
         volatile int never = 0;
         umma_commit(&ms.bar_drain);
         mbar_wait_bounded(&ms.bar_drain, 0, &never, nullptr, WAIT_LIMIT);
-        if (n_la > 0) mbar_wait_bounded(&ms.bar_la, (uint32_t)((n_la - 1) & 1), &never, nullptr, WAIT_LIMIT);
         if (n_raw > 0) mbar_wait_bounded(&ms.bar_raw, (uint32_t)((n_raw - 1) & 1), &never, nullptr, WAIT_LIMIT);
         if (n_vw > 0) mbar_wait_bounded(&ms.bar_vw, (uint32_t)((n_vw - 1) & 1), &never, nullptr, WAIT_LIMIT);
+      }
+    }
+    __syncwarp();  // the warp reconverges before the block-wide barrier
+  } else if (warp == NCOMP / 32 + 1) {
+    // ========================= store warp: output stores and log-alpha copies ===============
+    // The output of chunk c - 1 is staged over the decay tile once the operand build of
+    // chunk c has read it; as soon as the store has read the staging, the log alpha of chunk
+    // c + 1 is copied over it.  Kept off the control thread, whose MMA issue would otherwise
+    // delay that copy, and with it the cumulative decay of the next chunk.
+    if (tid == STW) {
+      int n_la = 0;
+      auto issue_la = [&](int c) {  // log alpha of chunk c: dk/32 boxes of 32 channels x 64 tokens
+        mbar_arrive_expect_tx(&ms.bar_la, (uint32_t)(C * dk * 4));
+        for (int pn = 0; pn < (dk >> 5); ++pn)
+          tma_load_4d(sm + OFF_LA + pn * R64, &tmLA, &ms.bar_la, 32 * pn, h, t0 + C * c, bb);
+        ++n_la;
+      };
+      auto store_o = [&](int cc) {  // the staged output tile of chunk cc (rows past T are clipped)
+        tma_store_4d(&tmO, sm + OFF_LA, 0, h, t0 + C * cc, bb);
+        bulk_commit();
+      };
+      uint32_t ph_stage = 0;
+      bool alive = true;
+      if (nch > 0) issue_la(0);
+      for (int c = 0; c < nch; ++c) {
+        if (!(alive = wait_on(&ms.bar_stage, ph_stage))) break;
+        if (c > 0) {
+          store_o(c - 1);
+          bulk_wait_read_all();
+        }
+        if (c + 1 < nch) issue_la(c + 1);
+        else mbar_arrive(&ms.bar_lastread);  // the last staging may overwrite the tile
+      }
+      // the last chunk's output, staged by the compute warps (a packed sequence's partial last
+      // chunk is written by the compute warps themselves: its box would spill into the next
+      // sequence's rows)
+      if (alive && nch > 0 && wait_on(&ms.bar_stage, ph_stage) && !(VARLEN && len % C)) store_o(nch - 1);
+      if (ms.abort && n_la > 0) {  // the last copy lands before the block releases its memory
+        volatile int never = 0;
+        mbar_wait_bounded(&ms.bar_la, (uint32_t)((n_la - 1) & 1), &never, nullptr, WAIT_LIMIT);
       }
       bulk_wait_all();  // output stores complete before the block exits
     }
@@ -781,7 +802,8 @@ __global__ void __launch_bounds__(NT, 1)
 
     // ---- last chunk's output and decay, then the final state -----------------------------
     if (!dead && nch > 0) {
-      const bool ok = ok_prev && wait_mma();
+      uint32_t ph_lr = 0;
+      const bool ok = ok_prev && wait_mma() && wait_on(&ms.bar_lastread, ph_lr);
       if (named_bar_or(BAR_COMP, NCOMP, !ok)) dead = true;
     }
     if (!dead && nch > 0) {
