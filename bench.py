@@ -227,19 +227,44 @@ def time_packed(args, dev):
         g.gdn2_chunk_fwd_varlen(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["cu_seqlens"], x["S0"],
                                 o=o, S_T=S_T)
 
-    for _ in range(args.warmup):
+    ms = _time_loop(step, args.steps, args.warmup)
+    return dict(ms=ms, tokens=T, token_heads=T * H, units=PACKED.B * H, n_seq=PACKED.B,
+                ok=g.gdn2_device_status() == 0)
+
+
+def _time_loop(step, steps, warmup):
+    """Mean device time of one call of ``step`` (ms): CUDA events on the current stream
+    around ``steps`` back-to-back calls, after ``warmup`` untimed ones."""
+    import torch
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(st)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     t1.record(st)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / args.steps
-    return dict(ms=ms, tokens=T, token_heads=T * H, units=PACKED.B * H, n_seq=PACKED.B,
-                ok=g.gdn2_device_status() == 0)
+    return t0.elapsed_time(t1) / steps
+
+
+def time_raw(args, dev):
+    """The prefill workload fed with raw projections (activations inside the kernel)."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    d = gi.raw_inputs(PREFILL)
+    x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    B, T, H = PREFILL.B, PREFILL.T, PREFILL.H
+    o = torch.empty((B, T, H, PREFILL.dv), dtype=torch.float32, device=dev)
+    S_T = torch.empty((B, H, PREFILL.dk, PREFILL.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        g.gdn2_chunk_fwd_raw(x["q_raw"], x["k_raw"], x["v"], x["a_raw"], x["b_raw"], x["w_raw"], None,
+                             decay_scale=x["decay_scale"], o=o, S_T=S_T)
+
+    ms = _time_loop(step, args.steps, args.warmup)
+    return dict(ms=ms, tokens=B * T, token_heads=B * T * H, ok=g.gdn2_device_status() == 0)
 
 
 def time_prefill_e2e(args, dev):
@@ -395,6 +420,8 @@ def main():
 
     dec = time_decode(dev, args.decode_steps, world)
     pak = time_packed(args, dev)
+    raw = time_raw(args, dev)
+    raw_gbs = raw["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (raw["ms"] * 1e-3) / 1e9
     # algorithmic bytes: the token streams plus each sequence's entering and final state
     pak_bytes = pak["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD + pak["units"] * DECODE_STATE_BYTES
     pak_gbs = pak_bytes / (pak["ms"] * 1e-3) / 1e9
@@ -435,9 +462,16 @@ def main():
                    "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (packed)", "achieved": pak_gbs,
                                 "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": pak_gbs / pk["hbm_gbs"],
                                 "traffic": None}},
+        "raw": {"metric": "GDN-2 prefill tokens/s per layer, raw projections", "value": raw["tokens"] / (raw["ms"] * 1e-3),
+                "unit": "tokens/s", "ms_per_step": raw["ms"], "steps": args.steps,
+                "workload": "prefill_b8_h16_t4096 fed with the raw projections: q, k L2-normalised, sigmoid "
+                            "gates and log alpha = -softplus(a)/16 applied inside the kernel",
+                "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (raw)", "achieved": raw_gbs,
+                             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": raw_gbs / pk["hbm_gbs"],
+                             "traffic": None}},
         "gpu_launches": args.steps,
         "clocks": pre["clocks"],
-        "device_status_ok": bool(pre["ok"] and dec["ok"] and pak["ok"]),
+        "device_status_ok": bool(pre["ok"] and dec["ok"] and pak["ok"] and raw["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)

@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -57,6 +57,8 @@ def lib():
         L.gdn2_chunk_fwd.restype = I
         L.gdn2_chunk_fwd_varlen.argtypes = [P] * 10 + [I] * 6 + [P]
         L.gdn2_chunk_fwd_varlen.restype = I
+        L.gdn2_chunk_fwd_raw.argtypes = [P] * 11 + [I] * 6 + [P]
+        L.gdn2_chunk_fwd_raw.restype = I
         L.gdn2_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
         L.gdn2_decode_step.restype = I
         L.gdn2_device_status.argtypes = []
@@ -87,7 +89,7 @@ def _check_tokens(name, tensors, dtype, device):
             raise ValueError(f"{name}: {n} must be a CUDA tensor on {device}")
         if not t.is_contiguous():
             raise ValueError(f"{name}: {n} must be contiguous")
-        want = torch.float32 if n in ("log_alpha", "S0", "S", "S_T", "o") else dtype
+        want = torch.float32 if n in ("log_alpha", "a_raw", "S0", "S", "S_T", "o", "decay_scale") else dtype
         if t.dtype != want:
             raise ValueError(f"{name}: {n} must be {want}, got {t.dtype}")
 
@@ -145,6 +147,48 @@ def gdn2_chunk_fwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, o=No
                                      _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd_varlen", rc)
+    return o, S_T
+
+
+def gdn2_chunk_fwd_raw(q_raw, k_raw, v, a_raw, b_raw, w_raw, S0=None, *, decay_scale=None, cu_seqlens=None,
+                       o=None, S_T=None, want_state=True, stream=None):
+    """Chunkwise prefill forward on the raw projections (q, k normalised, sigmoid gates and
+    log alpha = -decay_scale[h] * softplus(a_raw) inside the kernel).
+
+    Without cu_seqlens: q_raw, k_raw, b_raw [B, T, H, d_k], v, w_raw [B, T, H, d_v], a_raw fp32
+    [B, T, H, d_k]; returns (o [B, T, H, d_v], S_T [B, H, d_k, d_v] or None).  With cu_seqlens
+    (int32 [N + 1] on the device) the tensors are packed, [T, H, D], and S0 / S_T are
+    [N, H, d_k, d_v].  decay_scale: fp32 [H] on the device, or None for 1."""
+    if q_raw.dtype != torch.bfloat16:
+        raise ValueError("gdn2_chunk_fwd_raw: bf16 inputs only")
+    if cu_seqlens is None:
+        B, T, H, dk = q_raw.shape
+        o_shape = (B, T, H, v.shape[-1])
+    else:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+            raise ValueError("gdn2_chunk_fwd_raw: cu_seqlens must be a contiguous int32 vector")
+        if cu_seqlens.device != q_raw.device:
+            raise ValueError("gdn2_chunk_fwd_raw: cu_seqlens must be on the inputs' device")
+        T, H, dk = q_raw.shape
+        B = cu_seqlens.numel() - 1
+        o_shape = (T, H, v.shape[-1])
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(o_shape, dtype=torch.float32, device=q_raw.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q_raw.device)
+    ts = dict(q_raw=q_raw, k_raw=k_raw, v=v, a_raw=a_raw, b_raw=b_raw, w_raw=w_raw, o=o)
+    for n, t in (("S0", S0), ("S_T", S_T), ("decay_scale", decay_scale)):
+        if t is not None:
+            ts[n] = t
+    if decay_scale is not None and decay_scale.numel() != H:
+        raise ValueError("gdn2_chunk_fwd_raw: decay_scale must hold one value per head")
+    _check_tokens("gdn2_chunk_fwd_raw", ts, q_raw.dtype, q_raw.device)
+    rc = lib().gdn2_chunk_fwd_raw(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(w_raw),
+                                  _ptr(decay_scale), _ptr(cu_seqlens), _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk,
+                                  dv, _DT[q_raw.dtype], _stream(q_raw.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_chunk_fwd_raw", rc)
     return o, S_T
 
 

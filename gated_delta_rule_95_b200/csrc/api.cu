@@ -99,6 +99,30 @@ extern "C" gdn2_status gdn2_chunk_fwd_varlen(const void* q, const void* k, const
   return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
 }
 
+extern "C" gdn2_status gdn2_chunk_fwd_raw(const void* q_raw, const void* k_raw, const void* v, const float* a_raw,
+                                          const void* b_raw, const void* w_raw, const float* decay_scale,
+                                          const int* cu_seqlens, const float* S0, float* o, float* S_T, int B, int T,
+                                          int H, int d_k, int d_v, gdn2_dtype dt, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (dt != GDN2_BF16) return GDN2_ERR_DTYPE;  // raw projections: bf16 inputs only
+  const bool packed = cu_seqlens != nullptr;
+  if (!sizes_ok(packed ? 1 : B, T, H, d_k, d_v) || B < 0 || (long long)B * H > 0x7fffffffLL) return GDN2_ERR_SHAPE;
+  if ((long long)B * H == 0) return GDN2_OK;
+  if (T > 0 && (!q_raw || !k_raw || !v || !a_raw || !b_raw || !w_raw || !o)) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q_raw, k_raw, v, a_raw, b_raw, w_raw, S0, o, S_T};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return GDN2_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(decay_scale) & 3u) != 0) return GDN2_ERR_ALIGN;
+
+  ChunkArgs a{q_raw, k_raw, v, b_raw, w_raw, a_raw, S0, o, S_T, B, T, H, d_k, d_v, true, cu_seqlens};
+  a.raw = true;
+  a.decay_scale = decay_scale;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (T == 0) ? launch_state_copy(a, st) : launch_chunk_fwd_tc(a, st);
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
 extern "C" gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
                                         const void* b, const void* w, float* S, float* o, int B, int H, int d_k,
                                         int d_v, gdn2_dtype dt, void* stream) {

@@ -96,6 +96,7 @@ struct Misc {
   int abort;
   alignas(16) float gC[2][128];    // Gamma at the chunk end, per key channel (chunk parity)
   alignas(16) float segtot[2][128];  // per half chunk: sum of log2 alpha, per key channel
+  alignas(16) float rn[128];       // raw projections: 1 / |q_t| (t < 64) and 1 / |k_t| (64 + t)
 };
 constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 
@@ -122,8 +123,17 @@ struct TcParams {
   int T, H, dk, dv;
   const int* cu_seqlens;  // packed sequences: [N + 1] token offsets (device); NULL = fixed length T
   int nseq;               // packed sequences: N
+  const float* dscale;    // raw projections: per-head decay scale s_h (NULL = 1)
   unsigned* err;
 };
+
+// Gate activations of the raw-projection variant, from their definitions, on the
+// special-function unit.  sigmoid(x) = 1 / (1 + 2^(-x log2 e)); softplus in base-2 units,
+// softplus(a) log2 e = max(a, 0) log2 e + log2(1 + 2^(-|a| log2 e)), which never overflows.
+__device__ __forceinline__ float sigmoid_fast(float x) { return rcp_approx(1.f + ex2_approx(-LOG2E * x)); }
+__device__ __forceinline__ float softplus_log2(float a) {
+  return fmaxf(a, 0.f) * LOG2E + lg2_approx(1.f + ex2_approx(-LOG2E * fabsf(a)));
+}
 
 // fp32 -> tf32, round to nearest with ties away from zero on the magnitude (add half an
 // ulp of the 10-bit mantissa, clear the 13 dropped bits); two integer instructions.
@@ -150,8 +160,11 @@ __device__ __forceinline__ void st2_tf32(unsigned char* p, const float2& f) {
 // DK, DV: key and value head dimensions (64 or 128), fixed at compile time so that each
 // launch runs straight-line code for its own shape.  VARLEN: the batch is a packed set of
 // sequences (a CTA per (sequence, head), token range from cu_seqlens); otherwise B
-// sequences of T tokens.
-template <int DK, int DV, bool VARLEN>
+// sequences of T tokens.  PREP: the inputs are the raw projections, and the kernel applies
+// the layer's input activations itself: q and k L2-normalised per token, b = sigmoid(b),
+// w = sigmoid(w), log alpha = -s_h softplus(a) (Gated DeltaNet-2 guide, "Decoupled Erase and
+// Write Gates" and "Normalization and Short Convolutions").
+template <int DK, int DV, bool VARLEN, bool PREP>
 __global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
@@ -453,6 +466,7 @@ __global__ void __launch_bounds__(NT, 1)
     // Warps 8-15, one chunk ahead (chunk cc).  Thread (ch, hf) owns the 32 tokens
     // [32 hf, 32 hf + 32) of channel ch.
     uint32_t ph_la = 0, ph_raw = 0, ph_vw = 0;
+    const float dsc = PREP ? (p.dscale ? p.dscale[h] : 1.f) : 0.f;  // decay scale s_h
     // Vw^T = (W * V)^T into the tensor-memory buffer of chunk cc's parity (v and w are copied
     // as soon as [A; P] has read the Kn tile).
     auto vw_ahead = [&](int cc, bool ok) -> bool {
@@ -465,7 +479,9 @@ __global__ void __launch_bounds__(NT, 1)
       for (int r = 0; r < 32; ++r) {
         const uint32_t ro = pnl + sw128_off(32 * hf + r, chk) + byt;
         const bool tv = !VARLEN || C * cc + 32 * hf + r < len;
-        vw[r] = (vval && tv) ? bf16_at(sm + RAW_V + ro) * bf16_at(sm + RAW_W + ro) : 0.f;
+        float wr = bf16_at(sm + RAW_W + ro);
+        if constexpr (PREP) wr = sigmoid_fast(wr);
+        vw[r] = (vval && tv) ? bf16_at(sm + RAW_V + ro) * wr : 0.f;
       }
       tmem_st32(tlane + TM_VW + 64 * (cc & 1) + 32 * hf, vw);
       tmem_st_wait();
@@ -485,7 +501,14 @@ __global__ void __launch_bounds__(NT, 1)
       float acc = 0.f;
 #pragma unroll
       for (int r = 0; r < 32; ++r) {
-        acc = fmaf(x[r], LOG2E, acc);
+        if constexpr (PREP) {
+          // log2 alpha = -s_h softplus(a) log2 e.  Rows past the sequence add nothing (a
+          // fixed-length batch's tail rows read a = 0, whose softplus is not 0).
+          const bool vr = kval && C * cc + 32 * hf + r < len;
+          acc -= vr ? dsc * softplus_log2(x[r]) : 0.f;
+        } else {
+          acc = fmaf(x[r], LOG2E, acc);
+        }
         x[r] = acc;
       }
       ms.segtot[hf][ch] = acc;
@@ -499,10 +522,40 @@ __global__ void __launch_bounds__(NT, 1)
       if (hf == 1) ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
       return ok;
     };
+    // Raw projections: 1 / |q_t| and 1 / |k_t| of chunk cc (zero vectors stay zero), from the
+    // raw q, k tiles once they have landed.  Thread a = t - 256 sums the squares of one
+    // 128-byte row: row a / 2 of the stacked [q; k] rows, channel panel a mod 2.
+    uint32_t ph_rawa = 0;
+    auto norms_ahead = [&](bool ok) -> bool {
+      ok = ok && wait_on(&ms.bar_raw, ph_rawa);
+      const int a = tid - NSOLVE, row = a >> 1, pn = a & 1;
+      const int t = row & 63;
+      const unsigned char* base = sm + (row < 64 ? RAW_Q : RAW_K) + pn * R64;
+      float ss = 0.f;
+      if (pn * 64 < dk) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          // (the swizzle spreads rows t .. t + 7 over the eight 16-byte bank groups)
+          const uint4 u = *reinterpret_cast<const uint4*>(base + sw128_off(t, j));
+          const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float lo = __uint_as_float(wd[m] << 16), hi = __uint_as_float(wd[m] & 0xFFFF0000u);
+            ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+          }
+        }
+      }
+      ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 1);
+      if (pn == 0) ms.rn[row] = rsqrtf(fmaxf(ss, 1e-24f));
+      return ok;
+    };
 
     bool dead = false;
     bool ok_prev = true;  // failed waits of the previous chunk's tail, voted at the next barrier
-    if (nch > 0 && warp >= NSOLVE / 32) ok_prev = decay_ahead(0, vw_ahead(0, true));
+    if (nch > 0 && warp >= NSOLVE / 32) {
+      ok_prev = decay_ahead(0, vw_ahead(0, true));
+      if constexpr (PREP) ok_prev = norms_ahead(ok_prev);
+    }
     tc_fence_before();
     if (named_bar_or(BAR_COMP, NCOMP, !ok_prev)) dead = true;
     tc_fence_after();
@@ -515,7 +568,8 @@ __global__ void __launch_bounds__(NT, 1)
       const int cp = tid & 63, ts = tid >> 6, c2 = 2 * cp;
       const bool kv2 = c2 < dk;
       float2 nkb[8], qh[8], kn[8];
-      bool ok_raw = wait_on(&ms.bar_raw, ph_raw);
+      // (raw projections: warps 8-15 have seen these copies land already, for the norms)
+      bool ok_raw = (PREP && warp >= NSOLVE / 32) ? true : wait_on(&ms.bar_raw, ph_raw);
       {
         const unsigned char* la_t = sm + OFF_LA;
         const uint32_t pnl = (uint32_t)(c2 >> 6) * R64;  // raw tiles: panels of 64 channels
@@ -531,6 +585,12 @@ __global__ void __launch_bounds__(NT, 1)
             kk = bf16x2_at(sm + RAW_K + ro);
             bg = bf16x2_at(sm + RAW_B + ro);
             qq = bf16x2_at(sm + RAW_Q + ro);
+            if constexpr (PREP) {
+              const float rq = ms.rn[t], rk = ms.rn[64 + t];
+              kk = make_float2(kk.x * rk, kk.y * rk);
+              qq = make_float2(qq.x * rq, qq.y * rq);
+              bg = make_float2(sigmoid_fast(bg.x), sigmoid_fast(bg.y));
+            }
           }
           const float2 Gi = make_float2(rcp_approx(G.x), rcp_approx(G.y));
           nkb[r] = make_float2(-(kk.x * bg.x) * G.x, -(kk.y * bg.y) * G.y);
@@ -786,7 +846,10 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         warp_arrive(&ms.bar_tdiag);
         // ===== then one chunk ahead: Vw^T and the cumulative decay of the next chunk =========
-        if (c + 1 < nch) ok_s = decay_ahead(c + 1, vw_ahead(c + 1, ok_s));
+        if (c + 1 < nch) {
+          ok_s = decay_ahead(c + 1, vw_ahead(c + 1, ok_s));
+          if constexpr (PREP) ok_s = norms_ahead(ok_s);
+        }
         // These warps do not use U~; they step their phase bit past its product without
         // waiting (by now the chunk's last product may have completed as well, and a parity
         // wait must never trail its barrier by two phases).  Their next wait, on that last
@@ -875,31 +938,31 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
   return r == CUDA_SUCCESS;
 }
 
-template <int DK, int DV, bool VARLEN>
+template <int DK, int DV, bool VARLEN, bool PREP>
 cudaError_t launch_shape(int grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
                          const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw, const CUtensorMap& mla,
                          const CUtensorMap& mo, const TcParams& p) {
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV, VARLEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  chunk_fwd_tc_kernel<DK, DV, VARLEN><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
+  chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
   return cudaSuccess;
 }
 
 }  // namespace
 
-template <bool VARLEN>
+template <bool VARLEN, bool PREP>
 cudaError_t launch_dims(int grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
                         const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw, const CUtensorMap& mla,
                         const CUtensorMap& mo, const TcParams& p) {
-  if (p.dk == 128 && p.dv == 128) return launch_shape<128, 128, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
-  if (p.dk == 128 && p.dv == 64) return launch_shape<128, 64, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
-  if (p.dk == 64 && p.dv == 128) return launch_shape<64, 128, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
-  if (p.dk == 64 && p.dv == 64) return launch_shape<64, 64, VARLEN>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (p.dk == 128 && p.dv == 128) return launch_shape<128, 128, VARLEN, PREP>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (p.dk == 128 && p.dv == 64) return launch_shape<128, 64, VARLEN, PREP>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (p.dk == 64 && p.dv == 128) return launch_shape<64, 128, VARLEN, PREP>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (p.dk == 64 && p.dv == 64) return launch_shape<64, 64, VARLEN, PREP>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
   return cudaErrorInvalidValue;
 }
 
@@ -937,8 +1000,14 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   p.nseq = varlen ? a.B : 0;
   p.err = device_error_word();
   const int grid = a.B * a.H;
-  cudaError_t e = varlen ? launch_dims<true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
-                         : launch_dims<false>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  p.dscale = a.decay_scale;
+  cudaError_t e;
+  if (a.raw)
+    e = varlen ? launch_dims<true, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
+               : launch_dims<false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  else
+    e = varlen ? launch_dims<true, false>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
+               : launch_dims<false, false>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

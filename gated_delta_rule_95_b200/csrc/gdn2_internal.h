@@ -22,6 +22,10 @@ struct ChunkArgs {
   int B, T, H, dk, dv;  // packed sequences: B = number of sequences, T = total tokens
   bool bf16;
   const int* cu_seqlens;  // packed sequences: [B + 1] device token offsets; NULL otherwise
+  // raw projections: q, k un-normalised, b, w gate logits, log_alpha holds the decay
+  // pre-activation a (log alpha = -s_h softplus(a)); decay_scale: s_h per head (NULL = 1)
+  bool raw = false;
+  const float* decay_scale = nullptr;
 };
 
 // Device error word of this library: bits set by kernels, read and cleared by

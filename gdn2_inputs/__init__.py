@@ -168,6 +168,36 @@ def prefill_inputs(wl: Workload, B=None, T=None, H=None, seed=None):
     return out
 
 
+def raw_inputs(wl: Workload, B=None, T=None, H=None, seed=None):
+    """The raw projections behind a prefill workload: the same draws as
+    ``prefill_inputs`` before any activation, for the raw-projection entry point.
+
+    Returns dict(q_raw, k_raw, v, b_raw, w_raw: dtype [B,T,H,D]; a_raw: float32
+    [B,T,H,dk]; decay_scale: float32 [H]; S0).  The decay pre-activation and scale
+    reproduce the workload's gate: log alpha = -decay_scale * softplus(a_raw), with
+    a_raw = x and scale 1/16 ("base"), or a_raw = 2x and scale 1/8 ("heavy")."""
+    import torch
+    B = wl.B if B is None else B
+    T = wl.T if T is None else T
+    H = wl.H if H is None else H
+    key = [wl.seed if seed is None else seed]
+    sk, sv = (B, T, H, wl.dk), (B, T, H, wl.dv)
+    heavy = wl.decay == "heavy"
+    q = _draw(key, _TID["q"], sk)
+    k = _draw(key, _TID["k"], sk)
+    v = _draw(key, _TID["v"], sv)
+    a = _draw(key, _TID["alpha"], sk, (lambda x: 2.0 * x) if heavy else None)
+    b = _draw(key, _TID["b"], sk)
+    w = _draw(key, _TID["w"], sv)
+    S0 = None
+    if wl.state_std > 0:
+        S0 = torch.from_numpy(_draw(key, _TID["S"], (B, H, wl.dk, wl.dv), lambda x: wl.state_std * x))
+    scale = np.full(H, 1.0 / 8.0 if heavy else 1.0 / 16.0, dtype=np.float32)
+    return dict(q_raw=_round(q, wl.dtype), k_raw=_round(k, wl.dtype), v=_round(v, wl.dtype),
+                b_raw=_round(b, wl.dtype), w_raw=_round(w, wl.dtype), a_raw=torch.from_numpy(a),
+                decay_scale=torch.from_numpy(scale), S0=S0)
+
+
 def packed_lengths(n: int, lo: int, hi: int, seed: int):
     """A seeded serving-like length mix: n lengths log-uniform in [lo, hi] (integers)."""
     rng = np.random.default_rng([seed, 2000])

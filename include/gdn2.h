@@ -111,6 +111,32 @@ GDN2_API gdn2_status gdn2_chunk_fwd_varlen(const void* q, const void* k, const v
                                   void* stream);
 
 /*
+ * Chunkwise prefill forward fed with the raw projections, the layer's input
+ * activations applied inside the kernel as it loads each chunk (so they cost no
+ * extra pass over memory): q and k are L2-normalised per (token, head) (a zero
+ * vector stays zero), b = sigmoid(b_raw), w = sigmoid(w_raw) (Gated DeltaNet-2 guide,
+ * "Normalization and Short Convolutions" and "Decoupled Erase and Write Gates"), and
+ * log alpha = -s_h * softplus(a_raw) with a per-head scale s_h (a channel-wise decay
+ * in (0, 1): snilld.dk, "Hvad Gated DeltaNet-2 aendrer").  The result is gdn2_chunk_fwd (or
+ * gdn2_chunk_fwd_varlen) on the activated inputs, up to rounding: the activations are
+ * computed in fp32 and never rounded back to bf16.
+ *
+ *   q_raw, k_raw, b_raw : [B, T, H, d_k]  bf16 (packed: [T, H, d_k])
+ *   v, w_raw            : [B, T, H, d_v]  bf16 (packed: [T, H, d_v])
+ *   a_raw               : [B, T, H, d_k]  fp32, finite (packed: [T, H, d_k])
+ *   decay_scale         : [H] fp32 DEVICE array of s_h > 0, 4-byte aligned; NULL means 1
+ *   cu_seqlens          : NULL: B sequences of T tokens each.  Otherwise a packed batch
+ *                         of B sequences over T tokens in total, exactly as
+ *                         gdn2_chunk_fwd_varlen takes it (N = B).
+ *   S0, o, S_T          : as gdn2_chunk_fwd (packed: as gdn2_chunk_fwd_varlen)
+ *   dt                  : GDN2_BF16 (fp32 inputs return GDN2_ERR_DTYPE)
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_raw(const void* q_raw, const void* k_raw, const void* v, const float* a_raw,
+                               const void* b_raw, const void* w_raw, const float* decay_scale,
+                               const int* cu_seqlens, const float* S0, float* o, float* S_T, int B, int T,
+                               int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
+
+/*
  * One recurrent decode step: the update above for a single token per
  * (sequence, head), with the state updated in place (Gated DeltaNet-2 guide,
  * "4.5x Higher Decoding Throughput with Zero KV Cache": a fixed-size state

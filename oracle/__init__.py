@@ -9,6 +9,9 @@ this package, and this package imports nothing from the CUDA path.
   update; readout after the update as in the guide's PyTorch loop).
 * ``chunkwise.forward`` re-derives the chunkwise WY form in numpy; it is a
   second, independent route to the same numbers, used to pin chunk invariance.
+* ``activations`` maps the raw projections to the mixer's inputs (L2-normalised
+  q and k, sigmoid gates, log alpha = -s_h softplus(a)); composed with
+  ``forward`` it is what the raw-projection entry point computes.
 
 Every function takes float64 numpy arrays in the layouts of the C ABI:
 tokens [B, T, H, D], states [B, H, d_k, d_v].
@@ -111,6 +114,39 @@ def forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, nthreads=None,
         o[a:e] = o_n[0]
         S_T[n] = s_n[0]
     return o, S_T
+
+
+def _sigmoid(x):
+    # 1 / (1 + e^-x), evaluated on the side where the exponential cannot overflow
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def activations(q_raw, k_raw, a_raw, b_raw, w_raw, decay_scale=None):
+    """The layer's input activations, in float64, for tokens [..., H, D] (H the
+    second-to-last axis).
+
+    * q and k are divided by their Euclidean norm per (token, head) (Gated DeltaNet-2
+      guide, "Normalization and Short Convolutions"); a zero vector stays zero (the
+      norm is floored at 1e-12).
+    * b = sigmoid(b_raw), w = sigmoid(w_raw): the erase and write gates take values in
+      (0, 1) and come from sigmoid projections (same guide, "Decoupled Erase and Write
+      Gates"; snilld.dk, "Hvad Gated DeltaNet-2 aendrer").
+    * log alpha = -s_h softplus(a_raw) = -s_h log(1 + e^a), a channel-wise decay in
+      (0, 1) with a positive per-head scale s_h (decay_scale [H], default 1).
+
+    Returns dict(q, k, log_alpha, b, w)."""
+    q_raw, k_raw, a_raw, b_raw, w_raw = map(_f64, (q_raw, k_raw, a_raw, b_raw, w_raw))
+
+    def l2n(x):
+        n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+        return x / np.maximum(n, 1e-12)
+
+    H = q_raw.shape[-2]
+    s = np.ones(H) if decay_scale is None else np.asarray(decay_scale, dtype=np.float64).reshape(H)
+    softplus = np.logaddexp(0.0, a_raw)
+    return dict(q=l2n(q_raw), k=l2n(k_raw), log_alpha=-s[:, None] * softplus, b=_sigmoid(b_raw),
+                w=_sigmoid(w_raw))
 
 
 def decode_step(q, k, v, log_alpha, b, w, S, nthreads=None, lib=None):

@@ -82,6 +82,21 @@ def test_chunk_fwd_varlen_validation(kw, status):
     assert varlen(**kw) == status
 
 
+def raw(q=A, k=A, v=A, a=A, b=A, w=A, sc=None, cu=None, S0=None, o=A, ST=None, B=2, T=100, H=1, dk=128, dv=128,
+        dt=1):
+    return g.lib().gdn2_chunk_fwd_raw(q, k, v, a, b, w, sc, cu, S0, o, ST, B, T, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=96), 2), (dict(B=-1), 2), (dict(T=-1), 2), (dict(dt=0), 3), (dict(dt=7), 3),
+    (dict(q=None), 1), (dict(a=None), 1), (dict(w=None), 1), (dict(o=None), 1),
+    (dict(sc=P(0x10002)), 4), (dict(cu=P(0x10001)), 4), (dict(b=M), 4), (dict(S0=M), 4),
+    (dict(B=0), 0), (dict(H=0), 0), (dict(cu=A, B=0), 0),
+])
+def test_chunk_fwd_raw_validation(kw, status):
+    assert raw(**kw) == status
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)

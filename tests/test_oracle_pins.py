@@ -60,3 +60,46 @@ def test_packed_sequences_are_independent_runs():
     o2, S2 = oracle.forward_varlen(**packed, cu_seqlens=np.array([0, 40, 40, 80, 120]), S0=S0e)
     assert np.array_equal(S2[1], S0e[1]) and np.array_equal(o2, o)
     assert np.array_equal(S2[[0, 2, 3]], S)
+
+
+# ---- the input activations of the raw-projection entry point ------------------------------
+
+def _act(q=None, k=None, a=None, b=None, w=None, scale=None, H=1, D=4):
+    z = np.zeros((1, 1, H, D))
+    f = lambda x: z if x is None else np.asarray(x, dtype=np.float64).reshape(1, 1, H, D)
+    return oracle.activations(f(q), f(k), f(a), f(b), f(w), scale)
+
+
+def test_activations_closed_forms():
+    # a 3-4-5 vector normalises to (0.6, 0.8); a zero vector stays zero
+    r = _act(q=[3.0, 4.0, 0.0, 0.0], k=[0.0, 0.0, 0.0, 0.0])
+    assert np.allclose(r["q"].ravel(), [0.6, 0.8, 0.0, 0.0], rtol=0, atol=1e-15)
+    assert np.array_equal(r["k"].ravel(), np.zeros(4))
+    # sigmoid(0) = 1/2, sigmoid(ln 3) = 3/4, sigmoid(-ln 3) = 1/4
+    r = _act(b=[0.0, np.log(3.0), -np.log(3.0), 0.0], w=[np.log(3.0), 0.0, 0.0, -np.log(3.0)])
+    assert np.allclose(r["b"].ravel(), [0.5, 0.75, 0.25, 0.5], rtol=0, atol=1e-15)
+    assert np.allclose(r["w"].ravel(), [0.75, 0.5, 0.5, 0.25], rtol=0, atol=1e-15)
+    # softplus(0) = ln 2, softplus(ln(e - 1)) = 1, softplus(50) = 50 (to 2e-22),
+    # softplus(-50) = e^-50 (to first order): log alpha = -s softplus(a), s = 0.25
+    r = _act(a=[0.0, np.log(np.e - 1.0), 50.0, -50.0], scale=[0.25])
+    want = -0.25 * np.array([np.log(2.0), 1.0, 50.0, np.exp(-50.0)])
+    assert np.allclose(r["log_alpha"].ravel(), want, rtol=1e-14, atol=0)
+
+
+def test_activations_identities():
+    rng = np.random.default_rng(7)
+    x = 6.0 * rng.standard_normal((2, 3, 4, 8))
+    H = x.shape[-2]
+    p = oracle.activations(x, x, x, x, x, np.full(H, 1.0))
+    m = oracle.activations(-x, -x, -x, -x, -x, np.full(H, 1.0))
+    # sigmoid(x) + sigmoid(-x) = 1; softplus(x) - softplus(-x) = x; unit norms, directions kept
+    assert np.allclose(p["b"] + m["b"], 1.0, rtol=0, atol=1e-15)
+    assert np.allclose(-p["log_alpha"] + m["log_alpha"], x, rtol=0, atol=1e-13)
+    assert np.allclose(np.linalg.norm(p["q"], axis=-1), 1.0, rtol=0, atol=1e-15)
+    assert np.allclose(p["q"] * np.linalg.norm(x, axis=-1, keepdims=True), x, rtol=0, atol=1e-13)
+    # the per-head scale multiplies log alpha of its own head only
+    s = np.array([1.0, 2.0, 0.5, 3.0])
+    q = oracle.activations(x, x, x, x, x, s)
+    assert np.allclose(q["log_alpha"], p["log_alpha"] * s[:, None], rtol=1e-15, atol=0)
+    # every decay lies in (0, 1) and every gate in (0, 1)
+    assert np.all(p["log_alpha"] < 0) and np.all((p["w"] > 0) & (p["w"] < 1))
