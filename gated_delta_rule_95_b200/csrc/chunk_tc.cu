@@ -522,40 +522,40 @@ __global__ void __launch_bounds__(NT, 1)
       if (hf == 1) ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
       return ok;
     };
-    // Raw projections: 1 / |q_t| and 1 / |k_t| of chunk cc (zero vectors stay zero), from the
-    // raw q, k tiles once they have landed.  Thread a = t - 256 sums the squares of one
-    // 128-byte row: row a / 2 of the stacked [q; k] rows, channel panel a mod 2.
-    uint32_t ph_rawa = 0;
+    // Raw projections, warps 0-7, one chunk ahead once its q, k, b copies have landed:
+    // 1 / |q_t| and 1 / |k_t| (a zero vector stays zero).  Thread a = t mod 256 sums the
+    // squares of one 128-byte row: row a / 2 of the stacked [q; k] rows, channel panel a mod 2.
     auto norms_ahead = [&](bool ok) -> bool {
-      ok = ok && wait_on(&ms.bar_raw, ph_rawa);
-      const int a = tid - NSOLVE, row = a >> 1, pn = a & 1;
-      const int t = row & 63;
-      const unsigned char* base = sm + (row < 64 ? RAW_Q : RAW_K) + pn * R64;
-      float ss = 0.f;
-      if (pn * 64 < dk) {
+      ok = ok && wait_on(&ms.bar_raw, ph_raw);
+      const int a = tid & 255;
+      {
+        const int row = a >> 1, pn = a & 1, t = row & 63;
+        const unsigned char* base = sm + (row < 64 ? RAW_Q : RAW_K) + pn * R64;
+        float ss = 0.f;
+        if (pn * 64 < dk) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          // (the swizzle spreads rows t .. t + 7 over the eight 16-byte bank groups)
-          const uint4 u = *reinterpret_cast<const uint4*>(base + sw128_off(t, j));
-          const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+          for (int j = 0; j < 8; ++j) {
+            // (the swizzle spreads rows t .. t + 7 over the eight 16-byte bank groups)
+            const uint4 u = *reinterpret_cast<const uint4*>(base + sw128_off(t, j));
+            const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const float lo = __uint_as_float(wd[m] << 16), hi = __uint_as_float(wd[m] & 0xFFFF0000u);
-            ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+            for (int m = 0; m < 4; ++m) {
+              const float lo = __uint_as_float(wd[m] << 16), hi = __uint_as_float(wd[m] & 0xFFFF0000u);
+              ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+            }
           }
         }
+        ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 1);
+        if (pn == 0) ms.rn[row] = rsqrtf(fmaxf(ss, 1e-24f));
       }
-      ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 1);
-      if (pn == 0) ms.rn[row] = rsqrtf(fmaxf(ss, 1e-24f));
       return ok;
     };
 
     bool dead = false;
     bool ok_prev = true;  // failed waits of the previous chunk's tail, voted at the next barrier
-    if (nch > 0 && warp >= NSOLVE / 32) {
-      ok_prev = decay_ahead(0, vw_ahead(0, true));
-      if constexpr (PREP) ok_prev = norms_ahead(ok_prev);
-    }
+    if (nch > 0 && warp >= NSOLVE / 32) ok_prev = decay_ahead(0, vw_ahead(0, true));
+    if constexpr (PREP)
+      if (nch > 0 && warp < NSOLVE / 32) ok_prev = norms_ahead(true);
     tc_fence_before();
     if (named_bar_or(BAR_COMP, NCOMP, !ok_prev)) dead = true;
     tc_fence_after();
@@ -568,8 +568,8 @@ __global__ void __launch_bounds__(NT, 1)
       const int cp = tid & 63, ts = tid >> 6, c2 = 2 * cp;
       const bool kv2 = c2 < dk;
       float2 nkb[8], qh[8], kn[8];
-      // (raw projections: warps 8-15 have seen these copies land already, for the norms)
-      bool ok_raw = (PREP && warp >= NSOLVE / 32) ? true : wait_on(&ms.bar_raw, ph_raw);
+      // (raw projections: warps 0-7 have seen these copies land already, one chunk ahead)
+      bool ok_raw = (PREP && warp < NSOLVE / 32) ? true : wait_on(&ms.bar_raw, ph_raw);
       {
         const unsigned char* la_t = sm + OFF_LA;
         const uint32_t pnl = (uint32_t)(c2 >> 6) * R64;  // raw tiles: panels of 64 channels
@@ -828,7 +828,13 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         warp_arrive(&ms.bar_uround);
         ok_prev = ok_u;
+        if constexpr (PREP)
+          if (c + 1 < nch) ok_prev = norms_ahead(ok_prev);
       } else {
+        // (raw projections: the next chunk's Vw^T first, its sigmoid filling the wait for the
+        // state product)
+        if constexpr (PREP)
+          if (c + 1 < nch) ok_s = vw_ahead(c + 1, ok_s);
         // ===== R^T = Vw^T + X^T rounded to tf32 in place once the state product is done ======
         ok_s = ok_s && wait_on(&ms.bar_s, ph_s);
         tc_fence_after();
@@ -846,10 +852,7 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         warp_arrive(&ms.bar_tdiag);
         // ===== then one chunk ahead: Vw^T and the cumulative decay of the next chunk =========
-        if (c + 1 < nch) {
-          ok_s = decay_ahead(c + 1, vw_ahead(c + 1, ok_s));
-          if constexpr (PREP) ok_s = norms_ahead(ok_s);
-        }
+        if (c + 1 < nch) ok_s = decay_ahead(c + 1, PREP ? ok_s : vw_ahead(c + 1, ok_s));
         // These warps do not use U~; they step their phase bit past its product without
         // waiting (by now the chunk's last product may have completed as well, and a parity
         // wait must never trail its barrier by two phases).  Their next wait, on that last
