@@ -249,6 +249,27 @@ def _time_loop(step, steps, warmup):
     return t0.elapsed_time(t1) / steps
 
 
+def time_conv(args, dev):
+    """The short convolution over the q, k, v projections of the prefill workload, side by
+    side: [B, T, 3 H d] bf16 (each element read once and written once)."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    B, T, C = PREFILL.B, PREFILL.T, PREFILL.H * (2 * PREFILL.dk + PREFILL.dv)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(PREFILL.seed)
+    x = torch.randn((B, T, C), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    w = 0.5 * torch.randn((C, 4), generator=gen, device=dev, dtype=torch.float32)
+    b = 0.1 * torch.randn((C,), generator=gen, device=dev, dtype=torch.float32)
+    y = torch.empty_like(x)
+
+    def step():
+        g.gdn2_short_conv(x, w, b, y=y)
+
+    ms = _time_loop(step, args.steps, args.warmup)
+    return dict(ms=ms, bytes=2 * x.numel() * x.element_size(), tokens=B * T, C=C,
+                ok=g.gdn2_device_status() == 0)
+
+
 def time_raw(args, dev):
     """The prefill workload fed with raw projections (activations inside the kernel)."""
     import torch
@@ -421,6 +442,8 @@ def main():
     dec = time_decode(dev, args.decode_steps, world)
     pak = time_packed(args, dev)
     raw = time_raw(args, dev)
+    cv = time_conv(args, dev)
+    cv_gbs = cv["bytes"] / (cv["ms"] * 1e-3) / 1e9
     raw_gbs = raw["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (raw["ms"] * 1e-3) / 1e9
     # algorithmic bytes: the token streams plus each sequence's entering and final state
     pak_bytes = pak["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD + pak["units"] * DECODE_STATE_BYTES
@@ -469,9 +492,16 @@ def main():
                 "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (raw)", "achieved": raw_gbs,
                              "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": raw_gbs / pk["hbm_gbs"],
                              "traffic": None}},
+        "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
+                 "steps": args.steps,
+                 "workload": f"q, k, v projections of prefill_b8_h16_t4096 side by side: [8, 4096, {cv['C']}] bf16, "
+                             "4 taps + bias, zero history",
+                 "roofline": {"bound": "hbm", "kernel": "short_conv_kernel", "achieved": cv_gbs,
+                              "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": cv_gbs / pk["hbm_gbs"],
+                              "traffic": None}},
         "gpu_launches": args.steps,
         "clocks": pre["clocks"],
-        "device_status_ok": bool(pre["ok"] and dec["ok"] and pak["ok"] and raw["ok"]),
+        "device_status_ok": bool(pre["ok"] and dec["ok"] and pak["ok"] and raw["ok"] and cv["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)

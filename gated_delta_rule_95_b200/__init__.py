@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -59,6 +59,8 @@ def lib():
         L.gdn2_chunk_fwd_varlen.restype = I
         L.gdn2_chunk_fwd_raw.argtypes = [P] * 11 + [I] * 6 + [P]
         L.gdn2_chunk_fwd_raw.restype = I
+        L.gdn2_short_conv.argtypes = [P] * 7 + [I] * 4 + [P]
+        L.gdn2_short_conv.restype = I
         L.gdn2_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
         L.gdn2_decode_step.restype = I
         L.gdn2_device_status.argtypes = []
@@ -89,7 +91,8 @@ def _check_tokens(name, tensors, dtype, device):
             raise ValueError(f"{name}: {n} must be a CUDA tensor on {device}")
         if not t.is_contiguous():
             raise ValueError(f"{name}: {n} must be contiguous")
-        want = torch.float32 if n in ("log_alpha", "a_raw", "S0", "S", "S_T", "o", "decay_scale") else dtype
+        want = torch.float32 if n in ("log_alpha", "a_raw", "S0", "S", "S_T", "o", "decay_scale", "weight",
+                                      "bias") else dtype
         if t.dtype != want:
             raise ValueError(f"{name}: {n} must be {want}, got {t.dtype}")
 
@@ -190,6 +193,42 @@ def gdn2_chunk_fwd_raw(q_raw, k_raw, v, a_raw, b_raw, w_raw, S0=None, *, decay_s
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd_raw", rc)
     return o, S_T
+
+
+def gdn2_short_conv(x, weight, bias=None, *, cu_seqlens=None, hist=None, y=None, hist_out=None, want_hist=False,
+                    stream=None):
+    """Short causal depthwise convolution (4 taps) over the token axis.
+
+    x: [B, T, C] (or packed [T, C] with cu_seqlens int32 [N + 1] on the device); weight fp32
+    [C, 4] (or [C, 1, 4]); bias fp32 [C] or None; hist: [B, 3, C] carried history or None.
+    Returns (y like x, hist_out [B, 3, C] or None); hist_out may be hist (in-place update)."""
+    if x.dtype not in _DT:
+        raise ValueError(f"gdn2_short_conv: unsupported dtype {x.dtype}")
+    if cu_seqlens is None:
+        B, T, C = x.shape
+    else:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+            raise ValueError("gdn2_short_conv: cu_seqlens must be a contiguous int32 vector")
+        if cu_seqlens.device != x.device:
+            raise ValueError("gdn2_short_conv: cu_seqlens must be on the inputs' device")
+        T, C = x.shape
+        B = cu_seqlens.numel() - 1
+    if weight.numel() != 4 * C:
+        raise ValueError("gdn2_short_conv: weight must hold 4 taps per channel")
+    if y is None:
+        y = torch.empty_like(x)
+    if hist_out is None and want_hist:
+        hist_out = torch.empty((B, 3, C), dtype=x.dtype, device=x.device)
+    ts = dict(x=x, weight=weight, y=y)
+    for n, t in (("bias", bias), ("hist", hist), ("hist_out", hist_out)):
+        if t is not None:
+            ts[n] = t
+    _check_tokens("gdn2_short_conv", ts, x.dtype, x.device)
+    rc = lib().gdn2_short_conv(_ptr(x), _ptr(weight), _ptr(bias), _ptr(cu_seqlens), _ptr(hist), _ptr(y),
+                               _ptr(hist_out), B, T, C, _DT[x.dtype], _stream(x.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_short_conv", rc)
+    return y, hist_out
 
 
 def gdn2_decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):

@@ -123,6 +123,27 @@ extern "C" gdn2_status gdn2_chunk_fwd_raw(const void* q_raw, const void* k_raw, 
   return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
 }
 
+extern "C" gdn2_status gdn2_short_conv(const void* x, const float* weight, const float* bias, const int* cu_seqlens,
+                                       const void* hist_in, void* y, void* hist_out, int B, int T, int C,
+                                       gdn2_dtype dt, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  const bool packed = cu_seqlens != nullptr;
+  if (B < 0 || T < 0 || C < 0 || C % 8 != 0 || C > (1 << 24)) return GDN2_ERR_SHAPE;
+  const long long ntok = packed ? (long long)T : (long long)B * T;
+  if (ntok > 0x7fffffffLL - 64 || ntok * C > (1LL << 46)) return GDN2_ERR_SHAPE;
+  if (B == 0 || C == 0) return GDN2_OK;
+  if (ntok > 0 && (!x || !y || !weight)) return GDN2_ERR_NULL;
+  if (hist_out && !x && ntok > 0) return GDN2_ERR_NULL;
+  const void* ptrs[] = {x, weight, bias, hist_in, y, hist_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return GDN2_ERR_ALIGN;
+  if (x && x == y) return GDN2_ERR_SHAPE;  // the window reads inputs other threads would overwrite
+  ShortConvArgs a{x, weight, bias, cu_seqlens, hist_in, y, hist_out, B, T, C, dt == GDN2_BF16};
+  cudaError_t e = launch_short_conv(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
 extern "C" gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
                                         const void* b, const void* w, float* S, float* o, int B, int H, int d_k,
                                         int d_v, gdn2_dtype dt, void* stream) {

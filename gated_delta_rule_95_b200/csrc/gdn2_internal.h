@@ -36,6 +36,20 @@ enum : unsigned {
 };
 unsigned* device_error_word();
 
+// Short causal convolution (4 taps) over [B, T, C] (or packed [T, C] with cu_seqlens).
+struct ShortConvArgs {
+  const void* x;
+  const float* weight;    // [C, 4]
+  const float* bias;      // [C] or NULL
+  const int* cu_seqlens;  // packed: [B + 1] device offsets; NULL: B sequences of T tokens
+  const void* hist_in;    // [B, 3, C] or NULL (zeros)
+  void* y;
+  void* hist_out;         // [B, 3, C] or NULL; may alias hist_in
+  int B, T, C;
+  bool bf16;
+};
+cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t st);
+
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
 // bf16 inputs: tcgen05/TMEM kernel fed by TMA.
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st);

@@ -1,0 +1,226 @@
+// Short causal depthwise convolution (kernel size 4) over the token axis, applied to
+// q, k and v before the recurrence (Gated DeltaNet-2 guide, "Normalization and Short
+// Convolutions"; the guide's layer convolves each channel with 4 taps, padded on the
+// left so that token t sees tokens t-3 .. t, with a bias):
+//
+//     y[t, c] = bias[c] + sum_{j=0..3} weight[c, j] * x[t - 3 + j, c]
+//
+// where the tokens before a sequence's first come from its carried history (the last
+// three inputs of the previous call) or are zero.  Bandwidth-bound: every input element is
+// read once and every output written once.
+//
+// Work split: thread (strip, channel quad) walks STRIP consecutive tokens of four adjacent
+// channels with a three-token window in registers; a warp covers 128 consecutive channels
+// of one token per load (256 bytes for bf16), and a strip's loads are all issued before
+// the first output so that each thread keeps STRIP loads in flight.  A strip may cross
+// sequence boundaries (packed batches): the window is reloaded from the history at each
+// sequence start.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "gdn2_internal.h"
+
+namespace gdn2 {
+namespace {
+
+// tokens per thread: 32 of bf16 or 16 of fp32, i.e. 256 bytes of loads in flight per thread
+template <typename T>
+__host__ __device__ constexpr int strip_of() { return 512 / (int)sizeof(T) / 8; }
+constexpr int CONV_THREADS = 256;
+
+// Four adjacent channels of one token: 8 bytes of bf16 or 16 bytes of fp32.
+template <typename T>
+struct Quad;
+template <>
+struct Quad<float> {
+  using V = float4;
+  static __device__ __forceinline__ float4 load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+  static __device__ __forceinline__ void store(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+  static __device__ __forceinline__ float4 f(float4 v) { return v; }
+  static __device__ __forceinline__ float4 from(float4 v) { return v; }
+  static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+};
+template <>
+struct Quad<__nv_bfloat16> {
+  using V = uint2;
+  static __device__ __forceinline__ uint2 load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, uint2 v) { __stcs(reinterpret_cast<uint2*>(p), v); }
+  static __device__ __forceinline__ float4 f(uint2 v) {
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                       __uint_as_float(v.y & 0xFFFF0000u));
+  }
+  static __device__ __forceinline__ uint2 from(float4 v) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    return make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+  }
+  static __device__ __forceinline__ uint2 zero() { return make_uint2(0u, 0u); }
+};
+
+// Sequence of flat token g: fixed length T per sequence, or the packed offsets cu[0..nseq].
+__device__ __forceinline__ int seq_of(int g, const int* cu, int nseq, int T) {
+  if (!cu) return g / T;
+  int lo = 0, hi = nseq;  // cu[lo] <= g < cu[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu[mid] <= g) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Packed offsets are checked where they are used: a strip whose sequence lookup is not
+// consistent (offsets out of order or out of range) sets kErrBadSeqlens and writes nothing.
+// Block b covers channel block b mod ncb of strip b / ncb, so that consecutive blocks read
+// consecutive parts of the same token rows.
+template <typename T>
+__global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const T* __restrict__ x, const float* __restrict__ w,
+                                                                const float* __restrict__ bias, const int* cu,
+                                                                int nseq, const T* hist, T* __restrict__ y,
+                                                                int ntok, int T_seq, int C, int ncb, unsigned* err) {
+  using Q = Quad<T>;
+  constexpr int STRIP = strip_of<T>();
+  const int cb = blockIdx.x % ncb, strip = blockIdx.x / ncb;
+  const int c = 4 * (cb * CONV_THREADS + threadIdx.x);
+  if (c >= C) return;
+  const int g0 = strip * STRIP;
+  if (cu) {
+    const int n0 = seq_of(g0, cu, nseq, T_seq);
+    const bool bad = cu[0] != 0 || cu[nseq] != ntok || cu[n0] < 0 || cu[n0] > g0 || cu[n0 + 1] <= g0;
+    if (bad) {
+      if (threadIdx.x == 0 && err) atomicOr(err, kErrBadSeqlens);
+      return;
+    }
+  }
+  const int g1 = min(g0 + STRIP, ntok);
+  // taps of the four channels: wt[j] = (w[c][j], w[c+1][j], w[c+2][j], w[c+3][j])
+  float4 wt[4];
+  {
+    const float4 r0 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c));
+    const float4 r1 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 4));
+    const float4 r2 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 8));
+    const float4 r3 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 12));
+    wt[0] = make_float4(r0.x, r1.x, r2.x, r3.x);
+    wt[1] = make_float4(r0.y, r1.y, r2.y, r3.y);
+    wt[2] = make_float4(r0.z, r1.z, r2.z, r3.z);
+    wt[3] = make_float4(r0.w, r1.w, r2.w, r3.w);
+  }
+  const float4 b0 = bias ? __ldg(reinterpret_cast<const float4*>(bias + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+
+  // the strip's inputs first (STRIP independent loads in flight)
+  typename Q::V xs[STRIP];
+#pragma unroll
+  for (int i = 0; i < STRIP; ++i) xs[i] = (g0 + i < g1) ? Q::load(x + (size_t)(g0 + i) * C + c) : Q::zero();
+
+  int n = seq_of(g0, cu, nseq, T_seq);
+  int start = cu ? cu[n] : n * T_seq;
+  int next = cu ? cu[n + 1] : start + T_seq;  // first token of the next sequence
+  // window h[j] = input at token g - 3 + j (j = 0, 1, 2) for the strip's first token
+  float4 h[3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int gj = g0 - 3 + j;  // >= start - 3
+    if (gj >= start) {
+      h[j] = Q::f(Q::load(x + (size_t)gj * C + c));
+    } else if (hist) {  // history slot 3 - (start - gj) of sequence n, oldest first
+      h[j] = Q::f(Q::load(hist + ((size_t)n * 3 + 3 - (start - gj)) * C + c));
+    } else {
+      h[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < STRIP; ++i) {
+    const int g = g0 + i;
+    if (g >= g1) break;
+    if (g >= next) {  // a new sequence starts here (skipping empty ones): its own history
+      while (g >= next && n + 1 < nseq) {  // (g < cu[nseq] stops it first for valid offsets)
+        ++n;
+        start = next;
+        next = cu ? cu[n + 1] : start + T_seq;
+      }
+      if (g < start || g >= next) return;  // offsets out of order: nothing more is written
+#pragma unroll
+      for (int j = 0; j < 3; ++j)  // g == start: slot j of the new sequence's history
+        h[j] = hist ? Q::f(Q::load(hist + ((size_t)n * 3 + j) * C + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float4 xi = Q::f(xs[i]);
+    float4 o;
+    o.x = fmaf(wt[0].x, h[0].x, fmaf(wt[1].x, h[1].x, fmaf(wt[2].x, h[2].x, fmaf(wt[3].x, xi.x, b0.x))));
+    o.y = fmaf(wt[0].y, h[0].y, fmaf(wt[1].y, h[1].y, fmaf(wt[2].y, h[2].y, fmaf(wt[3].y, xi.y, b0.y))));
+    o.z = fmaf(wt[0].z, h[0].z, fmaf(wt[1].z, h[1].z, fmaf(wt[2].z, h[2].z, fmaf(wt[3].z, xi.z, b0.z))));
+    o.w = fmaf(wt[0].w, h[0].w, fmaf(wt[1].w, h[1].w, fmaf(wt[2].w, h[2].w, fmaf(wt[3].w, xi.w, b0.w))));
+    Q::store(y + (size_t)g * C + c, Q::from(o));
+    h[0] = h[1];
+    h[1] = h[2];
+    h[2] = xi;
+  }
+}
+
+// The history after the call: the last three inputs of each sequence, counting the carried
+// history before it (a sequence shorter than three tokens keeps part of its old history).
+// One thread per (sequence, channel pair) reads its three values before writing, so the
+// history may be updated in place.
+template <typename T>
+__global__ void short_conv_history_kernel(const T* __restrict__ x, const int* cu, const T* hist_in, T* hist_out,
+                                          int nseq, int ntok, int T_seq, int C, unsigned* err) {
+  using Q = Quad<T>;
+  const int c = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+  const int n = blockIdx.y;
+  if (c >= C || n >= nseq) return;
+  const int start = cu ? cu[n] : n * T_seq;
+  const int len = cu ? cu[n + 1] - start : T_seq;
+  if (start < 0 || len < 0 || start + len > ntok) {  // offsets out of order or out of range
+    if (c == 0 && err) atomicOr(err, kErrBadSeqlens);
+    return;
+  }
+  typename Q::V v[3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const int e = len + i;  // position in [history (3) | the sequence's tokens]
+    if (e >= 3) {
+      v[i] = Q::load(x + (size_t)(start + e - 3) * C + c);
+    } else if (hist_in) {
+      v[i] = *reinterpret_cast<const typename Q::V*>(hist_in + ((size_t)n * 3 + e) * C + c);
+    } else {
+      v[i] = Q::zero();
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 3; ++i) *reinterpret_cast<typename Q::V*>(hist_out + ((size_t)n * 3 + i) * C + c) = v[i];
+}
+
+template <typename T>
+cudaError_t launch_typed(const ShortConvArgs& a, cudaStream_t st) {
+  const T* x = static_cast<const T*>(a.x);
+  const T* hin = static_cast<const T*>(a.hist_in);
+  T* y = static_cast<T*>(a.y);
+  T* hout = static_cast<T*>(a.hist_out);
+  const int nseq = a.B;
+  const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
+  const int quads = a.C / 4;
+  if (ntok > 0) {
+    const int ncb = (quads + CONV_THREADS - 1) / CONV_THREADS;
+    constexpr int STRIP = strip_of<T>();
+    const long long blocks = (long long)((ntok + STRIP - 1) / STRIP) * ncb;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    short_conv_kernel<T><<<(unsigned)blocks, CONV_THREADS, 0, st>>>(x, a.weight, a.bias, a.cu_seqlens, nseq, hin, y,
+                                                                     ntok, a.T, a.C, ncb, device_error_word());
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (hout) {
+    dim3 grid((quads + 127) / 128, nseq);
+    short_conv_history_kernel<T><<<grid, 128, 0, st>>>(x, a.cu_seqlens, hin, hout, nseq, ntok, a.T, a.C,
+                                                        device_error_word());
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t st) {
+  if (a.B == 0 || a.C == 0) return cudaSuccess;
+  return a.bf16 ? launch_typed<__nv_bfloat16>(a, st) : launch_typed<float>(a, st);
+}
+
+}  // namespace gdn2

@@ -137,6 +137,36 @@ GDN2_API gdn2_status gdn2_chunk_fwd_raw(const void* q_raw, const void* k_raw, co
                                int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
 
 /*
+ * Short causal depthwise convolution with 4 taps over the token axis, the local mixing
+ * the layer applies to q, k and v before the recurrence (Gated DeltaNet-2 guide,
+ * "Normalization and Short Convolutions"; the guide's layer pads each channel on the
+ * left so that token t sees tokens t-3 .. t, and adds a bias):
+ *
+ *     y[t, c] = bias[c] + sum_{j=0..3} weight[c, j] * x[t - 3 + j, c]
+ *
+ * Tokens before a sequence's first are taken from its carried history (the last three
+ * inputs of the previous call, oldest first), or are zero.  Accumulation in fp32; y is
+ * rounded to dt.  Streaming decode is the case T = 1 with hist_out = hist_in.
+ *
+ *   x, y       : [B, T, C] dt (packed: [T, C]); y must not alias x
+ *   weight     : [C, 4] fp32 (the layout of a depthwise Conv1d weight [C, 1, 4])
+ *   bias       : [C] fp32, or NULL for none
+ *   cu_seqlens : NULL: B sequences of T tokens.  Otherwise [B + 1] int32 DEVICE offsets of
+ *                B packed sequences over T tokens, as gdn2_chunk_fwd_varlen takes them;
+ *                offsets out of order or out of range are reported by
+ *                gdn2_device_status() as GDN2_ERR_SHAPE (the affected outputs are not
+ *                written)
+ *   hist_in    : [B, 3, C] dt, read only, or NULL for zeros
+ *   hist_out   : [B, 3, C] dt, written with each sequence's last three inputs (for a
+ *                sequence shorter than three, the tail of its history first), or NULL;
+ *                may alias hist_in
+ *   C          : a multiple of 8 (16-byte rows), at most 2^24
+ */
+GDN2_API gdn2_status gdn2_short_conv(const void* x, const float* weight, const float* bias, const int* cu_seqlens,
+                            const void* hist_in, void* y, void* hist_out, int B, int T, int C, gdn2_dtype dt,
+                            void* stream);
+
+/*
  * One recurrent decode step: the update above for a single token per
  * (sequence, head), with the state updated in place (Gated DeltaNet-2 guide,
  * "4.5x Higher Decoding Throughput with Zero KV Cache": a fixed-size state

@@ -9,6 +9,8 @@ this package, and this package imports nothing from the CUDA path.
   update; readout after the update as in the guide's PyTorch loop).
 * ``chunkwise.forward`` re-derives the chunkwise WY form in numpy; it is a
   second, independent route to the same numbers, used to pin chunk invariance.
+* ``short_conv`` is the layer's 4-tap causal depthwise convolution, a plain loop
+  over taps.
 * ``activations`` maps the raw projections to the mixer's inputs (L2-normalised
   q and k, sigmoid gates, log alpha = -s_h softplus(a)); composed with
   ``forward`` it is what the raw-projection entry point computes.
@@ -147,6 +149,29 @@ def activations(q_raw, k_raw, a_raw, b_raw, w_raw, decay_scale=None):
     softplus = np.logaddexp(0.0, a_raw)
     return dict(q=l2n(q_raw), k=l2n(k_raw), log_alpha=-s[:, None] * softplus, b=_sigmoid(b_raw),
                 w=_sigmoid(w_raw))
+
+
+def short_conv(x, weight, bias=None, hist=None):
+    """Causal depthwise convolution with 4 taps over the token axis of one sequence
+    (Gated DeltaNet-2 guide, "Normalization and Short Convolutions": the layer convolves
+    each channel of q, k and v over tokens t-3 .. t, padding on the left, with a bias):
+    y[t, c] = bias[c] + sum_j weight[c, j] x[t - 3 + j, c], tokens before the first taken
+    from ``hist`` ([3, C], oldest first) or zero.
+
+    x: [T, C]; weight [C, 4]; bias [C] or None.  Returns (y [T, C], the last three inputs
+    [3, C] of the history followed by x)."""
+    x = _f64(x)
+    T, C = x.shape
+    w = _f64(weight).reshape(C, 4)
+    ext = np.zeros((T + 3, C))
+    if hist is not None:
+        ext[:3] = _f64(hist).reshape(3, C)
+    ext[3:] = x
+    y = np.zeros((T, C)) if bias is None else np.tile(_f64(bias).reshape(1, C), (T, 1))
+    for t in range(T):
+        for j in range(4):
+            y[t] += w[:, j] * ext[t + j]
+    return y, ext[T:T + 3].copy()
 
 
 def decode_step(q, k, v, log_alpha, b, w, S, nthreads=None, lib=None):

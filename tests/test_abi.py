@@ -97,6 +97,21 @@ def test_chunk_fwd_raw_validation(kw, status):
     assert raw(**kw) == status
 
 
+def conv(x=A, w=A, b=None, cu=None, hi=None, y=P(0x20000), ho=None, B=2, T=10, C=64, dt=1):
+    return g.lib().gdn2_short_conv(x, w, b, cu, hi, y, ho, B, T, C, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(C=60), 2), (dict(C=-8), 2), (dict(B=-1), 2), (dict(T=-1), 2), (dict(dt=4), 3),
+    (dict(x=None), 1), (dict(w=None), 1), (dict(y=None), 1),
+    (dict(y=A), 2),  # y aliasing x
+    (dict(b=P(0x10008)), 4), (dict(hi=P(0x10004)), 4), (dict(cu=P(0x10002)), 4),
+    (dict(B=0), 0), (dict(C=0), 0),
+])
+def test_short_conv_validation(kw, status):
+    assert conv(**kw) == status
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)

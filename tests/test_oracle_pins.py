@@ -103,3 +103,51 @@ def test_activations_identities():
     assert np.allclose(q["log_alpha"], p["log_alpha"] * s[:, None], rtol=1e-15, atol=0)
     # every decay lies in (0, 1) and every gate in (0, 1)
     assert np.all(p["log_alpha"] < 0) and np.all((p["w"] > 0) & (p["w"] < 1))
+
+
+# ---- the short convolution -----------------------------------------------------------------
+
+def test_short_conv_is_a_truncated_full_convolution():
+    # y[:, c] equals numpy's full convolution with the taps reversed, cut to the first T
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((37, 6))
+    w = rng.standard_normal((6, 4))
+    bias = rng.standard_normal(6)
+    y, _ = oracle.short_conv(x, w, bias)
+    for c in range(6):
+        ref = np.convolve(x[:, c], w[c, ::-1])[:37] + bias[c]
+        assert np.allclose(y[:, c], ref, rtol=0, atol=1e-13)
+
+
+def test_short_conv_impulse_and_causality():
+    w = np.arange(1.0, 9.0).reshape(2, 4)
+    x = np.zeros((8, 2))
+    x[2] = 1.0  # an impulse at token 2: y[2 + s] = w[:, 3 - s] for s = 0..3, zero elsewhere
+    y, hist = oracle.short_conv(x, w)
+    want = np.zeros((8, 2))
+    for s in range(4):
+        want[2 + s] = w[:, 3 - s]
+    assert np.array_equal(y, want)
+    assert np.array_equal(hist, x[-3:])
+    # a change at token 5 leaves tokens 0..4 alone
+    x2 = x.copy()
+    x2[5] = 7.0
+    y2, _ = oracle.short_conv(x2, w)
+    assert np.array_equal(y2[:5], y[:5]) and not np.array_equal(y2[5:], y[5:])
+
+
+@pytest.mark.parametrize("cut", [1, 2, 3, 10])
+def test_short_conv_history_handoff(cut):
+    # splitting a sequence and carrying the last three inputs equals one run, also when the
+    # first part is shorter than the window
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((20, 5))
+    w = rng.standard_normal((5, 4))
+    h0 = rng.standard_normal((3, 5))
+    y, h = oracle.short_conv(x, w, None, h0)
+    ya, ha = oracle.short_conv(x[:cut], w, None, h0)
+    yb, hb = oracle.short_conv(x[cut:], w, None, ha)
+    assert np.allclose(np.concatenate([ya, yb]), y, rtol=0, atol=1e-13)
+    assert np.array_equal(hb, h)
+    if cut < 3:  # the old history's tail survives in front of the new tokens
+        assert np.array_equal(ha[:3 - cut], h0[cut:])
