@@ -9,26 +9,34 @@
 // three inputs of the previous call) or are zero.  Bandwidth-bound: every input element is
 // read once and every output written once.
 //
-// Work split: thread (strip, channel quad) walks STRIP consecutive tokens of four adjacent
-// channels with a three-token window in registers; a warp covers 128 consecutive channels
-// of one token per load (256 bytes for bf16), and a strip's loads are all issued before
-// the first output so that each thread keeps STRIP loads in flight.  A strip may cross
-// sequence boundaries (packed batches): the window is reloaded from the history at each
-// sequence start.
+// Work split: a block of 256 threads takes a strip of tokens by a block of 1024 channels.
+// One thread copies the strip's rows (and the three rows before it) into shared memory
+// with 1-D bulk copies on one mbarrier, so that a block keeps its whole tile (70 KB for
+// bf16) in flight without holding it in registers and three blocks share an SM; then
+// thread t walks the strip for the four channels [4 t, 4 t + 4) of the block with a
+// three-token window in registers and stores y directly (a warp writes 256 contiguous
+// bytes of bf16 per token).  A strip may cross sequence boundaries (packed batches): the
+// window is reloaded from the history at each sequence start.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 #include "gdn2_internal.h"
+#include "ptx.cuh"
 
 namespace gdn2 {
 namespace {
 
-// tokens per thread: 32 of bf16 or 16 of fp32, i.e. 256 bytes of loads in flight per thread
-template <typename T>
-__host__ __device__ constexpr int strip_of() { return 512 / (int)sizeof(T) / 8; }
 constexpr int CONV_THREADS = 256;
+// tokens per strip: 32 of bf16 or 16 of fp32 (a tile of at most 35 or 19 rows of 2 or 4 KB)
+template <typename T>
+__host__ __device__ constexpr int strip_of() { return 64 / (int)sizeof(T); }
+template <typename T>
+__host__ __device__ constexpr uint32_t conv_smem_bytes() {
+  return (uint32_t)(strip_of<T>() + 3) * CONV_THREADS * 4 * (uint32_t)sizeof(T) + 16;
+}
+constexpr uint64_t CONV_WAIT_LIMIT = 2000000000ull;  // 2 s
 
 // Four adjacent channels of one token: 8 bytes of bf16 or 16 bytes of fp32.
 template <typename T>
@@ -81,8 +89,7 @@ __global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const T* __res
   using Q = Quad<T>;
   constexpr int STRIP = strip_of<T>();
   const int cb = blockIdx.x % ncb, strip = blockIdx.x / ncb;
-  const int c = 4 * (cb * CONV_THREADS + threadIdx.x);
-  if (c >= C) return;
+  const int c = 4 * (cb * CONV_THREADS + threadIdx.x);  // may be >= C in the last channel block
   const int g0 = strip * STRIP;
   if (cu) {
     const int n0 = seq_of(g0, cu, nseq, T_seq);
@@ -93,24 +100,49 @@ __global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const T* __res
     }
   }
   const int g1 = min(g0 + STRIP, ntok);
-  // taps of the four channels: wt[j] = (w[c][j], w[c+1][j], w[c+2][j], w[c+3][j])
-  float4 wt[4];
-  {
-    const float4 r0 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c));
-    const float4 r1 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 4));
-    const float4 r2 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 8));
-    const float4 r3 = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 12));
-    wt[0] = make_float4(r0.x, r1.x, r2.x, r3.x);
-    wt[1] = make_float4(r0.y, r1.y, r2.y, r3.y);
-    wt[2] = make_float4(r0.z, r1.z, r2.z, r3.z);
-    wt[3] = make_float4(r0.w, r1.w, r2.w, r3.w);
+  // the tile: rows r0 .. g1 - 1 (the strip and up to three rows before it) of this block's
+  // channels [c0, c0 + width), row i at tile + i * width
+  extern __shared__ __align__(16) unsigned char conv_smem[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(conv_smem);
+  T* tile = reinterpret_cast<T*>(conv_smem + 16);
+  const int c0 = cb * CONV_THREADS * 4;
+  const int width = min(CONV_THREADS * 4, C - c0);
+  const int r0 = max(g0 - 3, 0);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
   }
-  const float4 b0 = bias ? __ldg(reinterpret_cast<const float4*>(bias + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
-
-  // the strip's inputs first (STRIP independent loads in flight)
-  typename Q::V xs[STRIP];
-#pragma unroll
-  for (int i = 0; i < STRIP; ++i) xs[i] = (g0 + i < g1) ? Q::load(x + (size_t)(g0 + i) * C + c) : Q::zero();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t row_bytes = (uint32_t)width * sizeof(T);
+    mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)(g1 - r0));
+    for (int r = r0; r < g1; ++r)
+      bulk_load_1d(tile + (size_t)(r - r0) * width, x + (size_t)r * C + c0, row_bytes, bar);
+  }
+  // taps of the four channels: wt[j] = (w[c][j], w[c+1][j], w[c+2][j], w[c+3][j])
+  const bool active = c < C;
+  float4 wt[4];
+  float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) {
+    const float4 r0w = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c));
+    const float4 r1w = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 4));
+    const float4 r2w = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 8));
+    const float4 r3w = __ldg(reinterpret_cast<const float4*>(w + 4 * (size_t)c + 12));
+    wt[0] = make_float4(r0w.x, r1w.x, r2w.x, r3w.x);
+    wt[1] = make_float4(r0w.y, r1w.y, r2w.y, r3w.y);
+    wt[2] = make_float4(r0w.z, r1w.z, r2w.z, r3w.z);
+    wt[3] = make_float4(r0w.w, r1w.w, r2w.w, r3w.w);
+    if (bias) b0 = __ldg(reinterpret_cast<const float4*>(bias + c));
+  }
+  volatile int never = 0;
+  if (!mbar_wait_bounded(bar, 0, &never, err, CONV_WAIT_LIMIT)) {
+    // the copies must land before the block's shared memory is released
+    mbar_wait_bounded(bar, 0, &never, nullptr, CONV_WAIT_LIMIT);
+    return;
+  }
+  if (!active) return;
+  const T* tc = tile + 4 * threadIdx.x;  // this thread's channels in row 0 of the tile
+  auto row = [&](int g) { return Q::f(*reinterpret_cast<const typename Q::V*>(tc + (size_t)(g - r0) * width)); };
 
   int n = seq_of(g0, cu, nseq, T_seq);
   int start = cu ? cu[n] : n * T_seq;
@@ -120,8 +152,8 @@ __global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const T* __res
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
     const int gj = g0 - 3 + j;  // >= start - 3
-    if (gj >= start) {
-      h[j] = Q::f(Q::load(x + (size_t)gj * C + c));
+    if (gj >= start) {  // (start >= 0, so gj >= r0)
+      h[j] = row(gj);
     } else if (hist) {  // history slot 3 - (start - gj) of sequence n, oldest first
       h[j] = Q::f(Q::load(hist + ((size_t)n * 3 + 3 - (start - gj)) * C + c));
     } else {
@@ -143,7 +175,7 @@ __global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const T* __res
       for (int j = 0; j < 3; ++j)  // g == start: slot j of the new sequence's history
         h[j] = hist ? Q::f(Q::load(hist + ((size_t)n * 3 + j) * C + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float4 xi = Q::f(xs[i]);
+    const float4 xi = row(g);
     float4 o;
     o.x = fmaf(wt[0].x, h[0].x, fmaf(wt[1].x, h[1].x, fmaf(wt[2].x, h[2].x, fmaf(wt[3].x, xi.x, b0.x))));
     o.y = fmaf(wt[0].y, h[0].y, fmaf(wt[1].y, h[1].y, fmaf(wt[2].y, h[2].y, fmaf(wt[3].y, xi.y, b0.y))));
@@ -203,7 +235,14 @@ cudaError_t launch_typed(const ShortConvArgs& a, cudaStream_t st) {
     constexpr int STRIP = strip_of<T>();
     const long long blocks = (long long)((ntok + STRIP - 1) / STRIP) * ncb;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    short_conv_kernel<T><<<(unsigned)blocks, CONV_THREADS, 0, st>>>(x, a.weight, a.bias, a.cu_seqlens, nseq, hin, y,
+    static bool attr_set = false;  // per element type
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(short_conv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)conv_smem_bytes<T>());
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    short_conv_kernel<T><<<(unsigned)blocks, CONV_THREADS, conv_smem_bytes<T>(), st>>>(x, a.weight, a.bias, a.cu_seqlens, nseq, hin, y,
                                                                      ntok, a.T, a.C, ncb, device_error_word());
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
