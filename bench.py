@@ -322,7 +322,9 @@ def time_prefill_e2e(args, dev):
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 
 
-def time_decode(dev, n_steps, world=1):
+def time_decode(dev, n_steps, world=1, raw=False):
+    """Decode steps on the decode workload; raw=True runs the raw-projection step on the same
+    token draws read as raw projections (the timing does not depend on the values)."""
     import torch
     import gated_delta_rule_95_b200 as g
     S = gi.decode_state(DECODE).to(dev)
@@ -330,10 +332,14 @@ def time_decode(dev, n_steps, world=1):
     td = [{k: v.to(dev) for k, v in t.items()} for t in toks]
     del toks
     o = torch.empty((DECODE.B, DECODE.H, DECODE.dv), dtype=torch.float32, device=dev)
+    scale = torch.full((DECODE.H,), 1.0 / 16.0, dtype=torch.float32, device=dev)
 
     def run(j):
         t = td[j]
-        g.gdn2_decode_step(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], S, o=o)
+        if raw:
+            g.gdn2_decode_step_raw(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], S, decay_scale=scale, o=o)
+        else:
+            g.gdn2_decode_step(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], S, o=o)
 
     for j in range(3):
         run(j)
@@ -440,6 +446,7 @@ def main():
     traffic = profile_traffic("chunk_fwd_tc_kernel")
 
     dec = time_decode(dev, args.decode_steps, world)
+    dec_raw = time_decode(dev, args.decode_steps, world, raw=True)
     pak = time_packed(args, dev)
     raw = time_raw(args, dev)
     cv = time_conv(args, dev)
@@ -450,6 +457,7 @@ def main():
     pak_gbs = pak_bytes / (pak["ms"] * 1e-3) / 1e9
     dec_units = DECODE.B * DECODE.H
     dec_gbs = dec_units * DECODE_STATE_BYTES / (dec["ms_per_step"] * 1e-3) / 1e9
+    decr_gbs = dec_units * DECODE_STATE_BYTES / (dec_raw["ms_per_step"] * 1e-3) / 1e9
     barrier(world)
     if rank != 0:
         if world > 1:
@@ -478,6 +486,13 @@ def main():
                                 "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],
                                 "traffic": profile_traffic("decode_step_kernel")},
                    "clocks": dec["clocks"]},
+        "decode_raw": {"metric": "GDN-2 decode steps/s, raw projections", "value": 1e3 / dec_raw["ms_per_step"],
+                       "unit": "steps/s", "ms_per_step": dec_raw["ms_per_step"], "steps": args.decode_steps,
+                       "workload": "decode_b256_h16 through gdn2_decode_step_raw (q, k normalised, sigmoid gates "
+                                   "and softplus decay inside the step)",
+                       "roofline": {"bound": "hbm", "kernel": "decode_step_kernel (raw)", "achieved": decr_gbs,
+                                    "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": decr_gbs / pk["hbm_gbs"],
+                                    "traffic": None}},
         "packed": {"metric": "GDN-2 packed prefill tokens/s per layer", "value": pak["tokens"] / (pak["ms"] * 1e-3),
                    "unit": "tokens/s", "ms_per_step": pak["ms"], "steps": args.steps,
                    "workload": f"packed_n64_h16: {pak['n_seq']} sequences, lengths log-uniform in [16, 8192] "
@@ -501,7 +516,7 @@ def main():
                               "traffic": None}},
         "gpu_launches": args.steps,
         "clocks": pre["clocks"],
-        "device_status_ok": bool(pre["ok"] and dec["ok"] and pak["ok"] and raw["ok"] and cv["ok"]),
+        "device_status_ok": bool(pre["ok"] and dec["ok"] and dec_raw["ok"] and pak["ok"] and raw["ok"] and cv["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)

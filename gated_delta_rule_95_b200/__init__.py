@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -63,6 +63,8 @@ def lib():
         L.gdn2_short_conv.restype = I
         L.gdn2_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
         L.gdn2_decode_step.restype = I
+        L.gdn2_decode_step_raw.argtypes = [P] * 9 + [I] * 5 + [P]
+        L.gdn2_decode_step_raw.restype = I
         L.gdn2_device_status.argtypes = []
         L.gdn2_device_status.restype = I
         L.gdn2_status_string.argtypes = [I]
@@ -245,6 +247,30 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
                                 B, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_decode_step", rc)
+    return o
+
+
+def gdn2_decode_step_raw(q_raw, k_raw, v, a_raw, b_raw, w_raw, S, *, decay_scale=None, o=None, stream=None):
+    """One decode step on the raw projections (q, k normalised, sigmoid gates, log alpha =
+    -decay_scale[h] * softplus(a_raw) inside the step); S [B,H,d_k,d_v] fp32 is updated in
+    place.  Returns o [B,H,d_v]."""
+    B, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    if q_raw.dtype not in _DT:
+        raise ValueError(f"gdn2_decode_step_raw: unsupported dtype {q_raw.dtype}")
+    if decay_scale is not None and decay_scale.numel() != H:
+        raise ValueError("gdn2_decode_step_raw: decay_scale must hold one value per head")
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=torch.float32, device=q_raw.device)
+    ts = dict(q_raw=q_raw, k_raw=k_raw, v=v, a_raw=a_raw, b_raw=b_raw, w_raw=w_raw, S=S, o=o)
+    if decay_scale is not None:
+        ts["decay_scale"] = decay_scale
+    _check_tokens("gdn2_decode_step_raw", ts, q_raw.dtype, q_raw.device)
+    rc = lib().gdn2_decode_step_raw(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(w_raw),
+                                    _ptr(decay_scale), _ptr(S), _ptr(o), B, H, dk, dv, _DT[q_raw.dtype],
+                                    _stream(q_raw.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_decode_step_raw", rc)
     return o
 
 

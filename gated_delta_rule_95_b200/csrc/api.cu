@@ -159,6 +159,24 @@ extern "C" gdn2_status gdn2_decode_step(const void* q, const void* k, const void
   return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
 }
 
+extern "C" gdn2_status gdn2_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, const float* a_raw,
+                                            const void* b_raw, const void* w_raw, const float* decay_scale, float* S,
+                                            float* o, int B, int H, int d_k, int d_v, gdn2_dtype dt, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (!sizes_ok(B, 1, H, d_k, d_v)) return GDN2_ERR_SHAPE;
+  if ((long long)B * H == 0) return GDN2_OK;
+  if (!q_raw || !k_raw || !v || !a_raw || !b_raw || !w_raw || !S || !o) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q_raw, k_raw, v, a_raw, b_raw, w_raw, S, o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN2_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(decay_scale) & 3u) != 0) return GDN2_ERR_ALIGN;
+  DecodeArgs a{q_raw, k_raw, v, b_raw, w_raw, a_raw, S, o, B, H, d_k, d_v, dt == GDN2_BF16};
+  a.raw = true;
+  a.decay_scale = decay_scale;
+  cudaError_t e = launch_decode_step(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
 extern "C" gdn2_status gdn2_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e);

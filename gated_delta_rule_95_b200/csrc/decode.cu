@@ -11,6 +11,12 @@
 // so one pass over S (two key-axis reductions per value column) gives o, and a
 // second pass over the registers that already hold S writes S'.
 //
+// Raw projections (PREP): b = sigmoid(b), w = sigmoid(w) and log alpha = -s_h softplus(a)
+// (Gated DeltaNet-2 guide, "Normalization and Short Convolutions" and "Decoupled Erase and
+// Write Gates") in fp32 while the state loads are in flight; q and k are L2-normalised by
+// carrying 1/|q| and 1/|k| as factors (reduced with q . k) into e, S^T y, q . k and the
+// rank-one write, which are linear in them.
+//
 // Work split: one CTA of 256 threads per (sequence, head).  Warp r owns rows
 // [r*DK/8, (r+1)*DK/8); lane c owns value columns [c*DV/32, (c+1)*DV/32), so
 // every warp-wide load or store of S covers whole contiguous rows.
@@ -33,12 +39,15 @@ __device__ __forceinline__ float ld_tok<__nv_bfloat16>(const __nv_bfloat16* p) {
   return __bfloat162float(__ldg(p));
 }
 
-template <typename T, int DK, int DV>
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+
+template <typename T, int DK, int DV, bool PREP>
 __global__ void __launch_bounds__(256) decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v,
                                                           const float* __restrict__ log_alpha,
                                                           const T* __restrict__ bg, const T* __restrict__ wg,
-                                                          float* __restrict__ S, float* __restrict__ o) {
+                                                          float* __restrict__ S, float* __restrict__ o, int H,
+                                                          const float* __restrict__ dscale) {
   constexpr int ROWS = DK / 8;   // rows per warp
   constexpr int CPL = DV / 32;   // columns per lane (2 or 4)
   using vec_t = typename std::conditional<CPL == 4, float4, float2>::type;
@@ -46,7 +55,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const T* __restrict__ 
   __shared__ float s_alpha[DK], s_k[DK], s_x[DK], s_y[DK];
   __shared__ float s_wv[DV], s_delta[DV];
   __shared__ float s_red[2][8][DV];
-  __shared__ float s_qk;
+  __shared__ float s_qk, s_rq, s_rk;
 
   const int unit = blockIdx.x;               // b * H + h
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -64,8 +73,28 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const T* __restrict__ 
   }
 
   if (tid < DK) {
-    const float a = __expf(__ldg(log_alpha + tk + tid));
-    const float kk = ld_tok(k + tk + tid), qq = ld_tok(q + tk + tid), bb = ld_tok(bg + tk + tid);
+    float la = __ldg(log_alpha + tk + tid);
+    if constexpr (PREP) {  // log alpha = -s_h softplus(a)
+      const float sh = dscale ? __ldg(dscale + unit % H) : 1.f;
+      la = -sh * (fmaxf(la, 0.f) + log1pf(__expf(-fabsf(la))));
+    }
+    const float a = __expf(la);
+    const float kk = ld_tok(k + tk + tid), qq = ld_tok(q + tk + tid);
+    float bb = ld_tok(bg + tk + tid);
+    if constexpr (PREP) {
+      bb = sigmoid_f(bb);
+      // |q|^2 and |k|^2, reduced like q . k (slots 1 and 2 of the reduction buffer)
+      float pq = qq * qq, pk = kk * kk;
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        pq += __shfl_xor_sync(0xffffffffu, pq, off);
+        pk += __shfl_xor_sync(0xffffffffu, pk, off);
+      }
+      if (lane == 0) {
+        s_red[0][warp][1] = pq;
+        s_red[0][warp][2] = pk;
+      }
+    }
     s_alpha[tid] = a;
     s_k[tid] = kk;
     s_x[tid] = a * bb * kk;
@@ -76,12 +105,28 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const T* __restrict__ 
     for (int off = 16; off; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
     if (lane == 0) s_red[0][warp][0] = p;  // reuse of the reduction buffer before it is needed
   }
-  if (tid < DV) s_wv[tid] = ld_tok(wg + tv + tid) * ld_tok(v + tv + tid);
+  if (tid < DV) {
+    float ww = ld_tok(wg + tv + tid);
+    if constexpr (PREP) ww = sigmoid_f(ww);
+    s_wv[tid] = ww * ld_tok(v + tv + tid);
+  }
   __syncthreads();
   if (tid == 0) {
     float p = 0.f;
 #pragma unroll
     for (int w = 0; w < DK / 32; ++w) p += s_red[0][w][0];
+    if constexpr (PREP) {
+      float nq = 0.f, nk = 0.f;
+#pragma unroll
+      for (int w = 0; w < DK / 32; ++w) {
+        nq += s_red[0][w][1];
+        nk += s_red[0][w][2];
+      }
+      const float rq = rsqrtf(fmaxf(nq, 1e-24f)), rk = rsqrtf(fmaxf(nk, 1e-24f));  // zero stays zero
+      s_rq = rq;
+      s_rk = rk;
+      p *= rq * rk;
+    }
     s_qk = p;
   }
 
@@ -113,8 +158,12 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const T* __restrict__ 
       ee += s_red[0][w][tid];
       rr += s_red[1][w][tid];
     }
+    if constexpr (PREP) {
+      ee *= s_rk;
+      rr *= s_rq;
+    }
     const float d = s_wv[tid] - ee;
-    s_delta[tid] = d;
+    s_delta[tid] = PREP ? d * s_rk : d;  // (the write k delta^T with the raw k)
     o[tv + tid] = fmaf(s_qk, d, rr);
   }
   __syncthreads();
@@ -136,9 +185,14 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const T* __restrict__ 
 
 template <typename T, int DK, int DV>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
-  decode_step_kernel<T, DK, DV><<<a.B * a.H, 256, 0, st>>>(
-      static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.log_alpha,
-      static_cast<const T*>(a.b), static_cast<const T*>(a.w), a.S, a.o);
+  const T *q = static_cast<const T*>(a.q), *k = static_cast<const T*>(a.k), *v = static_cast<const T*>(a.v);
+  const T *b = static_cast<const T*>(a.b), *w = static_cast<const T*>(a.w);
+  if (a.raw)
+    decode_step_kernel<T, DK, DV, true><<<a.B * a.H, 256, 0, st>>>(q, k, v, a.log_alpha, b, w, a.S, a.o, a.H,
+                                                                   a.decay_scale);
+  else
+    decode_step_kernel<T, DK, DV, false><<<a.B * a.H, 256, 0, st>>>(q, k, v, a.log_alpha, b, w, a.S, a.o, a.H,
+                                                                    nullptr);
   return cudaGetLastError();
 }
 

@@ -11,6 +11,10 @@ struct DecodeArgs {
   float* o;
   int B, H, dk, dv;
   bool bf16;
+  // raw projections: q, k un-normalised, b, w gate logits, log_alpha holds the decay
+  // pre-activation a (log alpha = -s_h softplus(a)); decay_scale: s_h per head (NULL = 1)
+  bool raw = false;
+  const float* decay_scale = nullptr;
 };
 
 struct ChunkArgs {

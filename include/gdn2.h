@@ -182,6 +182,21 @@ GDN2_API gdn2_status gdn2_decode_step(const void* q, const void* k, const void* 
                              const void* b, const void* w, float* S, float* o,
                              int B, int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
 
+/*
+ * One decode step on the raw projections: the activations of gdn2_chunk_fwd_raw (q and k
+ * L2-normalised per (sequence, head), b = sigmoid(b_raw), w = sigmoid(w_raw), log alpha =
+ * -s_h softplus(a_raw)) computed in fp32 inside the step, then gdn2_decode_step.
+ *
+ *   q_raw, k_raw, b_raw : [B, H, d_k]  dt
+ *   v, w_raw            : [B, H, d_v]  dt
+ *   a_raw               : [B, H, d_k]  fp32, finite
+ *   decay_scale         : [H] fp32 DEVICE array of s_h > 0, 4-byte aligned; NULL means 1
+ *   S, o                : as gdn2_decode_step
+ */
+GDN2_API gdn2_status gdn2_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, const float* a_raw,
+                                 const void* b_raw, const void* w_raw, const float* decay_scale, float* S,
+                                 float* o, int B, int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
+
 /* Synchronises the current device, then reports and clears the device error
  * word: GDN2_OK, GDN2_ERR_TIMEOUT (a bounded wait gave up), GDN2_ERR_SHAPE (bad
  * cu_seqlens), or GDN2_ERR_CUDA if the sync itself failed. */

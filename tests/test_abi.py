@@ -112,6 +112,18 @@ def test_short_conv_validation(kw, status):
     assert conv(**kw) == status
 
 
+def decode_raw(q=A, k=A, v=A, a=A, b=A, w=A, sc=None, S=A, o=A, B=2, H=1, dk=128, dv=128, dt=1):
+    return g.lib().gdn2_decode_step_raw(q, k, v, a, b, w, sc, S, o, B, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=80), 2), (dict(B=-2), 2), (dict(dt=2), 3), (dict(S=None), 1), (dict(a=None), 1),
+    (dict(v=M), 4), (dict(sc=P(0x10002)), 4), (dict(B=0), 0),
+])
+def test_decode_step_raw_validation(kw, status):
+    assert decode_raw(**kw) == status
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)

@@ -119,3 +119,35 @@ def test_full_prefill_b8_h16_t4096_sampled():
     for n, (bb, h) in enumerate(units):
         assert rel_err(o_c[bb, :, h].numpy(), o_ref[n, :, 0]) <= TOL["bf16"], (bb, h)
         assert rel_err(S_c[bb, h].numpy(), S_ref[n, 0]) <= TOL["bf16"], (bb, h)
+
+
+# ---- decode on raw projections ---------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("bf16", 64, 128), ("f32", 128, 64), ("f32", 64, 64)])
+def test_decode_raw_matches_oracle(dtype, dk, dv):
+    wl = dataclasses.replace(BASE, dk=dk, dv=dv, dtype=dtype, state_std=0.05)
+    d = gi.raw_inputs(wl, B=4, T=1, H=3)
+    d["decay_scale"] = torch.tensor([1 / 16, 1 / 4, 1.0], dtype=torch.float32)
+    d["q_raw"][1, 0, 2] = 0  # a zero query
+    x = {n: d[n][:, 0].contiguous().cuda() for n in RAW}
+    S = d["S0"].clone().cuda()
+    o = g.gdn2_decode_step_raw(*(x[n] for n in RAW), S, decay_scale=d["decay_scale"].cuda())
+    torch.cuda.synchronize()
+    a = _act({n: d[n][:, 0] for n in RAW}, d["decay_scale"].numpy())
+    o_ref, S_ref = oracle.decode_step(a["q"], a["k"], a["v"], a["log_alpha"], a["b"], a["w"], gi.as_f64(d["S0"]))
+    assert rel_err(o.cpu().numpy(), o_ref) <= TOL[dtype]
+    assert rel_err(S.cpu().numpy(), S_ref) <= TOL[dtype]
+    assert torch.count_nonzero(o[1, 2].cpu()) == 0
+
+
+def test_decode_raw_steps_equal_chunk_forward_raw():
+    d = gi.raw_inputs(dataclasses.replace(BASE, state_std=0.05), B=2, T=70, H=2)
+    o_c, S_c = _run(d)
+    x = {n: d[n].cuda() for n in RAW}
+    S = d["S0"].clone().cuda()
+    outs = [g.gdn2_decode_step_raw(*(x[n][:, t].contiguous() for n in RAW), S,
+                                   decay_scale=d["decay_scale"].cuda()) for t in range(70)]
+    od = torch.stack(outs, 1)
+    torch.cuda.synchronize()
+    assert rel_err(od.cpu().numpy(), o_c.cpu().numpy()) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), S_c.cpu().numpy()) <= TOL["bf16"]
