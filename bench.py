@@ -270,6 +270,34 @@ def time_conv(args, dev):
                 ok=g.gdn2_device_status() == 0)
 
 
+def time_long(args, dev):
+    """The long-context workload (B1 H16 T65536: 16 (batch, head) units for 148 SMs), plain
+    and with the sequence split at the library's segment count."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    wl = gi.WORKLOADS["long_b1_h16_t65536"]
+    d = gi.prefill_inputs(wl)
+    x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=torch.float32, device=dev)
+    S_T = torch.empty((wl.B, wl.H, wl.dk, wl.dv), dtype=torch.float32, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    P = g.lib().gdn2_chunk_fwd_split_segments(wl.B, wl.T, wl.H, sms)
+    ws = torch.empty(max(1, g.lib().gdn2_chunk_fwd_split_workspace_bytes(wl.B, wl.H, wl.dk, wl.dv, P)),
+                     dtype=torch.uint8, device=dev)
+    args_t = [x[n] for n in ("q", "k", "v", "log_alpha", "b", "w")]
+
+    def plain():
+        g.gdn2_chunk_fwd(*args_t, None, o=o, S_T=S_T)
+
+    def split():
+        g.gdn2_chunk_fwd_split(*args_t, None, segments=P, workspace=ws, o=o, S_T=S_T)
+
+    ms_plain = _time_loop(plain, max(3, args.steps // 4), args.warmup)
+    ms_split = _time_loop(split, max(3, args.steps // 4), args.warmup)
+    return dict(ms_plain=ms_plain, ms_split=ms_split, P=P, tokens=wl.B * wl.T, token_heads=wl.B * wl.T * wl.H,
+                ok=g.gdn2_device_status() == 0)
+
+
 def time_raw(args, dev):
     """The prefill workload fed with raw projections (activations inside the kernel)."""
     import torch
@@ -450,6 +478,8 @@ def main():
     pak = time_packed(args, dev)
     raw = time_raw(args, dev)
     cv = time_conv(args, dev)
+    lg = time_long(args, dev)
+    lg_gbs = lg["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (lg["ms_split"] * 1e-3) / 1e9
     cv_gbs = cv["bytes"] / (cv["ms"] * 1e-3) / 1e9
     raw_gbs = raw["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (raw["ms"] * 1e-3) / 1e9
     # algorithmic bytes: the token streams plus each sequence's entering and final state
@@ -507,6 +537,14 @@ def main():
                 "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (raw)", "achieved": raw_gbs,
                              "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": raw_gbs / pk["hbm_gbs"],
                              "traffic": None}},
+        "long": {"metric": "GDN-2 prefill tokens/s per layer, long context", "value": lg["tokens"] / (lg["ms_split"] * 1e-3),
+                 "unit": "tokens/s", "ms_per_step": lg["ms_split"], "segments": lg["P"],
+                 "unsplit_ms_per_step": lg["ms_plain"],
+                 "workload": "long_b1_h16_t65536 (B=1 H=16 T=65536, heavy decay tail) through "
+                             "gdn2_chunk_fwd_split at the library's segment count",
+                 "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (split)", "achieved": lg_gbs,
+                              "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": lg_gbs / pk["hbm_gbs"],
+                              "traffic": None}},
         "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
                  "steps": args.steps,
                  "workload": f"q, k, v projections of prefill_b8_h16_t4096 side by side: [8, 4096, {cv['C']}] bf16, "
@@ -516,7 +554,8 @@ def main():
                               "traffic": None}},
         "gpu_launches": args.steps,
         "clocks": pre["clocks"],
-        "device_status_ok": bool(pre["ok"] and dec["ok"] and dec_raw["ok"] and pak["ok"] and raw["ok"] and cv["ok"]),
+        "device_status_ok": bool(pre["ok"] and dec["ok"] and dec_raw["ok"] and pak["ok"] and raw["ok"] and cv["ok"]
+                                 and lg["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)

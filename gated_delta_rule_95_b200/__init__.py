@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -55,6 +55,12 @@ def lib():
         P, I = ctypes.c_void_p, ctypes.c_int
         L.gdn2_chunk_fwd.argtypes = [P] * 9 + [I] * 6 + [P]
         L.gdn2_chunk_fwd.restype = I
+        L.gdn2_chunk_fwd_split.argtypes = [P] * 9 + [I] * 7 + [P, ctypes.c_size_t, P]
+        L.gdn2_chunk_fwd_split.restype = I
+        L.gdn2_chunk_fwd_split_segments.argtypes = [I] * 4
+        L.gdn2_chunk_fwd_split_segments.restype = I
+        L.gdn2_chunk_fwd_split_workspace_bytes.argtypes = [I] * 5
+        L.gdn2_chunk_fwd_split_workspace_bytes.restype = ctypes.c_size_t
         L.gdn2_chunk_fwd_varlen.argtypes = [P] * 10 + [I] * 6 + [P]
         L.gdn2_chunk_fwd_varlen.restype = I
         L.gdn2_chunk_fwd_raw.argtypes = [P] * 11 + [I] * 6 + [P]
@@ -119,6 +125,42 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_
                               _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd", rc)
+    return o, S_T
+
+
+def gdn2_chunk_fwd_split(q, k, v, log_alpha, b, w, S0=None, *, segments=None, workspace=None, o=None, S_T=None,
+                         want_state=True, stream=None):
+    """Chunkwise prefill forward with each sequence split into ``segments`` parallel segments
+    (bf16, d_k = d_v).  segments=None takes the library's choice for this device's SM count;
+    workspace (a uint8 CUDA tensor of at least gdn2_chunk_fwd_split_workspace_bytes) is
+    allocated when not given.  Returns (o [B,T,H,d_v], S_T [B,H,d_k,d_v] or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise ValueError("gdn2_chunk_fwd_split: bf16 inputs only")
+    L = lib()
+    if segments is None:
+        sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+        segments = L.gdn2_chunk_fwd_split_segments(B, T, H, sms)
+    need = L.gdn2_chunk_fwd_split_workspace_bytes(B, H, dk, dv, segments)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ts = dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, o=o)
+    if S0 is not None:
+        ts["S0"] = S0
+    if S_T is not None:
+        ts["S_T"] = S_T
+    _check_tokens("gdn2_chunk_fwd_split", ts, q.dtype, q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = L.gdn2_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                                _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], segments, _ptr(workspace), wbytes,
+                                _stream(q.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_chunk_fwd_split", rc)
     return o, S_T
 
 

@@ -77,6 +77,55 @@ extern "C" gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* 
   return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
 }
 
+extern "C" int gdn2_chunk_fwd_split_segments(int B, int T, int H, int sm_count) {
+  // waves of one CTA per SM: the first pass runs (2P - 1) B H segment runs, the last
+  // (P - 1) B H, each of ceil(chunks / P) chunks; one pass of B H full runs without a split
+  if (B <= 0 || T <= 0 || H <= 0 || sm_count <= 0) return 1;
+  const long long bh = (long long)B * H, nch = (T + 63) / 64, sms = sm_count;
+  auto waves = [&](long long units) { return (units + sms - 1) / sms; };
+  long long best = waves(bh) * nch;
+  int best_p = 1;
+  for (int P = 2; P <= 64 && P <= nch; ++P) {
+    const long long len = (nch + P - 1) / P;
+    const long long est = (waves(bh * (2 * P - 1)) + waves(bh * (P - 1))) * len + 1;  // + the chaining
+    if (est < best) {
+      best = est;
+      best_p = P;
+    }
+  }
+  return best_p;
+}
+
+extern "C" size_t gdn2_chunk_fwd_split_workspace_bytes(int B, int H, int d_k, int d_v, int segments) {
+  if (B <= 0 || H <= 0 || segments <= 1 || !head_dim_ok(d_k) || !head_dim_ok(d_v)) return 0;
+  return (size_t)3 * B * H * segments * d_k * d_v * sizeof(float);
+}
+
+extern "C" gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const void* v, const float* log_alpha,
+                                            const void* b, const void* w, const float* S0, float* o, float* S_T,
+                                            int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, int segments,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (dt != GDN2_BF16) return GDN2_ERR_DTYPE;  // the tensor-core path only
+  if (!sizes_ok(B, T, H, d_k, d_v) || d_k != d_v || segments < 1 || segments > 4096) return GDN2_ERR_SHAPE;
+  const bool tokens = (long long)B * T * H > 0;
+  if (tokens && (!q || !k || !v || !log_alpha || !b || !w || !o)) return GDN2_ERR_NULL;
+  if (segments > 1 && !workspace) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, b, w, S0, o, S_T, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if (segments > 1 && workspace_bytes < gdn2_chunk_fwd_split_workspace_bytes(B, H, d_k, d_v, segments))
+    return GDN2_ERR_SHAPE;
+  if ((long long)B * H == 0) return GDN2_OK;
+
+  ChunkArgs a{q, k, v, b, w, log_alpha, S0, o, S_T, B, T, H, d_k, d_v, true};
+  a.split = segments;
+  a.workspace = static_cast<float*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (T == 0) ? launch_state_copy(a, st) : launch_chunk_fwd_tc(a, st);
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
 extern "C" gdn2_status gdn2_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* log_alpha,
                                              const void* b, const void* w, const int* cu_seqlens, const float* S0,
                                              float* o, float* S_T, int N, int T, int H, int d_k, int d_v,

@@ -124,6 +124,12 @@ struct TcParams {
   const int* cu_seqlens;  // packed sequences: [N + 1] token offsets (device); NULL = fixed length T
   int nseq;               // packed sequences: N
   const float* dscale;    // raw projections: per-head decay scale s_h (NULL = 1)
+  // Sequence split (fixed-length batches): 0 = off; 1 = first pass (segment 0 from S0, and
+  // for every later segment its transition M and offset N); 3 = last pass (segments >= 1
+  // from their start states).  split_L: tokens per segment (a multiple of C); split_P:
+  // segments; ws: workspace [3][B H][P][d_k d_v] fp32 (M, N, start states).
+  int split_phase = 0, split_P = 0, split_L = 0;
+  float* ws = nullptr;
   unsigned* err;
 };
 
@@ -163,8 +169,9 @@ __device__ __forceinline__ void st2_tf32(unsigned char* p, const float2& f) {
 // sequences of T tokens.  PREP: the inputs are the raw projections, and the kernel applies
 // the layer's input activations itself: q and k L2-normalised per token, b = sigmoid(b),
 // w = sigmoid(w), log alpha = -s_h softplus(a) (Gated DeltaNet-2 guide, "Decoupled Erase and
-// Write Gates" and "Normalization and Short Convolutions").
-template <int DK, int DV, bool VARLEN, bool PREP>
+// Write Gates" and "Normalization and Short Convolutions").  SPLIT: one pass of the sequence
+// split (fixed-length batches, d_k = d_v), below.
+template <int DK, int DV, bool VARLEN, bool PREP, bool SPLIT>
 __global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
@@ -179,10 +186,33 @@ __global__ void __launch_bounds__(NT, 1)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int ch = tid & 127;  // channel (key i and value j) and tensor-memory lane
   const int sg = tid >> 7;   // token segment [16 sg, 16 sg + 16); column group of TMEM accesses
-  const int unit = blockIdx.x, h = unit % p.H;
+  const int unit = blockIdx.x;
+  int h = unit % p.H;
   // this CTA's sequence: batch coordinate bb, first token t0, length len, chunk count nch,
   // and su, the (sequence, head) index of its entering and final state
   int bb = unit / p.H, t0 = 0, len = p.T, su = unit;
+  const size_t st_sz = (size_t)DK * DV;
+  // Sequence split of a long sequence (SPLIT): segment s covers tokens [s L, s L + L).  By
+  // the recurrence's linearity in (S, v), the state after segment s is M_s S + N_s, with
+  // M_s the state reached from S = I with v = 0 (d_k = d_v) and N_s the one reached from
+  // S = 0; the host chains them between the passes.  First pass (phase 1): r = 0 runs
+  // segment 0 from S0, r in [1, P) gives N_r, r in [P, 2P - 1) gives M_{r-P+1}; last pass
+  // (phase 3): segment r + 1 from its start state.
+  int sp_r = 0, sp_seg = 0;
+  if constexpr (SPLIT) {
+    const int BH = p.nseq;
+    const int bh = unit % BH;
+    sp_r = unit / BH;
+    h = bh % p.H;
+    bb = bh / p.H;
+    su = bh;
+    sp_seg = p.split_phase == 1 ? (sp_r < p.split_P ? sp_r : sp_r - p.split_P + 1) : sp_r + 1;
+    t0 = sp_seg * p.split_L;
+    len = min(p.split_L, p.T - t0);
+  }
+  const bool sp_first = SPLIT && p.split_phase == 1;
+  const bool write_o = !SPLIT || !sp_first || sp_r == 0;          // outputs written
+  const bool sp_trans = SPLIT && sp_first && sp_r >= p.split_P;  // M_s: from I, no write term
   if constexpr (VARLEN) {
     int n = unit / p.H;
     if (p.nseq <= LPT_MAX_SEQ) {
@@ -393,7 +423,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (nch > 0) issue_la(0);
       for (int c = 0; c < nch; ++c) {
         if (!(alive = wait_on(&ms.bar_stage, ph_stage))) break;
-        if (c > 0) {
+        if (c > 0 && write_o) {
           store_o(c - 1);
           bulk_wait_read_all();
         }
@@ -403,7 +433,7 @@ __global__ void __launch_bounds__(NT, 1)
       // the last chunk's output, staged by the compute warps (a packed sequence's partial last
       // chunk is written by the compute warps themselves: its box would spill into the next
       // sequence's rows)
-      if (alive && nch > 0 && wait_on(&ms.bar_stage, ph_stage) && !(VARLEN && len % C)) store_o(nch - 1);
+      if (alive && nch > 0 && wait_on(&ms.bar_stage, ph_stage) && !(VARLEN && len % C) && write_o) store_o(nch - 1);
       if (ms.abort && n_la > 0) {  // the last copy lands before the block releases its memory
         volatile int never = 0;
         mbar_wait_bounded(&ms.bar_la, (uint32_t)((n_la - 1) & 1), &never, nullptr, WAIT_LIMIT);
@@ -416,12 +446,18 @@ __global__ void __launch_bounds__(NT, 1)
     // entering state S0 -> S^T in tensor memory: lane j = ch (a value channel), key-channel
     // columns [32 sg, 32 sg + 32)
     {
+      // (split: segment 0 from S0, N_s from zero, M_s from I, the last pass from the start
+      // states of the workspace)
+      const float* S0u = p.S0 ? p.S0 + (size_t)su * st_sz : nullptr;
+      if (SPLIT && (sp_first ? sp_r > 0 : true))
+        S0u = sp_first ? nullptr : p.ws + (2 * (size_t)p.nseq * p.split_P + (size_t)su * p.split_P + sp_seg) * st_sz;
       float v[32];
-      const bool ok = p.S0 && vval;
+      const bool ok = S0u && vval;
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
         const int i = 32 * sg + x;
-        v[x] = (ok && i < dk) ? p.S0[((size_t)su * dk + i) * dv + ch] : 0.f;
+        v[x] = (ok && i < dk) ? S0u[(size_t)i * dv + ch] : 0.f;
+        if (sp_trans) v[x] = (i == ch && vval) ? 1.f : 0.f;
       }
       tmem_st32(tlane + TM_S + 32 * sg, v);
       tmem_st_wait();
@@ -481,7 +517,7 @@ __global__ void __launch_bounds__(NT, 1)
         const bool tv = !VARLEN || C * cc + 32 * hf + r < len;
         float wr = bf16_at(sm + RAW_W + ro);
         if constexpr (PREP) wr = sigmoid_fast(wr);
-        vw[r] = (vval && tv) ? bf16_at(sm + RAW_V + ro) * wr : 0.f;
+        vw[r] = (vval && tv && !sp_trans) ? bf16_at(sm + RAW_V + ro) * wr : 0.f;
       }
       tmem_st32(tlane + TM_VW + 64 * (cc & 1) + 32 * hf, vw);
       tmem_st_wait();
@@ -896,14 +932,24 @@ __global__ void __launch_bounds__(NT, 1)
       warp_arrive(&ms.bar_stage);
     }
     // the final state (for an empty sequence: the entering one)
-    if (!dead && p.S_T && vval) {
+    // (split: the end of segment 0 starts segment 1, N_s and M_s go to the workspace, the
+    // last pass writes S_T from the last segment only)
+    float* STu = p.S_T ? p.S_T + (size_t)su * st_sz : nullptr;
+    if constexpr (SPLIT) {
+      const size_t blk = (size_t)p.nseq * p.split_P * st_sz, at = ((size_t)su * p.split_P + sp_seg) * st_sz;
+      if (sp_first)
+        STu = sp_r == 0 ? p.ws + 2 * blk + at + st_sz : (sp_trans ? p.ws + at : p.ws + blk + at);
+      else if (sp_seg != p.split_P - 1)
+        STu = nullptr;
+    }
+    if (!dead && STu && vval) {
       tc_fence_after();
       float v[32];
       tmem_ld32(tlane + TM_S + 32 * sg, v);
       tmem_ld_wait();
 #pragma unroll
       for (int x = 0; x < 32; ++x)
-        if (32 * sg + x < dk) p.S_T[((size_t)su * dk + 32 * sg + x) * dv + ch] = v[x];
+        if (32 * sg + x < dk) STu[(size_t)(32 * sg + x) * dv + ch] = v[x];
     }
   }
   // ---- teardown ---------------------------------------------------------------------------
@@ -911,6 +957,50 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+// Between the passes of the sequence split: start states S(s + 1) = M_s S(s) + N_s for
+// s = 1 .. P - 2 of every (batch, head), S(1) being the first pass's end of segment 0.  One
+// CTA per (batch, head, 16 value columns) walks the segments with the running state's
+// column slice in shared memory and M_s staged there row by row (rows padded by one
+// float so that the 16 rows a warp reads fall in 16 banks); fp32 throughout.
+template <int D>
+__global__ void __launch_bounds__(256) split_chain_kernel(float* __restrict__ ws, int BH, int P) {
+  constexpr int CPT = D / 16;      // value columns per thread
+  constexpr int GROUPS = 16 / CPT;  // threads per row
+  extern __shared__ float chain_sm[];
+  float* Ms = chain_sm;                // D x (D + 1)
+  float* Ss = chain_sm + D * (D + 1);  // D x 16
+  const int bh = blockIdx.x / (D / 16), j0 = 16 * (blockIdx.x % (D / 16));
+  const size_t st = (size_t)D * D;
+  const float* M = ws;
+  const float* N = ws + (size_t)BH * P * st;
+  float* S = ws + 2 * (size_t)BH * P * st;
+  const int tid = threadIdx.x, row = tid / GROUPS, jc = CPT * (tid % GROUPS);
+  for (int e = tid; e < D * 16; e += 256)
+    Ss[e] = S[((size_t)bh * P + 1) * st + (size_t)(e / 16) * D + j0 + e % 16];
+  for (int sgm = 1; sgm + 1 < P; ++sgm) {
+    const float* Mg = M + ((size_t)bh * P + sgm) * st;
+    for (int e = tid; e < D * D; e += 256) Ms[(e / D) * (D + 1) + e % D] = Mg[e];
+    __syncthreads();
+    const float* Ng = N + ((size_t)bh * P + sgm) * st + (size_t)row * D + j0 + jc;
+    float acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = Ng[c];
+    for (int i = 0; i < D; ++i) {
+      const float m = Ms[row * (D + 1) + i];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) acc[c] = fmaf(m, Ss[i * 16 + jc + c], acc[c]);
+    }
+    __syncthreads();  // every read of the slice and of M_s is done
+    float* Sg = S + ((size_t)bh * P + sgm + 1) * st + (size_t)row * D + j0 + jc;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      Ss[row * 16 + jc + c] = acc[c];
+      Sg[c] = acc[c];
+    }
+    __syncthreads();
+  }
 }
 
 // ---- host side ------------------------------------------------------------------------------
@@ -941,18 +1031,18 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
   return r == CUDA_SUCCESS;
 }
 
-template <int DK, int DV, bool VARLEN, bool PREP>
+template <int DK, int DV, bool VARLEN, bool PREP, bool SPLIT = false>
 cudaError_t launch_shape(int grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
                          const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw, const CUtensorMap& mla,
                          const CUtensorMap& mo, const TcParams& p) {
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
+  chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP, SPLIT><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
   return cudaSuccess;
 }
 
@@ -967,6 +1057,47 @@ cudaError_t launch_dims(int grid, cudaStream_t st, const CUtensorMap& mq, const 
   if (p.dk == 64 && p.dv == 128) return launch_shape<64, 128, VARLEN, PREP>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
   if (p.dk == 64 && p.dv == 64) return launch_shape<64, 64, VARLEN, PREP>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_split(const ChunkArgs& a, TcParams p, cudaStream_t st, const CUtensorMap& mq,
+                         const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw,
+                         const CUtensorMap& mla, const CUtensorMap& mo) {
+  const int nch = (a.T + C - 1) / C;
+  const int L = C * ((nch + a.split - 1) / a.split);  // tokens per segment
+  const int P = (a.T + L - 1) / L;                      // segments actually used (<= a.split)
+  const int BH = a.B * a.H;
+  if (P < 2) return launch_dims<false, false>(BH, st, mq, mk, mv, mb, mw, mla, mo, p);
+  p.nseq = BH;
+  p.split_P = P;
+  p.split_L = L;
+  p.ws = a.workspace;
+  auto pass = [&](int grid) {  // d_k = d_v
+    return a.dk == 128 ? launch_shape<128, 128, false, false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
+                       : launch_shape<64, 64, false, false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  };
+  p.split_phase = 1;
+  cudaError_t e = pass(BH * (2 * P - 1));
+  if (e != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (P > 2) {
+    const int D = a.dk;
+    const size_t smem = (size_t)(D * (D + 1) + D * 16) * sizeof(float);
+    if (D == 128) {
+      static bool attr = false;
+      if (!attr) {
+        if ((e = cudaFuncSetAttribute(split_chain_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+          return e;
+        attr = true;
+      }
+      split_chain_kernel<128><<<BH * (D / 16), 256, smem, st>>>(a.workspace, BH, P);
+    } else {
+      split_chain_kernel<64><<<BH * (D / 16), 256, smem, st>>>(a.workspace, BH, P);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  p.split_phase = 3;
+  return pass(BH * (P - 1));
 }
 
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
@@ -1005,6 +1136,11 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   const int grid = a.B * a.H;
   p.dscale = a.decay_scale;
   cudaError_t e;
+  if (a.split > 1 && !varlen && !a.raw && a.dk == a.dv) {
+    e = launch_split(a, p, st, mq, mk, mv, mb, mw, mla, mo);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (a.raw)
     e = varlen ? launch_dims<true, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
                : launch_dims<false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);

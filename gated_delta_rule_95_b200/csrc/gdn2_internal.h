@@ -30,6 +30,10 @@ struct ChunkArgs {
   // pre-activation a (log alpha = -s_h softplus(a)); decay_scale: s_h per head (NULL = 1)
   bool raw = false;
   const float* decay_scale = nullptr;
+  // sequence split: segments per sequence (<= 1: off) and the caller's workspace
+  // [3][B H][split][d_k d_v] fp32
+  int split = 0;
+  float* workspace = nullptr;
 };
 
 // Device error word of this library: bits set by kernels, read and cleared by

@@ -36,6 +36,8 @@
 #ifndef GDN2_H
 #define GDN2_H
 
+#include <stddef.h>
+
 #if defined(__GNUC__)
 #define GDN2_API __attribute__((visibility("default")))
 #else
@@ -81,6 +83,37 @@ typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
 GDN2_API gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
                            const void* b, const void* w, const float* S0, float* o, float* S_T,
                            int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, void* stream);
+
+/*
+ * Chunkwise prefill forward with every sequence split into `segments` consecutive
+ * segments that run in parallel: for long sequences with few (batch, head) pairs, which
+ * would otherwise occupy one SM each and leave the rest idle.  The result is
+ * gdn2_chunk_fwd's, up to rounding.
+ *
+ * The recurrence is linear in (state, v) (snilld.dk, "Hvad Gated DeltaNet-2 aendrer":
+ * S_t = (I - k_t (b_t * k_t)^T) D_t S_{t-1} + k_t (w_t * v_t)^T), so the state after
+ * segment s is M_s S + N_s, with M_s = the state reached from S = I with no writes and
+ * N_s = the state reached from S = 0.  A first pass computes segment 0 from S0 and
+ * (M_s, N_s) for every later segment; a small kernel chains the start states
+ * S(s+1) = M_s S(s) + N_s; a last pass recomputes segments 1 .. P-1 from their start
+ * states, writing o and, for the last segment, S_T.  This is the exchange step of a
+ * sequence-parallel prefill done within one GPU; it costs about 3x the work of the
+ * segments it splits, in exchange for P times the parallelism.
+ *
+ *   q .. S_T, B, T, H, dt : as gdn2_chunk_fwd; d_k = d_v required; dt = GDN2_BF16
+ *   segments              : >= 1 (1 = gdn2_chunk_fwd); gdn2_chunk_fwd_split_segments()
+ *                           gives the count a simple wave model prefers
+ *   workspace             : DEVICE scratch of at least
+ *                           gdn2_chunk_fwd_split_workspace_bytes(B, H, d_k, d_v, segments)
+ *                           bytes, 16-byte aligned, owned by the caller; overwritten; two
+ *                           calls in flight must not share it
+ */
+GDN2_API int gdn2_chunk_fwd_split_segments(int B, int T, int H, int sm_count);
+GDN2_API size_t gdn2_chunk_fwd_split_workspace_bytes(int B, int H, int d_k, int d_v, int segments);
+GDN2_API gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const void* v, const float* log_alpha,
+                                 const void* b, const void* w, const float* S0, float* o, float* S_T, int B,
+                                 int T, int H, int d_k, int d_v, gdn2_dtype dt, int segments, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /*
  * Chunkwise prefill forward over a packed batch of variable-length sequences, each

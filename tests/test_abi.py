@@ -124,6 +124,28 @@ def test_decode_step_raw_validation(kw, status):
     assert decode_raw(**kw) == status
 
 
+def split(q=A, k=A, v=A, la=A, b=A, w=A, S0=None, o=A, ST=None, B=1, T=1000, H=2, dk=128, dv=128, dt=1, seg=4,
+          ws=P(0x40000), wsb=1 << 30):
+    return g.lib().gdn2_chunk_fwd_split(q, k, v, la, b, w, S0, o, ST, B, T, H, dk, dv, dt, seg, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=64), 2), (dict(seg=0), 2), (dict(T=-1), 2), (dict(dt=0), 3), (dict(ws=None), 1),
+    (dict(ws=P(0x40008)), 4), (dict(wsb=1000), 2), (dict(q=None), 1), (dict(B=0), 0),
+])
+def test_chunk_fwd_split_validation(kw, status):
+    assert split(**kw) == status
+
+
+def test_split_segment_model_and_workspace():
+    L = g.lib()
+    assert L.gdn2_chunk_fwd_split_segments(8, 4096, 16, 148) == 1  # 128 units already fill the GPU
+    assert L.gdn2_chunk_fwd_split_segments(1, 65536, 16, 148) > 1
+    assert L.gdn2_chunk_fwd_split_segments(1, 64, 1, 148) == 1  # one chunk cannot be split
+    assert L.gdn2_chunk_fwd_split_workspace_bytes(2, 3, 128, 128, 5) == 3 * 2 * 3 * 5 * 128 * 128 * 4
+    assert L.gdn2_chunk_fwd_split_workspace_bytes(2, 3, 128, 128, 1) == 0
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
