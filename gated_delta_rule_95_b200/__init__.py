@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_static", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -57,6 +57,8 @@ def lib():
         L.gdn2_chunk_fwd.restype = I
         L.gdn2_chunk_fwd_split.argtypes = [P] * 9 + [I] * 7 + [P, ctypes.c_size_t, P]
         L.gdn2_chunk_fwd_split.restype = I
+        L.gdn2_chunk_fwd_split_static.argtypes = [P] * 9 + [I] * 7 + [P]
+        L.gdn2_chunk_fwd_split_static.restype = I
         L.gdn2_chunk_fwd_split_segments.argtypes = [I] * 4
         L.gdn2_chunk_fwd_split_segments.restype = I
         L.gdn2_chunk_fwd_split_workspace_bytes.argtypes = [I] * 5
@@ -161,6 +163,32 @@ def gdn2_chunk_fwd_split(q, k, v, log_alpha, b, w, S0=None, *, segments=None, wo
                                 _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd_split", rc)
+    return o, S_T
+
+
+def gdn2_chunk_fwd_split_static(q, k, v, log_alpha, b, w, S0=None, *, segments, o=None, S_T=None, want_state=True,
+                                stream=None):
+    """gdn2_chunk_fwd_split with the library's fixed 16 MiB device scratch instead of a
+    workspace (the call allocates nothing when o and S_T are given)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise ValueError("gdn2_chunk_fwd_split_static: bf16 inputs only")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ts = dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, o=o)
+    if S0 is not None:
+        ts["S0"] = S0
+    if S_T is not None:
+        ts["S_T"] = S_T
+    _check_tokens("gdn2_chunk_fwd_split_static", ts, q.dtype, q.device)
+    rc = lib().gdn2_chunk_fwd_split_static(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),
+                                           _ptr(o), _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], segments,
+                                           _stream(q.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_chunk_fwd_split_static", rc)
     return o, S_T
 
 

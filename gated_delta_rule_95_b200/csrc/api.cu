@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "gdn2.h"
 #include "gdn2_internal.h"
@@ -124,6 +125,58 @@ extern "C" gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = (T == 0) ? launch_state_copy(a, st) : launch_chunk_fwd_tc(a, st);
   return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
+namespace gdn2 {
+namespace {
+// Scratch of gdn2_chunk_fwd_split_static: a fixed array in the module's device memory,
+// so that the call allocates nothing.  Its address is looked up once per device.
+constexpr size_t kSplitScratchBytes = size_t(16) << 20;  // 16 MiB
+__device__ __align__(256) float g_split_scratch[kSplitScratchBytes / sizeof(float)];
+
+cudaError_t split_scratch_address(float** out) {
+  constexpr int kMaxDev = 64;
+  static float* ptrs[kMaxDev] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_split_scratch);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = static_cast<float*>(p);
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+}  // namespace
+}  // namespace gdn2
+
+extern "C" gdn2_status gdn2_chunk_fwd_split_static(const void* q, const void* k, const void* v,
+                                                   const float* log_alpha, const void* b, const void* w,
+                                                   const float* S0, float* o, float* S_T, int B, int T, int H,
+                                                   int d_k, int d_v, gdn2_dtype dt, int segments, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (!sizes_ok(B, T, H, d_k, d_v) || d_k != d_v || segments < 1 || segments > 4096) return GDN2_ERR_SHAPE;
+  const size_t need = gdn2_chunk_fwd_split_workspace_bytes(B, H, d_k, d_v, segments);
+  if (need > kSplitScratchBytes) return GDN2_ERR_SHAPE;  // beyond the fixed scratch
+  const bool tokens = (long long)B * T * H > 0;
+  if (tokens && (!q || !k || !v || !log_alpha || !b || !w || !o)) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, b, w, S0, o, S_T};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if ((long long)B * H == 0) return GDN2_OK;
+  float* scratch = nullptr;
+  if (need > 0) {
+    cudaError_t e = split_scratch_address(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return gdn2_chunk_fwd_split(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, dt, segments, scratch,
+                              kSplitScratchBytes, stream);
 }
 
 extern "C" gdn2_status gdn2_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* log_alpha,

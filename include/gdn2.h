@@ -116,6 +116,29 @@ GDN2_API gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const vo
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * gdn2_chunk_fwd_split without a caller workspace, for callers that cannot allocate: the
+ * scratch is a fixed 16 MiB array in the library's own device memory (reserved when the
+ * library's module loads).  The Gated DeltaNet-2 pages describe no counterpart of this
+ * entry point; it is an interface convenience over the same kernels.
+ *
+ *   arguments   : as gdn2_chunk_fwd_split, without workspace and workspace_bytes
+ *   limit       : gdn2_chunk_fwd_split_workspace_bytes(B, H, d_k, d_v, segments) must not
+ *                 exceed 16 MiB (e.g. 16 heads x 5 segments at d = 128); larger requests
+ *                 return GDN2_ERR_SHAPE before any work is queued
+ *   first call  : on each device, the first call looks up the scratch's address
+ *                 (cudaGetSymbolAddress, with that device current); make that first call
+ *                 outside any stream capture.  A failed lookup returns GDN2_ERR_CUDA.
+ *   zeroing     : nothing in the scratch needs to start at zero: every value is written
+ *                 before it is read within the call
+ *   concurrency : the scratch is shared by all calls on a device; two calls in flight at
+ *                 the same time (on different streams or host threads) race on it
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_split_static(const void* q, const void* k, const void* v, const float* log_alpha,
+                                        const void* b, const void* w, const float* S0, float* o, float* S_T,
+                                        int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, int segments,
+                                        void* stream);
+
+/*
  * Chunkwise prefill forward over a packed batch of variable-length sequences, each
  * with its own state: the serving case of many independent dialogues or documents
  * whose states are carried between calls (DeltaNet-2 AI architecture guide: the

@@ -137,6 +137,19 @@ def test_chunk_fwd_split_validation(kw, status):
     assert split(**kw) == status
 
 
+def split_static(q=A, k=A, v=A, la=A, b=A, w=A, S0=None, o=A, ST=None, B=1, T=8192, H=16, dk=128, dv=128, dt=1,
+                 seg=5):
+    return g.lib().gdn2_chunk_fwd_split_static(q, k, v, la, b, w, S0, o, ST, B, T, H, dk, dv, dt, seg, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(seg=6), 2), (dict(dk=64), 2), (dict(seg=0), 2), (dict(dt=0), 3), (dict(q=None), 1),
+    (dict(o=M), 4), (dict(B=0), 0),
+])
+def test_chunk_fwd_split_static_validation(kw, status):
+    assert split_static(**kw) == status
+
+
 def test_split_segment_model_and_workspace():
     L = g.lib()
     assert L.gdn2_chunk_fwd_split_segments(8, 4096, 16, 148) == 1  # 128 units already fill the GPU

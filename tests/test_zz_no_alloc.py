@@ -1,0 +1,60 @@
+"""The allocation-free sequence split (fixed device scratch) through the C ABI, against
+the workspace entry point: two calls in a row, and the size limit.  Named to run last."""
+import ctypes
+
+import pytest
+import torch
+
+import gdn2_inputs as gi
+import gated_delta_rule_95_b200 as g
+from tests.parity import TOL, rel_err
+
+pytestmark = pytest.mark.gpu
+NAMES = ("q", "k", "v", "log_alpha", "b", "w")
+GDN2_ERR_SHAPE = 2
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _static_call(x, o, S_T, segments):
+    B, T, H, dk = x["q"].shape
+    dv = x["v"].shape[-1]
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return g.lib().gdn2_chunk_fwd_split_static(*(_ptr(x[n]) for n in NAMES), _ptr(x["S0"]), _ptr(o), _ptr(S_T),
+                                               B, T, H, dk, dv, 1, segments, st)
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_static_scratch_matches_workspace_entry_two_calls(seed):
+    import dataclasses
+    wl = dataclasses.replace(gi.WORKLOADS["prefill_b8_h16_t4096"], state_std=0.05)
+    segments = 5
+    need = g.lib().gdn2_chunk_fwd_split_workspace_bytes(1, 16, 128, 128, segments)
+    assert 0 < need <= 16 << 20
+    outs = []
+    for call in range(2):  # two calls in a row, on different inputs
+        d = gi.prefill_inputs(wl, B=1, T=8192, H=16, seed=seed * 10 + call)
+        x = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+        o = torch.full((1, 8192, 16, 128), float("nan"), device="cuda")
+        S_T = torch.full((1, 16, 128, 128), float("nan"), device="cuda")
+        assert _static_call(x, o, S_T, segments) == 0
+        o_ref, S_ref = g.gdn2_chunk_fwd_split(*(x[n] for n in NAMES), x["S0"], segments=segments)
+        torch.cuda.synchronize()
+        assert g.gdn2_device_status() == 0
+        assert rel_err(o.cpu().numpy(), o_ref.cpu().numpy()) <= TOL["bf16"]
+        assert rel_err(S_T.cpu().numpy(), S_ref.cpu().numpy()) <= TOL["bf16"]
+        outs.append(o)
+    assert not torch.equal(outs[0], outs[1])
+
+
+def test_static_scratch_rejects_sizes_beyond_its_limit():
+    L = g.lib()
+    # 16 heads x 6 segments of 128 x 128 fp32 states, three sets: 18.9 MB > 16 MiB
+    assert L.gdn2_chunk_fwd_split_workspace_bytes(1, 16, 128, 128, 6) > 16 << 20
+    x = {n: torch.zeros((1, 8192, 16, 128), dtype=torch.bfloat16 if n != "log_alpha" else torch.float32,
+                        device="cuda") for n in NAMES}
+    x["S0"] = None
+    o = torch.empty((1, 8192, 16, 128), device="cuda")
+    assert _static_call(x, o, None, 6) == GDN2_ERR_SHAPE
