@@ -9,6 +9,9 @@ this package, and this package imports nothing from the CUDA path.
   update; readout after the update as in the guide's PyTorch loop).
 * ``chunkwise.forward`` re-derives the chunkwise WY form in numpy; it is a
   second, independent route to the same numbers, used to pin chunk invariance.
+* ``backward.backward`` is reverse mode of the token-by-token recurrence (fp64, every
+  state kept), pinned against central finite differences of ``forward``;
+  ``chunkwise.backward`` re-derives it in chunk form (the blueprint of the GPU backward).
 * ``short_conv`` is the layer's 4-tap causal depthwise convolution, a plain loop
   over taps.
 * ``activations`` maps the raw projections to the mixer's inputs (L2-normalised
