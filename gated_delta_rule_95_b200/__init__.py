@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_static", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_bwd", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_static", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -55,6 +55,10 @@ def lib():
         P, I = ctypes.c_void_p, ctypes.c_int
         L.gdn2_chunk_fwd.argtypes = [P] * 9 + [I] * 6 + [P]
         L.gdn2_chunk_fwd.restype = I
+        L.gdn2_chunk_bwd.argtypes = [P] * 16 + [I] * 6 + [P, ctypes.c_size_t, P]
+        L.gdn2_chunk_bwd.restype = I
+        L.gdn2_chunk_bwd_workspace_bytes.argtypes = [I] * 5
+        L.gdn2_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.gdn2_chunk_fwd_split.argtypes = [P] * 9 + [I] * 7 + [P, ctypes.c_size_t, P]
         L.gdn2_chunk_fwd_split.restype = I
         L.gdn2_chunk_fwd_split_static.argtypes = [P] * 9 + [I] * 7 + [P]
@@ -128,6 +132,43 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd", rc)
     return o, S_T
+
+
+def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, *, workspace=None, want_dS0=True, out=None,
+                   stream=None):
+    """Backward of gdn2_chunk_fwd: gradients of L given dO = dL/do [B,T,H,d_v] fp32 and
+    dS_T = dL/dS_T (or None).  Returns dict(dq, dk, dv, dlog_alpha, db, dw: fp32 like the
+    inputs; dS0 [B,H,d_k,d_v] or None).  workspace (uint8 CUDA tensor of at least
+    gdn2_chunk_bwd_workspace_bytes) is allocated when not given."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DT:
+        raise ValueError(f"gdn2_chunk_bwd: unsupported dtype {q.dtype}")
+    L = lib()
+    need = L.gdn2_chunk_bwd_workspace_bytes(B, T, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = out if out is not None else dict(
+        dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+        dv=torch.empty((B, T, H, dv), **f32), dlog_alpha=torch.empty((B, T, H, dk), **f32),
+        db=torch.empty((B, T, H, dk), **f32), dw=torch.empty((B, T, H, dv), **f32),
+        dS0=torch.empty((B, H, dk, dv), **f32) if want_dS0 else None)
+    ts = dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, o=dO)
+    for n, t in (("S0", S0), ("S_T", dS_T)):
+        if t is not None:
+            ts[n] = t
+    _check_tokens("gdn2_chunk_bwd", ts, q.dtype, q.device)
+    for n, t in g.items():
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != q.device):
+            raise ValueError(f"gdn2_chunk_bwd: {n} must be a contiguous fp32 tensor on {q.device}")
+    rc = L.gdn2_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
+                          _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]),
+                          _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), B, T, H, dk, dv, _DT[q.dtype],
+                          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(q.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_chunk_bwd", rc)
+    return g
 
 
 def gdn2_chunk_fwd_split(q, k, v, log_alpha, b, w, S0=None, *, segments=None, workspace=None, o=None, S_T=None,

@@ -179,6 +179,42 @@ extern "C" gdn2_status gdn2_chunk_fwd_split_static(const void* q, const void* k,
                               kSplitScratchBytes, stream);
 }
 
+extern "C" size_t gdn2_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v) {
+  if (!sizes_ok(B, T, H, d_k, d_v)) return 0;
+  return chunk_bwd_workspace_bytes(B, T, H, d_k, d_v);
+}
+
+extern "C" gdn2_status gdn2_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                                      const void* b, const void* w, const float* S0, const float* dO,
+                                      const float* dS_T, float* dq, float* dk, float* dv, float* dlog_alpha,
+                                      float* db, float* dw, float* dS0, int B, int T, int H, int d_k, int d_v,
+                                      gdn2_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (!sizes_ok(B, T, H, d_k, d_v)) return GDN2_ERR_SHAPE;
+  const bool tokens = (long long)B * T * H > 0;
+  if (tokens && (!q || !k || !v || !log_alpha || !b || !w || !dO || !dq || !dk || !dv || !dlog_alpha || !db ||
+                 !dw || !workspace))
+    return GDN2_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk, dv, dlog_alpha, db, dw, dS0, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if (tokens && workspace_bytes < chunk_bwd_workspace_bytes(B, T, H, d_k, d_v)) return GDN2_ERR_SHAPE;
+  if ((long long)B * H == 0) return GDN2_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (T == 0) {  // no tokens: the gradient passes straight to the entering state
+    if (dS0) {
+      const size_t n = (size_t)B * H * d_k * d_v * sizeof(float);
+      e = dS_T ? cudaMemcpyAsync(dS0, dS_T, n, cudaMemcpyDeviceToDevice, st) : cudaMemsetAsync(dS0, 0, n, st);
+    }
+  } else {
+    ChunkBwdArgs a{q, k, v, b, w, log_alpha, S0, dO, dS_T, dq, dk, dv, dlog_alpha, db, dw, dS0,
+                   static_cast<float*>(workspace), B, T, H, d_k, d_v, dt == GDN2_BF16};
+    e = launch_chunk_bwd(a, st);
+  }
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
 extern "C" gdn2_status gdn2_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* log_alpha,
                                              const void* b, const void* w, const int* cu_seqlens, const float* S0,
                                              float* o, float* S_T, int N, int T, int H, int d_k, int d_v,

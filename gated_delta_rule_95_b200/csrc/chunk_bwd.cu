@@ -1,0 +1,504 @@
+// Backward pass of the chunkwise forward: gradients of o and S_T with respect to q, k, v,
+// log alpha, b, w and S0, by reverse mode of the chunk form (Gated DeltaNet-2 guide,
+// "Chunkwise Parallel Algorithm for GPU Training"; WY form with the cumulative decay folded
+// into the factors, snilld.dk, "Hvad betyder det for traening og inferens").  Per chunk,
+// with entering state S, rows = the chunk's tokens, Kb = K*B*Gamma, Qh = Q*Gamma,
+// Kn = K/Gamma, Vw = W*V, A = strictly lower part of Kb Kn^T, P = lower part of Qh Kn^T,
+// T = (I + A)^-1, R = Vw - Kb S, U = T R, O = Qh S + P U, St = S + Kn^T U and
+// S_next = Diag(Gamma_C) St; given dO and dS_next:
+//
+//     dSt = Diag(Gamma_C) dS_next,   dGamma_C = rowsum(dS_next * St)
+//     dU  = P^T dO + Kn dSt,   dR = T^T dU (= dVw),   dP = lower(dO U^T)
+//     dA  = strictly lower part of -T^T (dU R^T) T^T
+//     dKb = -dR S^T + dA Kn,   dKn = U dSt^T + dA^T Kb + dP^T Qh,   dQh = dO S^T + dP Kn
+//     dS  = Qh^T dO + dSt - Kb^T dR
+//
+// and, elementwise, dK = dKb*B*Gamma + dKn/Gamma, dB = dKb*K*Gamma, dQ = dQh*Gamma,
+// dW = dVw*V, dV = dVw*W, dg = dKb*Kb + dQh*Qh - dKn*Kn (+ dGamma_C*Gamma_C on the last
+// row), dlog alpha = reverse cumsum of dg over the chunk.
+//
+// Kernels: chunk_bwd_kernel, one CTA of 256 threads per (batch, head, 32 value columns)
+// (value columns never mix in the recurrence, so dS, U, R and the per-column gradients
+// split by columns; the key-side gradients dKb, dKn, dQh, dGamma_C are sums over the
+// column slices and are accumulated with atomics).  It first sweeps the chunks forward to
+// store each chunk's entering state (its column slice) in the workspace, then sweeps them
+// in reverse.  chunk_bwd_finish_kernel turns the summed dKb, dKn, dQh into dq, dk, db and
+// dlog alpha.  All arithmetic is fp32 on the CUDA cores, operands in shared memory.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "gdn2_internal.h"
+
+namespace gdn2 {
+namespace {
+
+constexpr int BC = 64;        // chunk size
+constexpr int BJ = 32;        // value columns per CTA
+constexpr int BT = 256;       // threads per CTA
+constexpr int LJ = BJ + 1;    // padded row of the [.][BJ] tiles
+constexpr int LC = BC + 1;    // padded row of the [BC][BC] tiles
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T* p);
+template <>
+__device__ __forceinline__ float ldf<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(__ldg(p)); }
+
+// C[M][N] = sum_k fa(m, k) fb(k, n), spread over the 256 threads: thread (tm, tn) owns rows
+// tm*TM .. +TM and columns tn, tn + N/TN, ... (consecutive threads take consecutive
+// columns), handing each result to epi(m, n, value).
+template <int M, int N, int TM, int TN, class FA, class FB, class FE>
+__device__ __forceinline__ void gemm(int K, FA fa, FB fb, FE epi) {
+  constexpr int NC = N / TN;
+  static_assert((M / TM) * NC == BT, "thread tiling must cover the output");
+  const int tn = threadIdx.x % NC, tm = threadIdx.x / NC;
+  float acc[TM][TN];
+#pragma unroll
+  for (int x = 0; x < TM; ++x)
+#pragma unroll
+    for (int y = 0; y < TN; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < K; ++k) {
+    float av[TM], bv[TN];
+#pragma unroll
+    for (int x = 0; x < TM; ++x) av[x] = fa(tm * TM + x, k);
+#pragma unroll
+    for (int y = 0; y < TN; ++y) bv[y] = fb(k, tn + y * NC);
+#pragma unroll
+    for (int x = 0; x < TM; ++x)
+#pragma unroll
+      for (int y = 0; y < TN; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+  }
+#pragma unroll
+  for (int x = 0; x < TM; ++x)
+#pragma unroll
+    for (int y = 0; y < TN; ++y) epi(tm * TM + x, tn + y * NC, acc[x][y]);
+}
+
+template <typename E>
+struct BwdParams {
+  const E *q, *k, *v, *b, *w;
+  const float* la;
+  const float* S0;
+  const float* dO;
+  const float* dST;
+  float *dq, *dk, *db;  // on entry zero; receive the summed dQh, dKb, dKn
+  float *dv, *dw, *dS0;
+  float* states;        // [B H][nch][DK][DV]: each chunk's entering state
+  float* dgc;           // [B H][nch][DK]: dGamma_C, zero on entry
+  int T, H, nch;
+};
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) {
+  constexpr int LK = DK + 1;  // padded row of the [BC][DK] tiles
+  constexpr int NS = DV / BJ;
+  extern __shared__ float sm[];
+  float* Kb = sm;
+  float* Qh = Kb + BC * LK;
+  float* Kn = Qh + BC * LK;
+  float* Sj = Kn + BC * LK;      // [DK][LJ]  entering state, this CTA's columns
+  float* dS = Sj + DK * LJ;      // [DK][LJ]  gradient of the state after the chunk (then before it)
+  float* Tm = dS + DK * LJ;      // [BC][LC]  T
+  float* Pm = Tm + BC * LC;      // [BC][LC]  P, then dP
+  float* X1 = Pm + BC * LC;      // [BC][LC]  A, then dT, then dA
+  float* Rm = X1 + BC * LC;      // [BC][LJ]  R         } together: Y = dT T^T ([BC][LC])
+  float* dU = Rm + BC * LJ;      // [BC][LJ]  dU        }
+  float* Um = dU + BC * LJ;      // [BC][LJ]  U
+  float* dOj = Um + BC * LJ;     // [BC][LJ]  dO
+  float* dR = dOj + BC * LJ;     // [BC][LJ]  dR
+  float* gC = dR + BC * LJ;      // [DK]      Gamma_C
+  float* dgC = gC + DK;          // [DK]      dGamma_C, this CTA's part
+  float* Ym = Rm;
+
+  const int tid = threadIdx.x;
+  const int sl = blockIdx.x % NS, bh = blockIdx.x / NS;
+  const int h = bh % p.H, bb = bh / p.H;
+  const int j0 = sl * BJ;
+  const size_t rowstride = (size_t)p.H;  // tokens are [B][T][H][D]
+  auto tok = [&](int t) { return ((size_t)bb * p.T + t) * rowstride + h; };  // (token, head) index
+
+  // Kb, Kn (and Qh) of chunk c, Gamma_C; rows past the sequence are zero.  The raw inputs
+  // are loaded by all threads (log alpha into the free T, P, A tiles), then thread i < DK
+  // walks the rows of key channel i, summing log alpha, and folds the decay in place.
+  auto build = [&](int c, bool with_q) {
+    const int t0 = c * BC;
+    float* raw_la = Tm;  // [BC][DK] over T, P and A (3 BC LC >= BC DK floats)
+#pragma unroll 4
+    for (int e = tid; e < BC * DK; e += BT) {
+      const int t = e / DK, i = e % DK, tt = t0 + t;
+      float la = 0.f, kk = 0.f, bg = 0.f, qq = 0.f;
+      if (tt < p.T) {
+        const size_t x = tok(tt) * DK + i;
+        la = __ldg(p.la + x);
+        kk = ldf(p.k + x);
+        bg = ldf(p.b + x);
+        if (with_q) qq = ldf(p.q + x);
+      }
+      raw_la[e] = la;
+      Kn[t * LK + i] = kk;
+      Kb[t * LK + i] = bg;
+      if (with_q) Qh[t * LK + i] = qq;
+    }
+    __syncthreads();
+    if (tid < DK) {
+      const int i = tid;
+      float g = 0.f;
+      for (int t = 0; t < BC; ++t) {
+        g += raw_la[t * DK + i];
+        const float G = __expf(g), kk = Kn[t * LK + i];
+        Kb[t * LK + i] *= kk * G;
+        Kn[t * LK + i] = kk / G;
+        if (with_q) Qh[t * LK + i] *= G;
+      }
+      gC[i] = __expf(g);
+    }
+  };
+  // T = (I + A)^-1 from A (strictly lower, in X1) by forward substitution per column: four
+  // threads per column s split each row's dot product.
+  auto solve = [&]() {
+    const int s = tid >> 2, part = tid & 3;
+    for (int t = 0; t < BC; ++t) Tm[t * LC + s] = 0.f;
+    __syncwarp();
+    if (part == 0) Tm[s * LC + s] = 1.f;
+    __syncwarp();
+    for (int t = 1; t < BC; ++t) {
+      float acc = 0.f;
+      if (t > s)
+        for (int r = s + part; r < t; r += 4) acc = fmaf(X1[t * LC + r], Tm[r * LC + s], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (t > s && part == 0) Tm[t * LC + s] = -acc;
+      __syncwarp();
+    }
+  };
+  // R = Vw - Kb S and U = T R for chunk c
+  auto r_and_u = [&](int c) {
+    const int t0 = c * BC;
+    gemm<BC, BJ, 2, 4>(DK, [&](int t, int i) { return Kb[t * LK + i]; }, [&](int i, int j) { return Sj[i * LJ + j]; },
+                       [&](int t, int j, float acc) {
+                         const int tt = t0 + t;
+                         float vw = 0.f;
+                         if (tt < p.T) {
+                           const size_t x = tok(tt) * DV + j0 + j;
+                           vw = ldf(p.w + x) * ldf(p.v + x);
+                         }
+                         Rm[t * LJ + j] = vw - acc;
+                       });
+    __syncthreads();
+    gemm<BC, BJ, 2, 4>(BC, [&](int t, int s) { return Tm[t * LC + s]; }, [&](int s, int j) { return Rm[s * LJ + j]; },
+                       [&](int t, int j, float acc) { Um[t * LJ + j] = acc; });
+  };
+  auto strict_lower_kk = [&](float* dst, const float* Lhs, bool incl_diag) {
+    gemm<BC, BC, 4, 4>(DK, [&](int t, int i) { return Lhs[t * LK + i]; }, [&](int i, int s) { return Kn[s * LK + i]; },
+                       [&](int t, int s, float acc) { dst[t * LC + s] = (s < t || (incl_diag && s == t)) ? acc : 0.f; });
+  };
+
+  // ---- forward sweep: every chunk's entering state -----------------------------------------
+  for (int e = tid; e < DK * BJ; e += BT) {
+    const int i = e / BJ, j = e % BJ;
+    Sj[i * LJ + j] = p.S0 ? p.S0[((size_t)bh * DK + i) * DV + j0 + j] : 0.f;
+  }
+  __syncthreads();
+  for (int c = 0; c < p.nch; ++c) {
+    float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
+    for (int e = tid; e < DK * BJ; e += BT) {
+      const int i = e / BJ, j = e % BJ;
+      st[(size_t)i * DV + j0 + j] = Sj[i * LJ + j];
+    }
+    build(c, false);
+    __syncthreads();
+    strict_lower_kk(X1, Kb, false);
+    __syncthreads();
+    solve();
+    __syncthreads();
+    r_and_u(c);
+    __syncthreads();
+    // S <- Diag(Gamma_C) (S + Kn^T U)
+    gemm<DK, BJ, DK / 32, 4>(BC, [&](int i, int s) { return Kn[s * LK + i]; },
+                             [&](int s, int j) { return Um[s * LJ + j]; },
+                             [&](int i, int j, float acc) { Sj[i * LJ + j] = gC[i] * (Sj[i * LJ + j] + acc); });
+    __syncthreads();
+  }
+
+  // ---- reverse sweep -------------------------------------------------------------------------
+  for (int e = tid; e < DK * BJ; e += BT) {
+    const int i = e / BJ, j = e % BJ;
+    dS[i * LJ + j] = p.dST ? p.dST[((size_t)bh * DK + i) * DV + j0 + j] : 0.f;
+  }
+  __syncthreads();
+  for (int c = p.nch - 1; c >= 0; --c) {
+    const int t0 = c * BC;
+    const float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
+    for (int e = tid; e < DK * BJ; e += BT) {
+      const int i = e / BJ, j = e % BJ;
+      Sj[i * LJ + j] = st[(size_t)i * DV + j0 + j];
+    }
+    for (int e = tid; e < BC * BJ; e += BT) {
+      const int t = e / BJ, j = e % BJ, tt = t0 + t;
+      dOj[t * LJ + j] = tt < p.T ? __ldg(p.dO + tok(tt) * DV + j0 + j) : 0.f;
+    }
+    if (tid < DK) dgC[tid] = 0.f;
+    build(c, true);
+    __syncthreads();
+    strict_lower_kk(X1, Kb, false);  // A
+    strict_lower_kk(Pm, Qh, true);   // P
+    __syncthreads();
+    solve();
+    __syncthreads();
+    r_and_u(c);
+    __syncthreads();
+    // dGamma_C = rowsum(dS_next * (S + Kn^T U)), this CTA's columns
+    gemm<DK, BJ, DK / 32, 4>(BC, [&](int i, int s) { return Kn[s * LK + i]; },
+                             [&](int s, int j) { return Um[s * LJ + j]; }, [&](int i, int j, float acc) {
+                               atomicAdd(&dgC[i], dS[i * LJ + j] * (Sj[i * LJ + j] + acc));
+                             });
+    __syncthreads();
+    if (tid < DK) atomicAdd(p.dgc + ((size_t)bh * p.nch + c) * DK + tid, dgC[tid]);
+    // dSt = Diag(Gamma_C) dS_next, in place
+    for (int e = tid; e < DK * BJ; e += BT) {
+      const int i = e / BJ, j = e % BJ;
+      dS[i * LJ + j] *= gC[i];
+    }
+    __syncthreads();
+    // dU = P^T dO + Kn dSt
+    gemm<BC, BJ, 2, 4>(BC, [&](int t, int s) { return Pm[s * LC + t]; }, [&](int s, int j) { return dOj[s * LJ + j]; },
+                       [&](int t, int j, float acc) { dU[t * LJ + j] = acc; });
+    gemm<BC, BJ, 2, 4>(DK, [&](int t, int i) { return Kn[t * LK + i]; }, [&](int i, int j) { return dS[i * LJ + j]; },
+                       [&](int t, int j, float acc) { dU[t * LJ + j] += acc; });
+    __syncthreads();
+    // dR = T^T dU (= dVw): dW = dVw * V, dV = dVw * W; dP = lower(dO U^T) over P
+    gemm<BC, BJ, 2, 4>(BC, [&](int t, int s) { return Tm[s * LC + t]; }, [&](int s, int j) { return dU[s * LJ + j]; },
+                       [&](int t, int j, float acc) {
+                         dR[t * LJ + j] = acc;
+                         const int tt = t0 + t;
+                         if (tt < p.T) {
+                           const size_t x = tok(tt) * DV + j0 + j;
+                           p.dw[x] = acc * ldf(p.v + x);
+                           p.dv[x] = acc * ldf(p.w + x);
+                         }
+                       });
+    gemm<BC, BC, 4, 4>(BJ, [&](int t, int j) { return dOj[t * LJ + j]; }, [&](int j, int s) { return Um[s * LJ + j]; },
+                       [&](int t, int s, float acc) { Pm[t * LC + s] = s <= t ? acc : 0.f; });
+    // dT = dU R^T over A
+    gemm<BC, BC, 4, 4>(BJ, [&](int t, int j) { return dU[t * LJ + j]; }, [&](int j, int s) { return Rm[s * LJ + j]; },
+                       [&](int t, int s, float acc) { X1[t * LC + s] = acc; });
+    __syncthreads();
+    // Y = dT T^T over R and dU; then dA = strictly lower part of -T^T Y over dT
+    gemm<BC, BC, 4, 4>(BC, [&](int t, int r) { return X1[t * LC + r]; }, [&](int r, int s) { return Tm[s * LC + r]; },
+                       [&](int t, int s, float acc) { Ym[t * LC + s] = acc; });
+    __syncthreads();
+    gemm<BC, BC, 4, 4>(BC, [&](int t, int r) { return Tm[r * LC + t]; }, [&](int r, int s) { return Ym[r * LC + s]; },
+                       [&](int t, int s, float acc) { X1[t * LC + s] = s < t ? -acc : 0.f; });
+    __syncthreads();
+    // key-side gradients of this CTA's columns, summed over the slices in global memory:
+    //   dKb = -dR S^T + dA Kn,  dKn = U dSt^T + dA^T Kb + dP^T Qh,  dQh = dO S^T + dP Kn
+    {
+      constexpr int TN = DK / 16, NC = 16;  // 64 x DK outputs: 4 rows x TN columns per thread
+      const int tn = tid % NC, tm = tid / NC;
+      float akb[4][TN], akn[4][TN], aqh[4][TN];
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < TN; ++y) akb[x][y] = akn[x][y] = aqh[x][y] = 0.f;
+#pragma unroll 2
+      for (int j = 0; j < BJ; ++j) {
+        float sv[TN], dsv[TN];
+#pragma unroll
+        for (int y = 0; y < TN; ++y) {
+          sv[y] = Sj[(tn + y * NC) * LJ + j];
+          dsv[y] = dS[(tn + y * NC) * LJ + j];
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int t = tm * 4 + x;
+          const float r = dR[t * LJ + j], u = Um[t * LJ + j], o = dOj[t * LJ + j];
+#pragma unroll
+          for (int y = 0; y < TN; ++y) {
+            akb[x][y] = fmaf(-r, sv[y], akb[x][y]);
+            akn[x][y] = fmaf(u, dsv[y], akn[x][y]);
+            aqh[x][y] = fmaf(o, sv[y], aqh[x][y]);
+          }
+        }
+      }
+#pragma unroll 2
+      for (int s = 0; s < BC; ++s) {
+        float knv[TN], kbv[TN], qhv[TN];
+#pragma unroll
+        for (int y = 0; y < TN; ++y) {
+          const int i = tn + y * NC;
+          knv[y] = Kn[s * LK + i];
+          kbv[y] = Kb[s * LK + i];
+          qhv[y] = Qh[s * LK + i];
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int t = tm * 4 + x;
+          const float da = X1[t * LC + s], daT = X1[s * LC + t], dp = Pm[t * LC + s], dpT = Pm[s * LC + t];
+#pragma unroll
+          for (int y = 0; y < TN; ++y) {
+            akb[x][y] = fmaf(da, knv[y], akb[x][y]);
+            akn[x][y] = fmaf(daT, kbv[y], fmaf(dpT, qhv[y], akn[x][y]));
+            aqh[x][y] = fmaf(dp, knv[y], aqh[x][y]);
+          }
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int tt = t0 + tm * 4 + x;
+        if (tt >= p.T) continue;
+#pragma unroll
+        for (int y = 0; y < TN; ++y) {
+          const size_t xi = tok(tt) * DK + tn + y * NC;
+          atomicAdd(p.dk + xi, akb[x][y]);
+          atomicAdd(p.db + xi, akn[x][y]);
+          atomicAdd(p.dq + xi, aqh[x][y]);
+        }
+      }
+    }
+    // dS (before the chunk) = Qh^T dO + dSt - Kb^T dR
+    {
+      constexpr int TM = DK / 32;
+      const int tn = tid % 8, tm = tid / 8;
+      float acc[TM][4];
+#pragma unroll
+      for (int x = 0; x < TM; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = dS[(tm * TM + x) * LJ + tn + 8 * y];
+#pragma unroll 4
+      for (int t = 0; t < BC; ++t) {
+        float qv[TM], kv[TM], ov[4], rv[4];
+#pragma unroll
+        for (int x = 0; x < TM; ++x) {
+          qv[x] = Qh[t * LK + tm * TM + x];
+          kv[x] = Kb[t * LK + tm * TM + x];
+        }
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          ov[y] = dOj[t * LJ + tn + 8 * y];
+          rv[y] = dR[t * LJ + tn + 8 * y];
+        }
+#pragma unroll
+        for (int x = 0; x < TM; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(qv[x], ov[y], fmaf(-kv[x], rv[y], acc[x][y]));
+      }
+      __syncthreads();  // every read of dSt is done
+#pragma unroll
+      for (int x = 0; x < TM; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) dS[(tm * TM + x) * LJ + tn + 8 * y] = acc[x][y];
+    }
+    __syncthreads();
+  }
+  if (p.dS0)
+    for (int e = tid; e < DK * BJ; e += BT) {
+      const int i = e / BJ, j = e % BJ;
+      p.dS0[((size_t)bh * DK + i) * DV + j0 + j] = dS[i * LJ + j];
+    }
+}
+
+// dq, dk, db and dlog alpha from the summed dQh, dKb, dKn (held in dq, dk, db): thread i of
+// CTA (batch, head, chunk) walks the chunk's rows of key channel i.
+template <typename T, int DK>
+__global__ void __launch_bounds__(DK) chunk_bwd_finish_kernel(const BwdParams<T> p, float* dla) {
+  const int i = threadIdx.x;
+  const int c = blockIdx.x % p.nch, bh = blockIdx.x / p.nch;
+  const int h = bh % p.H, bb = bh / p.H;
+  const int t0 = c * BC, n = min(BC, p.T - t0);
+  float G[BC];  // Gamma of each row
+  float g = 0.f;
+#pragma unroll
+  for (int t = 0; t < BC; ++t) {
+    if (t < n) g += __ldg(p.la + (((size_t)bb * p.T + t0 + t) * p.H + h) * DK + i);
+    G[t] = __expf(g);
+  }
+  // the last row of the chunk carries dGamma_C (rows past the sequence decay no further)
+  float run = p.dgc[((size_t)bh * p.nch + c) * DK + i] * G[BC - 1];
+#pragma unroll
+  for (int t = BC - 1; t >= 0; --t) {
+    if (t >= n) continue;
+    const size_t x = (((size_t)bb * p.T + t0 + t) * p.H + h) * DK + i;
+    const float kk = ldf(p.k + x), bg = ldf(p.b + x), qq = ldf(p.q + x);
+    const float dkb = p.dk[x], dkn = p.db[x], dqh = p.dq[x];
+    const float Gt = G[t];
+    run += dkb * kk * bg * Gt + dqh * qq * Gt - dkn * kk / Gt;
+    dla[x] = run;
+    p.dk[x] = dkb * bg * Gt + dkn / Gt;
+    p.db[x] = dkb * kk * Gt;
+    p.dq[x] = dqh * Gt;
+  }
+}
+
+template <int DK>
+constexpr size_t bwd_smem_bytes() {
+  return sizeof(float) * ((size_t)3 * BC * (DK + 1) + 2 * (size_t)DK * LJ + 3 * (size_t)BC * LC +
+                          5 * (size_t)BC * LJ + 2 * DK);
+}
+
+template <typename T, int DK, int DV>
+cudaError_t launch_bwd_t(const ChunkBwdArgs& a, cudaStream_t st) {
+  BwdParams<T> p;
+  p.q = static_cast<const T*>(a.q);
+  p.k = static_cast<const T*>(a.k);
+  p.v = static_cast<const T*>(a.v);
+  p.b = static_cast<const T*>(a.b);
+  p.w = static_cast<const T*>(a.w);
+  p.la = a.log_alpha;
+  p.S0 = a.S0;
+  p.dO = a.dO;
+  p.dST = a.dS_T;
+  p.dq = a.dq;
+  p.dk = a.dk;
+  p.db = a.db;
+  p.dv = a.dv;
+  p.dw = a.dw;
+  p.dS0 = a.dS0;
+  p.T = a.T;
+  p.H = a.H;
+  p.nch = (a.T + BC - 1) / BC;
+  const size_t BH = (size_t)a.B * a.H;
+  p.states = a.workspace;
+  p.dgc = a.workspace + BH * p.nch * DK * DV;
+  const size_t tok = (size_t)a.B * a.T * a.H * DK;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(a.dq, 0, tok * sizeof(float), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(a.dk, 0, tok * sizeof(float), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(a.db, 0, tok * sizeof(float), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(p.dgc, 0, BH * p.nch * DK * sizeof(float), st)) != cudaSuccess) return e;
+  constexpr size_t smem = bwd_smem_bytes<DK>();
+  static bool attr = false;
+  if (!attr) {
+    if ((e = cudaFuncSetAttribute(chunk_bwd_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+      return e;
+    attr = true;
+  }
+  chunk_bwd_kernel<T, DK, DV><<<(unsigned)(BH * (DV / BJ)), BT, smem, st>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  chunk_bwd_finish_kernel<T, DK><<<(unsigned)(BH * p.nch), DK, 0, st>>>(p, a.dlog_alpha);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_bwd_dims(const ChunkBwdArgs& a, cudaStream_t st) {
+  if (a.dk_ == 128 && a.dv_ == 128) return launch_bwd_t<T, 128, 128>(a, st);
+  if (a.dk_ == 128 && a.dv_ == 64) return launch_bwd_t<T, 128, 64>(a, st);
+  if (a.dk_ == 64 && a.dv_ == 128) return launch_bwd_t<T, 64, 128>(a, st);
+  return launch_bwd_t<T, 64, 64>(a, st);
+}
+
+}  // namespace
+
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  const size_t nch = (size_t)(T + BC - 1) / BC, BH = (size_t)B * H;
+  return sizeof(float) * BH * nch * ((size_t)dk * dv + dk);
+}
+
+cudaError_t launch_chunk_bwd(const ChunkBwdArgs& a, cudaStream_t st) {
+  if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
+  return a.bf16 ? launch_bwd_dims<__nv_bfloat16>(a, st) : launch_bwd_dims<float>(a, st);
+}
+
+}  // namespace gdn2

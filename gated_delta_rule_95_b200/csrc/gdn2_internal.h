@@ -44,7 +44,22 @@ enum : unsigned {
 };
 unsigned* device_error_word();
 
-// Short causal convolution (4 taps) over [B, T, C] (or packed [T, C] with cu_seqlens).
+// Backward of the chunkwise forward (gradients fp32; dq, dk, db are zeroed and accumulated).
+struct ChunkBwdArgs {
+  const void *q, *k, *v, *b, *w;
+  const float* log_alpha;
+  const float* S0;
+  const float* dO;
+  const float* dS_T;
+  float *dq, *dk, *dv, *dlog_alpha, *db, *dw, *dS0;
+  float* workspace;  // chunk_bwd_workspace_bytes
+  int B, T, H, dk_, dv_;
+  bool bf16;
+};
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_chunk_bwd(const ChunkBwdArgs& a, cudaStream_t st);
+
+// Short causal (4 taps) over [B, T, C] (or packed [T, C] with cu_seqlens).
 struct ShortConvArgs {
   const void* x;
   const float* weight;    // [C, 4]

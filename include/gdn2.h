@@ -116,6 +116,31 @@ GDN2_API gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const vo
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * Backward of gdn2_chunk_fwd: given dO = dL/do and dS_T = dL/dS_T, the gradients of L with
+ * respect to q, k, v, log_alpha, b, w and S0 (reverse mode of the chunkwise WY form of
+ * the Gated DeltaNet-2 guide's "Chunkwise Parallel Algorithm for GPU Training", the
+ * training-time counterpart of the forward).  The forward's inputs are passed again; the
+ * chunk states are recomputed in fp32.  All arithmetic fp32 (CUDA cores).
+ *
+ *   q .. w, S0, B, T, H, d_k, d_v, dt : as gdn2_chunk_fwd (the forward's inputs)
+ *   dO          : [B, T, H, d_v] fp32
+ *   dS_T        : [B, H, d_k, d_v] fp32, or NULL for zero
+ *   dq, dk, db, dlog_alpha : [B, T, H, d_k] fp32, written
+ *   dv, dw      : [B, T, H, d_v] fp32, written
+ *   dS0         : [B, H, d_k, d_v] fp32, written, or NULL for "not needed"
+ *   workspace   : DEVICE scratch of gdn2_chunk_bwd_workspace_bytes(B, T, H, d_k, d_v)
+ *                 bytes (every chunk's entering state), 16-byte aligned, owned by the
+ *                 caller; two calls in flight must not share it
+ * Gradient buffers must not alias the inputs or each other.
+ */
+GDN2_API size_t gdn2_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v);
+GDN2_API gdn2_status gdn2_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const void* b, const void* w, const float* S0, const float* dO, const float* dS_T,
+                           float* dq, float* dk, float* dv, float* dlog_alpha, float* db, float* dw,
+                           float* dS0, int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
  * gdn2_chunk_fwd_split without a caller workspace, for callers that cannot allocate: the
  * scratch is a fixed 16 MiB array in the library's own device memory (reserved when the
  * library's module loads).  The Gated DeltaNet-2 pages describe no counterpart of this
