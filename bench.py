@@ -41,6 +41,12 @@ PREFILL_FLOP_PER_TOKEN_HEAD = 2 * 64 * (3 * 128 + 2 * 128) + 6 * 128 * 128
 DECODE_STATE_BYTES = 2 * 128 * 128 * 4
 # nominal dense tf32 : bf16 tensor throughput on B200 (1.1 : 2.25 PFLOP/s); the products run in tf32
 TF32_PER_BF16 = 1.1 / 2.25
+# backward: dense matrix-product FLOPs per chunk-head (C = 64, d = 128) of the chunkwise
+# reverse mode including its forward recomputation: 7 products of C^2 d_k, 10 of C d_k d_v,
+# 6 of C^2 d_v and 2 of C^3 multiply-adds
+BWD_FLOP_PER_CHUNK_HEAD = 2 * (7 * 64 * 64 * 128 + 10 * 64 * 128 * 128 + 6 * 64 * 64 * 128 + 2 * 64 ** 3)
+# CUDA-core fp32 peak: 148 SMs x 128 FMA lanes x 2 FLOP x 1.965 GHz
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def peaks():
@@ -298,6 +304,33 @@ def time_long(args, dev):
                 ok=g.gdn2_device_status() == 0)
 
 
+def time_bwd(args, dev):
+    """The backward of the prefill workload (gradients of all inputs and S0 given dO, dS_T)."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    d = gi.prefill_inputs(PREFILL)
+    x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    B, T, H, dk, dv = PREFILL.B, PREFILL.T, PREFILL.H, PREFILL.dk, PREFILL.dv
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(PREFILL.seed)
+    dO = torch.randn((B, T, H, dv), generator=gen, device=dev)
+    dS = torch.randn((B, H, dk, dv), generator=gen, device=dev)
+    ws = torch.empty(g.lib().gdn2_chunk_bwd_workspace_bytes(B, T, H, dk, dv), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+               dv=torch.empty((B, T, H, dv), **f32), dlog_alpha=torch.empty((B, T, H, dk), **f32),
+               db=torch.empty((B, T, H, dk), **f32), dw=torch.empty((B, T, H, dv), **f32),
+               dS0=torch.empty((B, H, dk, dv), **f32))
+    args_t = [x[n] for n in ("q", "k", "v", "log_alpha", "b", "w")]
+
+    def step():
+        g.gdn2_chunk_bwd(*args_t, None, dO, dS, workspace=ws, out=out)
+
+    ms = _time_loop(step, max(3, args.steps // 4), args.warmup)
+    return dict(ms=ms, tokens=B * T, token_heads=B * T * H, chunk_heads=B * H * (T // 64),
+                ok=g.gdn2_device_status() == 0)
+
+
 def time_raw(args, dev):
     """The prefill workload fed with raw projections (activations inside the kernel)."""
     import torch
@@ -479,6 +512,8 @@ def main():
     raw = time_raw(args, dev)
     cv = time_conv(args, dev)
     lg = time_long(args, dev)
+    bw = time_bwd(args, dev)
+    bw_tflops = bw["chunk_heads"] * BWD_FLOP_PER_CHUNK_HEAD / (bw["ms"] * 1e-3) / 1e12
     lg_gbs = lg["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (lg["ms_split"] * 1e-3) / 1e9
     cv_gbs = cv["bytes"] / (cv["ms"] * 1e-3) / 1e9
     raw_gbs = raw["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (raw["ms"] * 1e-3) / 1e9
@@ -545,6 +580,13 @@ def main():
                  "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (split)", "achieved": lg_gbs,
                               "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": lg_gbs / pk["hbm_gbs"],
                               "traffic": None}},
+        "bwd": {"metric": "GDN-2 backward tokens/s per layer", "value": bw["tokens"] / (bw["ms"] * 1e-3),
+                "unit": "tokens/s", "ms_per_step": bw["ms"],
+                "workload": "prefill_b8_h16_t4096 backward: dq, dk, dv, dlog_alpha, db, dw, dS0 from dO and dS_T "
+                            "(fp32 on the CUDA cores)",
+                "roofline": {"bound": "alu", "kernel": "chunk_bwd_kernel", "achieved": bw_tflops,
+                             "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s", "frac": bw_tflops / FP32_FMA_TFLOPS,
+                             "flop_per_chunk_head": BWD_FLOP_PER_CHUNK_HEAD, "traffic": None}},
         "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
                  "steps": args.steps,
                  "workload": f"q, k, v projections of prefill_b8_h16_t4096 side by side: [8, 4096, {cv['C']}] bf16, "
@@ -555,7 +597,7 @@ def main():
         "gpu_launches": args.steps,
         "clocks": pre["clocks"],
         "device_status_ok": bool(pre["ok"] and dec["ok"] and dec_raw["ok"] and pak["ok"] and raw["ok"] and cv["ok"]
-                                 and lg["ok"]),
+                                 and lg["ok"] and bw["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)

@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   auto build = [&](int c, bool with_q) {
     const int t0 = c * BC;
     float* raw_la = Tm;  // [BC][DK] over T, P and A (3 BC LC >= BC DK floats)
-#pragma unroll 4
+#pragma unroll 8
     for (int e = tid; e < BC * DK; e += BT) {
       const int t = e / DK, i = e % DK, tt = t0 + t;
       float la = 0.f, kk = 0.f, bg = 0.f, qq = 0.f;
@@ -149,28 +149,104 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
         g += raw_la[t * DK + i];
         const float G = __expf(g), kk = Kn[t * LK + i];
         Kb[t * LK + i] *= kk * G;
-        Kn[t * LK + i] = kk / G;
+        Kn[t * LK + i] = kk * __expf(-g);
         if (with_q) Qh[t * LK + i] *= G;
       }
       gC[i] = __expf(g);
     }
   };
-  // T = (I + A)^-1 from A (strictly lower, in X1) by forward substitution per column: four
-  // threads per column s split each row's dot product.
+  // the inputs of chunk c into L2 while the current chunk computes (q and dO only for the
+  // reverse sweep): one 128-byte line per thread and row segment
+  auto prefetch = [&](int c, bool rev) {
+    if (c < 0 || c >= p.nch) return;
+    const int t0 = c * BC;
+    constexpr int KL = DK * (int)sizeof(T) / 128, VL = DV * (int)sizeof(T) / 128;  // lines per row
+    constexpr int LL = DK * 4 / 128, OL = DV * 4 / 128;
+    const int nseg = 2 * KL + LL + 2 * VL + (rev ? KL + OL : 0);
+    for (int e = tid; e < BC * nseg; e += BT) {
+      const int t = e % BC, r = e / BC, tt = t0 + t;
+      if (tt >= p.T) continue;
+      const char* a;
+      int m = r;
+      if (m < KL) a = reinterpret_cast<const char*>(p.k + tok(tt) * DK) + 128 * m;
+      else if ((m -= KL) < KL) a = reinterpret_cast<const char*>(p.b + tok(tt) * DK) + 128 * m;
+      else if ((m -= KL) < LL) a = reinterpret_cast<const char*>(p.la + tok(tt) * DK) + 128 * m;
+      else if ((m -= LL) < VL) a = reinterpret_cast<const char*>(p.v + tok(tt) * DV) + 128 * m;
+      else if ((m -= VL) < VL) a = reinterpret_cast<const char*>(p.w + tok(tt) * DV) + 128 * m;
+      else if ((m -= VL) < KL) a = reinterpret_cast<const char*>(p.q + tok(tt) * DK) + 128 * m;
+      else a = reinterpret_cast<const char*>(p.dO + tok(tt) * DV) + 128 * (m - KL);
+      asm volatile("prefetch.global.L2 [%0];" :: "l"(a));
+    }
+  };
+  // T = (I + A)^-1 from A (strictly lower, in X1), by blocks: the 16 x 16 diagonal blocks by
+  // forward substitution (four threads per column split each row's dot product), then the
+  // 2 x 2 block merges T21 = -T22 (A21 T11) at 32 and 64 (products staged in the R tile,
+  // free at this point).
   auto solve = [&]() {
-    const int s = tid >> 2, part = tid & 3;
-    for (int t = 0; t < BC; ++t) Tm[t * LC + s] = 0.f;
-    __syncwarp();
-    if (part == 0) Tm[s * LC + s] = 1.f;
-    __syncwarp();
-    for (int t = 1; t < BC; ++t) {
-      float acc = 0.f;
-      if (t > s)
-        for (int r = s + part; r < t; r += 4) acc = fmaf(X1[t * LC + r], Tm[r * LC + s], acc);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if (t > s && part == 0) Tm[t * LC + s] = -acc;
+    for (int e = tid; e < BC * BC; e += BT) Tm[(e / BC) * LC + e % BC] = 0.f;
+    __syncthreads();
+    {
+      const int s = tid >> 2, part = tid & 3, base = s & ~15;  // a warp's 8 columns share a block
+      if (part == 0) Tm[s * LC + s] = 1.f;
       __syncwarp();
+      for (int t = base + 1; t < base + 16; ++t) {
+        float acc = 0.f;
+        if (t > s)
+          for (int r = s + part; r < t; r += 4) acc = fmaf(X1[t * LC + r], Tm[r * LC + s], acc);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (t > s && part == 0) Tm[t * LC + s] = -acc;
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    float* Xs = Rm;  // [32][LJ]
+    {
+      // 32: blocks q = 0, 1 at offset 32 q; thread: row r of the block, columns c, c + 1
+      const int q = tid >> 7, r = (tid >> 3) & 15, c = 2 * (tid & 7), o = 32 * q;
+      float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const float a = X1[(o + 16 + r) * LC + o + m];
+        x0 = fmaf(a, Tm[(o + m) * LC + o + c], x0);
+        x1 = fmaf(a, Tm[(o + m) * LC + o + c + 1], x1);
+      }
+      Xs[(16 * q + r) * LJ + c] = x0;
+      Xs[(16 * q + r) * LJ + c + 1] = x1;
+      __syncthreads();
+      float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const float t22 = Tm[(o + 16 + r) * LC + o + 16 + m];
+        y0 = fmaf(t22, Xs[(16 * q + m) * LJ + c], y0);
+        y1 = fmaf(t22, Xs[(16 * q + m) * LJ + c + 1], y1);
+      }
+      Tm[(o + 16 + r) * LC + o + c] = -y0;
+      Tm[(o + 16 + r) * LC + o + c + 1] = -y1;
+    }
+    __syncthreads();
+    {
+      // 64: thread: row r of the lower half, columns [4 c4, 4 c4 + 4)
+      const int r = tid >> 3, c4 = 4 * (tid & 7);
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int m = 0; m < 32; ++m) {
+        const float a = X1[(32 + r) * LC + m];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) x[y] = fmaf(a, Tm[m * LC + c4 + y], x[y]);
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y) Xs[r * LJ + c4 + y] = x[y];
+      __syncthreads();
+      float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int m = 0; m < 32; ++m) {
+        const float t22 = Tm[(32 + r) * LC + 32 + m];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) z[y] = fmaf(t22, Xs[m * LJ + c4 + y], z[y]);
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y) Tm[(32 + r) * LC + c4 + y] = -z[y];
     }
   };
   // R = Vw - Kb S and U = T R for chunk c
@@ -202,6 +278,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   }
   __syncthreads();
   for (int c = 0; c < p.nch; ++c) {
+    prefetch(c + 1, false);
     float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
     for (int e = tid; e < DK * BJ; e += BT) {
       const int i = e / BJ, j = e % BJ;
@@ -230,11 +307,14 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   __syncthreads();
   for (int c = p.nch - 1; c >= 0; --c) {
     const int t0 = c * BC;
+    prefetch(c - 1, true);
     const float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
+#pragma unroll
     for (int e = tid; e < DK * BJ; e += BT) {
       const int i = e / BJ, j = e % BJ;
       Sj[i * LJ + j] = st[(size_t)i * DV + j0 + j];
     }
+#pragma unroll
     for (int e = tid; e < BC * BJ; e += BT) {
       const int t = e / BJ, j = e % BJ, tt = t0 + t;
       dOj[t * LJ + j] = tt < p.T ? __ldg(p.dO + tok(tt) * DV + j0 + j) : 0.f;
