@@ -150,6 +150,26 @@ def test_chunk_fwd_split_static_validation(kw, status):
     assert split_static(**kw) == status
 
 
+def bwd(q=A, k=A, v=A, la=A, b=A, w=A, S0=None, dO=A, dST=None, dq=A, dk_=A, dv_=A, dla=A, db=A, dw=A, dS0=None,
+        B=1, T=100, H=2, dk=128, dv=128, dt=1, ws=P(0x40000), wsb=1 << 30):
+    return g.lib().gdn2_chunk_bwd(q, k, v, la, b, w, S0, dO, dST, dq, dk_, dv_, dla, db, dw, dS0, B, T, H, dk, dv, dt,
+                                  ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=96), 2), (dict(T=-1), 2), (dict(dt=5), 3), (dict(dO=None), 1), (dict(ws=None), 1), (dict(dw=None), 1),
+    (dict(dq=M), 4), (dict(ws=P(0x40008)), 4), (dict(wsb=1000), 2), (dict(B=0), 0), (dict(T=0), 0),
+])
+def test_chunk_bwd_validation(kw, status):
+    assert bwd(**kw) == status
+
+
+def test_bwd_workspace_size():
+    L = g.lib()
+    assert L.gdn2_chunk_bwd_workspace_bytes(2, 100, 3, 128, 64) == 4 * 2 * 3 * 2 * (128 * 64 + 128)
+    assert L.gdn2_chunk_bwd_workspace_bytes(2, 100, 3, 96, 64) == 0
+
+
 def test_split_segment_model_and_workspace():
     L = g.lib()
     assert L.gdn2_chunk_fwd_split_segments(8, 4096, 16, 148) == 1  # 128 units already fill the GPU
