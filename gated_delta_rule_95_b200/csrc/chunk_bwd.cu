@@ -38,6 +38,14 @@ constexpr int BT = 256;       // threads per CTA
 constexpr int LJ = BJ + 1;    // padded row of the [.][BJ] tiles
 constexpr int LC = BC + 1;    // padded row of the [BC][BC] tiles
 
+// four consecutive elements (8- or 16-byte aligned) as fp32
+__device__ __forceinline__ float4 ld4f(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 ld4f(const __nv_bfloat16* p) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xFFFF0000u));
+}
+
 template <typename T>
 __device__ __forceinline__ float ldf(const T* p);
 template <>
@@ -125,21 +133,34 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   auto build = [&](int c, bool with_q) {
     const int t0 = c * BC;
     float* raw_la = Tm;  // [BC][DK] over T, P and A (3 BC LC >= BC DK floats)
-#pragma unroll 8
-    for (int e = tid; e < BC * DK; e += BT) {
-      const int t = e / DK, i = e % DK, tt = t0 + t;
-      float la = 0.f, kk = 0.f, bg = 0.f, qq = 0.f;
+    // four consecutive key channels per load, every load of the thread in flight at once
+    constexpr int Q4 = BC * DK / 4 / BT;
+    float4 la4[Q4], k4[Q4], b4[Q4], q4[Q4];
+#pragma unroll
+    for (int m = 0; m < Q4; ++m) {
+      const int e4 = tid + BT * m, t = e4 / (DK / 4), i = 4 * (e4 % (DK / 4)), tt = t0 + t;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      la4[m] = k4[m] = b4[m] = q4[m] = z;
       if (tt < p.T) {
         const size_t x = tok(tt) * DK + i;
-        la = __ldg(p.la + x);
-        kk = ldf(p.k + x);
-        bg = ldf(p.b + x);
-        if (with_q) qq = ldf(p.q + x);
+        la4[m] = ld4f(p.la + x);
+        k4[m] = ld4f(p.k + x);
+        b4[m] = ld4f(p.b + x);
+        if (with_q) q4[m] = ld4f(p.q + x);
       }
-      raw_la[e] = la;
-      Kn[t * LK + i] = kk;
-      Kb[t * LK + i] = bg;
-      if (with_q) Qh[t * LK + i] = qq;
+    }
+#pragma unroll
+    for (int m = 0; m < Q4; ++m) {
+      const int e4 = tid + BT * m, t = e4 / (DK / 4), i = 4 * (e4 % (DK / 4));
+      const float la[4] = {la4[m].x, la4[m].y, la4[m].z, la4[m].w}, kk[4] = {k4[m].x, k4[m].y, k4[m].z, k4[m].w};
+      const float bg[4] = {b4[m].x, b4[m].y, b4[m].z, b4[m].w}, qq[4] = {q4[m].x, q4[m].y, q4[m].z, q4[m].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        raw_la[t * DK + i + u] = la[u];
+        Kn[t * LK + i + u] = kk[u];
+        Kb[t * LK + i + u] = bg[u];
+        if (with_q) Qh[t * LK + i + u] = qq[u];
+      }
     }
     __syncthreads();
     if (tid < DK) {
@@ -309,15 +330,35 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     const int t0 = c * BC;
     prefetch(c - 1, true);
     const float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
+    {
+      constexpr int NSQ = DK * BJ / 4 / BT, NOQ = BC * BJ / 4 / BT;
+      float4 sv[NSQ], ov[NOQ];
 #pragma unroll
-    for (int e = tid; e < DK * BJ; e += BT) {
-      const int i = e / BJ, j = e % BJ;
-      Sj[i * LJ + j] = st[(size_t)i * DV + j0 + j];
-    }
+      for (int m = 0; m < NSQ; ++m) {
+        const int e4 = tid + BT * m, i = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
+        sv[m] = ld4f(st + (size_t)i * DV + j0 + j);
+      }
 #pragma unroll
-    for (int e = tid; e < BC * BJ; e += BT) {
-      const int t = e / BJ, j = e % BJ, tt = t0 + t;
-      dOj[t * LJ + j] = tt < p.T ? __ldg(p.dO + tok(tt) * DV + j0 + j) : 0.f;
+      for (int m = 0; m < NOQ; ++m) {
+        const int e4 = tid + BT * m, t = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4)), tt = t0 + t;
+        ov[m] = tt < p.T ? ld4f(p.dO + tok(tt) * DV + j0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int m = 0; m < NSQ; ++m) {
+        const int e4 = tid + BT * m, i = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
+        Sj[i * LJ + j] = sv[m].x;
+        Sj[i * LJ + j + 1] = sv[m].y;
+        Sj[i * LJ + j + 2] = sv[m].z;
+        Sj[i * LJ + j + 3] = sv[m].w;
+      }
+#pragma unroll
+      for (int m = 0; m < NOQ; ++m) {
+        const int e4 = tid + BT * m, t = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
+        dOj[t * LJ + j] = ov[m].x;
+        dOj[t * LJ + j + 1] = ov[m].y;
+        dOj[t * LJ + j + 2] = ov[m].z;
+        dOj[t * LJ + j + 3] = ov[m].w;
+      }
     }
     if (tid < DK) dgC[tid] = 0.f;
     build(c, true);
