@@ -977,16 +977,37 @@ __global__ void __launch_bounds__(256) split_chain_kernel(float* __restrict__ ws
   const float* N = ws + (size_t)BH * P * st;
   float* S = ws + 2 * (size_t)BH * P * st;
   const int tid = threadIdx.x, row = tid / GROUPS, jc = CPT * (tid % GROUPS);
+  constexpr int NQ = D * D / 4 / 256;  // float4 of M per thread
+  float4 mq[NQ];                       // the next M, in flight while the current one is used
+  auto fetch = [&](int sgm) {
+    const float4* Mg = reinterpret_cast<const float4*>(M + ((size_t)bh * P + sgm) * st);
+#pragma unroll
+    for (int m = 0; m < NQ; ++m) mq[m] = __ldg(Mg + tid + 256 * m);
+  };
+  auto stage = [&]() {
+#pragma unroll
+    for (int m = 0; m < NQ; ++m) {
+      const int e = 4 * (tid + 256 * m), r = e / D, c = e % D;
+      Ms[r * (D + 1) + c] = mq[m].x;
+      Ms[r * (D + 1) + c + 1] = mq[m].y;
+      Ms[r * (D + 1) + c + 2] = mq[m].z;
+      Ms[r * (D + 1) + c + 3] = mq[m].w;
+    }
+  };
   for (int e = tid; e < D * 16; e += 256)
     Ss[e] = S[((size_t)bh * P + 1) * st + (size_t)(e / 16) * D + j0 + e % 16];
+  if (P > 2) {
+    fetch(1);
+    stage();
+  }
+  __syncthreads();
   for (int sgm = 1; sgm + 1 < P; ++sgm) {
-    const float* Mg = M + ((size_t)bh * P + sgm) * st;
-    for (int e = tid; e < D * D; e += 256) Ms[(e / D) * (D + 1) + e % D] = Mg[e];
-    __syncthreads();
+    if (sgm + 2 < P) fetch(sgm + 1);
     const float* Ng = N + ((size_t)bh * P + sgm) * st + (size_t)row * D + j0 + jc;
     float acc[CPT];
 #pragma unroll
     for (int c = 0; c < CPT; ++c) acc[c] = Ng[c];
+#pragma unroll 8
     for (int i = 0; i < D; ++i) {
       const float m = Ms[row * (D + 1) + i];
 #pragma unroll
@@ -999,6 +1020,7 @@ __global__ void __launch_bounds__(256) split_chain_kernel(float* __restrict__ ws
       Ss[row * 16 + jc + c] = acc[c];
       Sg[c] = acc[c];
     }
+    if (sgm + 2 < P) stage();
     __syncthreads();
   }
 }
