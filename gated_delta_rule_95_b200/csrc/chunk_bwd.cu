@@ -96,6 +96,7 @@ struct BwdParams {
   float* states;        // [B H][nch][DK][DV]: each chunk's entering state
   float* dgc;           // [B H][nch][DK]: dGamma_C, zero on entry
   int T, H, nch;
+  int states_given;     // the entering states are already in `states`
 };
 
 template <typename T, int DK, int DV>
@@ -292,13 +293,13 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
                        [&](int t, int s, float acc) { dst[t * LC + s] = (s < t || (incl_diag && s == t)) ? acc : 0.f; });
   };
 
-  // ---- forward sweep: every chunk's entering state -----------------------------------------
-  for (int e = tid; e < DK * BJ; e += BT) {
+  // ---- forward sweep: every chunk's entering state (unless given) ---------------------------
+  for (int e = tid; e < DK * BJ && !p.states_given; e += BT) {
     const int i = e / BJ, j = e % BJ;
     Sj[i * LJ + j] = p.S0 ? p.S0[((size_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
   __syncthreads();
-  for (int c = 0; c < p.nch; ++c) {
+  for (int c = 0; c < p.nch && !p.states_given; ++c) {
     prefetch(c + 1, false);
     float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
     for (int e = tid; e < DK * BJ; e += BT) {
@@ -370,11 +371,40 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     __syncthreads();
     r_and_u(c);
     __syncthreads();
-    // dGamma_C = rowsum(dS_next * (S + Kn^T U)), this CTA's columns
-    gemm<DK, BJ, DK / 32, 4>(BC, [&](int i, int s) { return Kn[s * LK + i]; },
-                             [&](int s, int j) { return Um[s * LJ + j]; }, [&](int i, int j, float acc) {
-                               atomicAdd(&dgC[i], dS[i * LJ + j] * (Sj[i * LJ + j] + acc));
-                             });
+    // dGamma_C = rowsum(dS_next * (S + Kn^T U)), this CTA's columns: thread (row group,
+    // column group) sums its products, then the 8 threads of a row group add theirs
+    {
+      constexpr int TM = DK / 32;
+      const int tn = tid % 8, tm = tid / 8;
+      float acc[TM][4];
+#pragma unroll
+      for (int x = 0; x < TM; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
+      for (int t = 0; t < BC; ++t) {
+        float kv[TM], uv[4];
+#pragma unroll
+        for (int x = 0; x < TM; ++x) kv[x] = Kn[t * LK + tm * TM + x];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) uv[y] = Um[t * LJ + tn + 8 * y];
+#pragma unroll
+        for (int x = 0; x < TM; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(kv[x], uv[y], acc[x][y]);
+      }
+#pragma unroll
+      for (int x = 0; x < TM; ++x) {
+        const int i = tm * TM + x;
+        float r = 0.f;
+#pragma unroll
+        for (int y = 0; y < 4; ++y) r = fmaf(dS[i * LJ + tn + 8 * y], Sj[i * LJ + tn + 8 * y] + acc[x][y], r);
+        r += __shfl_xor_sync(0xffffffffu, r, 1);
+        r += __shfl_xor_sync(0xffffffffu, r, 2);
+        r += __shfl_xor_sync(0xffffffffu, r, 4);
+        if (tn == 0) dgC[i] = r;
+      }
+    }
     __syncthreads();
     if (tid < DK) atomicAdd(p.dgc + ((size_t)bh * p.nch + c) * DK + tid, dgC[tid]);
     // dSt = Diag(Gamma_C) dS_next, in place
@@ -588,6 +618,13 @@ cudaError_t launch_bwd_t(const ChunkBwdArgs& a, cudaStream_t st) {
   if ((e = cudaMemsetAsync(a.dk, 0, tok * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.db, 0, tok * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(p.dgc, 0, BH * p.nch * DK * sizeof(float), st)) != cudaSuccess) return e;
+  // bf16 with d_k = d_v: the entering states from the tensor-core forward's checkpoint phase
+  p.states_given = 0;
+  if (a.bf16 && DK == DV) {
+    ChunkArgs f{a.q, a.k, a.v, a.b, a.w, a.log_alpha, a.S0, nullptr, nullptr, a.B, a.T, a.H, DK, DV, true};
+    if ((e = launch_chunk_states_tc(f, p.states, st)) != cudaSuccess) return e;
+    p.states_given = 1;
+  }
   constexpr size_t smem = bwd_smem_bytes<DK>();
   static bool attr = false;
   if (!attr) {

@@ -197,7 +197,9 @@ __global__ void __launch_bounds__(NT, 1)
   // M_s the state reached from S = I with v = 0 (d_k = d_v) and N_s the one reached from
   // S = 0; the host chains them between the passes.  First pass (phase 1): r = 0 runs
   // segment 0 from S0, r in [1, P) gives N_r, r in [P, 2P - 1) gives M_{r-P+1}; last pass
-  // (phase 3): segment r + 1 from its start state.
+  // (phase 3): segment r + 1 from its start state.  The same instantiation also runs the
+  // whole sequence writing the state entering every chunk to the workspace [B H][chunk]
+  // [d_k][d_v] and no outputs (phase 5, the checkpoints of the backward pass).
   int sp_r = 0, sp_seg = 0;
   if constexpr (SPLIT) {
     const int BH = p.nseq;
@@ -209,9 +211,15 @@ __global__ void __launch_bounds__(NT, 1)
     sp_seg = p.split_phase == 1 ? (sp_r < p.split_P ? sp_r : sp_r - p.split_P + 1) : sp_r + 1;
     t0 = sp_seg * p.split_L;
     len = min(p.split_L, p.T - t0);
+    if (p.split_phase == 5) {
+      sp_seg = 0;
+      t0 = 0;
+      len = p.T;
+    }
   }
   const bool sp_first = SPLIT && p.split_phase == 1;
-  const bool write_o = !SPLIT || !sp_first || sp_r == 0;          // outputs written
+  const bool sp_ckpt = SPLIT && p.split_phase == 5;
+  const bool write_o = !SPLIT || (sp_first ? sp_r == 0 : !sp_ckpt);  // outputs written
   const bool sp_trans = SPLIT && sp_first && sp_r >= p.split_P;  // M_s: from I, no write term
   if constexpr (VARLEN) {
     int n = unit / p.H;
@@ -449,7 +457,7 @@ __global__ void __launch_bounds__(NT, 1)
       // (split: segment 0 from S0, N_s from zero, M_s from I, the last pass from the start
       // states of the workspace)
       const float* S0u = p.S0 ? p.S0 + (size_t)su * st_sz : nullptr;
-      if (SPLIT && (sp_first ? sp_r > 0 : true))
+      if (SPLIT && !sp_ckpt && (sp_first ? sp_r > 0 : true))
         S0u = sp_first ? nullptr : p.ws + (2 * (size_t)p.nseq * p.split_P + (size_t)su * p.split_P + sp_seg) * st_sz;
       float v[32];
       const bool ok = S0u && vval;
@@ -458,6 +466,12 @@ __global__ void __launch_bounds__(NT, 1)
         const int i = 32 * sg + x;
         v[x] = (ok && i < dk) ? S0u[(size_t)i * dv + ch] : 0.f;
         if (sp_trans) v[x] = (i == ch && vval) ? 1.f : 0.f;
+      }
+      if (sp_ckpt && vval && nch > 0) {  // the state entering chunk 0
+        float* ck = p.ws + (size_t)su * nch * st_sz + ch;
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          if (32 * sg + x < dk) ck[(size_t)(32 * sg + x) * dv] = v[x];
       }
       tmem_st32(tlane + TM_S + 32 * sg, v);
       tmem_st_wait();
@@ -470,8 +484,9 @@ __global__ void __launch_bounds__(NT, 1)
     float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);  // block product, 32 x LDX fp32
     const int lane = tid & 31;
     auto wait_mma = [&]() -> bool { return wait_on(&ms.bar_mma, ph_mma); };
-    // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory.
-    auto decay_state = [&](int gb) {
+    // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory (checkpoint
+    // phase: also written out as the state entering chunk cst, if cst >= 0).
+    auto decay_state = [&](int gb, int cst) {
       float v[32];
       tmem_ld32(tlane + TM_S + 32 * sg, v);
       tmem_ld_wait();
@@ -484,6 +499,12 @@ __global__ void __launch_bounds__(NT, 1)
         v[x + 3] *= gq.w;
       }
       tmem_st32(tlane + TM_S + 32 * sg, v);
+      if (sp_ckpt && cst >= 0 && vval) {
+        float* ck = p.ws + ((size_t)su * nch + cst) * st_sz + ch;
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          if (32 * sg + x < dk) ck[(size_t)(32 * sg + x) * dv] = v[x];
+      }
     };
     // Output of the last finished chunk (O^T in tensor memory) into the shared-memory tile
     // [t][j] (rows of d_v floats, over the log-decay tile, whose reads are done) that the
@@ -670,7 +691,7 @@ __global__ void __launch_bounds__(NT, 1)
       // decay ==================================================================================
       if (c > 0) {
         stage_o();
-        decay_state(ob ^ 1);
+        decay_state(ob ^ 1, c);
       }
       tmem_st_wait();
       fence_proxy_async_smem();
@@ -925,7 +946,7 @@ __global__ void __launch_bounds__(NT, 1)
       } else {
         stage_o();
       }
-      decay_state((nch - 1) & 1);
+      decay_state((nch - 1) & 1, -1);
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -937,7 +958,9 @@ __global__ void __launch_bounds__(NT, 1)
     float* STu = p.S_T ? p.S_T + (size_t)su * st_sz : nullptr;
     if constexpr (SPLIT) {
       const size_t blk = (size_t)p.nseq * p.split_P * st_sz, at = ((size_t)su * p.split_P + sp_seg) * st_sz;
-      if (sp_first)
+      if (sp_ckpt)
+        STu = nullptr;
+      else if (sp_first)
         STu = sp_r == 0 ? p.ws + 2 * blk + at + st_sz : (sp_trans ? p.ws + at : p.ws + blk + at);
       else if (sp_seg != p.split_P - 1)
         STu = nullptr;
@@ -1120,6 +1143,52 @@ cudaError_t launch_split(const ChunkArgs& a, TcParams p, cudaStream_t st, const 
   }
   p.split_phase = 3;
   return pass(BH * (P - 1));
+}
+
+// The state entering every chunk ([B H][chunk][d_k][d_v] fp32 at `states`), for the backward
+// pass: the split instantiation's checkpoint phase over whole sequences (bf16, d_k = d_v).
+cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st) {
+  if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
+  if (a.dk != a.dv || !a.bf16) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, mb, mw, mla, mo;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  // o is never written in this phase: the map only needs a valid, aligned address
+  bool ok = make_map(&mq, a.q, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
+            make_map(&mk, a.k, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
+            make_map(&mb, a.b, BF, 2, a.B, a.T, a.H, a.dk, 64, SW) &&
+            make_map(&mv, a.v, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
+            make_map(&mw, a.w, BF, 2, a.B, a.T, a.H, a.dv, 64, SW) &&
+            make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dk, 32, SW) &&
+            make_map(&mo, states, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, a.dv, a.dv,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return cudaErrorInvalidValue;
+  TcParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.k = static_cast<const __nv_bfloat16*>(a.k);
+  p.v = static_cast<const __nv_bfloat16*>(a.v);
+  p.b = static_cast<const __nv_bfloat16*>(a.b);
+  p.w = static_cast<const __nv_bfloat16*>(a.w);
+  p.S0 = a.S0;
+  p.S_T = nullptr;
+  p.o = nullptr;
+  p.T = a.T;
+  p.H = a.H;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.cu_seqlens = nullptr;
+  p.nseq = a.B * a.H;
+  p.dscale = nullptr;
+  p.err = device_error_word();
+  p.split_phase = 5;
+  p.split_P = 1;
+  p.split_L = a.T;
+  p.ws = states;
+  const int grid = a.B * a.H;
+  cudaError_t e = a.dk == 128 ? launch_shape<128, 128, false, false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
+                              : launch_shape<64, 64, false, false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {

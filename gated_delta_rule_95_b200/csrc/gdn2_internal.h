@@ -76,6 +76,8 @@ cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t st);
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
 // bf16 inputs: tcgen05/TMEM kernel fed by TMA.
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st);
+// bf16, d_k = d_v: the state entering every chunk, [B H][chunk][d_k][d_v] fp32 (no outputs).
+cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st);
 // fp32 inputs: fp32 CUDA-core kernel of the same chunkwise algorithm.
 cudaError_t launch_chunk_fwd_f32(const ChunkArgs& a, cudaStream_t st);
 // T = 0: S_T = S0 (or zeros).
