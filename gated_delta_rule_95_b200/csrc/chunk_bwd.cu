@@ -446,8 +446,11 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     // key-side gradients of this CTA's columns, summed over the slices in global memory:
     //   dKb = -dR S^T + dA Kn,  dKn = U dSt^T + dA^T Kb + dP^T Qh,  dQh = dO S^T + dP Kn
     {
-      constexpr int TN = DK / 16, NC = 16;  // 64 x DK outputs: 4 rows x TN columns per thread
+      // 64 x DK outputs: thread (tm, tn) takes rows 4 tm .. +4 and the key channels
+      // 4 tn + 64 g + u (u < 4), so that its sums leave as 16-byte vector atomics
+      constexpr int TN = DK / 16, NC = 16;
       const int tn = tid % NC, tm = tid / NC;
+      auto col = [&](int y) { return 4 * tn + 64 * (y >> 2) + (y & 3); };
       float akb[4][TN], akn[4][TN], aqh[4][TN];
 #pragma unroll
       for (int x = 0; x < 4; ++x)
@@ -458,8 +461,8 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
         float sv[TN], dsv[TN];
 #pragma unroll
         for (int y = 0; y < TN; ++y) {
-          sv[y] = Sj[(tn + y * NC) * LJ + j];
-          dsv[y] = dS[(tn + y * NC) * LJ + j];
+          sv[y] = Sj[col(y) * LJ + j];
+          dsv[y] = dS[col(y) * LJ + j];
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
@@ -478,7 +481,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
         float knv[TN], kbv[TN], qhv[TN];
 #pragma unroll
         for (int y = 0; y < TN; ++y) {
-          const int i = tn + y * NC;
+          const int i = col(y);
           knv[y] = Kn[s * LK + i];
           kbv[y] = Kb[s * LK + i];
           qhv[y] = Qh[s * LK + i];
@@ -500,11 +503,11 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
         const int tt = t0 + tm * 4 + x;
         if (tt >= p.T) continue;
 #pragma unroll
-        for (int y = 0; y < TN; ++y) {
-          const size_t xi = tok(tt) * DK + tn + y * NC;
-          atomicAdd(p.dk + xi, akb[x][y]);
-          atomicAdd(p.db + xi, akn[x][y]);
-          atomicAdd(p.dq + xi, aqh[x][y]);
+        for (int y = 0; y < TN; y += 4) {
+          const size_t xi = tok(tt) * DK + col(y);  // 16-byte aligned
+          atomicAdd(reinterpret_cast<float4*>(p.dk + xi), make_float4(akb[x][y], akb[x][y + 1], akb[x][y + 2], akb[x][y + 3]));
+          atomicAdd(reinterpret_cast<float4*>(p.db + xi), make_float4(akn[x][y], akn[x][y + 1], akn[x][y + 2], akn[x][y + 3]));
+          atomicAdd(reinterpret_cast<float4*>(p.dq + xi), make_float4(aqh[x][y], aqh[x][y + 1], aqh[x][y + 2], aqh[x][y + 3]));
         }
       }
     }
