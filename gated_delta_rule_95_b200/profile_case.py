@@ -2,6 +2,7 @@
 
     python -m gated_delta_rule_95_b200.profile_case --kind prefill --B 8 --H 16 --T 1024 --reps 2
     python -m gated_delta_rule_95_b200.profile_case --kind decode --B 256 --H 16 --reps 4
+    python -m gated_delta_rule_95_b200.profile_case --kind bwd --B 2 --H 16 --T 1024 --reps 2
 
 Inputs follow the recipe of the named workload (gdn2_inputs) with the given
 sizes; it exits 0 after a device synchronisation and a clean device status.
@@ -19,7 +20,7 @@ if ROOT not in sys.path:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", choices=["prefill", "decode"], required=True)
+    ap.add_argument("--kind", choices=["prefill", "decode", "bwd"], required=True)
     ap.add_argument("--workload", default=None)
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--H", type=int, default=None)
@@ -39,6 +40,17 @@ def main():
         x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
         for _ in range(a.reps):
             g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
+    elif a.kind == "bwd":
+        wl = gi.WORKLOADS[a.workload or "prefill_b8_h16_t4096"]
+        d = gi.prefill_inputs(wl, B=a.B, T=a.T, H=a.H)
+        x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+        B, T, H = x["q"].shape[:3]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(wl.seed)
+        dO = torch.randn((B, T, H, wl.dv), generator=gen, device=dev)
+        dS = torch.randn((B, H, wl.dk, wl.dv), generator=gen, device=dev)
+        for _ in range(a.reps):
+            g.gdn2_chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], dO, dS)
     else:
         wl = gi.WORKLOADS[a.workload or "decode_b256_h16"]
         S = gi.decode_state(wl, B=a.B, H=a.H).to(dev)
