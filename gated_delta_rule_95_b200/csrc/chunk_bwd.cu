@@ -27,7 +27,10 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "gdn2_internal.h"
+#include "ptx.cuh"
 
 namespace gdn2 {
 namespace {
@@ -35,8 +38,11 @@ namespace {
 constexpr int BC = 64;        // chunk size
 constexpr int BJ = 32;        // value columns per CTA
 constexpr int BT = 256;       // threads per CTA
-constexpr int LJ = BJ + 1;    // padded row of the [.][BJ] tiles
-constexpr int LC = BC + 1;    // padded row of the [BC][BC] tiles
+// Row padding of the shared-memory tiles: 1 float for the CUDA-core products (whose
+// column-wise reads then meet 32 banks), 4 floats for the tensor-core fragments (the 8 x 4
+// element groups of an mma fragment then meet 32 banks)
+template <bool TC>
+__host__ __device__ constexpr int pad() { return TC ? 4 : 1; }
 
 // four consecutive elements (8- or 16-byte aligned) as fp32
 __device__ __forceinline__ float4 ld4f(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
@@ -84,6 +90,71 @@ __device__ __forceinline__ void gemm(int K, FA fa, FB fb, FE epi) {
     for (int y = 0; y < TN; ++y) epi(tm * TM + x, tn + y * NC, acc[x][y]);
 }
 
+// The same products on the tensor cores (bf16 inputs): mma.sync m16n8k8 with operands
+// rounded to tf32 (nearest), fp32 accumulation.  The 16 x 8 output tiles go to the 8 warps
+// in row-major order, TPW consecutive tiles per warp sharing one 16-row block, so that a
+// warp loads each A fragment once per k step.  d holds the warp's tiles' accumulators.
+__device__ __forceinline__ uint32_t tf32r(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
+
+template <int M, int N>
+struct MT {
+  static constexpr int NT = N / 8, TPW = (M / 16) * NT / 8;
+  static_assert(TPW >= 1 && NT % TPW == 0, "a warp's tiles must share a row block");
+};
+template <int M, int N>
+__device__ __forceinline__ void mzero(float (&d)[MT<M, N>::TPW][4]) {
+#pragma unroll
+  for (int q = 0; q < MT<M, N>::TPW; ++q) d[q][0] = d[q][1] = d[q][2] = d[q][3] = 0.f;
+}
+template <int M, int N, class FA, class FB>
+__device__ __forceinline__ void mmac(float (&d)[MT<M, N>::TPW][4], int K, FA fa, FB fb) {
+  constexpr int NT = MT<M, N>::NT, TPW = MT<M, N>::TPW;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int m0 = (warp * TPW / NT) * 16, nb = (warp * TPW) % NT;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const uint32_t a[4] = {tf32r(fa(m0 + g, k0 + t)), tf32r(fa(m0 + g + 8, k0 + t)), tf32r(fa(m0 + g, k0 + t + 4)),
+                           tf32r(fa(m0 + g + 8, k0 + t + 4))};
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) {
+      const int n0 = 8 * (nb + q);
+      const uint32_t b[2] = {tf32r(fb(k0 + t, n0 + g)), tf32r(fb(k0 + t + 4, n0 + g))};
+      mma_16x8x8_tf32(d[q], a, b);
+    }
+  }
+}
+// epi(m, n, value) for every element of the warp's tiles, and the row/column of element e
+// of tile q
+template <int M, int N, class FE>
+__device__ __forceinline__ void mepi(const float (&d)[MT<M, N>::TPW][4], FE epi) {
+  constexpr int NT = MT<M, N>::NT, TPW = MT<M, N>::TPW;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int m0 = (warp * TPW / NT) * 16, nb = (warp * TPW) % NT;
+#pragma unroll
+  for (int q = 0; q < TPW; ++q) {
+    const int n0 = 8 * (nb + q);
+    epi(m0 + g, n0 + 2 * t, d[q][0]);
+    epi(m0 + g, n0 + 2 * t + 1, d[q][1]);
+    epi(m0 + g + 8, n0 + 2 * t, d[q][2]);
+    epi(m0 + g + 8, n0 + 2 * t + 1, d[q][3]);
+  }
+}
+template <int M, int N, class FA, class FB, class FE>
+__device__ __forceinline__ void mgemm(int K, FA fa, FB fb, FE epi) {
+  float d[MT<M, N>::TPW][4];
+  mzero<M, N>(d);
+  mmac<M, N>(d, K, fa, fb);
+  mepi<M, N>(d, epi);
+}
+// the products of the kernel: tensor cores for bf16 inputs, CUDA-core fp32 for fp32 inputs
+template <bool TC, int M, int N, int TM, int TN, class FA, class FB, class FE>
+__device__ __forceinline__ void prod(int K, FA fa, FB fb, FE epi) {
+  if constexpr (TC)
+    mgemm<M, N>(K, fa, fb, epi);
+  else
+    gemm<M, N, TM, TN>(K, fa, fb, epi);
+}
+
 template <typename E>
 struct BwdParams {
   const E *q, *k, *v, *b, *w;
@@ -101,7 +172,10 @@ struct BwdParams {
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) {
-  constexpr int LK = DK + 1;  // padded row of the [BC][DK] tiles
+  constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;  // products on the tensor cores
+  constexpr int LK = DK + pad<TC>();  // padded rows: [BC][DK] tiles
+  constexpr int LJ = BJ + pad<TC>();  //              [.][BJ] tiles
+  constexpr int LC = BC + pad<TC>();  //              [BC][BC] tiles
   constexpr int NS = DV / BJ;
   extern __shared__ float sm[];
   float* Kb = sm;
@@ -110,16 +184,16 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   float* Sj = Kn + BC * LK;      // [DK][LJ]  entering state, this CTA's columns
   float* dS = Sj + DK * LJ;      // [DK][LJ]  gradient of the state after the chunk (then before it)
   float* Tm = dS + DK * LJ;      // [BC][LC]  T
-  float* Pm = Tm + BC * LC;      // [BC][LC]  P, then dP
+  float* Pm = Tm + BC * LC;      // [BC][LC]  P, then Y = dT T^T, then dP
   float* X1 = Pm + BC * LC;      // [BC][LC]  A, then dT, then dA
-  float* Rm = X1 + BC * LC;      // [BC][LJ]  R         } together: Y = dT T^T ([BC][LC])
-  float* dU = Rm + BC * LJ;      // [BC][LJ]  dU        }
+  float* Rm = X1 + BC * LC;      // [BC][LJ]  R, then dR
+  float* dU = Rm + BC * LJ;      // [BC][LJ]  dGamma_C (first DK floats), then dU
   float* Um = dU + BC * LJ;      // [BC][LJ]  U
   float* dOj = Um + BC * LJ;     // [BC][LJ]  dO
-  float* dR = dOj + BC * LJ;     // [BC][LJ]  dR
-  float* gC = dR + BC * LJ;      // [DK]      Gamma_C
-  float* dgC = gC + DK;          // [DK]      dGamma_C, this CTA's part
-  float* Ym = Rm;
+  float* gC = dOj + BC * LJ;     // [DK]      Gamma_C
+  float* dgC = dU;               // [DK]      dGamma_C, this CTA's part
+  float* Ym = Pm;
+  float* dR = Rm;
 
   const int tid = threadIdx.x;
   const int sl = blockIdx.x % NS, bh = blockIdx.x / NS;
@@ -274,7 +348,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   // R = Vw - Kb S and U = T R for chunk c
   auto r_and_u = [&](int c) {
     const int t0 = c * BC;
-    gemm<BC, BJ, 2, 4>(DK, [&](int t, int i) { return Kb[t * LK + i]; }, [&](int i, int j) { return Sj[i * LJ + j]; },
+    prod<TC, BC, BJ, 2, 4>(DK, [&](int t, int i) { return Kb[t * LK + i]; }, [&](int i, int j) { return Sj[i * LJ + j]; },
                        [&](int t, int j, float acc) {
                          const int tt = t0 + t;
                          float vw = 0.f;
@@ -285,11 +359,11 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
                          Rm[t * LJ + j] = vw - acc;
                        });
     __syncthreads();
-    gemm<BC, BJ, 2, 4>(BC, [&](int t, int s) { return Tm[t * LC + s]; }, [&](int s, int j) { return Rm[s * LJ + j]; },
+    prod<TC, BC, BJ, 2, 4>(BC, [&](int t, int s) { return Tm[t * LC + s]; }, [&](int s, int j) { return Rm[s * LJ + j]; },
                        [&](int t, int j, float acc) { Um[t * LJ + j] = acc; });
   };
   auto strict_lower_kk = [&](float* dst, const float* Lhs, bool incl_diag) {
-    gemm<BC, BC, 4, 4>(DK, [&](int t, int i) { return Lhs[t * LK + i]; }, [&](int i, int s) { return Kn[s * LK + i]; },
+    prod<TC, BC, BC, 4, 4>(DK, [&](int t, int i) { return Lhs[t * LK + i]; }, [&](int i, int s) { return Kn[s * LK + i]; },
                        [&](int t, int s, float acc) { dst[t * LC + s] = (s < t || (incl_diag && s == t)) ? acc : 0.f; });
   };
 
@@ -315,7 +389,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     r_and_u(c);
     __syncthreads();
     // S <- Diag(Gamma_C) (S + Kn^T U)
-    gemm<DK, BJ, DK / 32, 4>(BC, [&](int i, int s) { return Kn[s * LK + i]; },
+    prod<TC, DK, BJ, DK / 32, 4>(BC, [&](int i, int s) { return Kn[s * LK + i]; },
                              [&](int s, int j) { return Um[s * LJ + j]; },
                              [&](int i, int j, float acc) { Sj[i * LJ + j] = gC[i] * (Sj[i * LJ + j] + acc); });
     __syncthreads();
@@ -373,7 +447,25 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     __syncthreads();
     // dGamma_C = rowsum(dS_next * (S + Kn^T U)), this CTA's columns: thread (row group,
     // column group) sums its products, then the 8 threads of a row group add theirs
-    {
+    if constexpr (TC) {
+      float d[MT<DK, BJ>::TPW][4];
+      mzero<DK, BJ>(d);
+      mmac<DK, BJ>(d, BC, [&](int i, int s) { return Kn[s * LK + i]; }, [&](int s, int j) { return Um[s * LJ + j]; });
+      float rs[2] = {0.f, 0.f};  // rows g and g + 8 of the warp's row block
+      int rows[2] = {0, 0};
+      mepi<DK, BJ>(d, [&](int i, int j, float acc) {
+        const int h8 = ((i & 15) >= 8);
+        rows[h8] = i;
+        rs[h8] = fmaf(dS[i * LJ + j], Sj[i * LJ + j] + acc, rs[h8]);
+      });
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float r = rs[u];
+        r += __shfl_xor_sync(0xffffffffu, r, 1);
+        r += __shfl_xor_sync(0xffffffffu, r, 2);
+        if ((tid & 3) == 0) atomicAdd(&dgC[rows[u]], r);
+      }
+    } else {
       constexpr int TM = DK / 32;
       const int tn = tid % 8, tm = tid / 8;
       float acc[TM][4];
@@ -414,38 +506,67 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     }
     __syncthreads();
     // dU = P^T dO + Kn dSt
-    gemm<BC, BJ, 2, 4>(BC, [&](int t, int s) { return Pm[s * LC + t]; }, [&](int s, int j) { return dOj[s * LJ + j]; },
+    prod<TC, BC, BJ, 2, 4>(BC, [&](int t, int s) { return Pm[s * LC + t]; }, [&](int s, int j) { return dOj[s * LJ + j]; },
                        [&](int t, int j, float acc) { dU[t * LJ + j] = acc; });
-    gemm<BC, BJ, 2, 4>(DK, [&](int t, int i) { return Kn[t * LK + i]; }, [&](int i, int j) { return dS[i * LJ + j]; },
+    prod<TC, BC, BJ, 2, 4>(DK, [&](int t, int i) { return Kn[t * LK + i]; }, [&](int i, int j) { return dS[i * LJ + j]; },
                        [&](int t, int j, float acc) { dU[t * LJ + j] += acc; });
     __syncthreads();
-    // dR = T^T dU (= dVw): dW = dVw * V, dV = dVw * W; dP = lower(dO U^T) over P
-    gemm<BC, BJ, 2, 4>(BC, [&](int t, int s) { return Tm[s * LC + t]; }, [&](int s, int j) { return dU[s * LJ + j]; },
-                       [&](int t, int j, float acc) {
-                         dR[t * LJ + j] = acc;
-                         const int tt = t0 + t;
-                         if (tt < p.T) {
-                           const size_t x = tok(tt) * DV + j0 + j;
-                           p.dw[x] = acc * ldf(p.v + x);
-                           p.dv[x] = acc * ldf(p.w + x);
-                         }
-                       });
-    gemm<BC, BC, 4, 4>(BJ, [&](int t, int j) { return dOj[t * LJ + j]; }, [&](int j, int s) { return Um[s * LJ + j]; },
-                       [&](int t, int s, float acc) { Pm[t * LC + s] = s <= t ? acc : 0.f; });
     // dT = dU R^T over A
-    gemm<BC, BC, 4, 4>(BJ, [&](int t, int j) { return dU[t * LJ + j]; }, [&](int j, int s) { return Rm[s * LJ + j]; },
-                       [&](int t, int s, float acc) { X1[t * LC + s] = acc; });
+    prod<TC, BC, BC, 4, 4>(BJ, [&](int t, int j) { return dU[t * LJ + j]; }, [&](int j, int s) { return Rm[s * LJ + j]; },
+                           [&](int t, int s, float acc) { X1[t * LC + s] = acc; });
     __syncthreads();
-    // Y = dT T^T over R and dU; then dA = strictly lower part of -T^T Y over dT
-    gemm<BC, BC, 4, 4>(BC, [&](int t, int r) { return X1[t * LC + r]; }, [&](int r, int s) { return Tm[s * LC + r]; },
-                       [&](int t, int s, float acc) { Ym[t * LC + s] = acc; });
+    // dR = T^T dU (= dVw) over R: dW = dVw * V, dV = dVw * W; Y = dT T^T over P
+    prod<TC, BC, BJ, 2, 4>(BC, [&](int t, int s) { return Tm[s * LC + t]; }, [&](int s, int j) { return dU[s * LJ + j]; },
+                           [&](int t, int j, float acc) {
+                             dR[t * LJ + j] = acc;
+                             const int tt = t0 + t;
+                             if (tt < p.T) {
+                               const size_t x = tok(tt) * DV + j0 + j;
+                               p.dw[x] = acc * ldf(p.v + x);
+                               p.dv[x] = acc * ldf(p.w + x);
+                             }
+                           });
+    prod<TC, BC, BC, 4, 4>(BC, [&](int t, int r) { return X1[t * LC + r]; }, [&](int r, int s) { return Tm[s * LC + r]; },
+                           [&](int t, int s, float acc) { Ym[t * LC + s] = acc; });
     __syncthreads();
-    gemm<BC, BC, 4, 4>(BC, [&](int t, int r) { return Tm[r * LC + t]; }, [&](int r, int s) { return Ym[r * LC + s]; },
-                       [&](int t, int s, float acc) { X1[t * LC + s] = s < t ? -acc : 0.f; });
+    // dA = strictly lower part of -T^T Y over dT
+    prod<TC, BC, BC, 4, 4>(BC, [&](int t, int r) { return Tm[r * LC + t]; }, [&](int r, int s) { return Ym[r * LC + s]; },
+                           [&](int t, int s, float acc) { X1[t * LC + s] = s < t ? -acc : 0.f; });
+    __syncthreads();
+    // dP = lower(dO U^T) over Y
+    prod<TC, BC, BC, 4, 4>(BJ, [&](int t, int j) { return dOj[t * LJ + j]; }, [&](int j, int s) { return Um[s * LJ + j]; },
+                           [&](int t, int s, float acc) { Pm[t * LC + s] = s <= t ? acc : 0.f; });
     __syncthreads();
     // key-side gradients of this CTA's columns, summed over the slices in global memory:
     //   dKb = -dR S^T + dA Kn,  dKn = U dSt^T + dA^T Kb + dP^T Qh,  dQh = dO S^T + dP Kn
-    {
+    if constexpr (TC) {
+      float d[MT<BC, DK>::TPW][4];
+      auto out = [&](float* dst) {  // pairs of adjacent key channels leave as 8-byte atomics
+        constexpr int NT = MT<BC, DK>::NT, TPW = MT<BC, DK>::TPW;
+        const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+        const int m0 = (warp * TPW / NT) * 16, nb = (warp * TPW) % NT;
+#pragma unroll
+        for (int q = 0; q < TPW; ++q) {
+          const int i = 8 * (nb + q) + 2 * tq;
+          const int ta = t0 + m0 + g, tb = ta + 8;
+          if (ta < p.T) atomicAdd(reinterpret_cast<float2*>(dst + tok(ta) * DK + i), make_float2(d[q][0], d[q][1]));
+          if (tb < p.T) atomicAdd(reinterpret_cast<float2*>(dst + tok(tb) * DK + i), make_float2(d[q][2], d[q][3]));
+        }
+      };
+      mzero<BC, DK>(d);
+      mmac<BC, DK>(d, BJ, [&](int t, int j) { return -dR[t * LJ + j]; }, [&](int j, int i) { return Sj[i * LJ + j]; });
+      mmac<BC, DK>(d, BC, [&](int t, int s) { return X1[t * LC + s]; }, [&](int s, int i) { return Kn[s * LK + i]; });
+      out(p.dk);
+      mzero<BC, DK>(d);
+      mmac<BC, DK>(d, BJ, [&](int t, int j) { return Um[t * LJ + j]; }, [&](int j, int i) { return dS[i * LJ + j]; });
+      mmac<BC, DK>(d, BC, [&](int t, int s) { return X1[s * LC + t]; }, [&](int s, int i) { return Kb[s * LK + i]; });
+      mmac<BC, DK>(d, BC, [&](int t, int s) { return Pm[s * LC + t]; }, [&](int s, int i) { return Qh[s * LK + i]; });
+      out(p.db);
+      mzero<BC, DK>(d);
+      mmac<BC, DK>(d, BJ, [&](int t, int j) { return dOj[t * LJ + j]; }, [&](int j, int i) { return Sj[i * LJ + j]; });
+      mmac<BC, DK>(d, BC, [&](int t, int s) { return Pm[t * LC + s]; }, [&](int s, int i) { return Kn[s * LK + i]; });
+      out(p.dq);
+    } else {
       // 64 x DK outputs: thread (tm, tn) takes rows 4 tm .. +4 and the key channels
       // 4 tn + 64 g + u (u < 4), so that its sums leave as 16-byte vector atomics
       constexpr int TN = DK / 16, NC = 16;
@@ -512,7 +633,25 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
       }
     }
     // dS (before the chunk) = Qh^T dO + dSt - Kb^T dR
-    {
+    if constexpr (TC) {
+      float d[MT<DK, BJ>::TPW][4];
+      mzero<DK, BJ>(d);
+      mmac<DK, BJ>(d, BC, [&](int i, int t) { return Qh[t * LK + i]; }, [&](int t, int j) { return dOj[t * LJ + j]; });
+      mmac<DK, BJ>(d, BC, [&](int i, int t) { return -Kb[t * LK + i]; }, [&](int t, int j) { return dR[t * LJ + j]; });
+      float acc[MT<DK, BJ>::TPW][4];
+      int e = 0;
+      mepi<DK, BJ>(d, [&](int i, int j, float v) {
+        acc[e >> 2][e & 3] = v + dS[i * LJ + j];
+        ++e;
+      });
+      __syncthreads();  // every read of dSt is done
+      e = 0;
+      mepi<DK, BJ>(d, [&](int i, int j, float v) {
+        static_cast<void>(v);
+        dS[i * LJ + j] = acc[e >> 2][e & 3];
+        ++e;
+      });
+    } else {
       constexpr int TM = DK / 32;
       const int tn = tid % 8, tm = tid / 8;
       float acc[TM][4];
@@ -585,10 +724,10 @@ __global__ void __launch_bounds__(DK) chunk_bwd_finish_kernel(const BwdParams<T>
   }
 }
 
-template <int DK>
+template <int DK, bool TC>
 constexpr size_t bwd_smem_bytes() {
-  return sizeof(float) * ((size_t)3 * BC * (DK + 1) + 2 * (size_t)DK * LJ + 3 * (size_t)BC * LC +
-                          5 * (size_t)BC * LJ + 2 * DK);
+  constexpr size_t P = pad<TC>(), LK = DK + P, LJ = BJ + P, LC = BC + P;
+  return sizeof(float) * (3 * BC * LK + 2 * (size_t)DK * LJ + 3 * BC * LC + 4 * BC * LJ + DK);
 }
 
 template <typename T, int DK, int DV>
@@ -628,7 +767,8 @@ cudaError_t launch_bwd_t(const ChunkBwdArgs& a, cudaStream_t st) {
     if ((e = launch_chunk_states_tc(f, p.states, st)) != cudaSuccess) return e;
     p.states_given = 1;
   }
-  constexpr size_t smem = bwd_smem_bytes<DK>();
+  constexpr size_t smem = bwd_smem_bytes<DK, std::is_same<T, __nv_bfloat16>::value>();
+  static_assert(smem <= 227 * 1024, "shared memory of the backward CTA");
   static bool attr = false;
   if (!attr) {
     if ((e = cudaFuncSetAttribute(chunk_bwd_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
