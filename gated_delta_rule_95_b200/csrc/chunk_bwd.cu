@@ -227,29 +227,46 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
 #pragma unroll
     for (int m = 0; m < Q4; ++m) {
       const int e4 = tid + BT * m, t = e4 / (DK / 4), i = 4 * (e4 % (DK / 4));
-      const float la[4] = {la4[m].x, la4[m].y, la4[m].z, la4[m].w}, kk[4] = {k4[m].x, k4[m].y, k4[m].z, k4[m].w};
-      const float bg[4] = {b4[m].x, b4[m].y, b4[m].z, b4[m].w}, qq[4] = {q4[m].x, q4[m].y, q4[m].z, q4[m].w};
+      *reinterpret_cast<float4*>(raw_la + t * DK + i) = la4[m];
+      if constexpr (LK % 4 == 0) {  // 16-byte aligned rows: one vector store each
+        *reinterpret_cast<float4*>(Kn + t * LK + i) = k4[m];
+        *reinterpret_cast<float4*>(Kb + t * LK + i) = b4[m];
+        if (with_q) *reinterpret_cast<float4*>(Qh + t * LK + i) = q4[m];
+      } else {
+        const float kk[4] = {k4[m].x, k4[m].y, k4[m].z, k4[m].w}, bg[4] = {b4[m].x, b4[m].y, b4[m].z, b4[m].w};
+        const float qq[4] = {q4[m].x, q4[m].y, q4[m].z, q4[m].w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        raw_la[t * DK + i + u] = la[u];
-        Kn[t * LK + i + u] = kk[u];
-        Kb[t * LK + i + u] = bg[u];
-        if (with_q) Qh[t * LK + i + u] = qq[u];
+        for (int u = 0; u < 4; ++u) {
+          Kn[t * LK + i + u] = kk[u];
+          Kb[t * LK + i + u] = bg[u];
+          if (with_q) Qh[t * LK + i + u] = qq[u];
+        }
       }
     }
     __syncthreads();
-    if (tid < DK) {
-      const int i = tid;
-      float g = 0.f;
-      for (int t = 0; t < BC; ++t) {
-        g += raw_la[t * DK + i];
-        const float G = __expf(g), kk = Kn[t * LK + i];
-        Kb[t * LK + i] *= kk * G;
-        Kn[t * LK + i] = kk * __expf(-g);
-        if (with_q) Qh[t * LK + i] *= G;
-      }
-      gC[i] = __expf(g);
+    // the cumulative log decay, RS threads per key channel each over BC / RS rows: segment
+    // sums first, then each segment's scan from the sum of the segments before it
+    constexpr int RS = BT / DK, RL = BC / RS;
+    float* part = raw_la + BC * DK;  // [RS][DK], past the raw log alpha (3 BC LC >= BC DK + BT)
+    const int i = tid % DK, sgm = tid / DK;
+    {
+      float sum = 0.f;
+#pragma unroll 8
+      for (int t = sgm * RL; t < sgm * RL + RL; ++t) sum += raw_la[t * DK + i];
+      part[sgm * DK + i] = sum;
     }
+    __syncthreads();
+    float g = 0.f;
+    for (int r = 0; r < sgm; ++r) g += part[r * DK + i];
+#pragma unroll 4
+    for (int t = sgm * RL; t < sgm * RL + RL; ++t) {
+      g += raw_la[t * DK + i];
+      const float G = __expf(g), kk = Kn[t * LK + i];
+      Kb[t * LK + i] *= kk * G;
+      Kn[t * LK + i] = kk * __expf(-g);
+      if (with_q) Qh[t * LK + i] *= G;
+    }
+    if (sgm == RS - 1) gC[i] = __expf(g);
   };
   // the inputs of chunk c into L2 while the current chunk computes (q and dO only for the
   // reverse sweep): one 128-byte line per thread and row segment
@@ -273,6 +290,11 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
       else a = reinterpret_cast<const char*>(p.dO + tok(tt) * DV) + 128 * (m - KL);
       asm volatile("prefetch.global.L2 [%0];" :: "l"(a));
     }
+    if (rev)  // the chunk's entering state, this CTA's columns: one line per key channel
+      for (int i = tid; i < DK; i += BT) {
+        const float* a = p.states + (((size_t)bh * p.nch + c) * DK + i) * DV + j0;
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(a));
+      }
   };
   // T = (I + A)^-1 from A (strictly lower, in X1), by blocks: the 16 x 16 diagonal blocks by
   // forward substitution (four threads per column split each row's dot product), then the
