@@ -583,9 +583,12 @@ def main():
         "bwd": {"metric": "GDN-2 backward tokens/s per layer", "value": bw["tokens"] / (bw["ms"] * 1e-3),
                 "unit": "tokens/s", "ms_per_step": bw["ms"],
                 "workload": "prefill_b8_h16_t4096 backward: dq, dk, dv, dlog_alpha, db, dw, dS0 from dO and dS_T "
-                            "(fp32 on the CUDA cores)",
-                "roofline": {"bound": "alu", "kernel": "chunk_bwd_kernel", "achieved": bw_tflops,
-                             "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s", "frac": bw_tflops / FP32_FMA_TFLOPS,
+                            "(products as tf32 warp-level MMAs)",
+                "roofline": {"bound": "tensor", "kernel": "chunk_bwd_kernel", "achieved": bw_tflops,
+                             "peak": pk["bf16_tflops"] * TF32_PER_BF16, "unit": "TFLOP/s",
+                             "frac": bw_tflops / (pk["bf16_tflops"] * TF32_PER_BF16),
+                             "peak_src": "measured bf16 x nominal tf32/bf16 ratio",
+                             "frac_of_fp32_cuda_core_peak": bw_tflops / FP32_FMA_TFLOPS,
                              "flop_per_chunk_head": BWD_FLOP_PER_CHUNK_HEAD, "traffic": None}},
         "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
                  "steps": args.steps,
