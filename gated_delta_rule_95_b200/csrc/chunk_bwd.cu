@@ -123,8 +123,30 @@ __device__ __forceinline__ void mmac(float (&d)[MT<M, N>::TPW][4], int K, FA fa,
     }
   }
 }
-// epi(m, n, value) for every element of the warp's tiles, and the row/column of element e
-// of tile q
+// two products sharing their B operand: d1 (+)= A1 B and d2 (+)= A2 B, each B fragment
+// loaded once for both
+template <int M, int N, class FA1, class FA2, class FB>
+__device__ __forceinline__ void mmac2(float (&d1)[MT<M, N>::TPW][4], float (&d2)[MT<M, N>::TPW][4], int K, FA1 fa1,
+                                      FA2 fa2, FB fb) {
+  constexpr int NT = MT<M, N>::NT, TPW = MT<M, N>::TPW;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int m0 = (warp * TPW / NT) * 16, nb = (warp * TPW) % NT;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const uint32_t a1[4] = {tf32r(fa1(m0 + g, k0 + t)), tf32r(fa1(m0 + g + 8, k0 + t)),
+                            tf32r(fa1(m0 + g, k0 + t + 4)), tf32r(fa1(m0 + g + 8, k0 + t + 4))};
+    const uint32_t a2[4] = {tf32r(fa2(m0 + g, k0 + t)), tf32r(fa2(m0 + g + 8, k0 + t)),
+                            tf32r(fa2(m0 + g, k0 + t + 4)), tf32r(fa2(m0 + g + 8, k0 + t + 4))};
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) {
+      const int n0 = 8 * (nb + q);
+      const uint32_t b[2] = {tf32r(fb(k0 + t, n0 + g)), tf32r(fb(k0 + t + 4, n0 + g))};
+      mma_16x8x8_tf32(d1[q], a1, b);
+      mma_16x8x8_tf32(d2[q], a2, b);
+    }
+  }
+}
+// epi(m, n, value) for every element of the warp's tiles
 template <int M, int N, class FE>
 __device__ __forceinline__ void mepi(const float (&d)[MT<M, N>::TPW][4], FE epi) {
   constexpr int NT = MT<M, N>::NT, TPW = MT<M, N>::TPW;
@@ -207,7 +229,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   // walks the rows of key channel i, summing log alpha, and folds the decay in place.
   auto build = [&](int c, bool with_q) {
     const int t0 = c * BC;
-    float* raw_la = Tm;  // [BC][DK] over T, P and A (3 BC LC >= BC DK floats)
+    float* raw_la = Pm;  // [BC][DK] over P, A and R (free at this point; T keeps its zeros)
     // four consecutive key channels per load, every load of the thread in flight at once
     constexpr int Q4 = BC * DK / 4 / BT;
     float4 la4[Q4], k4[Q4], b4[Q4], q4[Q4];
@@ -247,7 +269,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     // the cumulative log decay, RS threads per key channel each over BC / RS rows: segment
     // sums first, then each segment's scan from the sum of the segments before it
     constexpr int RS = BT / DK, RL = BC / RS;
-    float* part = raw_la + BC * DK;  // [RS][DK], past the raw log alpha (3 BC LC >= BC DK + BT)
+    float* part = raw_la + BC * DK;  // [RS][DK], past the raw log alpha (2 BC LC + BC LJ >= BC DK + BT)
     const int i = tid % DK, sgm = tid / DK;
     {
       float sum = 0.f;
@@ -300,9 +322,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   // forward substitution (four threads per column split each row's dot product), then the
   // 2 x 2 block merges T21 = -T22 (A21 T11) at 32 and 64 (products staged in the R tile,
   // free at this point).
-  auto solve = [&]() {
-    for (int e = tid; e < BC * BC; e += BT) Tm[(e / BC) * LC + e % BC] = 0.f;
-    __syncthreads();
+  auto solve = [&]() {  // (every entry above the diagonal of T is zero from the start)
     {
       const int s = tid >> 2, part = tid & 3, base = s & ~15;  // a warp's 8 columns share a block
       if (part == 0) Tm[s * LC + s] = 1.f;
@@ -389,6 +409,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
                        [&](int t, int s, float acc) { dst[t * LC + s] = (s < t || (incl_diag && s == t)) ? acc : 0.f; });
   };
 
+  for (int e = tid; e < BC * LC; e += BT) Tm[e] = 0.f;  // T: zero above the diagonal for good
   // ---- forward sweep: every chunk's entering state (unless given) ---------------------------
   for (int e = tid; e < DK * BJ && !p.states_given; e += BT) {
     const int i = e / BJ, j = e % BJ;
@@ -562,8 +583,8 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     // key-side gradients of this CTA's columns, summed over the slices in global memory:
     //   dKb = -dR S^T + dA Kn,  dKn = U dSt^T + dA^T Kb + dP^T Qh,  dQh = dO S^T + dP Kn
     if constexpr (TC) {
-      float d[MT<BC, DK>::TPW][4];
-      auto out = [&](float* dst) {  // pairs of adjacent key channels leave as 8-byte atomics
+      float d[MT<BC, DK>::TPW][4], d2[MT<BC, DK>::TPW][4];
+      auto out = [&](float* dst, const float (&d)[MT<BC, DK>::TPW][4]) {  // 8-byte atomics
         constexpr int NT = MT<BC, DK>::NT, TPW = MT<BC, DK>::TPW;
         const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
         const int m0 = (warp * TPW / NT) * 16, nb = (warp * TPW) % NT;
@@ -575,19 +596,20 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
           if (tb < p.T) atomicAdd(reinterpret_cast<float2*>(dst + tok(tb) * DK + i), make_float2(d[q][2], d[q][3]));
         }
       };
+      // dKb and dQh share their B operands (S, then Kn)
       mzero<BC, DK>(d);
-      mmac<BC, DK>(d, BJ, [&](int t, int j) { return -dR[t * LJ + j]; }, [&](int j, int i) { return Sj[i * LJ + j]; });
-      mmac<BC, DK>(d, BC, [&](int t, int s) { return X1[t * LC + s]; }, [&](int s, int i) { return Kn[s * LK + i]; });
-      out(p.dk);
+      mzero<BC, DK>(d2);
+      mmac2<BC, DK>(d, d2, BJ, [&](int t, int j) { return -dR[t * LJ + j]; }, [&](int t, int j) { return dOj[t * LJ + j]; },
+                    [&](int j, int i) { return Sj[i * LJ + j]; });
+      mmac2<BC, DK>(d, d2, BC, [&](int t, int s) { return X1[t * LC + s]; }, [&](int t, int s) { return Pm[t * LC + s]; },
+                    [&](int s, int i) { return Kn[s * LK + i]; });
+      out(p.dk, d);
+      out(p.dq, d2);
       mzero<BC, DK>(d);
       mmac<BC, DK>(d, BJ, [&](int t, int j) { return Um[t * LJ + j]; }, [&](int j, int i) { return dS[i * LJ + j]; });
       mmac<BC, DK>(d, BC, [&](int t, int s) { return X1[s * LC + t]; }, [&](int s, int i) { return Kb[s * LK + i]; });
       mmac<BC, DK>(d, BC, [&](int t, int s) { return Pm[s * LC + t]; }, [&](int s, int i) { return Qh[s * LK + i]; });
-      out(p.db);
-      mzero<BC, DK>(d);
-      mmac<BC, DK>(d, BJ, [&](int t, int j) { return dOj[t * LJ + j]; }, [&](int j, int i) { return Sj[i * LJ + j]; });
-      mmac<BC, DK>(d, BC, [&](int t, int s) { return Pm[t * LC + s]; }, [&](int s, int i) { return Kn[s * LK + i]; });
-      out(p.dq);
+      out(p.db, d);
     } else {
       // 64 x DK outputs: thread (tm, tn) takes rows 4 tm .. +4 and the key channels
       // 4 tn + 64 g + u (u < 4), so that its sums leave as 16-byte vector atomics
