@@ -37,7 +37,8 @@ namespace {
 
 constexpr int BC = 64;        // chunk size
 constexpr int BJ = 32;        // value columns per CTA
-constexpr int BT = 256;       // threads per CTA
+constexpr int BT = 256;       // threads per CTA of the CUDA-core path
+constexpr int MW = 16;        // warps per CTA of the tensor-core path
 // Row padding of the shared-memory tiles: 1 float for the CUDA-core products (whose
 // column-wise reads then meet 32 banks), 4 floats for the tensor-core fragments (the 8 x 4
 // element groups of an mma fragment then meet 32 banks)
@@ -91,14 +92,14 @@ __device__ __forceinline__ void gemm(int K, FA fa, FB fb, FE epi) {
 }
 
 // The same products on the tensor cores (bf16 inputs): mma.sync m16n8k8 with operands
-// rounded to tf32 (nearest), fp32 accumulation.  The 16 x 8 output tiles go to the 8 warps
+// rounded to tf32 (nearest), fp32 accumulation.  The 16 x 8 output tiles go to the MW warps
 // in row-major order, TPW consecutive tiles per warp sharing one 16-row block, so that a
 // warp loads each A fragment once per k step.  d holds the warp's tiles' accumulators.
 __device__ __forceinline__ uint32_t tf32r(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
 
 template <int M, int N>
 struct MT {
-  static constexpr int NT = N / 8, TPW = (M / 16) * NT / 8;
+  static constexpr int NT = N / 8, TPW = (M / 16) * NT / MW;
   static_assert(TPW >= 1 && NT % TPW == 0, "a warp's tiles must share a row block");
 };
 template <int M, int N>
@@ -193,8 +194,10 @@ struct BwdParams {
 };
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) {
+__global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * MW : BT, 1)
+    chunk_bwd_kernel(const BwdParams<T> p) {
   constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;  // products on the tensor cores
+  constexpr int NTH = TC ? 32 * MW : BT;                       // threads of the CTA
   constexpr int LK = DK + pad<TC>();  // padded rows: [BC][DK] tiles
   constexpr int LJ = BJ + pad<TC>();  //              [.][BJ] tiles
   constexpr int LC = BC + pad<TC>();  //              [BC][BC] tiles
@@ -231,11 +234,11 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     const int t0 = c * BC;
     float* raw_la = Pm;  // [BC][DK] over P, A and R (free at this point; T keeps its zeros)
     // four consecutive key channels per load, every load of the thread in flight at once
-    constexpr int Q4 = BC * DK / 4 / BT;
+    constexpr int Q4 = BC * DK / 4 / NTH;
     float4 la4[Q4], k4[Q4], b4[Q4], q4[Q4];
 #pragma unroll
     for (int m = 0; m < Q4; ++m) {
-      const int e4 = tid + BT * m, t = e4 / (DK / 4), i = 4 * (e4 % (DK / 4)), tt = t0 + t;
+      const int e4 = tid + NTH * m, t = e4 / (DK / 4), i = 4 * (e4 % (DK / 4)), tt = t0 + t;
       const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
       la4[m] = k4[m] = b4[m] = q4[m] = z;
       if (tt < p.T) {
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     }
 #pragma unroll
     for (int m = 0; m < Q4; ++m) {
-      const int e4 = tid + BT * m, t = e4 / (DK / 4), i = 4 * (e4 % (DK / 4));
+      const int e4 = tid + NTH * m, t = e4 / (DK / 4), i = 4 * (e4 % (DK / 4));
       *reinterpret_cast<float4*>(raw_la + t * DK + i) = la4[m];
       if constexpr (LK % 4 == 0) {  // 16-byte aligned rows: one vector store each
         *reinterpret_cast<float4*>(Kn + t * LK + i) = k4[m];
@@ -268,8 +271,8 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     __syncthreads();
     // the cumulative log decay, RS threads per key channel each over BC / RS rows: segment
     // sums first, then each segment's scan from the sum of the segments before it
-    constexpr int RS = BT / DK, RL = BC / RS;
-    float* part = raw_la + BC * DK;  // [RS][DK], past the raw log alpha (2 BC LC + BC LJ >= BC DK + BT)
+    constexpr int RS = NTH / DK, RL = BC / RS;
+    float* part = raw_la + BC * DK;  // [RS][DK], past the raw log alpha (2 BC LC + BC LJ >= BC DK + NTH)
     const int i = tid % DK, sgm = tid / DK;
     {
       float sum = 0.f;
@@ -298,7 +301,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     constexpr int KL = DK * (int)sizeof(T) / 128, VL = DV * (int)sizeof(T) / 128;  // lines per row
     constexpr int LL = DK * 4 / 128, OL = DV * 4 / 128;
     const int nseg = 2 * KL + LL + 2 * VL + (rev ? KL + OL : 0);
-    for (int e = tid; e < BC * nseg; e += BT) {
+    for (int e = tid; e < BC * nseg; e += NTH) {
       const int t = e % BC, r = e / BC, tt = t0 + t;
       if (tt >= p.T) continue;
       const char* a;
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
       asm volatile("prefetch.global.L2 [%0];" :: "l"(a));
     }
     if (rev)  // the chunk's entering state, this CTA's columns: one line per key channel
-      for (int i = tid; i < DK; i += BT) {
+      for (int i = tid; i < DK; i += NTH) {
         const float* a = p.states + (((size_t)bh * p.nch + c) * DK + i) * DV + j0;
         asm volatile("prefetch.global.L2 [%0];" :: "l"(a));
       }
@@ -322,8 +325,9 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   // forward substitution (four threads per column split each row's dot product), then the
   // 2 x 2 block merges T21 = -T22 (A21 T11) at 32 and 64 (products staged in the R tile,
   // free at this point).
-  auto solve = [&]() {  // (every entry above the diagonal of T is zero from the start)
-    {
+  auto solve = [&]() {  // (every entry above the diagonal of T is zero from the start; the
+                        // first 256 threads work, the rest only meet the barriers)
+    if (tid < 256) {
       const int s = tid >> 2, part = tid & 3, base = s & ~15;  // a warp's 8 columns share a block
       if (part == 0) Tm[s * LC + s] = 1.f;
       __syncwarp();
@@ -341,50 +345,58 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     float* Xs = Rm;  // [32][LJ]
     {
       // 32: blocks q = 0, 1 at offset 32 q; thread: row r of the block, columns c, c + 1
-      const int q = tid >> 7, r = (tid >> 3) & 15, c = 2 * (tid & 7), o = 32 * q;
-      float x0 = 0.f, x1 = 0.f;
+      const int q = (tid >> 7) & 1, r = (tid >> 3) & 15, c = 2 * (tid & 7), o = 32 * q;
+      if (tid < 256) {
+        float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const float a = X1[(o + 16 + r) * LC + o + m];
-        x0 = fmaf(a, Tm[(o + m) * LC + o + c], x0);
-        x1 = fmaf(a, Tm[(o + m) * LC + o + c + 1], x1);
+        for (int m = 0; m < 16; ++m) {
+          const float a = X1[(o + 16 + r) * LC + o + m];
+          x0 = fmaf(a, Tm[(o + m) * LC + o + c], x0);
+          x1 = fmaf(a, Tm[(o + m) * LC + o + c + 1], x1);
+        }
+        Xs[(16 * q + r) * LJ + c] = x0;
+        Xs[(16 * q + r) * LJ + c + 1] = x1;
       }
-      Xs[(16 * q + r) * LJ + c] = x0;
-      Xs[(16 * q + r) * LJ + c + 1] = x1;
       __syncthreads();
-      float y0 = 0.f, y1 = 0.f;
+      if (tid < 256) {
+        float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const float t22 = Tm[(o + 16 + r) * LC + o + 16 + m];
-        y0 = fmaf(t22, Xs[(16 * q + m) * LJ + c], y0);
-        y1 = fmaf(t22, Xs[(16 * q + m) * LJ + c + 1], y1);
+        for (int m = 0; m < 16; ++m) {
+          const float t22 = Tm[(o + 16 + r) * LC + o + 16 + m];
+          y0 = fmaf(t22, Xs[(16 * q + m) * LJ + c], y0);
+          y1 = fmaf(t22, Xs[(16 * q + m) * LJ + c + 1], y1);
+        }
+        Tm[(o + 16 + r) * LC + o + c] = -y0;
+        Tm[(o + 16 + r) * LC + o + c + 1] = -y1;
       }
-      Tm[(o + 16 + r) * LC + o + c] = -y0;
-      Tm[(o + 16 + r) * LC + o + c + 1] = -y1;
     }
     __syncthreads();
     {
       // 64: thread: row r of the lower half, columns [4 c4, 4 c4 + 4)
-      const int r = tid >> 3, c4 = 4 * (tid & 7);
-      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      const int r = (tid >> 3) & 31, c4 = 4 * (tid & 7);
+      if (tid < 256) {
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-      for (int m = 0; m < 32; ++m) {
-        const float a = X1[(32 + r) * LC + m];
+        for (int m = 0; m < 32; ++m) {
+          const float a = X1[(32 + r) * LC + m];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) x[y] = fmaf(a, Tm[m * LC + c4 + y], x[y]);
+          for (int y = 0; y < 4; ++y) x[y] = fmaf(a, Tm[m * LC + c4 + y], x[y]);
+        }
+#pragma unroll
+        for (int y = 0; y < 4; ++y) Xs[r * LJ + c4 + y] = x[y];
       }
-#pragma unroll
-      for (int y = 0; y < 4; ++y) Xs[r * LJ + c4 + y] = x[y];
       __syncthreads();
-      float z[4] = {0.f, 0.f, 0.f, 0.f};
+      if (tid < 256) {
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-      for (int m = 0; m < 32; ++m) {
-        const float t22 = Tm[(32 + r) * LC + 32 + m];
+        for (int m = 0; m < 32; ++m) {
+          const float t22 = Tm[(32 + r) * LC + 32 + m];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) z[y] = fmaf(t22, Xs[m * LJ + c4 + y], z[y]);
+          for (int y = 0; y < 4; ++y) z[y] = fmaf(t22, Xs[m * LJ + c4 + y], z[y]);
+        }
+#pragma unroll
+        for (int y = 0; y < 4; ++y) Tm[(32 + r) * LC + c4 + y] = -z[y];
       }
-#pragma unroll
-      for (int y = 0; y < 4; ++y) Tm[(32 + r) * LC + c4 + y] = -z[y];
     }
   };
   // R = Vw - Kb S and U = T R for chunk c
@@ -409,9 +421,9 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
                        [&](int t, int s, float acc) { dst[t * LC + s] = (s < t || (incl_diag && s == t)) ? acc : 0.f; });
   };
 
-  for (int e = tid; e < BC * LC; e += BT) Tm[e] = 0.f;  // T: zero above the diagonal for good
+  for (int e = tid; e < BC * LC; e += NTH) Tm[e] = 0.f;  // T: zero above the diagonal for good
   // ---- forward sweep: every chunk's entering state (unless given) ---------------------------
-  for (int e = tid; e < DK * BJ && !p.states_given; e += BT) {
+  for (int e = tid; e < DK * BJ && !p.states_given; e += NTH) {
     const int i = e / BJ, j = e % BJ;
     Sj[i * LJ + j] = p.S0 ? p.S0[((size_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
@@ -419,7 +431,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   for (int c = 0; c < p.nch && !p.states_given; ++c) {
     prefetch(c + 1, false);
     float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
-    for (int e = tid; e < DK * BJ; e += BT) {
+    for (int e = tid; e < DK * BJ; e += NTH) {
       const int i = e / BJ, j = e % BJ;
       st[(size_t)i * DV + j0 + j] = Sj[i * LJ + j];
     }
@@ -439,7 +451,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
   }
 
   // ---- reverse sweep -------------------------------------------------------------------------
-  for (int e = tid; e < DK * BJ; e += BT) {
+  for (int e = tid; e < DK * BJ; e += NTH) {
     const int i = e / BJ, j = e % BJ;
     dS[i * LJ + j] = p.dST ? p.dST[((size_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
@@ -449,21 +461,21 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     prefetch(c - 1, true);
     const float* st = p.states + ((size_t)bh * p.nch + c) * DK * DV;
     {
-      constexpr int NSQ = DK * BJ / 4 / BT, NOQ = BC * BJ / 4 / BT;
+      constexpr int NSQ = DK * BJ / 4 / NTH, NOQ = BC * BJ / 4 / NTH;
       float4 sv[NSQ], ov[NOQ];
 #pragma unroll
       for (int m = 0; m < NSQ; ++m) {
-        const int e4 = tid + BT * m, i = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
+        const int e4 = tid + NTH * m, i = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
         sv[m] = ld4f(st + (size_t)i * DV + j0 + j);
       }
 #pragma unroll
       for (int m = 0; m < NOQ; ++m) {
-        const int e4 = tid + BT * m, t = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4)), tt = t0 + t;
+        const int e4 = tid + NTH * m, t = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4)), tt = t0 + t;
         ov[m] = tt < p.T ? ld4f(p.dO + tok(tt) * DV + j0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int m = 0; m < NSQ; ++m) {
-        const int e4 = tid + BT * m, i = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
+        const int e4 = tid + NTH * m, i = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
         Sj[i * LJ + j] = sv[m].x;
         Sj[i * LJ + j + 1] = sv[m].y;
         Sj[i * LJ + j + 2] = sv[m].z;
@@ -471,7 +483,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
       }
 #pragma unroll
       for (int m = 0; m < NOQ; ++m) {
-        const int e4 = tid + BT * m, t = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
+        const int e4 = tid + NTH * m, t = e4 / (BJ / 4), j = 4 * (e4 % (BJ / 4));
         dOj[t * LJ + j] = ov[m].x;
         dOj[t * LJ + j + 1] = ov[m].y;
         dOj[t * LJ + j + 2] = ov[m].z;
@@ -543,7 +555,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     __syncthreads();
     if (tid < DK) atomicAdd(p.dgc + ((size_t)bh * p.nch + c) * DK + tid, dgC[tid]);
     // dSt = Diag(Gamma_C) dS_next, in place
-    for (int e = tid; e < DK * BJ; e += BT) {
+    for (int e = tid; e < DK * BJ; e += NTH) {
       const int i = e / BJ, j = e % BJ;
       dS[i * LJ + j] *= gC[i];
     }
@@ -730,7 +742,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const BwdParams<T> p) 
     __syncthreads();
   }
   if (p.dS0)
-    for (int e = tid; e < DK * BJ; e += BT) {
+    for (int e = tid; e < DK * BJ; e += NTH) {
       const int i = e / BJ, j = e % BJ;
       p.dS0[((size_t)bh * DK + i) * DV + j0 + j] = dS[i * LJ + j];
     }
@@ -820,7 +832,8 @@ cudaError_t launch_bwd_t(const ChunkBwdArgs& a, cudaStream_t st) {
       return e;
     attr = true;
   }
-  chunk_bwd_kernel<T, DK, DV><<<(unsigned)(BH * (DV / BJ)), BT, smem, st>>>(p);
+  constexpr int nth = std::is_same<T, __nv_bfloat16>::value ? 32 * MW : BT;
+  chunk_bwd_kernel<T, DK, DV><<<(unsigned)(BH * (DV / BJ)), nth, smem, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   chunk_bwd_finish_kernel<T, DK><<<(unsigned)(BH * p.nch), DK, 0, st>>>(p, a.dlog_alpha);
   return cudaGetLastError();
