@@ -67,3 +67,23 @@ def test_bwd_no_tokens():
     gg = g.gdn2_chunk_bwd(*(x[n] for n in NAMES), x["S0"], do.cuda(), dS.cuda())
     torch.cuda.synchronize()
     assert torch.equal(gg["dS0"].cpu(), dS)
+
+
+def test_bwd_full_prefill_b8_h16_t4096_sampled_units():
+    # the bench's backward workload; two (batch, head) units against the oracle, whose
+    # gradients depend on that unit's inputs and cotangents only
+    wl = BASE
+    d = gi.prefill_inputs(wl)
+    do, dS = _cot(wl.B, wl.T, wl.H, wl.dk, wl.dv, 11)
+    x = {k_: (None if v_ is None else v_.cuda()) for k_, v_ in d.items()}
+    gg = g.gdn2_chunk_bwd(*(x[n] for n in NAMES), x["S0"], do.cuda(), dS.cuda())
+    torch.cuda.synchronize()
+    assert g.gdn2_device_status() == 0
+    for bb, h in [(0, 0), (6, 11)]:
+        sl = {n: gi.as_f64(d[n][bb:bb + 1, :, h:h + 1]) for n in NAMES}
+        ref = ob.backward(**sl, S0=None, do=do[bb:bb + 1, :, h:h + 1].double().numpy(),
+                          dS_T=dS[bb:bb + 1, h:h + 1].double().numpy())
+        for n in GRADS:
+            got = gg[n][bb:bb + 1, h:h + 1] if n == "dS0" else gg[n][bb:bb + 1, :, h:h + 1]
+            err = rel_err(got.cpu().numpy(), ref[n])
+            assert err <= TOL["bf16"], (bb, h, n, err)
