@@ -331,6 +331,32 @@ def time_bwd(args, dev):
                 ok=g.gdn2_device_status() == 0)
 
 
+def time_csize(args, dev):
+    """The prefill workload at chunk sizes 32, 64 and 128 through gdn2_chunk_fwd_csize
+    (one kernel template for the three sizes): latency, and the on-chip footprint that
+    sets how many CTAs share an SM (the call needs no device memory besides its tensors)."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    d = gi.prefill_inputs(PREFILL)
+    x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    B, T, H, dk, dv = PREFILL.B, PREFILL.T, PREFILL.H, PREFILL.dk, PREFILL.dv
+    o = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    args_t = [x[n] for n in ("q", "k", "v", "log_alpha", "b", "w")]
+    sm_total = 228 * 1024  # shared memory of one SM, 1 KB of it reserved per resident CTA
+    out = {}
+    for C in (32, 64, 128):
+        def step(C=C):
+            g.gdn2_chunk_fwd_csize(*args_t, None, chunk=C, o=o, S_T=S_T)
+
+        ms = _time_loop(step, args.steps, args.warmup)
+        smem = g.lib().gdn2_chunk_fwd_csize_smem_bytes(C, dk)
+        out[C] = dict(ms=ms, smem=smem, ctas_per_sm=sm_total // (smem + 1024))
+    arg_bytes = sum(t.numel() * t.element_size() for t in args_t + [o, S_T])
+    return dict(sizes=out, tokens=B * T, token_heads=B * T * H, arg_bytes=arg_bytes, ctas=B * H * (dv // 32),
+                ok=g.gdn2_device_status() == 0)
+
+
 def time_raw(args, dev):
     """The prefill workload fed with raw projections (activations inside the kernel)."""
     import torch
@@ -513,6 +539,7 @@ def main():
     cv = time_conv(args, dev)
     lg = time_long(args, dev)
     bw = time_bwd(args, dev)
+    cs = time_csize(args, dev)
     bw_tflops = bw["chunk_heads"] * BWD_FLOP_PER_CHUNK_HEAD / (bw["ms"] * 1e-3) / 1e12
     lg_gbs = lg["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (lg["ms_split"] * 1e-3) / 1e9
     cv_gbs = cv["bytes"] / (cv["ms"] * 1e-3) / 1e9
@@ -590,6 +617,22 @@ def main():
                              "peak_src": "measured bf16 x nominal tf32/bf16 ratio",
                              "frac_of_fp32_cuda_core_peak": bw_tflops / FP32_FMA_TFLOPS,
                              "flop_per_chunk_head": BWD_FLOP_PER_CHUNK_HEAD, "traffic": None}},
+        "csize": {"metric": "GDN-2 prefill tokens/s per layer by chunk size",
+                  "workload": "prefill_b8_h16_t4096 through gdn2_chunk_fwd_csize (warp-level tf32 MMAs, one "
+                              f"template for every chunk size; {cs['ctas']} CTAs of (batch, head, 32 value columns))",
+                  "device_bytes": {"arguments": cs["arg_bytes"], "scratch": 0},
+                  "sizes": {str(C): {"value": cs["tokens"] / (r["ms"] * 1e-3), "unit": "tokens/s",
+                                     "ms_per_step": r["ms"], "smem_bytes_per_cta": r["smem"],
+                                     "ctas_per_sm_by_smem": r["ctas_per_sm"],
+                                     "flop_per_token_head": 2 * C * (3 * 128 + 2 * 128) + 6 * 128 * 128,
+                                     "roofline": {"bound": "hbm", "kernel": "chunk_fwd_csize_kernel",
+                                                  "achieved": cs["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD
+                                                  / (r["ms"] * 1e-3) / 1e9,
+                                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                                  "frac": cs["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD
+                                                  / (r["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                                  "traffic": None}}
+                            for C, r in cs["sizes"].items()}},
         "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
                  "steps": args.steps,
                  "workload": f"q, k, v projections of prefill_b8_h16_t4096 side by side: [8, 4096, {cv['C']}] bf16, "
@@ -600,7 +643,7 @@ def main():
         "gpu_launches": args.steps,
         "clocks": pre["clocks"],
         "device_status_ok": bool(pre["ok"] and dec["ok"] and dec_raw["ok"] and pak["ok"] and raw["ok"] and cv["ok"]
-                                 and lg["ok"] and bw["ok"]),
+                                 and lg["ok"] and bw["ok"] and cs["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)

@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_bwd", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_static", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_csize", "gdn2_chunk_bwd", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_static", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_raw", "gdn2_short_conv", "gdn2_decode_step", "gdn2_decode_step_raw", "gdn2_device_status", "GDN2Error", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -67,6 +67,10 @@ def lib():
         L.gdn2_chunk_fwd_split_segments.restype = I
         L.gdn2_chunk_fwd_split_workspace_bytes.argtypes = [I] * 5
         L.gdn2_chunk_fwd_split_workspace_bytes.restype = ctypes.c_size_t
+        L.gdn2_chunk_fwd_csize.argtypes = [P] * 9 + [I] * 7 + [P]
+        L.gdn2_chunk_fwd_csize.restype = I
+        L.gdn2_chunk_fwd_csize_smem_bytes.argtypes = [I] * 2
+        L.gdn2_chunk_fwd_csize_smem_bytes.restype = ctypes.c_size_t
         L.gdn2_chunk_fwd_varlen.argtypes = [P] * 10 + [I] * 6 + [P]
         L.gdn2_chunk_fwd_varlen.restype = I
         L.gdn2_chunk_fwd_raw.argtypes = [P] * 11 + [I] * 6 + [P]
@@ -131,6 +135,32 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_
                               _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd", rc)
+    return o, S_T
+
+
+def gdn2_chunk_fwd_csize(q, k, v, log_alpha, b, w, S0=None, *, chunk=64, o=None, S_T=None, want_state=True,
+                         stream=None):
+    """Chunkwise prefill forward at chunk size 32, 64 or 128 (bf16 inputs).  Returns
+    (o [B,T,H,d_v], S_T [B,H,d_k,d_v] or None), like gdn2_chunk_fwd."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DT:
+        raise ValueError(f"gdn2_chunk_fwd_csize: unsupported dtype {q.dtype}")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ts = dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, o=o)
+    if S0 is not None:
+        ts["S0"] = S0
+    if S_T is not None:
+        ts["S_T"] = S_T
+    _check_tokens("gdn2_chunk_fwd_csize", ts, q.dtype, q.device)
+    rc = lib().gdn2_chunk_fwd_csize(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),
+                                    _ptr(o), _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], int(chunk),
+                                    _stream(q.device, stream))
+    if rc != 0:
+        raise GDN2Error("gdn2_chunk_fwd_csize", rc)
     return o, S_T
 
 

@@ -179,6 +179,29 @@ extern "C" gdn2_status gdn2_chunk_fwd_split_static(const void* q, const void* k,
                               kSplitScratchBytes, stream);
 }
 
+extern "C" size_t gdn2_chunk_fwd_csize_smem_bytes(int chunk, int d_k) {
+  return chunk_fwd_csize_smem_bytes(chunk, d_k);
+}
+
+extern "C" gdn2_status gdn2_chunk_fwd_csize(const void* q, const void* k, const void* v, const float* log_alpha,
+                                            const void* b, const void* w, const float* S0, float* o, float* S_T,
+                                            int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, int chunk,
+                                            void* stream) {
+  if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+  if (dt != GDN2_BF16) return GDN2_ERR_DTYPE;  // the tensor-core path only
+  if (!sizes_ok(B, T, H, d_k, d_v) || chunk_fwd_csize_smem_bytes(chunk, d_k) == 0) return GDN2_ERR_SHAPE;
+  const bool tokens = (long long)B * T * H > 0;
+  if (tokens && (!q || !k || !v || !log_alpha || !b || !w || !o)) return GDN2_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, b, w, S0, o, S_T};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+  if ((long long)B * H == 0) return GDN2_OK;
+  ChunkArgs a{q, k, v, b, w, log_alpha, S0, o, S_T, B, T, H, d_k, d_v, true};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (T == 0) ? launch_state_copy(a, st) : launch_chunk_fwd_csize(a, chunk, st);
+  return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
+}
+
 extern "C" size_t gdn2_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v) {
   if (!sizes_ok(B, T, H, d_k, d_v)) return 0;
   return chunk_bwd_workspace_bytes(B, T, H, d_k, d_v);

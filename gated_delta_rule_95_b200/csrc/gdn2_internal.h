@@ -80,6 +80,10 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st);
 // fp32 inputs: fp32 CUDA-core kernel of the same chunkwise algorithm.
 cudaError_t launch_chunk_fwd_f32(const ChunkArgs& a, cudaStream_t st);
+// bf16, chunk size 32, 64 or 128: the chunk-size study kernel (warp-level tf32 MMAs);
+// shared memory per CTA, 0 for an unsupported (chunk, d_k).
+size_t chunk_fwd_csize_smem_bytes(int chunk, int dk);
+cudaError_t launch_chunk_fwd_csize(const ChunkArgs& a, int chunk, cudaStream_t st);
 // T = 0: S_T = S0 (or zeros).
 cudaError_t launch_state_copy(const ChunkArgs& a, cudaStream_t st);
 

@@ -185,3 +185,27 @@ def test_binding_rejects_cpu_tensors():
     la = torch.zeros(1, 64, 1, 128)
     with pytest.raises(ValueError):
         g.gdn2_chunk_fwd(x, x, x, la, x, x, o=x, S_T=torch.zeros(1, 1, 128, 128))
+
+
+def csize(q=A, k=A, v=A, la=A, b=A, w=A, S0=None, o=A, ST=None, B=1, T=300, H=2, dk=128, dv=128, dt=1, chunk=32):
+    return g.lib().gdn2_chunk_fwd_csize(q, k, v, la, b, w, S0, o, ST, B, T, H, dk, dv, dt, chunk, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(chunk=16), 2), (dict(chunk=96), 2), (dict(chunk=256), 2), (dict(chunk=0), 2), (dict(dk=96), 2),
+    (dict(dv=32), 2), (dict(T=-1), 2), (dict(dt=0), 3), (dict(dt=4), 3), (dict(q=None), 1), (dict(la=None), 1),
+    (dict(o=None), 1), (dict(w=M), 4), (dict(ST=M), 4), (dict(B=0), 0), (dict(H=0, chunk=128), 0),
+])
+def test_chunk_fwd_csize_validation(kw, status):
+    assert csize(**kw) == status
+
+
+def test_csize_shared_memory_footprint():
+    # Kn and Kb/Qh [C][d_k], A/P [C][C], U [C][32], state [d_k][32], Gamma_C [d_k], cumsum
+    # partials [256], all fp32
+    L = g.lib()
+    for C in (32, 64, 128):
+        for dk in (64, 128):
+            assert L.gdn2_chunk_fwd_csize_smem_bytes(C, dk) == 4 * (2 * C * dk + C * C + 32 * C + 33 * dk + 256)
+    assert L.gdn2_chunk_fwd_csize_smem_bytes(128, 128) <= 227 * 1024
+    assert L.gdn2_chunk_fwd_csize_smem_bytes(16, 128) == 0 and L.gdn2_chunk_fwd_csize_smem_bytes(64, 96) == 0

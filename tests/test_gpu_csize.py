@@ -1,0 +1,120 @@
+"""Chunk sizes 32, 64 and 128 on the GPU against the CPU oracle (parity): ragged lengths
+that end inside a chunk, both head sizes and mixed ones, entering states, state
+aliasing, the heavy-decay recipe at the largest chunk, and the prefill and mixed-gate
+workloads at full size on sampled units."""
+import dataclasses
+
+import pytest
+import torch
+
+import gdn2_inputs as gi
+import gated_delta_rule_95_b200 as g
+import oracle
+from tests.parity import TOL, oracle_units, rel_err
+
+pytestmark = pytest.mark.gpu
+BASE = gi.WORKLOADS["prefill_b8_h16_t4096"]
+NAMES = ("q", "k", "v", "log_alpha", "b", "w")
+CHUNKS = (32, 64, 128)
+
+
+def _cuda(d):
+    return {k: (None if v is None else v.cuda()) for k, v in d.items()}
+
+
+def _run(x, chunk, S0="input", **kw):
+    # outputs start as NaN, so that anything the call fails to write shows
+    B, T, H, dk = x["q"].shape
+    dv = x["v"].shape[-1]
+    o = torch.full((B, T, H, dv), float("nan"), device="cuda")
+    S_T = kw.pop("S_T", torch.full((B, H, dk, dv), float("nan"), device="cuda"))
+    s0 = x["S0"] if isinstance(S0, str) else S0
+    o, S = g.gdn2_chunk_fwd_csize(*(x[n] for n in NAMES), s0, chunk=chunk, o=o, S_T=S_T, **kw)
+    torch.cuda.synchronize()
+    return o, S
+
+
+def _oracle(d):
+    f = {n: gi.as_f64(d[n]) for n in NAMES}
+    return oracle.forward(**f, S0=None if d["S0"] is None else gi.as_f64(d["S0"]))
+
+
+SHAPES = [  # B, T, H, dk, dv, entering state
+    (2, 300, 2, 128, 128, True), (1, 1000, 2, 128, 128, False), (2, 77, 2, 64, 64, True),
+    (1, 1, 3, 128, 128, True), (1, 31, 1, 128, 64, True), (2, 129, 1, 64, 128, False),
+    (1, 256, 2, 128, 128, True),
+]
+
+
+@pytest.mark.parametrize("chunk", CHUNKS)
+@pytest.mark.parametrize("B,T,H,dk,dv,s0", SHAPES)
+def test_matches_oracle(chunk, B, T, H, dk, dv, s0):
+    wl = dataclasses.replace(BASE, dk=dk, dv=dv, state_std=0.05 if s0 else 0.0, seed=300 + T)
+    d = gi.prefill_inputs(wl, B=B, T=T, H=H)
+    o, S = _run(_cuda(d), chunk)
+    assert g.gdn2_device_status() == 0
+    o_ref, S_ref = _oracle(d)
+    assert rel_err(o.cpu().numpy(), o_ref) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), S_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("chunk", CHUNKS)
+def test_close_to_the_tensor_memory_kernel(chunk):
+    d = gi.prefill_inputs(dataclasses.replace(BASE, state_std=0.05), B=2, T=700, H=4)
+    x = _cuda(d)
+    o, S = _run(x, chunk)
+    o2, S2 = g.gdn2_chunk_fwd(*(x[n] for n in NAMES), x["S0"])
+    torch.cuda.synchronize()
+    assert rel_err(o.cpu().numpy(), o2.cpu().numpy()) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), S2.cpu().numpy()) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("chunk", CHUNKS)
+def test_state_aliasing_no_state_out_and_empty(chunk):
+    d = gi.prefill_inputs(dataclasses.replace(BASE, state_std=0.05, seed=11), B=2, T=150, H=2)
+    x = _cuda(d)
+    o1, S1 = _run(x, chunk)
+    S_io = x["S0"].clone()
+    o2, S2 = _run(x, chunk, S0=S_io, S_T=S_io)
+    o3, S3 = _run(x, chunk, S_T=None, want_state=False)
+    assert S3 is None
+    assert torch.equal(o1, o2) and torch.equal(o1, o3) and torch.equal(S1, S2)
+    e = gi.prefill_inputs(dataclasses.replace(BASE, state_std=0.05, seed=12), B=2, T=0, H=3)
+    o, S = _run(_cuda(e), chunk)
+    assert o.shape == (2, 0, 3, 128) and torch.equal(S.cpu(), e["S0"])
+
+
+def test_chunk_sizes_agree_with_each_other():
+    d = gi.prefill_inputs(dataclasses.replace(BASE, state_std=0.05, seed=13), B=1, T=1000, H=4)
+    x = _cuda(d)
+    outs = [_run(x, c) for c in CHUNKS]
+    for o, S in outs[1:]:
+        assert rel_err(o.cpu().numpy(), outs[0][0].cpu().numpy()) <= TOL["bf16"]
+        assert rel_err(S.cpu().numpy(), outs[0][1].cpu().numpy()) <= TOL["bf16"]
+
+
+def test_heavy_decay_at_the_largest_chunk():
+    # the long-context recipe (heavier decay) over 128-token chunks: the chunk-start
+    # decay reference needs the in-chunk cumulative log decay > -80
+    wl = gi.WORKLOADS["long_b1_h16_t65536"]
+    d = gi.prefill_inputs(wl, T=2048, H=4)
+    la = d["log_alpha"].view(1, -1, 128, 4, 128)
+    assert float(torch.cumsum(la, dim=2).min()) > -80.0
+    o, S = _run(_cuda(d), 128)
+    o_ref, S_ref = _oracle(d)
+    assert rel_err(o.cpu().numpy(), o_ref) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), S_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("chunk", CHUNKS)
+@pytest.mark.parametrize("name,units", [("prefill_b8_h16_t4096", [(0, 0), (6, 11)]),
+                                        ("mixed_b4_h32_t8192", [(0, 0), (1, 1), (3, 29)])])
+def test_full_size_sampled(chunk, name, units):
+    d = gi.prefill_inputs(gi.WORKLOADS[name])
+    o, S = _run(_cuda(d), chunk)
+    assert g.gdn2_device_status() == 0
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    o_c, S_c = o.cpu(), S.cpu()
+    for (bb, h), (o_ref, S_ref) in zip(units, oracle_units(d, units)):
+        assert rel_err(o_c[bb, :, h].numpy(), o_ref) <= TOL["bf16"], (bb, h)
+        assert rel_err(S_c[bb, h].numpy(), S_ref) <= TOL["bf16"], (bb, h)
