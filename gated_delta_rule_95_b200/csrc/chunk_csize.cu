@@ -21,8 +21,11 @@
 // in shared memory as the operand of the next chunk's products.  The inverse of each 16 x 16
 // diagonal block of (I + A) is formed in fp32 by one warp; the off-diagonal substitution
 // steps are MMAs.  All tiles are fp32 in shared memory, unpadded, with an XOR swizzle of
-// the column (see swz) that keeps every fragment read free of bank conflicts; the C x C
-// tile and the two C x d_k tiles set the footprint, 231 KB at C = 128, d_k = 128.
+// the column (see swz) that keeps every fragment read free of bank conflicts (row-major
+// operands are read with ldmatrix); the C x C tile and the two C x d_k tiles set the
+// footprint, 231 KB at C = 128, d_k = 128.  Per chunk, log alpha is copied in with 16-byte
+// asynchronous copies, its cumsum formed in place, and the bf16 inputs folded in by one
+// vectorised pass; Qh is built the same way by the warps that do not run the substitution.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -47,8 +50,6 @@ __device__ __forceinline__ int swz(int r, int c) {
   return r * L + (c ^ (((r & 3) << 3) | (r & 4)));
 }
 
-__device__ __forceinline__ uint32_t bits(float x) { return __float_as_uint(x); }
-__device__ __forceinline__ uint32_t nbits(float x) { return __float_as_uint(x) ^ 0x80000000u; }
 // four consecutive bf16 (8-byte aligned) as raw bits, and their fp32 values
 __device__ __forceinline__ uint2 ld_bf4(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
 __device__ __forceinline__ float4 bf4f(uint2 u) {
@@ -56,24 +57,132 @@ __device__ __forceinline__ float4 bf4f(uint2 u) {
                      __uint_as_float(u.y & 0xFFFF0000u));
 }
 
-// d[q] += sum over k in [k0, k1) of A(m0 + r, k) B(k, n0 + 8q + c) for the 16 x 8 tiles
-// q < NQ that share the rows m0 .. m0 + 15; fa / fb return the tf32 bit pattern of an
-// element.  Fragment layout as in mma_16x8x8_tf32.
-template <int NQ, class FA, class FB>
-__device__ __forceinline__ void mma_run(float (&d)[NQ][4], int m0, int n0, int k0, int k1, FA fa, FB fb) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll 2
-  for (int k = k0; k < k1; k += 8) {
-    const uint32_t a[4] = {fa(m0 + g, k + t), fa(m0 + g + 8, k + t), fa(m0 + g, k + t + 4),
-                           fa(m0 + g + 8, k + t + 4)};
+// Fragment loads for the MMAs, with g = lane / 4 and t = lane % 4 (layout of
+// mma_16x8x8_tf32).  A row-major swizzled tile gives an 8 x 4 block of tf32 per 16-byte row
+// segment, which is what ldmatrix reads (8 rows of 16 bytes per matrix; lane l receives
+// word l % 4 of row l / 4), so a whole A fragment, or the B fragments of two 8-column tiles
+// stored as rows (B = X^T), take one ldmatrix.x4 each.  Operands stored the other way round
+// ([k][m] or [k][n]) are read as single words; since k advances by 8 and the swizzle only
+// depends on the row mod 8, each lane's offsets are fixed and only k * L moves.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p))
+               : "memory");
+}
+// swizzle term of a row (the row mod 8 decides it)
+__device__ __forceinline__ int swf(int r) { return ((r & 3) << 3) | (r & 4); }
+
+// A operand: rows m0 .. m0 + 15 of a row-major tile with rows of L floats, columns k .. k + 7
+template <int L>
+struct ARow {
+  const float* p;  // this lane's ldmatrix row, column 0
+  int cx;          // its column offset (0 or 4), to be XOR-ed with the row's swizzle
+  int f;
+  __device__ __forceinline__ ARow(const float* tile, int m0) {
+    const int lane = threadIdx.x & 31, j = lane >> 3, r = m0 + (lane & 7) + 8 * (j & 1);
+    p = tile + r * L;
+    cx = 4 * (j >> 1);
+    f = swf(r);
+  }
+  __device__ __forceinline__ void load(uint32_t (&a)[4], int k) const { ldsm_x4(a, p + ((k + cx) ^ f)); }
+};
+// B operand of two 8-column tiles q, q + 1 stored as rows X[n][k] (B = X^T), rows n0 .. n0 + 15
+template <int L>
+struct BRows {
+  const float* p;
+  int cx, f;
+  __device__ __forceinline__ BRows(const float* tile, int n0) {
+    const int lane = threadIdx.x & 31, j = lane >> 3, r = n0 + (lane & 7) + 8 * (j >> 1);
+    p = tile + r * L;
+    cx = 4 * (j & 1);
+    f = swf(r);
+  }
+  // b0 = {tile q: k + t, k + t + 4}, b1 = the same for tile q + 1
+  __device__ __forceinline__ void load(uint32_t (&b0)[2], uint32_t (&b1)[2], int k) const {
+    uint32_t r[4];
+    ldsm_x4(r, p + ((k + cx) ^ f));
+    b0[0] = r[0];
+    b0[1] = r[1];
+    b1[0] = r[2];
+    b1[1] = r[3];
+  }
+};
+// an operand stored [k][c] with rows of L floats, read at (k + t, c0 + g) and (k + t + 4, c0 + g)
+// for the 8-column groups c0 = base + 8 q: as a B operand (c = n) or, twice, as a transposed
+// A operand (c = m, m + 8)
+template <int L, int NQ>
+struct KRow {
+  const float* p;
+  int o0[NQ], o1[NQ];
+  __device__ __forceinline__ KRow(const float* tile, int base) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    p = tile + t * L;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
-      const uint32_t b[2] = {fb(k + t, n0 + 8 * q + g), fb(k + t + 4, n0 + 8 * q + g)};
+      o0[q] = (base + 8 * q + g) ^ swf(t);
+      o1[q] = 4 * L + ((base + 8 * q + g) ^ swf(t + 4));
+    }
+  }
+  __device__ __forceinline__ void load(uint32_t (&b)[2], int q, int k) const {
+    b[0] = __float_as_uint(p[k * L + o0[q]]);
+    b[1] = __float_as_uint(p[k * L + o1[q]]);
+  }
+};
+
+__device__ __forceinline__ void neg4(uint32_t (&a)[4]) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) a[e] ^= 0x80000000u;
+}
+
+// d[q] (+)= A B over k in [k0, k1) for the 8-column tiles q < NQ, with A from ARow (negated
+// when NEG) and B from KRow
+template <int NQ, bool NEG, int LA, int LB>
+__device__ __forceinline__ void mma_ak(float (&d)[NQ][4], const ARow<LA>& A, const KRow<LB, NQ>& Bk, int k0, int k1) {
+#pragma unroll 2
+  for (int k = k0; k < k1; k += 8) {
+    uint32_t a[4];
+    A.load(a, k);
+    if (NEG) neg4(a);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      uint32_t b[2];
+      Bk.load(b, q, k);
       mma_16x8x8_tf32(d[q], a, b);
     }
   }
 }
-// f(row, col, d[q][e]) for every accumulator element of the tiles of mma_run
+// d[0..1] (+)= A X^T over k in [0, K): a 16 x 16 block, A from ARow, X from BRows
+template <int K, int LA, int LB>
+__device__ __forceinline__ void mma_ab(float (&d)[2][4], const ARow<LA>& A, const BRows<LB>& X) {
+#pragma unroll 4
+  for (int k = 0; k < K; k += 8) {
+    uint32_t a[4], b0[2], b1[2];
+    A.load(a, k);
+    X.load(b0, b1, k);
+    mma_16x8x8_tf32(d[0], a, b0);
+    mma_16x8x8_tf32(d[1], a, b1);
+  }
+}
+// d[q] += A B with A = Y^T read from a [k][m] tile (rows m0 .. m0 + 15) and B from KRow
+template <int NQ, int LA, int LB>
+__device__ __forceinline__ void mma_kk(float (&d)[NQ][4], const KRow<LA, 2>& At, const KRow<LB, NQ>& Bk, int k0,
+                                       int k1) {
+#pragma unroll 2
+  for (int k = k0; k < k1; k += 8) {
+    uint32_t lo[2], hi[2];
+    At.load(lo, 0, k);  // (k + t, m0 + g), (k + t + 4, m0 + g)
+    At.load(hi, 1, k);  // rows m0 + g + 8
+    const uint32_t a[4] = {lo[0], hi[0], lo[1], hi[1]};
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      uint32_t b[2];
+      Bk.load(b, q, k);
+      mma_16x8x8_tf32(d[q], a, b);
+    }
+  }
+}
+// f(row, col, d[q][e]) for every accumulator element of 16 x 8 tiles at (m0, n0 + 8q)
 template <int NQ, class F>
 __device__ __forceinline__ void for_frag(float (&d)[NQ][4], int m0, int n0, F f) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -97,8 +206,7 @@ template <int C, int DK>
 struct CsLayout {
   static constexpr int KN = 0;                // Kn [C][DK]
   static constexpr int KQ = KN + C * DK;      // Kb, then Qh [C][DK]
-  static constexpr int AP = KQ + C * DK;      // A with (I + A_II)^-1 on its diagonal blocks, then P
-                                              // [C][C]; cumsum partials while the operands are built
+  static constexpr int AP = KQ + C * DK;      // A with (I + A_II)^-1 on its diagonal blocks, then P [C][C]
   static constexpr int UM = AP + C * C;       // Vw, then R, then U [C][NV]
   static constexpr int SM = UM + C * NV;      // state, tf32 copy [DK][NV]
   static constexpr int GC = SM + DK * NV;     // Gamma_C [DK]
@@ -239,8 +347,7 @@ __global__ void __launch_bounds__(NTH, csize_min_blocks<C>()) chunk_fwd_csize_ke
       while ((mb + 1) * (mb + 2) / 2 <= blk) ++mb;
       const int jb = blk - mb * (mb + 1) / 2;
       float d[2][4] = {};
-      mma_run<2>(d, 16 * mb, 16 * jb, 0, DK, [&](int m, int k) { return bits(KQ[swz<DK>(m, k)]); },
-                 [&](int k, int s) { return bits(Kn[swz<DK>(s, k)]); });
+      mma_ab<DK>(d, ARow<DK>(KQ, 16 * mb), BRows<DK>(Kn, 16 * jb));
       for_frag<2>(d, 16 * mb, 16 * jb, [&](int m, int s, float& x) {
         AP[swz<C>(m, s)] = s < m ? (jb == mb ? x : to_tf32(x)) : 0.f;
       });
@@ -248,8 +355,7 @@ __global__ void __launch_bounds__(NTH, csize_min_blocks<C>()) chunk_fwd_csize_ke
     {
       float d[RQ][4];
       for_frag<RQ>(d, r_m0, r_n0, [&](int t, int j, float& x) { x = Um[swz<NV>(t, j)]; });
-      mma_run<RQ>(d, r_m0, r_n0, 0, DK, [&](int m, int k) { return nbits(KQ[swz<DK>(m, k)]); },
-                  [&](int k, int j) { return bits(Sm[swz<NV>(k, j)]); });
+      mma_ak<RQ, true>(d, ARow<DK>(KQ, r_m0), KRow<NV, RQ>(Sm, r_n0), 0, DK);
       for_frag<RQ>(d, r_m0, r_n0, [&](int t, int j, float& x) { Um[swz<NV>(t, j)] = x; });
     }
     __syncthreads();
@@ -280,13 +386,11 @@ __global__ void __launch_bounds__(NTH, csize_min_blocks<C>()) chunk_fwd_csize_ke
         const int m0 = 16 * mb;
         float d[1][4];
         for_frag<1>(d, m0, n0, [&](int t, int j, float& x) { x = Um[swz<NV>(t, j)]; });
-        mma_run<1>(d, m0, n0, 0, m0, [&](int m, int k) { return nbits(AP[swz<C>(m, k)]); },
-                   [&](int k, int j) { return bits(Um[swz<NV>(k, j)]); });
+        mma_ak<1, true>(d, ARow<C>(AP, m0), KRow<NV, 1>(Um, n0), 0, m0);
         for_frag<1>(d, m0, n0, [&](int t, int j, float& x) { Um[swz<NV>(t, j)] = to_tf32(x); });
         __syncwarp();
         float e[1][4] = {};
-        mma_run<1>(e, m0, n0, m0, m0 + 16, [&](int m, int k) { return bits(AP[swz<C>(m, k)]); },
-                   [&](int k, int j) { return bits(Um[swz<NV>(k, j)]); });
+        mma_ak<1, false>(e, ARow<C>(AP, m0), KRow<NV, 1>(Um, n0), m0, m0 + 16);
         __syncwarp();
         for_frag<1>(e, m0, n0, [&](int t, int j, float& x) { Um[swz<NV>(t, j)] = to_tf32(x); });
         __syncwarp();
@@ -338,17 +442,14 @@ __global__ void __launch_bounds__(NTH, csize_min_blocks<C>()) chunk_fwd_csize_ke
       while ((mb + 1) * (mb + 2) / 2 <= blk) ++mb;
       const int jb = blk - mb * (mb + 1) / 2;
       float d[2][4] = {};
-      mma_run<2>(d, 16 * mb, 16 * jb, 0, DK, [&](int m, int k) { return bits(KQ[swz<DK>(m, k)]); },
-                 [&](int k, int s) { return bits(Kn[swz<DK>(s, k)]); });
+      mma_ab<DK>(d, ARow<DK>(KQ, 16 * mb), BRows<DK>(Kn, 16 * jb));
       for_frag<2>(d, 16 * mb, 16 * jb, [&](int m, int s, float& x) { AP[swz<C>(m, s)] = s <= m ? to_tf32(x) : 0.f; });
     }
     float Oacc[RQ][4] = {};
-    mma_run<RQ>(Oacc, r_m0, r_n0, 0, DK, [&](int m, int k) { return bits(KQ[swz<DK>(m, k)]); },
-                [&](int k, int j) { return bits(Sm[swz<NV>(k, j)]); });
+    mma_ak<RQ, false>(Oacc, ARow<DK>(KQ, r_m0), KRow<NV, RQ>(Sm, r_n0), 0, DK);
     __syncthreads();
     // (6) O += P U and store; S = Diag(Gamma_C) (S + Kn^T U)
-    mma_run<RQ>(Oacc, r_m0, r_n0, 0, r_m0 + 16, [&](int m, int s) { return bits(AP[swz<C>(m, s)]); },
-                [&](int s, int j) { return bits(Um[swz<NV>(s, j)]); });
+    mma_ak<RQ, false>(Oacc, ARow<C>(AP, r_m0), KRow<NV, RQ>(Um, r_n0), 0, r_m0 + 16);
 #pragma unroll
     for (int q = 0; q < RQ; ++q)
 #pragma unroll
@@ -358,8 +459,7 @@ __global__ void __launch_bounds__(NTH, csize_min_blocks<C>()) chunk_fwd_csize_ke
           *reinterpret_cast<float2*>(p.o + tok(t0 + t) * p.dv + j0 + r_n0 + 8 * q + 2 * t4) =
               make_float2(Oacc[q][2 * hf], Oacc[q][2 * hf + 1]);
       }
-    mma_run<SQ>(Sacc, s_m0, s_n0, 0, C, [&](int i, int s) { return bits(Kn[swz<DK>(s, i)]); },
-                [&](int s, int j) { return bits(Um[swz<NV>(s, j)]); });
+    mma_kk<SQ>(Sacc, KRow<DK, 2>(Kn, s_m0), KRow<NV, SQ>(Um, s_n0), 0, C);
     for_frag<SQ>(Sacc, s_m0, s_n0, [&](int i, int, float& x) { x *= gC[i]; });
     __syncthreads();
   }

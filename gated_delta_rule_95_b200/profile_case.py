@@ -3,6 +3,7 @@
     python -m gated_delta_rule_95_b200.profile_case --kind prefill --B 8 --H 16 --T 1024 --reps 2
     python -m gated_delta_rule_95_b200.profile_case --kind decode --B 256 --H 16 --reps 4
     python -m gated_delta_rule_95_b200.profile_case --kind bwd --B 2 --H 16 --T 1024 --reps 2
+    python -m gated_delta_rule_95_b200.profile_case --kind csize --chunk 128 --B 8 --H 16 --T 1024 --reps 2
 
 Inputs follow the recipe of the named workload (gdn2_inputs) with the given
 sizes; it exits 0 after a device synchronisation and a clean device status.
@@ -20,12 +21,13 @@ if ROOT not in sys.path:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", choices=["prefill", "decode", "bwd"], required=True)
+    ap.add_argument("--kind", choices=["prefill", "decode", "bwd", "csize"], required=True)
     ap.add_argument("--workload", default=None)
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--H", type=int, default=None)
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--reps", type=int, default=2)
+    ap.add_argument("--chunk", type=int, default=64)
     a = ap.parse_args()
 
     import torch
@@ -40,6 +42,12 @@ def main():
         x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
         for _ in range(a.reps):
             g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
+    elif a.kind == "csize":
+        wl = gi.WORKLOADS[a.workload or "prefill_b8_h16_t4096"]
+        d = gi.prefill_inputs(wl, B=a.B, T=a.T, H=a.H)
+        x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+        for _ in range(a.reps):
+            g.gdn2_chunk_fwd_csize(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], chunk=a.chunk)
     elif a.kind == "bwd":
         wl = gi.WORKLOADS[a.workload or "prefill_b8_h16_t4096"]
         d = gi.prefill_inputs(wl, B=a.B, T=a.T, H=a.H)
