@@ -14,8 +14,8 @@
 //     O  = Qh S + P U
 //     S  = Diag(Gamma_C) (S + Kn^T U)
 //
-// One CTA of 8 warps owns one (batch, head) and 32 value columns (value columns never mix
-// in the recurrence) and walks the chunks in order.  Products run on warp-level tensor-core
+// One CTA of 8 warps (16 at C = 128) owns one (batch, head) and 32 value columns (value
+// columns never mix in the recurrence) and walks the chunks in order.  Products run on warp-level tensor-core
 // MMAs (m16n8k8, tf32 operands rounded to nearest, fp32 accumulation); the state lives in
 // the registers of its owning warps as an fp32 accumulator across chunks, with a tf32 copy
 // in shared memory as the operand of the next chunk's products.  The inverse of each 16 x 16
@@ -37,9 +37,14 @@
 namespace gdn2 {
 namespace {
 
-constexpr int NW = 8;         // warps per CTA
-constexpr int NTH = 32 * NW;  // threads per CTA
 constexpr int NV = 32;        // value columns per CTA
+
+// Warps per CTA: 8, or 16 at C = 128, where the shared memory leaves one CTA per SM
+template <int C>
+struct CsWarps {
+  static constexpr int NW = C == 128 ? 16 : 8;
+  static constexpr int NTH = 32 * NW;
+};
 
 // Element (r, c) of a tile with rows of L floats (L a multiple of 32).  The column is
 // XOR-ed with f(r) = 8 (r mod 4) + 4 ((r mod 8) >= 4): the fragment reads of an MMA touch
@@ -211,7 +216,7 @@ struct CsLayout {
   static constexpr int SM = UM + C * NV;      // state, tf32 copy [DK][NV]
   static constexpr int GC = SM + DK * NV;     // Gamma_C [DK]
   static constexpr int TOT = GC + DK;         // cumsum partials [token range][DK]
-  static constexpr int FLOATS = TOT + NTH;
+  static constexpr int FLOATS = TOT + CsWarps<C>::NTH;
   static constexpr size_t BYTES = FLOATS * sizeof(float);
   static_assert(BYTES <= 232448, "shared memory per CTA");
 };
@@ -221,20 +226,22 @@ template <int C>
 constexpr int csize_min_blocks() { return C == 32 ? 3 : C == 64 ? 2 : 1; }
 
 template <int C, int DK>
-__global__ void __launch_bounds__(NTH, csize_min_blocks<C>()) chunk_fwd_csize_kernel(const CsParams p) {
+__global__ void __launch_bounds__(CsWarps<C>::NTH, csize_min_blocks<C>()) chunk_fwd_csize_kernel(const CsParams p) {
   using Lay = CsLayout<C, DK>;
+  constexpr int NW = CsWarps<C>::NW, NTH = CsWarps<C>::NTH;
   constexpr int NB = C / 16;                    // 16-row blocks of a chunk
   constexpr int NBLK = NB * (NB + 1) / 2;       // 16 x 16 blocks on and below the diagonal
   constexpr int SQ = (DK / 16) * (NV / 8) / NW; // state tiles per warp (one row block)
   constexpr int RQ = (C / 16) * (NV / 8) / NW;  // output tiles per warp (C >= 32: >= 1)
   constexpr int PT = NTH / DK, TP = C / PT;     // operand build: threads per key channel, tokens each
-  constexpr int QTH = NTH - 32 * (NV / 8);      // Qh build: the warps not in the substitution
+  constexpr int QTH = NTH - 32 * (NV / 8) < 2 * DK ? NTH - 32 * (NV / 8) : 2 * DK;  // Qh build: warps
+                                                // not in the substitution, at most two per channel
   constexpr int QPT = QTH / DK, QTP = C / QPT;
   constexpr int Q4K = C * DK / 4 / NTH, Q4V = C * NV / 4 / NTH, Q4Q = C * DK / 4 / QTH;  // 4-element groups per thread
   static_assert(Q4K * 4 * NTH == C * DK && Q4V * 4 * NTH == C * NV && Q4Q * 4 * QTH == C * DK, "copy split");
   static_assert((DK / 16) * (NV / 8) % NW == 0 && SQ >= 1 && SQ <= NV / 8, "state tiles: one row block per warp");
   static_assert((C / 16) * (NV / 8) % NW == 0 && RQ >= 1 && RQ <= NV / 8, "output tiles: one row block per warp");
-  static_assert(QPT >= 1 && QTH % DK == 0, "Qh build threads");
+  static_assert(QPT >= 1 && QTH % DK == 0 && QTH % 32 == 0 && C % QPT == 0, "Qh build threads");
   static_assert(NB <= NW, "one warp per diagonal block");
 
   extern __shared__ __align__(16) float sm[];
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(NTH, csize_min_blocks<C>()) chunk_fwd_csize_ke
         for_frag<1>(e, m0, n0, [&](int t, int j, float& x) { Um[swz<NV>(t, j)] = to_tf32(x); });
         __syncwarp();
       }
-    } else {
+    } else if (tid - 32 * (NV / 8) < QTH) {
       // Qh = Q*Gamma into KQ (free since the A and R products): log alpha copied in, its
       // cumsum formed in place, then multiplied out; barrier 1 spans these warps only
       const int qt = tid - 32 * (NV / 8), qi = qt % DK, qp = qt / DK;
@@ -481,7 +488,7 @@ cudaError_t launch_c(const ChunkArgs& a, cudaStream_t st) {
              static_cast<const __nv_bfloat16*>(a.w), a.log_alpha, a.S0, a.o, a.S_T, a.T, a.H, a.dv};
   const long long grid = (long long)a.B * a.H * (a.dv / NV);
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-  chunk_fwd_csize_kernel<C, DK><<<(unsigned)grid, NTH, smem, st>>>(p);
+  chunk_fwd_csize_kernel<C, DK><<<(unsigned)grid, CsWarps<C>::NTH, smem, st>>>(p);
   return cudaGetLastError();
 }
 
