@@ -47,6 +47,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "gdn2_internal.h"
 #include "ptx.cuh"
 
@@ -532,14 +534,20 @@ __global__ void __launch_bounds__(NT, 1)
       float vw[32];
       const uint32_t pnl = (uint32_t)(ch >> 6) * R64;
       const int chk = (ch & 63) >> 3, byt = (ch & 7) * 2;
+      const int lim = len - (C * cc + 32 * hf);  // rows of this half inside the sequence
+      // (packed sequences: the rows past the end, only in a sequence's last chunk, are masked)
+      auto fill = [&](auto masked) {
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        const uint32_t ro = pnl + sw128_off(32 * hf + r, chk) + byt;
-        const bool tv = !VARLEN || C * cc + 32 * hf + r < len;
-        float wr = bf16_at(sm + RAW_W + ro);
-        if constexpr (PREP) wr = sigmoid_fast(wr);
-        vw[r] = (vval && tv && !sp_trans) ? bf16_at(sm + RAW_V + ro) * wr : 0.f;
-      }
+        for (int r = 0; r < 32; ++r) {
+          const uint32_t ro = pnl + sw128_off(32 * hf + r, chk) + byt;
+          const bool tv = !decltype(masked)::value || r < lim;
+          float wr = bf16_at(sm + RAW_W + ro);
+          if constexpr (PREP) wr = sigmoid_fast(wr);
+          vw[r] = (vval && tv && !sp_trans) ? bf16_at(sm + RAW_V + ro) * wr : 0.f;
+        }
+      };
+      if (VARLEN && lim < 32) fill(std::true_type{});
+      else fill(std::false_type{});
       tmem_st32(tlane + TM_VW + 64 * (cc & 1) + 32 * hf, vw);
       tmem_st_wait();
       return ok;
@@ -551,23 +559,30 @@ __global__ void __launch_bounds__(NT, 1)
       unsigned char* la_w = sm + OFF_LA;
       ok = ok && wait_on(&ms.bar_la, ph_la);
       float x[32];
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-        x[r] = (kval && (!VARLEN || C * cc + 32 * hf + r < len))
-                   ? *reinterpret_cast<const float*>(la_w + f32_off(32 * hf + r, ch, R64)) : 0.f;
       float acc = 0.f;
+      const int lim = len - (C * cc + 32 * hf);  // rows of this half inside the sequence
+      // rows past the sequence add nothing: masked only in its last chunk (packed sequences,
+      // whose tile rows there belong to the next sequence; raw projections, whose tail rows
+      // read a = 0, and softplus(0) is not 0)
+      auto scan = [&](auto masked) {
+        constexpr bool M = decltype(masked)::value;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        if constexpr (PREP) {
-          // log2 alpha = -s_h softplus(a) log2 e.  Rows past the sequence add nothing (a
-          // fixed-length batch's tail rows read a = 0, whose softplus is not 0).
-          const bool vr = kval && C * cc + 32 * hf + r < len;
-          acc -= vr ? dsc * softplus_log2(x[r]) : 0.f;
-        } else {
-          acc = fmaf(x[r], LOG2E, acc);
+        for (int r = 0; r < 32; ++r)
+          x[r] = (kval && (!M || r < lim)) ? *reinterpret_cast<const float*>(la_w + f32_off(32 * hf + r, ch, R64))
+                                           : 0.f;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          if constexpr (PREP) {  // log2 alpha = -s_h softplus(a) log2 e
+            const bool vr = kval && (!M || r < lim);
+            acc -= vr ? dsc * softplus_log2(x[r]) : 0.f;
+          } else {
+            acc = fmaf(x[r], LOG2E, acc);
+          }
+          x[r] = acc;
         }
-        x[r] = acc;
-      }
+      };
+      if ((VARLEN || PREP) && lim < 32) scan(std::true_type{});
+      else scan(std::false_type{});
       ms.segtot[hf][ch] = acc;
       named_bar_sync(BAR_AUX, NCOMP - NSOLVE);
       const float off = hf ? ms.segtot[0][ch] : 0.f;
@@ -627,7 +642,7 @@ __global__ void __launch_bounds__(NT, 1)
       float2 nkb[8], qh[8], kn[8];
       // (raw projections: warps 0-7 have seen these copies land already, one chunk ahead)
       bool ok_raw = (PREP && warp < NSOLVE / 32) ? true : wait_on(&ms.bar_raw, ph_raw);
-      {
+      auto build = [&](auto masked) {
         const unsigned char* la_t = sm + OFF_LA;
         const uint32_t pnl = (uint32_t)(c2 >> 6) * R64;  // raw tiles: panels of 64 channels
         const int chk = (c2 & 63) >> 3, byt = (c2 & 7) * 2;
@@ -636,8 +651,9 @@ __global__ void __launch_bounds__(NT, 1)
           const int t = 8 * ts + r;
           const uint32_t ro = pnl + sw128_off(t, chk) + byt;
           float2 G = make_float2(1.f, 1.f), kk = make_float2(0.f, 0.f), bg = kk, qq = kk;
-          // (packed sequences: the tile rows past this sequence's end hold the next one's tokens)
-          if (kv2 && (!VARLEN || C * c + t < len)) {
+          // (packed sequences: the tile rows past this sequence's end hold the next one's
+          // tokens; masked only in its last chunk)
+          if (kv2 && (!decltype(masked)::value || C * c + t < len)) {
             G = *reinterpret_cast<const float2*>(la_t + f32_off(t, c2, R64));
             kk = bf16x2_at(sm + RAW_K + ro);
             bg = bf16x2_at(sm + RAW_B + ro);
@@ -654,7 +670,9 @@ __global__ void __launch_bounds__(NT, 1)
           qh[r] = make_float2(qq.x * G.x, qq.y * G.y);
           kn[r] = make_float2(kk.x * Gi.x, kk.y * Gi.y);
         }
-      }
+      };
+      if (VARLEN && C * c + C > len) build(std::true_type{});
+      else build(std::false_type{});
       // the previous chunk's last product must be done before Kn^T, O and S are touched,
       // and every raw read before the operand tiles overwrite the staging
       {
