@@ -550,11 +550,17 @@ __global__ void __launch_bounds__(NT, 1)
           const bool tv = !decltype(masked)::value || r < lim;
           float wr = bf16_at(sm + RAW_W + ro);
           if constexpr (PREP) wr = sigmoid_fast(wr);
-          vw[r] = (vval && tv && !sp_trans) ? bf16_at(sm + RAW_V + ro) * wr : 0.f;
+          vw[r] = (vval && tv) ? bf16_at(sm + RAW_V + ro) * wr : 0.f;
         }
       };
-      if (VARLEN && lim < 32) fill(std::true_type{});
-      else fill(std::false_type{});
+      if (sp_trans) {  // transition runs of the sequence split: no write term
+#pragma unroll
+        for (int r = 0; r < 32; ++r) vw[r] = 0.f;
+      } else if (VARLEN && lim < 32) {
+        fill(std::true_type{});
+      } else {
+        fill(std::false_type{});
+      }
       tmem_st32(tlane + TM_VW + 64 * (cc & 1) + 32 * hf, vw);
       tmem_st_wait();
       return ok;
