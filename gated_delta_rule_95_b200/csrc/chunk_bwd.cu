@@ -322,23 +322,45 @@ __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * M
       }
   };
   // T = (I + A)^-1 from A (strictly lower, in X1), by blocks: the 16 x 16 diagonal blocks by
-  // forward substitution (four threads per column split each row's dot product), then the
+  // forward substitution (one warp per block, a column per lane, in registers), then the
   // 2 x 2 block merges T21 = -T22 (A21 T11) at 32 and 64 (products staged in the R tile,
   // free at this point).
   auto solve = [&]() {  // (every entry above the diagonal of T is zero from the start; the
-                        // first 256 threads work, the rest only meet the barriers)
-    if (tid < 256) {
-      const int s = tid >> 2, part = tid & 3, base = s & ~15;  // a warp's 8 columns share a block
-      if (part == 0) Tm[s * LC + s] = 1.f;
-      __syncwarp();
-      for (int t = base + 1; t < base + 16; ++t) {
-        float acc = 0.f;
-        if (t > s)
-          for (int r = s + part; r < t; r += 4) acc = fmaf(X1[t * LC + r], Tm[r * LC + s], acc);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (t > s && part == 0) Tm[t * LC + s] = -acc;
-        __syncwarp();
+                        // first 128 or 256 threads work, the rest only meet the barriers)
+    if (tid < 128) {
+      // warp w: diagonal block w (rows 16 w ..); lane j < 16 forms column j of its inverse in
+      // registers by forward substitution (x[s] = 0 for s < j, so each row sums over s < r)
+      const int base = 16 * (tid >> 5), j = tid & 15;
+      const float* Ab = X1 + base * LC + base;
+      float x[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float ar[16];
+        if constexpr (LC % 4 == 0) {  // 16-byte aligned rows: vector loads
+#pragma unroll
+          for (int q4 = 0; q4 < (r + 3) / 4; ++q4) {
+            const float4 a = *reinterpret_cast<const float4*>(Ab + r * LC + 4 * q4);
+            ar[4 * q4] = a.x;
+            ar[4 * q4 + 1] = a.y;
+            ar[4 * q4 + 2] = a.z;
+            ar[4 * q4 + 3] = a.w;
+          }
+        } else {
+#pragma unroll
+          for (int s2 = 0; s2 < r; ++s2) ar[s2] = Ab[r * LC + s2];
+        }
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 + 1 < r; s2 += 2) {
+          acc0 = fmaf(ar[s2], x[s2], acc0);
+          acc1 = fmaf(ar[s2 + 1], x[s2 + 1], acc1);
+        }
+        if (r & 1) acc0 = fmaf(ar[r - 1], x[r - 1], acc0);
+        x[r] = r == j ? 1.f : (r > j ? -(acc0 + acc1) : 0.f);
+      }
+      if ((tid & 31) < 16) {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tm[(base + r) * LC + base + j] = x[r];
       }
     }
     __syncthreads();
