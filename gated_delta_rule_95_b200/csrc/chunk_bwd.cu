@@ -17,13 +17,17 @@
 // dW = dVw*V, dV = dVw*W, dg = dKb*Kb + dQh*Qh - dKn*Kn (+ dGamma_C*Gamma_C on the last
 // row), dlog alpha = reverse cumsum of dg over the chunk.
 //
-// Kernels: chunk_bwd_kernel, one CTA of 256 threads per (batch, head, 32 value columns)
-// (value columns never mix in the recurrence, so dS, U, R and the per-column gradients
-// split by columns; the key-side gradients dKb, dKn, dQh, dGamma_C are sums over the
-// column slices and are accumulated with atomics).  It first sweeps the chunks forward to
-// store each chunk's entering state (its column slice) in the workspace, then sweeps them
+// Kernels: chunk_bwd_kernel, one CTA per (batch, head, 32 value columns) — 16 warps for
+// bf16 inputs, 8 for fp32 — (value columns never mix in the recurrence, so dS, U, R and
+// the per-column gradients split by columns; the key-side gradients dKb, dKn, dQh,
+// dGamma_C are sums over the column slices and are accumulated with atomics).  The state
+// entering each chunk comes first: for bf16 inputs with d_k = d_v from the tensor-core
+// forward's checkpoint pass (a separate launch), otherwise from a forward sweep of this
+// kernel over the chunks (its column slice, into the workspace); then the chunks are swept
 // in reverse.  chunk_bwd_finish_kernel turns the summed dKb, dKn, dQh into dq, dk, db and
-// dlog alpha.  All arithmetic is fp32 on the CUDA cores, operands in shared memory.
+// dlog alpha.  Operands live in shared memory; the products run as tf32 warp-level MMAs
+// (fp32 accumulation) for bf16 inputs and as fp32 FFMA on the CUDA cores for fp32 inputs
+// (their 1e-4 accuracy bar); everything else is fp32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

@@ -120,7 +120,9 @@ GDN2_API gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const vo
  * respect to q, k, v, log_alpha, b, w and S0 (reverse mode of the chunkwise WY form of
  * the Gated DeltaNet-2 guide's "Chunkwise Parallel Algorithm for GPU Training", the
  * training-time counterpart of the forward).  The forward's inputs are passed again; the
- * chunk states are recomputed in fp32.  All arithmetic fp32 (CUDA cores).
+ * chunk states are recomputed (bf16 inputs with d_k = d_v: by the tensor-core forward, tf32
+ * products; otherwise in fp32).  Products: tf32 warp-level tensor-core MMAs with fp32
+ * accumulation for bf16 inputs, fp32 on the CUDA cores for fp32 inputs.
  *
  *   q .. w, S0, B, T, H, d_k, d_v, dt : as gdn2_chunk_fwd (the forward's inputs)
  *   dO          : [B, T, H, d_v] fp32
