@@ -851,13 +851,8 @@ cudaError_t launch_bwd_t(const ChunkBwdArgs& a, cudaStream_t st) {
   }
   constexpr size_t smem = bwd_smem_bytes<DK, std::is_same<T, __nv_bfloat16>::value>();
   static_assert(smem <= 227 * 1024, "shared memory of the backward CTA");
-  static bool attr = false;
-  if (!attr) {
-    if ((e = cudaFuncSetAttribute(chunk_bwd_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem)) != cudaSuccess)
-      return e;
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if ((e = smem_limit_once(chunk_bwd_kernel<T, DK, DV>, (int)smem, attr_done)) != cudaSuccess) return e;
   constexpr int nth = std::is_same<T, __nv_bfloat16>::value ? 32 * MW : BT;
   chunk_bwd_kernel<T, DK, DV><<<(unsigned)(BH * (DV / BJ)), nth, smem, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

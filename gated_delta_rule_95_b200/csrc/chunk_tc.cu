@@ -1111,13 +1111,9 @@ template <int DK, int DV, bool VARLEN, bool PREP, bool SPLIT = false>
 cudaError_t launch_shape(int grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
                          const CUtensorMap& mv, const CUtensorMap& mb, const CUtensorMap& mw, const CUtensorMap& mla,
                          const CUtensorMap& mo, const TcParams& p) {
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};  // per instantiation, a bit per device
+  cudaError_t e = smem_limit_once(chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP, SPLIT>, (int)SMEM_BYTES, attr_done);
+  if (e != cudaSuccess) return e;
   chunk_fwd_tc_kernel<DK, DV, VARLEN, PREP, SPLIT><<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mb, mw, mla, mo, p);
   return cudaSuccess;
 }
@@ -1159,13 +1155,8 @@ cudaError_t launch_split(const ChunkArgs& a, TcParams p, cudaStream_t st, const 
     const int D = a.dk;
     const size_t smem = (size_t)(D * (D + 1) + D * 16) * sizeof(float);
     if (D == 128) {
-      static bool attr = false;
-      if (!attr) {
-        if ((e = cudaFuncSetAttribute(split_chain_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem)) != cudaSuccess)
-          return e;
-        attr = true;
-      }
+      static std::atomic<unsigned long long> attr_done{0};
+      if ((e = smem_limit_once(split_chain_kernel<128>, (int)smem, attr_done)) != cudaSuccess) return e;
       split_chain_kernel<128><<<BH * (D / 16), 256, smem, st>>>(a.workspace, BH, P);
     } else {
       split_chain_kernel<64><<<BH * (D / 16), 256, smem, st>>>(a.workspace, BH, P);

@@ -2,6 +2,8 @@
 #pragma once
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 namespace gdn2 {
 
 struct DecodeArgs {
@@ -43,6 +45,22 @@ enum : unsigned {
   kErrBadSeqlens = 2u    // packed-sequence offsets out of order or out of range
 };
 unsigned* device_error_word();
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// device (the attribute belongs to each device's context): `done` holds one bit per device
+// index below 64 (higher indices set the attribute on every call).  Safe from several host
+// threads: a race sets the same value twice.
+template <class K>
+cudaError_t smem_limit_once(K* kernel, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Backward of the chunkwise forward (gradients fp32; dq, dk, db are zeroed and accumulated).
 struct ChunkBwdArgs {

@@ -235,16 +235,12 @@ cudaError_t launch_typed(const ShortConvArgs& a, cudaStream_t st) {
     constexpr int STRIP = strip_of<T>();
     const long long blocks = (long long)((ntok + STRIP - 1) / STRIP) * ncb;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    static bool attr_set = false;  // per element type
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(short_conv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)conv_smem_bytes<T>());
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};  // per element type, a bit per device
+    cudaError_t e = smem_limit_once(short_conv_kernel<T>, (int)conv_smem_bytes<T>(), attr_done);
+    if (e != cudaSuccess) return e;
     short_conv_kernel<T><<<(unsigned)blocks, CONV_THREADS, conv_smem_bytes<T>(), st>>>(x, a.weight, a.bias, a.cu_seqlens, nseq, hin, y,
                                                                      ntok, a.T, a.C, ncb, device_error_word());
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (hout) {
