@@ -33,8 +33,10 @@ DECODE = gi.WORKLOADS["decode_b256_h16"]
 PACKED = gi.WORKLOADS["packed_n64_h16"]
 METRIC = "GDN-2 prefill tokens/s per layer"
 UNIT = "tokens/s"
-# algorithmic HBM bytes per token-head: q,k,v,b,w bf16 + log-alpha fp32 in, o fp32 out
-PREFILL_BYTES_PER_TOKEN_HEAD = 5 * 128 * 2 + 128 * 4 + 128 * 4
+# algorithmic HBM bytes per token-head: q,k,v,b,w bf16 + log-alpha fp32 in, o out (bf16 in
+# the algorithmic figure of the hot path; the library writes o in fp32, 256 B more)
+PREFILL_BYTES_PER_TOKEN_HEAD = 5 * 128 * 2 + 128 * 4 + 128 * 2
+PREFILL_BYTES_FP32_O = PREFILL_BYTES_PER_TOKEN_HEAD + 128 * 2
 # dense-tile tensor FLOPs per token-head at C=64, d=128: 2C(3dk + 2dv) + 6 dk dv
 PREFILL_FLOP_PER_TOKEN_HEAD = 2 * 64 * (3 * 128 + 2 * 128) + 6 * 128 * 128
 # state read + write per (sequence, head) and step, fp32 128x128
@@ -413,10 +415,10 @@ def time_prefill_e2e(args, dev):
         drained[j].record(s_out)
 
     with torch.cuda.stream(s_in):
-        for i in range(max(1, min(args.warmup, 2))):
+        for i in range(args.warmup):
             step(i)
         torch.cuda.synchronize()
-        n = max(1, min(args.steps, 5))
+        n = args.steps
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(s_in)
@@ -427,7 +429,7 @@ def time_prefill_e2e(args, dev):
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / n
     return {"value": B * T / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms,
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n, "warmup": args.warmup,
             "pipelining": "two streams: step i's device->host copy overlaps step i+1's host->device copy"}
 
 
@@ -579,60 +581,38 @@ def main():
             dist.destroy_process_group()
         return
 
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "tf32", "data": "synthetic (seeded, see DESIGN.md)",
-        "config": config_dict(),
-        "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel", "achieved": achieved,
-                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                     "traffic": traffic, "peak_src": pk["src"],
-                     "bytes_per_token_head": PREFILL_BYTES_PER_TOKEN_HEAD,
-                     "tensor": {"achieved_tflops": tflops, "peak_tflops": pk["bf16_tflops"],
-                                "frac": tflops / pk["bf16_tflops"],
-                                "peak_tflops_tf32": pk["bf16_tflops"] * TF32_PER_BF16,
-                                "frac_tf32": tflops / (pk["bf16_tflops"] * TF32_PER_BF16),
-                                "flop_per_token_head": PREFILL_FLOP_PER_TOKEN_HEAD}},
-        "decode": {"metric": "GDN-2 decode steps/s", "value": 1e3 / dec["ms_per_step"], "unit": "steps/s",
-                   "ms_per_step": dec["ms_per_step"], "steps": args.decode_steps,
-                   "workload": "decode_b256_h16: B=256 H=16 d_k=d_v=128, bf16 tokens, fp32 state",
-                   "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": dec_gbs,
-                                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],
-                                "traffic": profile_traffic("decode_step_kernel")},
-                   "clocks": dec["clocks"]},
+    def hbm(kernel, gbs, traffic=None):
+        return {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"], "traffic": traffic}
+
+    # secondary legs: one JSON line of their own, printed before the result line
+    legs = {
+        "legs": "secondary workloads (the result line follows)",
         "decode_raw": {"metric": "GDN-2 decode steps/s, raw projections", "value": 1e3 / dec_raw["ms_per_step"],
                        "unit": "steps/s", "ms_per_step": dec_raw["ms_per_step"], "steps": args.decode_steps,
                        "workload": "decode_b256_h16 through gdn2_decode_step_raw (q, k normalised, sigmoid gates "
                                    "and softplus decay inside the step)",
-                       "roofline": {"bound": "hbm", "kernel": "decode_step_kernel (raw)", "achieved": decr_gbs,
-                                    "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": decr_gbs / pk["hbm_gbs"],
-                                    "traffic": None}},
+                       "roofline": hbm("decode_step_kernel (raw)", decr_gbs)},
         "packed": {"metric": "GDN-2 packed prefill tokens/s per layer", "value": pak["tokens"] / (pak["ms"] * 1e-3),
                    "unit": "tokens/s", "ms_per_step": pak["ms"], "steps": args.steps,
                    "workload": f"packed_n64_h16: {pak['n_seq']} sequences, lengths log-uniform in [16, 8192] "
                                f"({pak['tokens']} tokens), H=16 d_k=d_v=128, bf16, entering states N(0, 0.02)",
-                   "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (packed)", "achieved": pak_gbs,
-                                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": pak_gbs / pk["hbm_gbs"],
-                                "traffic": None}},
-        "raw": {"metric": "GDN-2 prefill tokens/s per layer, raw projections", "value": raw["tokens"] / (raw["ms"] * 1e-3),
-                "unit": "tokens/s", "ms_per_step": raw["ms"], "steps": args.steps,
+                   "roofline": hbm("chunk_fwd_tc_kernel (packed)", pak_gbs)},
+        "raw": {"metric": "GDN-2 prefill tokens/s per layer, raw projections",
+                "value": raw["tokens"] / (raw["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": raw["ms"],
+                "steps": args.steps,
                 "workload": "prefill_b8_h16_t4096 fed with the raw projections: q, k L2-normalised, sigmoid "
                             "gates and log alpha = -softplus(a)/16 applied inside the kernel",
-                "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (raw)", "achieved": raw_gbs,
-                             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": raw_gbs / pk["hbm_gbs"],
-                             "traffic": None}},
-        "long": {"metric": "GDN-2 prefill tokens/s per layer, long context", "value": lg["tokens"] / (lg["ms_split"] * 1e-3),
-                 "unit": "tokens/s", "ms_per_step": lg["ms_split"], "segments": lg["P"],
-                 "unsplit_ms_per_step": lg["ms_plain"],
+                "roofline": hbm("chunk_fwd_tc_kernel (raw)", raw_gbs)},
+        "long": {"metric": "GDN-2 prefill tokens/s per layer, long context",
+                 "value": lg["tokens"] / (lg["ms_split"] * 1e-3), "unit": "tokens/s", "ms_per_step": lg["ms_split"],
+                 "segments": lg["P"], "unsplit_ms_per_step": lg["ms_plain"],
                  "workload": "long_b1_h16_t65536 (B=1 H=16 T=65536, heavy decay tail) through "
                              "gdn2_chunk_fwd_split at the library's segment count",
-                 "roofline": {"bound": "hbm", "kernel": "chunk_fwd_tc_kernel (split)", "achieved": lg_gbs,
-                              "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": lg_gbs / pk["hbm_gbs"],
-                              "traffic": None}},
+                 "roofline": hbm("chunk_fwd_tc_kernel (split)", lg_gbs)},
         "bwd": {"metric": "GDN-2 backward tokens/s per layer", "value": bw["tokens"] / (bw["ms"] * 1e-3),
                 "unit": "tokens/s", "ms_per_step": bw["ms"],
-                "workload": "prefill_b8_h16_t4096 backward: dq, dk, dv, dlog_alpha, db, dw, dS0 from dO and dS_T "
-                            "(products as tf32 warp-level MMAs)",
+                "workload": "prefill_b8_h16_t4096 backward: dq, dk, dv, dlog_alpha, db, dw, dS0 from dO and dS_T",
                 "roofline": {"bound": "tensor", "kernel": "chunk_bwd_kernel", "achieved": bw_tflops,
                              "peak": pk["bf16_tflops"] * TF32_PER_BF16, "unit": "TFLOP/s",
                              "frac": bw_tflops / (pk["bf16_tflops"] * TF32_PER_BF16),
@@ -640,30 +620,39 @@ def main():
                              "frac_of_fp32_cuda_core_peak": bw_tflops / FP32_FMA_TFLOPS,
                              "flop_per_chunk_head": BWD_FLOP_PER_CHUNK_HEAD, "traffic": None}},
         "csize": {"metric": "GDN-2 prefill tokens/s per layer by chunk size",
-                  "workload": "prefill_b8_h16_t4096 through gdn2_chunk_fwd_csize (warp-level tf32 MMAs, one "
-                              f"template for every chunk size; {cs['ctas']} CTAs of (batch, head, 32 value columns))",
+                  "workload": "prefill_b8_h16_t4096 through gdn2_chunk_fwd_csize",
                   "device_bytes": {"arguments": cs["arg_bytes"], "scratch": 0},
                   "sizes": {str(C): {"value": cs["tokens"] / (r["ms"] * 1e-3), "unit": "tokens/s",
                                      "ms_per_step": r["ms"], "smem_bytes_per_cta": r["smem"],
                                      "ctas_per_sm_by_smem": r["ctas_per_sm"],
-                                     "flop_per_token_head": 2 * C * (3 * 128 + 2 * 128) + 6 * 128 * 128,
-                                     "roofline": {"bound": "hbm", "kernel": "chunk_fwd_csize_kernel",
-                                                  "achieved": cs["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD
-                                                  / (r["ms"] * 1e-3) / 1e9,
-                                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                                  "frac": cs["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD
-                                                  / (r["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"],
-                                                  "traffic": None}}
+                                     "roofline": hbm("chunk_fwd_csize_kernel",
+                                                     cs["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD
+                                                     / (r["ms"] * 1e-3) / 1e9)}
                             for C, r in cs["sizes"].items()}},
         "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
                  "steps": args.steps,
                  "workload": f"q, k, v projections of prefill_b8_h16_t4096 side by side: [8, 4096, {cv['C']}] bf16, "
                              "4 taps + bias, zero history",
-                 "roofline": {"bound": "hbm", "kernel": "short_conv_kernel", "achieved": cv_gbs,
-                              "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": cv_gbs / pk["hbm_gbs"],
-                              "traffic": None}},
+                 "roofline": hbm("short_conv_kernel", cv_gbs)},
+    }
+    print(json.dumps(legs), flush=True)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "tf32", "data": "synthetic (seeded normal draws, layer shape)",
+        "config": config_dict(),
+        "roofline": dict(hbm("chunk_fwd_tc_kernel", achieved, traffic), peak_src=pk["src"],
+                         bytes_per_token_head=PREFILL_BYTES_PER_TOKEN_HEAD,
+                         frac_fp32_o=achieved * PREFILL_BYTES_FP32_O / PREFILL_BYTES_PER_TOKEN_HEAD / pk["hbm_gbs"],
+                         tensor={"achieved_tflops": tflops, "frac_bf16": tflops / pk["bf16_tflops"],
+                                 "frac_tf32": tflops / (pk["bf16_tflops"] * TF32_PER_BF16)}),
+        "decode": {"value": 1e3 / dec["ms_per_step"], "unit": "steps/s", "ms_per_step": dec["ms_per_step"],
+                   "steps": args.decode_steps, "workload": "decode_b256_h16",
+                   "roofline": hbm("decode_step_kernel", dec_gbs, profile_traffic("decode_step_kernel")),
+                   "clocks": {k: dec["clocks"].get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons")}},
         "gpu_launches": args.steps,
-        "clocks": pre["clocks"],
+        "clocks": {k: pre["clocks"].get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
         "device_status_ok": bool(pre["ok"] and dec["ok"] and dec_raw["ok"] and pak["ok"] and raw["ok"] and cv["ok"]
                                  and lg["ok"] and bw["ok"] and cs["ok"]),
     }

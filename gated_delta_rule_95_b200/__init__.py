@@ -103,6 +103,13 @@ def _stream(dev, stream):
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def _on(device, fn, *args):
+    """Calls ``fn`` with ``device`` current (the library keys its per-device state, the
+    error word, scratch address and kernel attributes, by the current device)."""
+    with torch.cuda.device(device):
+        return fn(*args)
+
+
 def _check_tokens(name, tensors, dtype, device):
     for n, t in tensors.items():
         if not t.is_cuda or t.device != device:
@@ -131,7 +138,7 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_
     if S_T is not None:
         ts["S_T"] = S_T
     _check_tokens("gdn2_chunk_fwd", ts, q.dtype, q.device)
-    rc = lib().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+    rc = _on(q.device, lib().gdn2_chunk_fwd, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
                               _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_chunk_fwd", rc)
@@ -156,7 +163,7 @@ def gdn2_chunk_fwd_csize(q, k, v, log_alpha, b, w, S0=None, *, chunk=64, o=None,
     if S_T is not None:
         ts["S_T"] = S_T
     _check_tokens("gdn2_chunk_fwd_csize", ts, q.dtype, q.device)
-    rc = lib().gdn2_chunk_fwd_csize(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),
+    rc = _on(q.device, lib().gdn2_chunk_fwd_csize, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),
                                     _ptr(o), _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], int(chunk),
                                     _stream(q.device, stream))
     if rc != 0:
@@ -192,7 +199,7 @@ def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, *, workspace=Non
     for n, t in g.items():
         if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != q.device):
             raise ValueError(f"gdn2_chunk_bwd: {n} must be a contiguous fp32 tensor on {q.device}")
-    rc = L.gdn2_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
+    rc = _on(q.device, L.gdn2_chunk_bwd, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
                           _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]),
                           _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), B, T, H, dk, dv, _DT[q.dtype],
                           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(q.device, stream))
@@ -229,7 +236,7 @@ def gdn2_chunk_fwd_split(q, k, v, log_alpha, b, w, S0=None, *, segments=None, wo
         ts["S_T"] = S_T
     _check_tokens("gdn2_chunk_fwd_split", ts, q.dtype, q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = L.gdn2_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+    rc = _on(q.device, L.gdn2_chunk_fwd_split, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
                                 _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], segments, _ptr(workspace), wbytes,
                                 _stream(q.device, stream))
     if rc != 0:
@@ -255,7 +262,7 @@ def gdn2_chunk_fwd_split_static(q, k, v, log_alpha, b, w, S0=None, *, segments, 
     if S_T is not None:
         ts["S_T"] = S_T
     _check_tokens("gdn2_chunk_fwd_split_static", ts, q.dtype, q.device)
-    rc = lib().gdn2_chunk_fwd_split_static(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),
+    rc = _on(q.device, lib().gdn2_chunk_fwd_split_static, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),
                                            _ptr(o), _ptr(S_T), B, T, H, dk, dv, _DT[q.dtype], segments,
                                            _stream(q.device, stream))
     if rc != 0:
@@ -288,7 +295,7 @@ def gdn2_chunk_fwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, o=No
     if S_T is not None:
         ts["S_T"] = S_T
     _check_tokens("gdn2_chunk_fwd_varlen", ts, q.dtype, q.device)
-    rc = lib().gdn2_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(cu_seqlens),
+    rc = _on(q.device, lib().gdn2_chunk_fwd_varlen, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(cu_seqlens),
                                      _ptr(S0), _ptr(o), _ptr(S_T), N, T, H, dk, dv, _DT[q.dtype],
                                      _stream(q.device, stream))
     if rc != 0:
@@ -330,7 +337,7 @@ def gdn2_chunk_fwd_raw(q_raw, k_raw, v, a_raw, b_raw, w_raw, S0=None, *, decay_s
     if decay_scale is not None and decay_scale.numel() != H:
         raise ValueError("gdn2_chunk_fwd_raw: decay_scale must hold one value per head")
     _check_tokens("gdn2_chunk_fwd_raw", ts, q_raw.dtype, q_raw.device)
-    rc = lib().gdn2_chunk_fwd_raw(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(w_raw),
+    rc = _on(q_raw.device, lib().gdn2_chunk_fwd_raw, _ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(w_raw),
                                   _ptr(decay_scale), _ptr(cu_seqlens), _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk,
                                   dv, _DT[q_raw.dtype], _stream(q_raw.device, stream))
     if rc != 0:
@@ -367,7 +374,7 @@ def gdn2_short_conv(x, weight, bias=None, *, cu_seqlens=None, hist=None, y=None,
         if t is not None:
             ts[n] = t
     _check_tokens("gdn2_short_conv", ts, x.dtype, x.device)
-    rc = lib().gdn2_short_conv(_ptr(x), _ptr(weight), _ptr(bias), _ptr(cu_seqlens), _ptr(hist), _ptr(y),
+    rc = _on(x.device, lib().gdn2_short_conv, _ptr(x), _ptr(weight), _ptr(bias), _ptr(cu_seqlens), _ptr(hist), _ptr(y),
                                _ptr(hist_out), B, T, C, _DT[x.dtype], _stream(x.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_short_conv", rc)
@@ -384,7 +391,7 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
         o = torch.empty((B, H, dv), dtype=torch.float32, device=q.device)
     _check_tokens("gdn2_decode_step", dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, S=S, o=o), q.dtype,
                   q.device)
-    rc = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
+    rc = _on(q.device, lib().gdn2_decode_step, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
                                 B, H, dk, dv, _DT[q.dtype], _stream(q.device, stream))
     if rc != 0:
         raise GDN2Error("gdn2_decode_step", rc)
@@ -407,7 +414,7 @@ def gdn2_decode_step_raw(q_raw, k_raw, v, a_raw, b_raw, w_raw, S, *, decay_scale
     if decay_scale is not None:
         ts["decay_scale"] = decay_scale
     _check_tokens("gdn2_decode_step_raw", ts, q_raw.dtype, q_raw.device)
-    rc = lib().gdn2_decode_step_raw(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(w_raw),
+    rc = _on(q_raw.device, lib().gdn2_decode_step_raw, _ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(w_raw),
                                     _ptr(decay_scale), _ptr(S), _ptr(o), B, H, dk, dv, _DT[q_raw.dtype],
                                     _stream(q_raw.device, stream))
     if rc != 0:

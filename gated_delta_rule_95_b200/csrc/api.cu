@@ -15,12 +15,15 @@ namespace gdn2 {
 
 __device__ unsigned g_error_word = 0;
 
-// Address of the error word on the current device (looked up once per device).
+// Address of the error word on the current device (looked up once per device; several host
+// threads may ask at once, so the cache is filled under a lock).
 unsigned* device_error_word() {
   constexpr int kMaxDev = 64;
   static unsigned* ptrs[kMaxDev] = {};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!ptrs[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) ptrs[dev] = static_cast<unsigned*>(p);

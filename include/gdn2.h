@@ -144,8 +144,9 @@ GDN2_API gdn2_status gdn2_chunk_bwd(const void* q, const void* k, const void* v,
 
 /*
  * gdn2_chunk_fwd_split without a caller workspace, for callers that cannot allocate: the
- * scratch is a fixed 16 MiB array in the library's own device memory (reserved when the
- * library's module loads).  The Gated DeltaNet-2 pages describe no counterpart of this
+ * scratch is a fixed 16 MiB array in the library's own device memory, reserved when the
+ * library's device module is loaded on a device (with CUDA's lazy module loading, at the
+ * first call that touches the module there) and held until the process exits.  The Gated DeltaNet-2 pages describe no counterpart of this
  * entry point; it is an interface convenience over the same kernels.
  *
  *   arguments   : as gdn2_chunk_fwd_split, without workspace and workspace_bytes

@@ -45,3 +45,21 @@ def oracle_units(d, units, S0=None):
         s0 = np.concatenate([p["S0"] for p in per], axis=0)
     o, S = oracle.forward(cat["q"], cat["k"], cat["v"], cat["log_alpha"], cat["b"], cat["w"], s0)
     return [(o[n, :, 0], S[n, 0]) for n in range(len(units))]
+
+
+def check_units(d, o_gpu, S_gpu, tol, units=None, group=32):
+    """Element-wise parity of every listed (batch, head) unit (all of them by default):
+    o [B,T,H,dv] and S_T [B,H,dk,dv] of the GPU (CPU tensors) against the oracle, unit by
+    unit, in groups of ``group`` units per oracle call.  Returns the worst errors."""
+    B, H = d["q"].shape[0], d["q"].shape[2]
+    if units is None:
+        units = [(bb, h) for bb in range(B) for h in range(H)]
+    worst_o = worst_s = 0.0
+    for i in range(0, len(units), group):
+        part = units[i:i + group]
+        for (bb, h), (o_ref, S_ref) in zip(part, oracle_units(d, part)):
+            eo = rel_err(o_gpu[bb, :, h].double().numpy(), o_ref)
+            es = rel_err(S_gpu[bb, h].double().numpy(), S_ref)
+            assert eo <= tol and es <= tol, (bb, h, eo, es)
+            worst_o, worst_s = max(worst_o, eo), max(worst_s, es)
+    return worst_o, worst_s

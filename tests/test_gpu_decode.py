@@ -44,14 +44,15 @@ def test_decode_small(dtype, dk, dv):
     assert g.gdn2_device_status() == 0
 
 
-def test_decode_full_size_1000_steps_sampled():
-    """The benchmarked workload: B=256, H=16, d=128, 1000 steps, fresh tokens per
-    step; o checked at sampled steps and S after step 1000 on sampled units."""
+def test_decode_full_size_1000_steps_256_units():
+    """The benchmarked workload: B=256, H=16, d=128, 1000 steps, fresh tokens per step.
+    o is checked element by element at steps 0, 1, 500 and 999 and S after step 1000, on
+    256 (sequence, head) units spread over every sequence block and every head."""
     steps = WL.steps
     S = gi.decode_state(WL)
     toks = gi.decode_tokens_many(WL, range(steps))
     Sd = S.cuda()
-    check_steps = {0, 1, 2, 500, steps - 1}
+    check_steps = (0, 1, 500, steps - 1)
     o_at = {}
     for j, t in enumerate(toks):
         td = _to(t)
@@ -60,13 +61,21 @@ def test_decode_full_size_1000_steps_sampled():
             o_at[j] = o.float().cpu()
     S_gpu = Sd.cpu()
     assert torch.isfinite(S_gpu).all()
-    units = [(0, 0), (17, 3), (128, 8), (255, 15), (200, 11)]
-    seq = {k: np.stack([np.stack([gi.as_f64(t[k][b, h]) for t in toks]) for b, h in units])[:, :, None]
+    # unit n = (sequence n, head (7 n) mod 16): all 256 sequences, every head 16 times
+    bs = np.arange(WL.B)
+    hs = (7 * bs) % WL.H
+    seq = {k: np.stack([gi.as_f64(t[k][bs, hs]) for t in toks], axis=1)[:, :, None]
            for k in ("q", "k", "v", "log_alpha", "b", "w")}
-    S0 = np.stack([gi.as_f64(S[b, h]) for b, h in units])[:, None]
+    S0 = gi.as_f64(S[bs, hs])[:, None]
     o_ref, S_ref = oracle.forward(**seq, S0=S0)
-    for n, (b, h) in enumerate(units):
+    worst = 0.0
+    for n, (b, h) in enumerate(zip(bs, hs)):
         for j in check_steps:
-            assert rel_err(o_at[j][b, h].numpy(), o_ref[n, j, 0]) <= TOL["bf16"], (b, h, j)
-        assert rel_err(S_gpu[b, h].numpy(), S_ref[n, 0]) <= TOL["bf16"], (b, h)
+            e = rel_err(o_at[j][b, h].numpy(), o_ref[n, j, 0])
+            assert e <= TOL["bf16"], (b, h, j, e)
+            worst = max(worst, e)
+        e = rel_err(S_gpu[b, h].numpy(), S_ref[n, 0])
+        assert e <= TOL["bf16"], (b, h, e)
+        worst = max(worst, e)
+    print(f"decode 1000 steps, 256 units: worst error {worst:.2e}")
     assert g.gdn2_device_status() == 0

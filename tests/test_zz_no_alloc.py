@@ -49,6 +49,26 @@ def test_static_scratch_matches_workspace_entry_two_calls(seed):
     assert not torch.equal(outs[0], outs[1])
 
 
+def test_static_scratch_call_takes_no_device_memory():
+    """After a first call (which may load the module and with it the fixed array), further
+    calls leave the device's free memory unchanged: the entry point allocates nothing."""
+    import dataclasses
+    wl = dataclasses.replace(gi.WORKLOADS["prefill_b8_h16_t4096"], state_std=0.05)
+    d = gi.prefill_inputs(wl, B=1, T=4096, H=16, seed=3)
+    x = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+    o = torch.empty((1, 4096, 16, 128), device="cuda")
+    S_T = torch.empty((1, 16, 128, 128), device="cuda")
+    assert _static_call(x, o, S_T, 4) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _static_call(x, o, S_T, 4) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    assert g.gdn2_device_status() == 0
+
+
 def test_static_scratch_rejects_sizes_beyond_its_limit():
     L = g.lib()
     # 16 heads x 6 segments of 128 x 128 fp32 states, three sets: 18.9 MB > 16 MiB
