@@ -43,11 +43,15 @@ def library_path() -> str:
     return os.path.join(_HERE, "libgdn2.so")
 
 
-def lib():
-    """The loaded C library (ctypes).  Raises if it has not been built."""
+def lib(path=None):
+    """The loaded C library (ctypes).  Raises if it has not been built.  ``path`` loads
+    another build of the same library in its place (the instrumented build of the
+    profiling driver)."""
     global _LIB
+    if path is not None and (_LIB is None or _LIB._name != path):
+        _LIB = None
     if _LIB is None:
-        path = library_path()
+        path = path or library_path()
         if not os.path.exists(path):
             raise RuntimeError(f"{path} is missing: build it with `python -m gated_delta_rule_95_b200.build` "
                                "(or __graft_entry__.build()); there is no fallback path")

@@ -31,6 +31,27 @@ unsigned* device_error_word() {
   return ptrs[dev];
 }
 
+#ifdef GDN2_STAMPS
+// Instrumented build only: per-chunk clock stamps of the chunk kernel's first CTA.
+constexpr int kStampWords = 64 * 32;
+__device__ unsigned long long g_stamps[kStampWords];
+unsigned long long* stamp_buffer() {
+  constexpr int kMaxDev = 64;
+  static unsigned long long* ptrs[kMaxDev] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_stamps) == cudaSuccess) ptrs[dev] = static_cast<unsigned long long*>(p);
+  }
+  return ptrs[dev];
+}
+#else
+unsigned long long* stamp_buffer() { return nullptr; }
+#endif
+
 namespace {
 
 thread_local char g_last_cuda[256] = "";
@@ -82,7 +103,7 @@ extern "C" gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* 
 }
 
 extern "C" int gdn2_chunk_fwd_split_segments(int B, int T, int H, int sm_count) {
-  // waves of one CTA per SM: the first pass runs (2P - 1) B H segment runs, the last
+  // waves of one CTA per SM: the first pass runs (2P - 3) B H segment runs, the last
   // (P - 1) B H, each of ceil(chunks / P) chunks; one pass of B H full runs without a split
   if (B <= 0 || T <= 0 || H <= 0 || sm_count <= 0) return 1;
   const long long bh = (long long)B * H, nch = (T + 63) / 64, sms = sm_count;
@@ -91,7 +112,7 @@ extern "C" int gdn2_chunk_fwd_split_segments(int B, int T, int H, int sm_count) 
   int best_p = 1;
   for (int P = 2; P <= 64 && P <= nch; ++P) {
     const long long len = (nch + P - 1) / P;
-    const long long est = (waves(bh * (2 * P - 1)) + waves(bh * (P - 1))) * len + 1;  // + the chaining
+    const long long est = (waves(bh * (2 * P - 3)) + waves(bh * (P - 1))) * len + 1;  // + the chaining
     if (est < best) {
       best = est;
       best_p = P;
@@ -350,7 +371,9 @@ extern "C" gdn2_status gdn2_device_status(void) {
   if (word) {
     e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_fail(e);
-    return (word & kErrBadSeqlens) ? GDN2_ERR_SHAPE : GDN2_ERR_TIMEOUT;
+    if (word & kErrBadSeqlens) return GDN2_ERR_SHAPE;
+    if (word & kErrWaitTimeout) return GDN2_ERR_TIMEOUT;
+    return GDN2_ERR_RANGE;
   }
   return GDN2_OK;
 }
@@ -364,10 +387,23 @@ extern "C" const char* gdn2_status_string(int status) {
     case GDN2_ERR_ALIGN: return "pointer not 16-byte aligned";
     case GDN2_ERR_CUDA: return "CUDA error";
     case GDN2_ERR_TIMEOUT: return "device-side wait timed out";
+    case GDN2_ERR_RANGE: return "decay out of range (cumulative log decay within a chunk below -80)";
     default: return "unknown status";
   }
 }
 
 extern "C" const char* gdn2_last_cuda_error(void) { return g_last_cuda; }
 
-extern "C" int gdn2_version(void) { return 100; }
+extern "C" int gdn2_version(void) { return 200; }
+
+#ifdef GDN2_STAMPS
+// Instrumented build only: copies the stamp words ([chunk][slot] clock64 values of the last
+// chunk launch's first CTA) to host memory; returns the number of words copied.
+extern "C" GDN2_API int gdn2_stamps_read(unsigned long long* host, int n) {
+  if (!host || n <= 0) return 0;
+  if (n > kStampWords) n = kStampWords;
+  if (cudaDeviceSynchronize() != cudaSuccess) return 0;
+  if (cudaMemcpyFromSymbol(host, g_stamps, (size_t)n * sizeof(unsigned long long)) != cudaSuccess) return 0;
+  return n;
+}
+#endif

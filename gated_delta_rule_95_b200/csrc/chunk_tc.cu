@@ -60,10 +60,13 @@ constexpr int NCOMP = 512;                      // warps 0-15: elementwise work
 constexpr int NT = NCOMP + 64;                  // + the control warp and the store warp
 constexpr int CTL = NCOMP;                      // the thread that issues MMAs and the input copies
 constexpr int STW = NCOMP + 32;                 // the thread that issues output stores and log-alpha copies
-constexpr int NSOLVE = 256;                     // warps 0-7 run the triangular solve
-constexpr int BAR_COMP = 1, BAR_SOLVE = 2, BAR_AUX = 3;  // named barriers: compute warps; warps 0-7; 8-15
+constexpr int NSOLVE = 256;                     // warps 0-7: A read-out, the solve (warps 0-3), U~ rounding
+constexpr int BAR_COMP = 1, BAR_SOLVE = 2, BAR_AUX = 3;  // named barriers: compute warps; warps 0-3; 8-15
+constexpr int BAR_PAIR = 4;                     // named barriers 4, 5: warp pairs (0, 1) and (2, 3)
 constexpr uint64_t WAIT_LIMIT = 2000000000ull;  // 2 s of wall time per wait
 constexpr float LOG2E = 1.4426950408889634f;
+// in-chunk cumulative log2 decay below which 2^-g leaves the fp32 range (natural log -80)
+constexpr float G2_MIN = -115.4f;
 constexpr int PF_AHEAD = 2;                     // chunks of input prefetched into L2 ahead of use
 constexpr int LPT_MAX_SEQ = 1024;               // packed batches up to this many sequences start longest first
 
@@ -79,14 +82,14 @@ constexpr uint32_t OFF_T = OFF_PK + 2 * R192;   // T [t][s]: 2 panels x 64 rows
 constexpr uint32_t OFF_LA = OFF_T + 2 * R64;    // log alpha [t][i] fp32 (TMA, 128B swizzle): 4 panels x 64 rows,
                                                 // turned in place into the in-chunk cumulative log2 decay;
                                                 // between uses: the output tile [t][j] fp32 of a TMA store
-constexpr uint32_t OFF_SCR = OFF_LA + 4 * R64;  // solve scratch: fp32 64 x LDM, then 32 x LDX
+constexpr uint32_t OFF_SCR = OFF_LA + 4 * R64;  // solve scratch: fp32 64 x LDM, then 4 x 32 x LDW
 // raw bf16 staging (TMA, 128B swizzle): a [64 tokens][128 channels] tile = 2 panels of
 // 64 channels x 64 rows
 constexpr uint32_t B16 = 2 * R64;
 constexpr uint32_t RAW_Q = OFF_KQ, RAW_K = OFF_KQ + B16, RAW_B = OFF_KQ + 2 * B16;  // free once the
 constexpr uint32_t RAW_V = OFF_KN, RAW_W = OFF_KN + B16;  // state product (KQ) / [A; P] (Kn) has read them
 constexpr int LDM = 68;                         // padded row (floats) of the 64 x 64 solve matrix
-constexpr int LDX = 36;                         // padded row of the 32 x 32 block product
+constexpr int LDW = 8;                          // row of a solve warp's block-product scratch (32 x 8)
 constexpr uint32_t TILES = OFF_SCR + 22528;     // 214 KB
 
 struct Misc {
@@ -133,7 +136,24 @@ struct TcParams {
   int split_phase = 0, split_P = 0, split_L = 0;
   float* ws = nullptr;
   unsigned* err;
+  unsigned long long* stamps = nullptr;  // instrumented build only: per-chunk clock stamps
 };
+
+#ifdef GDN2_STAMPS
+// Instrumented build (GDN2_STAMPS): clock64 of the SM at fixed points of the per-chunk
+// schedule, for the first STAMP_CHUNKS chunks of the launch's first CTA, written by the one
+// thread named at each point into [chunk][slot].
+constexpr int STAMP_CHUNKS = 64, STAMP_SLOTS = 32;
+#define STAMP(cc, slot)                                                                      \
+  do {                                                                                       \
+    if (p.stamps && blockIdx.x == 0 && (cc) >= 0 && (cc) < STAMP_CHUNKS)                     \
+      p.stamps[(size_t)(cc) * STAMP_SLOTS + (slot)] = (unsigned long long)clock64();         \
+  } while (0)
+#else
+#define STAMP(cc, slot) \
+  do {                  \
+  } while (0)
+#endif
 
 // Gate activations of the raw-projection variant, from their definitions, on the
 // special-function unit.  sigmoid(x) = (1 + tanh(x / 2)) / 2, one special-function
@@ -159,6 +179,8 @@ __device__ __forceinline__ void st4_tf32(unsigned char* p, const float* f) {
   *reinterpret_cast<float4*>(p) = make_float4(rna_tf32(f[0]), rna_tf32(f[1]), rna_tf32(f[2]), rna_tf32(f[3]));
 }
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+// tf32 operand of a warp-level MMA (fp32 bit pattern, low 13 bits cleared)
+__device__ __forceinline__ uint32_t tfu(float x) { return __float_as_uint(rna_tf32(x)); }
 // one bf16 element of shared memory as fp32
 __device__ __forceinline__ float bf16_at(const unsigned char* p) {
   return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short*>(p)) << 16);
@@ -205,7 +227,8 @@ __global__ void __launch_bounds__(NT, 1)
   // the recurrence's linearity in (S, v), the state after segment s is M_s S + N_s, with
   // M_s the state reached from S = I with v = 0 (d_k = d_v) and N_s the one reached from
   // S = 0; the host chains them between the passes.  First pass (phase 1): r = 0 runs
-  // segment 0 from S0, r in [1, P) gives N_r, r in [P, 2P - 1) gives M_{r-P+1}; last pass
+  // segment 0 from S0, r in [1, P - 1) gives N_r, r in [P - 1, 2P - 3) gives M_{r-P+2} (the
+  // last segment needs neither: it starts from its chained state); last pass
   // (phase 3): segment r + 1 from its start state.  The same instantiation also runs the
   // whole sequence writing the state entering every chunk to the workspace [B H][chunk]
   // [d_k][d_v] and no outputs (phase 5, the checkpoints of the backward pass).
@@ -217,7 +240,7 @@ __global__ void __launch_bounds__(NT, 1)
     h = bh % p.H;
     bb = bh / p.H;
     su = bh;
-    sp_seg = p.split_phase == 1 ? (sp_r < p.split_P ? sp_r : sp_r - p.split_P + 1) : sp_r + 1;
+    sp_seg = p.split_phase == 1 ? (sp_r < p.split_P - 1 ? sp_r : sp_r - p.split_P + 2) : sp_r + 1;
     t0 = sp_seg * p.split_L;
     len = min(p.split_L, p.T - t0);
     if (p.split_phase == 5) {
@@ -229,7 +252,7 @@ __global__ void __launch_bounds__(NT, 1)
   const bool sp_first = SPLIT && p.split_phase == 1;
   const bool sp_ckpt = SPLIT && p.split_phase == 5;
   const bool write_o = !SPLIT || (sp_first ? sp_r == 0 : !sp_ckpt);  // outputs written
-  const bool sp_trans = SPLIT && sp_first && sp_r >= p.split_P;  // M_s: from I, no write term
+  const bool sp_trans = SPLIT && sp_first && sp_r >= p.split_P - 1;  // M_s: from I, no write term
   if constexpr (VARLEN) {
     int n = unit / p.H;
     if (p.nseq <= LPT_MAX_SEQ) {
@@ -355,6 +378,7 @@ __global__ void __launch_bounds__(NT, 1)
           umma_tf32_ss(tmem + TM_AP, aKQ, bKN, ID_64, ks > 0);
         }
         umma_commit(&ms.bar_mma);
+        STAMP(c, 0);
         // [X^T | O^T] = S^T [-Kb; Qh]^T : A = S^T (tensor memory), B = the KQ tile (N = 128);
         // X^T = -S^T Kb^T becomes R^T = Vw^T + X^T when warps 8-15 round it
         if (!(alive = wait_on(&ms.bar_stage, ph_stage))) break;
@@ -369,6 +393,7 @@ __global__ void __launch_bounds__(NT, 1)
           umma_tf32_ts(tmem + TM_R, tmem + TM_S + 8 * ks, bKQ, ID_128, ks > 0);
         }
         umma_commit(&ms.bar_s);
+        STAMP(c, 1);
         // the state product has read the KQ tile: the next chunk's q, k, b
         if (!(alive = wait_on(&ms.bar_s, ph_s))) break;
         if (c + 1 < nch) issue_qkb(c + 1);
@@ -388,6 +413,7 @@ __global__ void __launch_bounds__(NT, 1)
           const uint64_t bT = sdesc_sw128(sbase + OFF_T + R64 + 32 * 128 + (ks & 3) * 32, 16, 1024);
           umma_tf32_ts(tmem + TM_U + 32, tmem + TM_R + 8 * ks, bT, ID_32, ks > 4);
         }
+        STAMP(c, 2);
         if (!(alive = wait_on(&ms.bar_solved, ph_solved))) break;
         tc_fence_after();
 #pragma unroll
@@ -396,6 +422,7 @@ __global__ void __launch_bounds__(NT, 1)
           umma_tf32_ts(tmem + TM_U + 32, tmem + TM_R + 8 * ks, bT, ID_32, 1);
         }
         umma_commit(&ms.bar_mma);
+        STAMP(c, 3);
         // [O^T | S^T] += U~^T [P; Kn^T]^T : O^T += U~^T P^T and S^T += U~^T Kn in one N = 192 product
         if (!(alive = wait_on(&ms.bar_uround, ph_uround))) break;
         tc_fence_after();
@@ -405,6 +432,7 @@ __global__ void __launch_bounds__(NT, 1)
           umma_tf32_ts(tmem + TM_O, tmem + TM_U + 8 * ks, bPK, ID_192, 1);
         }
         umma_commit(&ms.bar_mma);
+        STAMP(c, 4);
       }
       // after a give-up: every MMA issued so far (a fresh commit tracks all of them) and
       // the last copies must land before the block releases its memory
@@ -444,6 +472,7 @@ __global__ void __launch_bounds__(NT, 1)
           store_o(c - 1);
           bulk_wait_read_all();
         }
+        STAMP(c, 16);
         if (c + 1 < nch) issue_la(c + 1);
         else mbar_arrive(&ms.bar_lastread);  // the last staging may overwrite the tile
       }
@@ -490,7 +519,7 @@ __global__ void __launch_bounds__(NT, 1)
       *reinterpret_cast<float4*>(sm + OFF_T + 16 * e) = make_float4(0.f, 0.f, 0.f, 0.f);
     uint32_t ph_mma = 0, ph_s = 0;
     float* Msc = reinterpret_cast<float*>(sm + OFF_SCR);                 // solve matrix, 64 x LDM fp32
-    float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);  // block product, 32 x LDX fp32
+    float* Xsc = reinterpret_cast<float*>(sm + OFF_SCR + 64 * LDM * 4);  // block products, 4 x 32 x LDW fp32
     const int lane = tid & 31;
     auto wait_mma = [&]() -> bool { return wait_on(&ms.bar_mma, ph_mma); };
     // S^T <- S^T Diag(Gamma_C of the chunk with parity gb), in tensor memory (checkpoint
@@ -604,7 +633,12 @@ __global__ void __launch_bounds__(NT, 1)
         for (int r = 0; r < 32; ++r)
           *reinterpret_cast<float*>(la_w + f32_off(32 * hf + r, ch, R64)) = ex2_approx(x[r] + off);
       }
-      if (hf == 1) ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
+      if (hf == 1) {
+        ms.gC[cc & 1][ch] = kval ? ex2_approx(off + acc) : 0.f;
+        // the chunk-start reference scales keys by 2^-g: beyond a cumulative log decay of -80
+        // (log2: G2_MIN) within the chunk that leaves the fp32 range; the result is flagged
+        if (kval && off + acc < G2_MIN && p.err) atomicOr(p.err, kErrDecayRange);
+      }
       return ok;
     };
     // Raw projections, warps 0-7, one chunk ahead once its q, k, b copies have landed:
@@ -655,6 +689,7 @@ __global__ void __launch_bounds__(NT, 1)
       float2 nkb[8], qh[8], kn[8];
       // (raw projections: warps 0-7 have seen these copies land already, one chunk ahead)
       bool ok_raw = (PREP && warp < NSOLVE / 32) ? true : wait_on(&ms.bar_raw, ph_raw);
+      if (tid == 0) STAMP(c, 5);
       auto build = [&](auto masked) {
         const unsigned char* la_t = sm + OFF_LA;
         const uint32_t pnl = (uint32_t)(c2 >> 6) * R64;  // raw tiles: panels of 64 channels
@@ -686,13 +721,10 @@ __global__ void __launch_bounds__(NT, 1)
       };
       if (VARLEN && C * c + C > len) build(std::true_type{});
       else build(std::false_type{});
-      // the previous chunk's last product must be done before Kn^T, O and S are touched,
-      // and every raw read before the operand tiles overwrite the staging
-      {
-        const bool ok = ok_raw && ((c == 0) || wait_mma());
-        if (named_bar_or(BAR_COMP, NCOMP, !ok)) { dead = true; break; }
-      }
-      tc_fence_after();
+      // every raw read must be done before the operand tiles overwrite the staging
+      if (named_bar_or(BAR_COMP, NCOMP, !ok_raw)) { dead = true; break; }
+      // the KQ and Kn tiles were last read by the previous chunk's state product and [A; P]:
+      // they are written while the previous chunk's output/state product may still run
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int t = 8 * ts + r;
@@ -700,8 +732,17 @@ __global__ void __launch_bounds__(NT, 1)
         st2_tf32(sm + OFF_KQ + f32_off(64 + t, c2, R128), qh[r]);
         st2_tf32(sm + OFF_KN + f32_off(t, c2, R64), kn[r]);
       }
+      // that product must be done before Kn^T, O and S are touched (and before this chunk's
+      // [A; P] is issued, so that no wait below trails the MMA barrier by two phases)
+      const bool ok_op = (c == 0) || wait_mma();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(&ms.bar_ops);
+      if (tid == 0) STAMP(c, 6);
+      tc_fence_after();
       {
-        // Kn^T rows 2 cp and 2 cp + 1, tokens [8 ts, 8 ts + 8).  The first store of each
+        // Kn^T rows 2 cp and 2 cp + 1, tokens [8 ts, 8 ts + 8) (read by this chunk's last
+        // product only; the staging arrival below publishes them).  The first store of each
         // thread goes to row 2 cp + ((cp >> 2) & 1), so that the 8 threads sharing a
         // 128-byte wavefront hit 8 different swizzle phases.
         const int sw = (cp >> 2) & 1;
@@ -715,9 +756,6 @@ __global__ void __launch_bounds__(NT, 1)
           st4_tf32(sm + OFF_PK + f32_off(64 + c2 + rsel, 8 * ts + 4, R192), f + 4);
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      warp_arrive(&ms.bar_ops);
       // ===== while [A; P] is on the tensor cores: the previous chunk's output and state
       // decay ==================================================================================
       if (c > 0) {
@@ -732,6 +770,7 @@ __global__ void __launch_bounds__(NT, 1)
       {
         const bool ok_ap = wait_mma();
         tc_fence_after();
+        if (tid == 0) STAMP(c, 7);
         float v[16];
         tmem_ld16(tlane + TM_AP + 16 * sg, v);
         tmem_ld_wait();
@@ -757,13 +796,16 @@ __global__ void __launch_bounds__(NT, 1)
             st4_tf32(sm + OFF_PK + f32_off(t, 16 * sg + x, R192), f);
           }
         }
-        if (named_bar_or(BAR_COMP, NCOMP, !ok_ap)) { dead = true; break; }
+        if (named_bar_or(BAR_COMP, NCOMP, !(ok_ap && ok_op))) { dead = true; break; }
       }
-      // ===== T = (I + A)^-1 on warps 0-7: 8x8 diagonal blocks by forward substitution (fp32),
-      // then 2x2 block merges T21 = -T22 (A21 T11) at 16, 32 and 64 (every entry above the
-      // diagonal is an explicit zero, so block products run dense).  Each level writes its
-      // blocks to the fp32 scratch (read by the next level) and, rounded, to the T operand
-      // tile.  Warps 8-15 meanwhile round R^T in tensor memory once the state product is done.
+      if (tid == 0) STAMP(c, 8);
+      // ===== T = (I + A)^-1 on warps 0-3 (warps 4-7 only round U~ below).  Warp k owns the
+      // 16-row block k: its two 8x8 diagonal blocks by forward substitution in fp32, then their
+      // 16-level merge T_21 = -T_22 (A_21 T_11), all within the warp; then the 32-level merges
+      // (warp pairs) and the 64-level merge (the four warps) on warp-level tf32 MMAs
+      // (mma.sync m16n8k8).  Every level writes its blocks to the fp32 scratch (read by the next
+      // level) and, rounded, to the T operand tile; entries above the 8x8 block diagonal stay
+      // zero.  Warps 8-15 meanwhile round R^T in tensor memory once the state product is done.
       bool ok_s = true;
       if (warp < 8) {
         auto put_t = [&](int row, int col, float x) {  // one element of the T operand tile
@@ -772,137 +814,150 @@ __global__ void __launch_bounds__(NT, 1)
         auto put_t2 = [&](int row, int col, float x0, float x1) {  // col even
           *reinterpret_cast<float2*>(sm + OFF_T + f32_off(row, col, R64)) = make_float2(rna_tf32(x0), rna_tf32(x1));
         };
-        if (tid < 64) {
-          // thread (blk, cc): column cc of the inverse of diagonal block blk (rows 8 blk ..)
-          const int r0 = 8 * (tid >> 3), cc = tid & 7;
-          const float* Ab = Msc + r0 * LDM + r0;
-          float x[8];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) x[r] = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-          for (int r = 1; r < 8; ++r) {
-            const float4 a0 = ld4(Ab + r * LDM), a1 = ld4(Ab + r * LDM + 4);
-            const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            float acc = 0.f;
-#pragma unroll
-            for (int s2 = 0; s2 < r; ++s2) acc = fmaf(ar[s2], x[s2], acc);
-            x[r] = (r > cc) ? -acc : x[r];
-          }
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            Msc[(r0 + r) * LDM + r0 + cc] = x[r];
-            put_t(r0 + r, r0 + cc, x[r]);
-          }
-        }
-        named_bar_sync(BAR_SOLVE, NSOLVE);
-        {
-          // 16x16 blocks q = 0..3: T_21 = -T_22 (A_21 T_11) with 8x8 blocks; thread (q, r, cc)
-          // computes one entry of each product.
-          const int q = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7;
-          const int i0 = 16 * q + 8, j0 = 16 * q;
-          float* Xq = Xsc + 64 * q;
+        if (warp < 4) {
+          const int k = warp, g4 = lane >> 2, t4 = lane & 3;
+          float* Xw = Xsc + warp * 32 * LDW;  // this warp's block-product scratch, 32 x LDW
           {
-            const float4 a0 = ld4(Msc + (i0 + r) * LDM + j0), a1 = ld4(Msc + (i0 + r) * LDM + j0 + 4);
-            const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            float z = 0.f;
+            // 8x8 diagonal blocks 2k (lanes 0-7) and 2k + 1 (lanes 8-15); a lane holds column
+            // lane mod 8 of its block (lanes 16-31 repeat lanes 0-15)
+            const int r0 = 8 * (2 * k + ((lane >> 3) & 1)), col = lane & 7;
+            float x[8];
 #pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) z = fmaf(ar[s2], Msc[(j0 + s2) * LDM + j0 + cc], z);
-            Xq[8 * r + cc] = z;
+            for (int r = 0; r < 8; ++r) x[r] = (r == col) ? 1.f : 0.f;
+#pragma unroll
+            for (int r = 1; r < 8; ++r) {
+              const float4 a0 = ld4(Msc + (r0 + r) * LDM + r0), a1 = ld4(Msc + (r0 + r) * LDM + r0 + 4);
+              const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+              float acc = 0.f;
+#pragma unroll
+              for (int s2 = 0; s2 < r; ++s2) acc = fmaf(ar[s2], x[s2], acc);
+              if (r > col) x[r] = -acc;
+            }
+            __syncwarp();
+            if (lane < 16) {
+#pragma unroll
+              for (int r = 0; r < 8; ++r) {
+                Msc[(r0 + r) * LDM + r0 + col] = x[r];
+                put_t(r0 + r, r0 + col, x[r]);
+              }
+            }
+            __syncwarp();
           }
-          named_bar_sync(BAR_SOLVE, NSOLVE);
           {
-            const float4 t0 = ld4(Msc + (i0 + r) * LDM + i0), t1 = ld4(Msc + (i0 + r) * LDM + i0 + 4);
-            const float tr[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-            float y = 0.f;
+            // 16-level: T_{2k+1,2k} (8x8) = -T_{2k+1,2k+1} (A_{2k+1,2k} T_{2k,2k}); lane l
+            // computes row l / 4, columns 2 (l mod 4) and + 1 of each product
+            const int I = 16 * k + 8, J = 16 * k, row = lane >> 2, c0 = 2 * (lane & 3);
+            float z0 = 0.f, z1 = 0.f;
 #pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) y = fmaf(tr[s2], Xq[8 * s2 + cc], y);
-            Msc[(i0 + r) * LDM + j0 + cc] = -y;
-            put_t(i0 + r, j0 + cc, -y);
+            for (int s2 = 0; s2 < 8; ++s2) {
+              const float a = Msc[(I + row) * LDM + J + s2];
+              const float2 tb = *reinterpret_cast<const float2*>(Msc + (J + s2) * LDM + J + c0);
+              z0 = fmaf(a, tb.x, z0);
+              z1 = fmaf(a, tb.y, z1);
+            }
+            *reinterpret_cast<float2*>(Xw + row * LDW + c0) = make_float2(z0, z1);
+            __syncwarp();
+            float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+              const float tt = Msc[(I + row) * LDM + I + s2];
+              const float2 xb = *reinterpret_cast<const float2*>(Xw + s2 * LDW + c0);
+              y0 = fmaf(tt, xb.x, y0);
+              y1 = fmaf(tt, xb.y, y1);
+            }
+            *reinterpret_cast<float2*>(Msc + (I + row) * LDM + J + c0) = make_float2(-y0, -y1);
+            put_t2(I + row, J + c0, -y0, -y1);
           }
-          named_bar_sync(BAR_SOLVE, NSOLVE);
-        }
-        // The block products of the next two levels run as warp-level tf32 MMAs
-        // (m16n8k8) on fragments read straight from the scratch matrices.
-        {
-          // 32x32 blocks: T_{2p+1,2p} = -T_{2p+1,2p+1} (A_{2p+1,2p} T_{2p,2p}), p = 0, 1;
-          // warp 2 p + nt computes the 16 x 8 output columns [8 nt, 8 nt + 8) of block p.
-          const int g = lane >> 2, t = lane & 3;
-          const int pp = warp >> 1, nt = warp & 1;
-          const int I = 2 * pp + 1, J = 2 * pp;
-          float* Xp = Xsc + 16 * pp * LDX;
-          if (warp < 4) {
+          if (tid == 0) STAMP(c, 9);
+          // ---- 32-level merges: T_{2m+1,2m} = -T_{2m+1,2m+1} (A_{2m+1,2m} T_{2m,2m}) in 16 x 16
+          // blocks; warp 2m + n computes the 8 output columns [8 n, 8 n + 8)
+          named_bar_sync(BAR_PAIR + (warp >> 1), 64);
+          {
+            const int m = warp >> 1, n = warp & 1;
+            const int I = 16 * (2 * m + 1), J = 16 * (2 * m);
             float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
-              const float* Ar = Msc + (16 * I + g) * LDM + 16 * J + 8 * ks + t;
-              const float* Bc = Msc + (16 * J + 8 * ks + t) * LDM + 16 * J + 8 * nt + g;
-              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
+              const float* Ar = Msc + (I + g4) * LDM + J + 8 * ks + t4;
+              const float* Bc = Msc + (J + 8 * ks + t4) * LDM + J + 8 * n + g4;
+              const uint32_t a[4] = {tfu(Ar[0]), tfu(Ar[8 * LDM]), tfu(Ar[4]), tfu(Ar[8 * LDM + 4])};
+              const uint32_t b[2] = {tfu(Bc[0]), tfu(Bc[4 * LDM])};
               mma_16x8x8_tf32(d, a, b);
             }
-            *reinterpret_cast<float2*>(Xp + g * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(Xp + (g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
-          }
-          named_bar_sync(BAR_SOLVE, NSOLVE);
-          if (warp < 4) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            __syncwarp();
+            *reinterpret_cast<float2*>(Xw + g4 * LDW + 2 * t4) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(Xw + (g4 + 8) * LDW + 2 * t4) = make_float2(d[2], d[3]);
+            __syncwarp();
+            d[0] = d[1] = d[2] = d[3] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
-              const float* Ar = Msc + (16 * I + g) * LDM + 16 * I + 8 * ks + t;
-              const float* Bc = Xp + (8 * ks + t) * LDX + 8 * nt + g;
-              const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                     __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-              const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
+              const float* Ar = Msc + (I + g4) * LDM + I + 8 * ks + t4;
+              const float* Bc = Xw + (8 * ks + t4) * LDW + g4;
+              const uint32_t a[4] = {tfu(Ar[0]), tfu(Ar[8 * LDM]), tfu(Ar[4]), tfu(Ar[8 * LDM + 4])};
+              const uint32_t b[2] = {tfu(Bc[0]), tfu(Bc[4 * LDW])};
               mma_16x8x8_tf32(d, a, b);
             }
-            const int row = 16 * I + g, col = 16 * J + 8 * nt + 2 * t;
-            *reinterpret_cast<float2*>(Msc + row * LDM + col) = make_float2(-d[0], -d[1]);
-            *reinterpret_cast<float2*>(Msc + (row + 8) * LDM + col) = make_float2(-d[2], -d[3]);
-            put_t2(row, col, -d[0], -d[1]);
-            put_t2(row + 8, col, -d[2], -d[3]);
+            const int row = I + g4, colo = J + 8 * n + 2 * t4;
+            *reinterpret_cast<float2*>(Msc + row * LDM + colo) = make_float2(-d[0], -d[1]);
+            *reinterpret_cast<float2*>(Msc + (row + 8) * LDM + colo) = make_float2(-d[2], -d[3]);
+            put_t2(row, colo, -d[0], -d[1]);
+            put_t2(row + 8, colo, -d[2], -d[3]);
           }
-          named_bar_sync(BAR_SOLVE, NSOLVE);
-        }
-        // the diagonal 32x32 blocks of T are in the operand tile: most of the U~ product can go
-        fence_proxy_async_smem();
-        tc_fence_before();
-        warp_arrive(&ms.bar_tdiag);
-        {
-          // 64x64: T_21 = -T_22 (A_21 T_11) with 32x32 blocks; warp 4 mt + nt (8 warps)
-          // computes the 16 x 8 output tile (rows [16 mt, +16), columns [8 nt, +8)).
-          const int g = lane >> 2, t = lane & 3;
-          const int mt = (warp >> 2) & 1, nt = warp & 3;
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
+          // the diagonal 32x32 blocks of T are in the operand tile: most of the U~ product can go
+          fence_proxy_async_smem();
+          tc_fence_before();
+          warp_arrive(&ms.bar_tdiag);
+          if (tid == 0) STAMP(c, 10);
+          named_bar_sync(BAR_SOLVE, 128);
+          {
+            // ---- 64-level merge: T_21 = -T_22 (A_21 T_11) in 32 x 32 blocks; warp k computes the
+            // 8 output columns [8 k, 8 k + 8) (T_11 and T_22 are zero above their diagonals, so
+            // those k-steps are skipped)
+            float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 8 * ks + t;
-            const float* Bc = Msc + (8 * ks + t) * LDM + 8 * nt + g;
-            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDM]))};
-            mma_16x8x8_tf32(d, a, b);
-          }
-          *reinterpret_cast<float2*>(Xsc + (16 * mt + g) * LDX + 8 * nt + 2 * t) = make_float2(d[0], d[1]);
-          *reinterpret_cast<float2*>(Xsc + (16 * mt + g + 8) * LDX + 8 * nt + 2 * t) = make_float2(d[2], d[3]);
-          named_bar_sync(BAR_SOLVE, NSOLVE);
-          d[0] = d[1] = d[2] = d[3] = 0.f;
+            for (int ks = 0; ks < 4; ++ks) {
+              if (ks < k) continue;
+              const float* Bc = Msc + (8 * ks + t4) * LDM + 8 * k + g4;
+              const uint32_t b[2] = {tfu(Bc[0]), tfu(Bc[4 * LDM])};
+              const float* A0 = Msc + (32 + g4) * LDM + 8 * ks + t4;
+              const float* A1 = A0 + 16 * LDM;
+              const uint32_t a0[4] = {tfu(A0[0]), tfu(A0[8 * LDM]), tfu(A0[4]), tfu(A0[8 * LDM + 4])};
+              const uint32_t a1[4] = {tfu(A1[0]), tfu(A1[8 * LDM]), tfu(A1[4]), tfu(A1[8 * LDM + 4])};
+              mma_16x8x8_tf32(d0, a0, b);
+              mma_16x8x8_tf32(d1, a1, b);
+            }
+            __syncwarp();
+            *reinterpret_cast<float2*>(Xw + g4 * LDW + 2 * t4) = make_float2(d0[0], d0[1]);
+            *reinterpret_cast<float2*>(Xw + (g4 + 8) * LDW + 2 * t4) = make_float2(d0[2], d0[3]);
+            *reinterpret_cast<float2*>(Xw + (g4 + 16) * LDW + 2 * t4) = make_float2(d1[0], d1[1]);
+            *reinterpret_cast<float2*>(Xw + (g4 + 24) * LDW + 2 * t4) = make_float2(d1[2], d1[3]);
+            __syncwarp();
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const float* Ar = Msc + (32 + 16 * mt + g) * LDM + 32 + 8 * ks + t;
-            const float* Bc = Xsc + (8 * ks + t) * LDX + 8 * nt + g;
-            const uint32_t a[4] = {__float_as_uint(rna_tf32(Ar[0])), __float_as_uint(rna_tf32(Ar[8 * LDM])),
-                                   __float_as_uint(rna_tf32(Ar[4])), __float_as_uint(rna_tf32(Ar[8 * LDM + 4]))};
-            const uint32_t b[2] = {__float_as_uint(rna_tf32(Bc[0])), __float_as_uint(rna_tf32(Bc[4 * LDX]))};
-            mma_16x8x8_tf32(d, a, b);
+            for (int mt = 0; mt < 2; ++mt) {
+              float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int ks = 0; ks < 2 + 2 * mt; ++ks) {
+                const float* Ar = Msc + (32 + 16 * mt + g4) * LDM + 32 + 8 * ks + t4;
+                const float* Bc = Xw + (8 * ks + t4) * LDW + g4;
+                const uint32_t a[4] = {tfu(Ar[0]), tfu(Ar[8 * LDM]), tfu(Ar[4]), tfu(Ar[8 * LDM + 4])};
+                const uint32_t b[2] = {tfu(Bc[0]), tfu(Bc[4 * LDW])};
+                mma_16x8x8_tf32(d, a, b);
+              }
+              const int row = 32 + 16 * mt + g4, colo = 8 * k + 2 * t4;
+              put_t2(row, colo, -d[0], -d[1]);
+              put_t2(row + 8, colo, -d[2], -d[3]);
+            }
           }
-          const int row = 32 + 16 * mt + g, col = 8 * nt + 2 * t;
-          put_t2(row, col, -d[0], -d[1]);
-          put_t2(row + 8, col, -d[2], -d[3]);
+          fence_proxy_async_smem();  // the T operand tile
+          tc_fence_before();
+          warp_arrive(&ms.bar_solved);
+        } else {
+          // warps 4-7 take no part in the solve: their arrivals go first
+          tc_fence_before();
+          warp_arrive(&ms.bar_tdiag);
+          warp_arrive(&ms.bar_solved);
         }
-        fence_proxy_async_smem();  // the T operand tile
-        tc_fence_before();
-        warp_arrive(&ms.bar_solved);
+        if (tid == 0) STAMP(c, 11);
         // ===== U~^T rounded to tf32 in place: the A operand of the chunk's last product =======
         const bool ok_u = wait_mma();
         tc_fence_after();
@@ -915,6 +970,7 @@ __global__ void __launch_bounds__(NT, 1)
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(&ms.bar_uround);
+        if (tid == 0) STAMP(c, 12);
         ok_prev = ok_u;
         if constexpr (PREP)
           if (c + 1 < nch) ok_prev = norms_ahead(ok_prev);
@@ -939,8 +995,10 @@ __global__ void __launch_bounds__(NT, 1)
         fence_proxy_async_smem();  // this warp's rows of the P operand tile
         tc_fence_before();
         warp_arrive(&ms.bar_tdiag);
+        if (tid == 256) STAMP(c, 13);
         // ===== then one chunk ahead: Vw^T and the cumulative decay of the next chunk =========
         if (c + 1 < nch) ok_s = decay_ahead(c + 1, PREP ? ok_s : vw_ahead(c + 1, ok_s));
+        if (tid == 256) STAMP(c, 14);
         // These warps do not use U~; they step their phase bit past its product without
         // waiting (by now the chunk's last product may have completed as well, and a parity
         // wait must never trail its barrier by two phases).  Their next wait, on that last
@@ -951,6 +1009,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       // the next chunk reads what warps 8-15 prepared
       if (named_bar_or(BAR_COMP, NCOMP, !ok_prev)) { dead = true; break; }
+      if (tid == 0) STAMP(c, 15);
       tc_fence_after();
     }
 
@@ -1148,7 +1207,8 @@ cudaError_t launch_split(const ChunkArgs& a, TcParams p, cudaStream_t st, const 
                        : launch_shape<64, 64, false, false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);
   };
   p.split_phase = 1;
-  cudaError_t e = pass(BH * (2 * P - 1));
+  // first pass: segment 0, and N_s, M_s for s = 1 .. P - 2 (the chain reads no others)
+  cudaError_t e = pass(BH * (2 * P - 3));
   if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (P > 2) {
@@ -1202,6 +1262,7 @@ cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream
   p.nseq = a.B * a.H;
   p.dscale = nullptr;
   p.err = device_error_word();
+  p.stamps = stamp_buffer();
   p.split_phase = 5;
   p.split_P = 1;
   p.split_L = a.T;
@@ -1246,6 +1307,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st) {
   p.cu_seqlens = a.cu_seqlens;
   p.nseq = varlen ? a.B : 0;
   p.err = device_error_word();
+  p.stamps = stamp_buffer();
   const int grid = a.B * a.H;
   p.dscale = a.decay_scale;
   cudaError_t e;

@@ -42,9 +42,13 @@ struct ChunkArgs {
 // gdn2_device_status().
 enum : unsigned {
   kErrWaitTimeout = 1u,  // a bounded wait gave up
-  kErrBadSeqlens = 2u    // packed-sequence offsets out of order or out of range
+  kErrBadSeqlens = 2u,   // packed-sequence offsets out of order or out of range
+  kErrDecayRange = 4u    // an in-chunk cumulative log decay fell below -80
 };
 unsigned* device_error_word();
+// Instrumented builds (GDN2_STAMPS): the device buffer of per-chunk clock stamps of the
+// chunk kernel on the current device; NULL in the product build.
+unsigned long long* stamp_buffer();
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
 // device (the attribute belongs to each device's context): `done` holds one bit per device

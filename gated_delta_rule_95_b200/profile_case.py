@@ -4,9 +4,16 @@
     python -m gated_delta_rule_95_b200.profile_case --kind decode --B 256 --H 16 --reps 4
     python -m gated_delta_rule_95_b200.profile_case --kind bwd --B 2 --H 16 --T 1024 --reps 2
     python -m gated_delta_rule_95_b200.profile_case --kind csize --chunk 128 --B 8 --H 16 --T 1024 --reps 2
+    python -m gated_delta_rule_95_b200.profile_case --kind prefill --stamps
 
 Inputs follow the recipe of the named workload (gdn2_inputs) with the given
 sizes; it exits 0 after a device synchronisation and a clean device status.
+
+--stamps runs the prefill on the instrumented library (libgdn2_stamps.so, built with
+GDN2_STAMPS: the chunk kernel's first CTA records clock64 at the points of its
+per-chunk schedule) and prints, per chunk, each point's cycle count relative to the
+point where the chunk's raw input tiles have landed, and the period between consecutive
+chunks.
 """
 from __future__ import annotations
 
@@ -28,12 +35,16 @@ def main():
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--reps", type=int, default=2)
     ap.add_argument("--chunk", type=int, default=64)
+    ap.add_argument("--stamps", action="store_true")
     a = ap.parse_args()
 
     import torch
 
     import gdn2_inputs as gi
     import gated_delta_rule_95_b200 as g
+
+    if a.stamps:
+        return stamps(a)
 
     dev = torch.device("cuda", 0)
     if a.kind == "prefill":
@@ -66,6 +77,52 @@ def main():
             t = {k: v.to(dev) for k, v in gi.decode_tokens(wl, j, B=a.B, H=a.H).items()}
             g.gdn2_decode_step(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], S)
     torch.cuda.synchronize()
+    status = g.gdn2_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status}")
+    print("ok")
+
+
+# stamp slots of the chunk kernel (its STAMP points), by role
+STAMP_SLOTS = 32
+SLOT_NAMES = {0: "AP issued", 1: "SP issued", 2: "U diag issued", 3: "U T21 issued", 4: "OP issued",
+              5: "raw landed", 6: "operands built", 7: "AP done", 8: "A/P read out", 9: "8x8 inverses",
+              10: "32-level done", 11: "64-level done", 12: "U rounded", 13: "R rounded",
+              14: "next decay ready", 15: "chunk end", 16: "o stored"}
+
+
+def stamps(a):
+    import ctypes
+
+    import numpy as np
+    import torch
+
+    import gdn2_inputs as gi
+    import gated_delta_rule_95_b200 as g
+    from gated_delta_rule_95_b200 import build as cuda_build
+
+    path = cuda_build.build(stamps=True)
+    lib = g.lib(path)  # the instrumented library in place of the product one
+    wl = gi.WORKLOADS[a.workload or "prefill_b8_h16_t4096"]
+    d = gi.prefill_inputs(wl, B=a.B, T=a.T, H=a.H)
+    x = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+    for _ in range(max(2, a.reps)):
+        g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
+    torch.cuda.synchronize()
+    buf = (ctypes.c_ulonglong * (64 * STAMP_SLOTS))()
+    lib.gdn2_stamps_read.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    n = lib.gdn2_stamps_read(buf, 64 * STAMP_SLOTS)
+    st = np.frombuffer(buf, dtype=np.uint64)[:n].astype(np.int64).reshape(-1, STAMP_SLOTS)
+    nch = min(64, (x["q"].shape[1] + 63) // 64)
+    base = st[:nch, 5]
+    print("cycles relative to the point where the chunk's raw tiles have landed (clock64 of the first CTA's SM)")
+    for c in range(nch):
+        per = base[c] - base[c - 1] if c > 0 else 0
+        row = sorted(((int(st[c, s] - base[c]), SLOT_NAMES[s]) for s in SLOT_NAMES if st[c, s]))
+        print(f"chunk {c} (period {per}): " + ", ".join(f"{n} {v}" for v, n in row))
+    per = np.diff(base[1:nch])
+    if len(per):
+        print(f"median period {int(np.median(per))} cycles")
     status = g.gdn2_device_status()
     if status != 0:
         raise SystemExit(f"device status {status}")

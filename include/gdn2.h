@@ -19,8 +19,12 @@
  *   - Tensors are dense, row-major (C order), and 16-byte aligned.
  *   - The decay gate is passed as log(alpha), fp32, finite and <= 0.  Within one
  *     chunk of 64 tokens the cumulative log decay of a channel must stay above
- *     about -80 (the chunk form scales keys by exp(-sum log alpha)); beyond that
- *     the result is undefined.
+ *     -80 (the chunk form scales keys by exp(-sum log alpha)); beyond that the
+ *     result is undefined, and the chunk kernels flag it: the next
+ *     gdn2_device_status() returns GDN2_ERR_RANGE.  This holds for the
+ *     raw-projection entry points too, where log alpha = -s_h softplus(a) is
+ *     formed inside the kernel (a_raw averaging above about 1.2 over a chunk at
+ *     s_h = 1 leaves the range).
  *   - dt selects the type of q, k, v, b and w: GDN2_BF16 or GDN2_F32.  The
  *     output o and the state (S0, S_T, S) are always fp32, and accumulation is
  *     fp32.  (o is stored in fp32 because its values are heavy-tailed: rounding
@@ -55,7 +59,10 @@ typedef enum {
   GDN2_ERR_DTYPE = 3,   /* dt is not a gdn2_dtype value */
   GDN2_ERR_ALIGN = 4,   /* a pointer is not 16-byte aligned */
   GDN2_ERR_CUDA = 5,    /* a CUDA runtime/driver call failed (see gdn2_last_cuda_error) */
-  GDN2_ERR_TIMEOUT = 6  /* a bounded device-side wait gave up (device error word set) */
+  GDN2_ERR_TIMEOUT = 6, /* a bounded device-side wait gave up (device error word set) */
+  GDN2_ERR_RANGE = 7    /* the decay left the supported range: some channel's cumulative log
+                           decay within one 64-token chunk fell below -80 (outputs undefined;
+                           reported by gdn2_device_status) */
 } gdn2_status;
 
 typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;

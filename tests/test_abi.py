@@ -33,8 +33,9 @@ def test_library_exports(name):
 def test_version_and_status_strings():
     L = g.lib()
     assert L.gdn2_version() >= 100
-    for s in range(7):
-        assert L.gdn2_status_string(s)
+    for s in range(8):
+        assert L.gdn2_status_string(s) and L.gdn2_status_string(s) != b"unknown status"
+    assert L.gdn2_status_string(8) == b"unknown status"
 
 
 P = ctypes.c_void_p

@@ -151,3 +151,35 @@ def test_decode_raw_steps_equal_chunk_forward_raw():
     torch.cuda.synchronize()
     assert rel_err(od.cpu().numpy(), o_c.cpu().numpy()) <= TOL["bf16"]
     assert rel_err(S.cpu().numpy(), S_c.cpu().numpy()) <= TOL["bf16"]
+
+
+GDN2_ERR_RANGE = 7
+
+
+def test_decay_beyond_the_chunk_range_is_flagged():
+    """The chunk form scales keys by exp(-g) with g the in-chunk cumulative log decay; below
+    g = -80 that leaves the fp32 range.  With s_h = 1 and a_raw shifted by +3 (softplus(3) is
+    about 3.05 per token, about -195 over a chunk), the raw entry must report the range
+    error through the device status; an in-range call afterwards reports clean again."""
+    wl = dataclasses.replace(BASE, seed=31)
+    d = gi.raw_inputs(wl, B=1, T=128, H=2)
+    d["a_raw"] = (d["a_raw"] + 3.0).contiguous()
+    _run(d, scale=None)
+    assert g.gdn2_device_status() == GDN2_ERR_RANGE
+    d = gi.raw_inputs(wl, B=1, T=128, H=2)
+    o, S = _run(d)
+    assert g.gdn2_device_status() == 0
+    o_ref, S_ref = _oracle(d, gi.as_f64(d["decay_scale"]))
+    assert rel_err(o.cpu().numpy(), o_ref) <= TOL["bf16"]
+
+
+def test_plain_entry_flags_decay_beyond_the_chunk_range():
+    """Same bound on the plain entry: log alpha = -2 per token gives -128 over a chunk."""
+    wl = dataclasses.replace(BASE, seed=32)
+    d = gi.prefill_inputs(wl, B=1, T=64, H=1)
+    x = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+    la = torch.full_like(x["log_alpha"], -2.0)
+    g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], la, x["b"], x["w"], None)
+    assert g.gdn2_device_status() == GDN2_ERR_RANGE
+    g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], None)
+    assert g.gdn2_device_status() == 0
