@@ -195,7 +195,23 @@ struct BwdParams {
   float* dgc;           // [B H][nch][DK]: dGamma_C, zero on entry
   int T, H, nch;
   int states_given;     // the entering states are already in `states`
+  unsigned long long* stamps = nullptr;  // instrumented build only: per-chunk clock stamps
 };
+
+#ifdef GDN2_STAMPS
+// Instrumented build (GDN2_STAMPS): clock64 at fixed points of the reverse sweep, for the
+// first CTA (batch 0, head 0, value columns 0-31), into [chunk][slot] of a 64 x 32 array;
+// thread 0 writes.
+#define BWD_STAMP(cc, slot)                                                                    \
+  do {                                                                                         \
+    if (p.stamps && blockIdx.x == 0 && threadIdx.x == 0 && (cc) >= 0 && (cc) < 64)             \
+      p.stamps[(size_t)(cc) * 32 + (slot)] = (unsigned long long)clock64();                    \
+  } while (0)
+#else
+#define BWD_STAMP(cc, slot) \
+  do {                      \
+  } while (0)
+#endif
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * MW : BT, 1)
@@ -516,16 +532,21 @@ __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * M
         dOj[t * LJ + j + 3] = ov[m].w;
       }
     }
+    BWD_STAMP(c, 0);
     if (tid < DK) dgC[tid] = 0.f;
     build(c, true);
     __syncthreads();
+    BWD_STAMP(c, 1);
     strict_lower_kk(X1, Kb, false);  // A
     strict_lower_kk(Pm, Qh, true);   // P
     __syncthreads();
+    BWD_STAMP(c, 2);
     solve();
     __syncthreads();
+    BWD_STAMP(c, 3);
     r_and_u(c);
     __syncthreads();
+    BWD_STAMP(c, 4);
     // dGamma_C = rowsum(dS_next * (S + Kn^T U)), this CTA's columns: thread (row group,
     // column group) sums its products, then the 8 threads of a row group add theirs
     if constexpr (TC) {
@@ -586,6 +607,7 @@ __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * M
       dS[i * LJ + j] *= gC[i];
     }
     __syncthreads();
+    BWD_STAMP(c, 5);
     // dU = P^T dO + Kn dSt
     prod<TC, BC, BJ, 2, 4>(BC, [&](int t, int s) { return Pm[s * LC + t]; }, [&](int s, int j) { return dOj[s * LJ + j]; },
                        [&](int t, int j, float acc) { dU[t * LJ + j] = acc; });
@@ -610,6 +632,7 @@ __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * M
     prod<TC, BC, BC, 4, 4>(BC, [&](int t, int r) { return X1[t * LC + r]; }, [&](int r, int s) { return Tm[s * LC + r]; },
                            [&](int t, int s, float acc) { Ym[t * LC + s] = acc; });
     __syncthreads();
+    BWD_STAMP(c, 6);
     // dA = strictly lower part of -T^T Y over dT
     prod<TC, BC, BC, 4, 4>(BC, [&](int t, int r) { return Tm[r * LC + t]; }, [&](int r, int s) { return Ym[r * LC + s]; },
                            [&](int t, int s, float acc) { X1[t * LC + s] = s < t ? -acc : 0.f; });
@@ -618,6 +641,7 @@ __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * M
     prod<TC, BC, BC, 4, 4>(BJ, [&](int t, int j) { return dOj[t * LJ + j]; }, [&](int j, int s) { return Um[s * LJ + j]; },
                            [&](int t, int s, float acc) { Pm[t * LC + s] = s <= t ? acc : 0.f; });
     __syncthreads();
+    BWD_STAMP(c, 7);
     // key-side gradients of this CTA's columns, summed over the slices in global memory:
     //   dKb = -dR S^T + dA Kn,  dKn = U dSt^T + dA^T Kb + dP^T Qh,  dQh = dO S^T + dP Kn
     if constexpr (TC) {
@@ -714,6 +738,7 @@ __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * M
         }
       }
     }
+    BWD_STAMP(c, 8);
     // dS (before the chunk) = Qh^T dO + dSt - Kb^T dR
     if constexpr (TC) {
       float d[MT<DK, BJ>::TPW][4];
@@ -766,6 +791,7 @@ __global__ void __launch_bounds__(std::is_same<T, __nv_bfloat16>::value ? 32 * M
         for (int y = 0; y < 4; ++y) dS[(tm * TM + x) * LJ + tn + 8 * y] = acc[x][y];
     }
     __syncthreads();
+    BWD_STAMP(c, 9);
   }
   if (p.dS0)
     for (int e = tid; e < DK * BJ; e += NTH) {
@@ -833,6 +859,7 @@ cudaError_t launch_bwd_t(const ChunkBwdArgs& a, cudaStream_t st) {
   p.T = a.T;
   p.H = a.H;
   p.nch = (a.T + BC - 1) / BC;
+  p.stamps = stamp_buffer();
   const size_t BH = (size_t)a.B * a.H;
   p.states = a.workspace;
   p.dgc = a.workspace + BH * p.nch * DK * DV;

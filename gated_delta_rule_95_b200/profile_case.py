@@ -5,13 +5,14 @@
     python -m gated_delta_rule_95_b200.profile_case --kind bwd --B 2 --H 16 --T 1024 --reps 2
     python -m gated_delta_rule_95_b200.profile_case --kind csize --chunk 128 --B 8 --H 16 --T 1024 --reps 2
     python -m gated_delta_rule_95_b200.profile_case --kind prefill --stamps
+    python -m gated_delta_rule_95_b200.profile_case --kind bwd --stamps
 
 Inputs follow the recipe of the named workload (gdn2_inputs) with the given
 sizes; it exits 0 after a device synchronisation and a clean device status.
 
---stamps runs the prefill on the instrumented library (libgdn2_stamps.so, built with
-GDN2_STAMPS: the chunk kernel's first CTA records clock64 at the points of its
-per-chunk schedule) and prints, per chunk, each point's cycle count relative to the
+--stamps runs the prefill (or the backward) on the instrumented library
+(libgdn2_stamps.so, built with GDN2_STAMPS: the kernel's first CTA records clock64 at the
+points of its per-chunk schedule) and prints, per chunk, each point's cycle count relative to the
 point where the chunk's raw input tiles have landed, and the period between consecutive
 chunks.
 """
@@ -85,6 +86,9 @@ def main():
 
 # stamp slots of the chunk kernel (its STAMP points), by role
 STAMP_SLOTS = 32
+BWD_SLOT_NAMES = {0: "loads done", 1: "operands built", 2: "A, P formed", 3: "T solved", 4: "R, U formed",
+                  5: "dGamma_C, dSt", 6: "dU, dR, dW, dV", 7: "dA, dP", 8: "key-side gradients",
+                  9: "dS updated"}
 SLOT_NAMES = {0: "AP issued", 1: "SP issued", 2: "U diag issued", 3: "U T21 issued", 4: "OP issued",
               5: "raw landed", 6: "operands built", 7: "AP done", 8: "A/P read out", 9: "8x8 inverses",
               10: "32-level done", 11: "64-level done", 12: "U rounded", 13: "R rounded",
@@ -106,21 +110,34 @@ def stamps(a):
     wl = gi.WORKLOADS[a.workload or "prefill_b8_h16_t4096"]
     d = gi.prefill_inputs(wl, B=a.B, T=a.T, H=a.H)
     x = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+    names, first = SLOT_NAMES, 5
+    if a.kind == "bwd":
+        B, T, H = x["q"].shape[:3]
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(wl.seed)
+        dO = torch.randn((B, T, H, wl.dv), generator=gen, device="cuda")
+        dS = torch.randn((B, H, wl.dk, wl.dv), generator=gen, device="cuda")
+        names, first = BWD_SLOT_NAMES, 0
     for _ in range(max(2, a.reps)):
-        g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
+        if a.kind == "bwd":
+            g.gdn2_chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], dO, dS)
+        else:
+            g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
     torch.cuda.synchronize()
     buf = (ctypes.c_ulonglong * (64 * STAMP_SLOTS))()
     lib.gdn2_stamps_read.argtypes = [ctypes.c_void_p, ctypes.c_int]
     n = lib.gdn2_stamps_read(buf, 64 * STAMP_SLOTS)
     st = np.frombuffer(buf, dtype=np.uint64)[:n].astype(np.int64).reshape(-1, STAMP_SLOTS)
     nch = min(64, (x["q"].shape[1] + 63) // 64)
-    base = st[:nch, 5]
-    print("cycles relative to the point where the chunk's raw tiles have landed (clock64 of the first CTA's SM)")
+    base = st[:nch, first]
+    print("cycles relative to the chunk's first point (clock64 of the first CTA's SM); the "
+          "backward visits the chunks in reverse")
     for c in range(nch):
-        per = base[c] - base[c - 1] if c > 0 else 0
-        row = sorted(((int(st[c, s] - base[c]), SLOT_NAMES[s]) for s in SLOT_NAMES if st[c, s]))
+        prev = c + 1 if a.kind == "bwd" else c - 1
+        per = base[c] - base[prev] if 0 <= prev < nch else 0
+        row = sorted(((int(st[c, s] - base[c]), names[s]) for s in names if st[c, s]))
         print(f"chunk {c} (period {per}): " + ", ".join(f"{n} {v}" for v, n in row))
-    per = np.diff(base[1:nch])
+    per = np.abs(np.diff(base[1:nch]))
     if len(per):
         print(f"median period {int(np.median(per))} cycles")
     status = g.gdn2_device_status()
