@@ -377,6 +377,24 @@ def time_raw(args, dev):
     return dict(ms=ms, tokens=B * T, token_heads=B * T * H, ok=g.gdn2_device_status() == 0)
 
 
+def time_tiny_f32(args, dev):
+    """The tiny fp32 workload (B1 H1 T256, d_k = d_v = 64, fp32 inputs: the 1e-4 parity bar)
+    through gdn2_chunk_fwd, which runs it on the fp32 kernel."""
+    import torch
+    import gated_delta_rule_95_b200 as g
+    wl = gi.WORKLOADS["tiny_f32"]
+    d = gi.prefill_inputs(wl)
+    x = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=torch.float32, device=dev)
+    S_T = torch.empty((wl.B, wl.H, wl.dk, wl.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], None, o=o, S_T=S_T)
+
+    ms = _time_loop(step, max(args.steps, 100), args.warmup)
+    return dict(ms=ms, tokens=wl.B * wl.T, ok=g.gdn2_device_status() == 0)
+
+
 def time_prefill_e2e(args, dev):
     """Same step through the public API with pinned host buffers, copies included: every
     step copies its inputs host->device, runs the forward and copies o and S_T back.  Steps
@@ -582,6 +600,7 @@ def main():
     lg = time_long(args, dev)
     bw = time_bwd(args, dev)
     cs = time_csize(args, dev)
+    tf = time_tiny_f32(args, dev)
     bw_tflops = bw["chunk_heads"] * BWD_FLOP_PER_CHUNK_HEAD / (bw["ms"] * 1e-3) / 1e12
     lg_gbs = lg["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD / (lg["ms_split"] * 1e-3) / 1e9
     cv_gbs = cv["bytes"] / (cv["ms"] * 1e-3) / 1e9
@@ -647,6 +666,10 @@ def main():
                                                      cs["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD
                                                      / (r["ms"] * 1e-3) / 1e9)}
                             for C, r in cs["sizes"].items()}},
+        "tiny_f32": {"metric": "GDN-2 prefill tokens/s per layer, fp32 inputs", "value": tf["tokens"] / (tf["ms"] * 1e-3),
+                     "unit": "tokens/s", "ms_per_step": tf["ms"],
+                     "workload": "tiny_f32: B=1 H=1 T=256 d_k=d_v=64, fp32 inputs (the fp32 CUDA-core kernel, "
+                                 "two CTAs of 32 value columns: latency-bound)"},
         "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
                  "steps": args.steps,
                  "workload": f"q, k, v projections of prefill_b8_h16_t4096 side by side: [8, 4096, {cv['C']}] bf16, "
@@ -674,7 +697,7 @@ def main():
         "gpu_launches": args.steps,
         "clocks": {k: pre["clocks"].get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
         "device_status_ok": bool(pre["ok"] and dec["ok"] and dec_b2b["ok"] and dec_raw["ok"] and pak["ok"] and raw["ok"] and cv["ok"]
-                                 and lg["ok"] and bw["ok"] and cs["ok"]),
+                                 and lg["ok"] and bw["ok"] and cs["ok"] and tf["ok"]),
     }
     if not args.no_e2e:
         line["e2e"] = time_prefill_e2e(args, dev)
