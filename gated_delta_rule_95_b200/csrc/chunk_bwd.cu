@@ -899,11 +899,18 @@ cudaError_t launch_bwd_dims(const ChunkBwdArgs& a, cudaStream_t st) {
 
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
   const size_t nch = (size_t)(T + BC - 1) / BC, BH = (size_t)B * H;
-  return sizeof(float) * BH * nch * ((size_t)dk * dv + dk);
+  const size_t warp_mma = sizeof(float) * BH * nch * ((size_t)dk * dv + dk);
+  // (the size does not depend on the dtype: d_k = d_v = 128 gets the tensor-core path's)
+  if (dk == 128 && dv == 128) {
+    const size_t tc = chunk_bwd_tc_workspace_bytes(B, T, H);
+    return tc > warp_mma ? tc : warp_mma;
+  }
+  return warp_mma;
 }
 
 cudaError_t launch_chunk_bwd(const ChunkBwdArgs& a, cudaStream_t st) {
   if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
+  if (a.bf16 && a.dk_ == 128 && a.dv_ == 128) return launch_chunk_bwd_tc(a, st);
   return a.bf16 ? launch_bwd_dims<__nv_bfloat16>(a, st) : launch_bwd_dims<float>(a, st);
 }
 

@@ -135,6 +135,9 @@ struct TcParams {
   // segments; ws: workspace [3][B H][P][d_k d_v] fp32 (M, N, start states).
   int split_phase = 0, split_P = 0, split_L = 0;
   float* ws = nullptr;
+  // checkpoint phase, for the tensor-core backward (NULL: not written): per (sequence, head,
+  // chunk) U~ [s][j], T^T [s][t] and P^T [t][s], fp32 with the tf32 rounding the products used
+  float *ck_u = nullptr, *ck_tt = nullptr, *ck_pt = nullptr;
   unsigned* err;
   unsigned long long* stamps = nullptr;  // instrumented build only: per-chunk clock stamps
 };
@@ -558,6 +561,17 @@ __global__ void __launch_bounds__(NT, 1)
       }
     };
 
+    // Checkpoint phase: T^T and P^T of chunk cc to the backward's workspace (both tiles stay
+    // intact until the next chunk's read-out and solve).
+    auto ckpt_tp = [&](int cc) {
+      const size_t at = ((size_t)su * nch + cc) * C * C;
+      for (int e = tid; e < C * C; e += NCOMP) {
+        const int r = e >> 6, x = e & 63;
+        p.ck_tt[at + e] = *reinterpret_cast<const float*>(sm + OFF_T + f32_off(x, r, R64));    // T[x][r]
+        p.ck_pt[at + e] = *reinterpret_cast<const float*>(sm + OFF_PK + f32_off(x, r, R192));  // P[x][r]
+      }
+    };
+
     // Warps 8-15, one chunk ahead (chunk cc).  Thread (ch, hf) owns the 32 tokens
     // [32 hf, 32 hf + 32) of channel ch.
     uint32_t ph_la = 0, ph_raw = 0, ph_vw = 0;
@@ -680,6 +694,7 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_after();
     for (int c = 0; c < nch && !dead; ++c) {
       const int ob = c & 1;
+      if (sp_ckpt && p.ck_tt && c > 0) ckpt_tp(c - 1);
       // ===== folded operands.  For this step thread t owns the key-channel pair
       // (2 cp, 2 cp + 1), cp = t mod 64, over the 8 tokens [8 ts, 8 ts + 8), ts = t / 64, so
       // that every raw load and tile store moves both channels at once.  Gamma = 2^g was
@@ -967,6 +982,11 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int x = 0; x < 32; ++x) v[x] = rna_tf32(v[x]);
         tmem_st32(tlane + TM_U + 32 * sg, v);
+        if (sp_ckpt && p.ck_u && vval) {  // U~ [s][j] of this chunk, for the backward
+          float* du = p.ck_u + ((size_t)su * nch + c) * C * dv + ch;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) du[(size_t)(32 * sg + x) * dv] = v[x];
+        }
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(&ms.bar_uround);
@@ -1013,6 +1033,7 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
     }
 
+    if (!dead && nch > 0 && sp_ckpt && p.ck_tt) ckpt_tp(nch - 1);
     // ---- last chunk's output and decay, then the final state -----------------------------
     if (!dead && nch > 0) {
       uint32_t ph_lr = 0;
@@ -1229,7 +1250,8 @@ cudaError_t launch_split(const ChunkArgs& a, TcParams p, cudaStream_t st, const 
 
 // The state entering every chunk ([B H][chunk][d_k][d_v] fp32 at `states`), for the backward
 // pass: the split instantiation's checkpoint phase over whole sequences (bf16, d_k = d_v).
-cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st) {
+cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st, float* ck_u, float* ck_tt,
+                                   float* ck_pt) {
   if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
   if (a.dk != a.dv || !a.bf16) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv, mb, mw, mla, mo;
@@ -1267,6 +1289,9 @@ cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream
   p.split_P = 1;
   p.split_L = a.T;
   p.ws = states;
+  p.ck_u = ck_u;
+  p.ck_tt = ck_tt;
+  p.ck_pt = ck_pt;
   const int grid = a.B * a.H;
   cudaError_t e = a.dk == 128 ? launch_shape<128, 128, false, false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p)
                               : launch_shape<64, 64, false, false, true>(grid, st, mq, mk, mv, mb, mw, mla, mo, p);

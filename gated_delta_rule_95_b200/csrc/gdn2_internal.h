@@ -80,6 +80,9 @@ struct ChunkBwdArgs {
 };
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_chunk_bwd(const ChunkBwdArgs& a, cudaStream_t st);
+// bf16, d_k = d_v = 128: the tensor-core backward (checkpoint pass, dS sweep, per-chunk pass)
+size_t chunk_bwd_tc_workspace_bytes(int B, int T, int H);
+cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs& a, cudaStream_t st);
 
 // Short causal (4 taps) over [B, T, C] (or packed [T, C] with cu_seqlens).
 struct ShortConvArgs {
@@ -98,8 +101,11 @@ cudaError_t launch_short_conv(const ShortConvArgs& a, cudaStream_t st);
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
 // bf16 inputs: tcgen05/TMEM kernel fed by TMA.
 cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st);
-// bf16, d_k = d_v: the state entering every chunk, [B H][chunk][d_k][d_v] fp32 (no outputs).
-cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st);
+// bf16, d_k = d_v: the state entering every chunk, [B H][chunk][d_k][d_v] fp32 (no outputs);
+// with ck_u, ck_tt, ck_pt also U~ [B H][chunk][64][d_v], T^T and P^T [B H][chunk][64][64] of
+// every chunk (the tensor-core backward's inputs).
+cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st, float* ck_u = nullptr,
+                                   float* ck_tt = nullptr, float* ck_pt = nullptr);
 // fp32 inputs: fp32 CUDA-core kernel of the same chunkwise algorithm.
 cudaError_t launch_chunk_fwd_f32(const ChunkArgs& a, cudaStream_t st);
 // bf16, chunk size 32, 64 or 128: the chunk-size study kernel (warp-level tf32 MMAs);

@@ -86,9 +86,11 @@ def main():
 
 # stamp slots of the chunk kernel (its STAMP points), by role
 STAMP_SLOTS = 32
-BWD_SLOT_NAMES = {0: "loads done", 1: "operands built", 2: "A, P formed", 3: "T solved", 4: "R, U formed",
-                  5: "dGamma_C, dSt", 6: "dU, dR, dW, dV", 7: "dA, dP", 8: "key-side gradients",
-                  9: "dS updated"}
+BWD_SLOT_NAMES = {0: "chunk start", 1: "dO^T stored", 2: "inputs loaded", 3: "operand tiles written",
+                  4: "dSn out, dSt formed", 5: "dU issued", 6: "dU done", 7: "dU rounded, dR issued",
+                  8: "dR done", 9: "-dR, dv, dw out, dS issued", 10: "dS done"}
+GRAD_SLOT_NAMES = {16: "unit start", 17: "copies landed, S in", 18: "operands built", 19: "first products done",
+                   20: "dP, dA, dSt written", 21: "second products done", 22: "gradients written"}
 SLOT_NAMES = {0: "AP issued", 1: "SP issued", 2: "U diag issued", 3: "U T21 issued", 4: "OP issued",
               5: "raw landed", 6: "operands built", 7: "AP done", 8: "A/P read out", 9: "8x8 inverses",
               10: "32-level done", 11: "64-level done", 12: "U rounded", 13: "R rounded",
@@ -140,6 +142,13 @@ def stamps(a):
     per = np.abs(np.diff(base[1:nch]))
     if len(per):
         print(f"median period {int(np.median(per))} cycles")
+    if a.kind == "bwd":
+        # the per-chunk pass: one CTA per (batch, head, chunk), rows = its first 64 CTAs
+        g0 = st[:nch, 16]
+        ok_rows = [c for c in range(nch) if g0[c]]
+        print("per-chunk pass, cycles from the start of a unit (each CTA's second), median over the first CTAs:")
+        print(", ".join(f"{GRAD_SLOT_NAMES[s]} {int(np.median([st[c, s] - g0[c] for c in ok_rows]))}"
+                        for s in sorted(GRAD_SLOT_NAMES) if all(st[c, s] for c in ok_rows)))
     status = g.gdn2_device_status()
     if status != 0:
         raise SystemExit(f"device status {status}")

@@ -128,8 +128,11 @@ GDN2_API gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const vo
  * the Gated DeltaNet-2 guide's "Chunkwise Parallel Algorithm for GPU Training", the
  * training-time counterpart of the forward).  The forward's inputs are passed again; the
  * chunk states are recomputed (bf16 inputs with d_k = d_v: by the tensor-core forward, tf32
- * products; otherwise in fp32).  Products: tf32 warp-level tensor-core MMAs with fp32
- * accumulation for bf16 inputs, fp32 on the CUDA cores for fp32 inputs.
+ * products; otherwise in fp32).  bf16 inputs with d_k = d_v = 128 run on the 5th-generation
+ * tensor cores (tcgen05, tf32 products, fp32 accumulation): the forward's checkpoint pass, a
+ * reverse sweep per (batch, head) carrying the state gradient, and a pass over all chunks in
+ * parallel for the other gradients.  Other bf16 shapes use tf32 warp-level MMAs; fp32
+ * inputs run fp32 products on the CUDA cores.
  *
  *   q .. w, S0, B, T, H, d_k, d_v, dt : as gdn2_chunk_fwd (the forward's inputs)
  *   dO          : [B, T, H, d_v] fp32
@@ -138,8 +141,9 @@ GDN2_API gdn2_status gdn2_chunk_fwd_split(const void* q, const void* k, const vo
  *   dv, dw      : [B, T, H, d_v] fp32, written
  *   dS0         : [B, H, d_k, d_v] fp32, written, or NULL for "not needed"
  *   workspace   : DEVICE scratch of gdn2_chunk_bwd_workspace_bytes(B, T, H, d_k, d_v)
- *                 bytes (every chunk's entering state), 16-byte aligned, owned by the
- *                 caller; two calls in flight must not share it
+ *                 bytes (per chunk: its entering state, and for d_k = d_v = 128 also the
+ *                 state gradient leaving it and the chunk's U, -dR, T^T, P^T), 16-byte
+ *                 aligned, owned by the caller; two calls in flight must not share it
  * Gradient buffers must not alias the inputs or each other.
  */
 GDN2_API size_t gdn2_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v);
