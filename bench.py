@@ -650,7 +650,9 @@ def main():
         "bwd": {"metric": "GDN-2 backward tokens/s per layer", "value": bw["tokens"] / (bw["ms"] * 1e-3),
                 "unit": "tokens/s", "ms_per_step": bw["ms"],
                 "workload": "prefill_b8_h16_t4096 backward: dq, dk, dv, dlog_alpha, db, dw, dS0 from dO and dS_T",
-                "roofline": {"bound": "tensor", "kernel": "chunk_bwd_kernel", "achieved": bw_tflops,
+                "kernels": "chunk_fwd_tc_kernel checkpoint pass (states, U, T^T, P^T), bwd_chain_kernel (reverse dS "
+                           "sweep, tcgen05), bwd_grad_kernel (per-chunk gradients, tcgen05)",
+                "roofline": {"bound": "tensor", "kernel": "the three launches together", "achieved": bw_tflops,
                              "peak": pk["bf16_tflops"] * TF32_PER_BF16, "unit": "TFLOP/s",
                              "frac": bw_tflops / (pk["bf16_tflops"] * TF32_PER_BF16),
                              "peak_src": "measured bf16 x nominal tf32/bf16 ratio",

@@ -55,9 +55,6 @@ constexpr uint32_t ID_128 = idesc_tf32(128, 128, 0, 0, 0, 0);
 __device__ __forceinline__ float rna(float x) {  // fp32 -> tf32, nearest (ties away), as fp32
   return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
-__device__ __forceinline__ float bf(const __nv_bfloat16* p, size_t x) {
-  return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p) + x) << 16);
-}
 __device__ __forceinline__ void st4r(unsigned char* p, float a, float b, float c, float d) {
   *reinterpret_cast<float4*>(p) = make_float4(rna(a), rna(b), rna(c), rna(d));
 }
@@ -83,26 +80,32 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t base, uint32_t panel, int ks)
 
 // ============================== (2) the dS sweep ==========================================
 struct ChainParams {
-  const __nv_bfloat16 *q, *k, *b, *v, *w;
-  const float* la;
-  const float* dO;
   const float* dS_T;  // [B H][d_k][d_v] or NULL
   float* dS0;         // [B H][d_k][d_v] or NULL
-  float *dv, *dw;     // [B][T][H][d_v]
   float* dsn;         // [B H][chunk][d_k][d_v]: gradient of the state leaving each chunk
-  float* nr;          // [B H][chunk][64][d_v]: -dR (tf32-rounded)
   int T, H, nch;
   unsigned* err;
   unsigned long long* stamps;  // instrumented build only
 };
+struct ChainMaps {  // panel-major token tiles (q, k, b, v, w bf16; log alpha, dO fp32), T^T, P^T;
+                    // the stores of dv, dw (fp32 tokens) and -dR
+  CUtensorMap q, k, b, v, w, la, dO, tt, pt, dv, dw, nr;
+};
 
 // shared memory (byte offsets from a 1024-byte aligned base)
-constexpr uint32_t K1_KN = 0;                // Kn [t][i]: 4 panels x 64 rows
+constexpr uint32_t K1_KN = 0;                 // Kn [t][i]: 4 panels x 64 rows
 constexpr uint32_t K1_KQT = K1_KN + 4 * R64;  // [Qh; Kb]^T [i][t']: 4 panels x 128 rows
-constexpr uint32_t K1_TP = K1_KQT + 4 * R128; // two buffers of {T^T [s][t], P^T [t][s]}: 2 + 2 panels x 64 rows
-constexpr uint32_t K1_TILES = K1_TP + 8 * R64;
+constexpr uint32_t K1_Y = K1_KQT + 4 * R128;  // dO [t][j] (fp32, 4 panels), v, w (bf16, 2 panels each)
+constexpr uint32_t K1_TP = K1_Y + 8 * R64;    // T^T [s][t] and P^T [t][s]: 2 + 2 panels x 64 rows
+constexpr uint32_t K1_TILES = K1_TP + 4 * R64;
+// staging of the raw log alpha, k, q, b over the Kn and [Qh; Kb]^T tiles they become
+constexpr uint32_t K1_RLA = 0, K1_RK = 4 * R64, K1_RQ = 6 * R64, K1_RB = 8 * R64;
+constexpr uint32_t K1_DO = K1_Y, K1_RV = K1_Y + 4 * R64, K1_RW = K1_Y + 6 * R64;
+// output staging (fp32 [t][j], 4 panels each) for TMA stores: dv over dO, dw over v and w,
+// -dR over T^T and P^T (each read before it is overwritten)
+constexpr uint32_t K1_ODV = K1_DO, K1_ODW = K1_RV, K1_ONR = K1_TP;
 struct ChainMisc {
-  uint64_t bar_tp[2], bar_mma, bar_drain;
+  uint64_t bar_x, bar_y, bar_tp, bar_mma, bar_drain;
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[D];
@@ -110,34 +113,70 @@ struct ChainMisc {
 };
 constexpr uint32_t K1_SMEM = K1_TILES + 1024 + sizeof(ChainMisc);
 // tensor memory columns (lanes = value channels j)
-constexpr uint32_t K1_DS = 0;     // dS^T fp32 accumulator [j][i]
-constexpr uint32_t K1_DSR = 128;  // dSt^T rounded [j][i]
-constexpr uint32_t K1_DO = 256;   // dO^T rounded [j][t]
-constexpr uint32_t K1_DU = 320;   // dU^T [j][t]
-constexpr uint32_t K1_DR = 384;   // dR^T [j][s], then -dR^T rounded
+constexpr uint32_t K1_TDS = 0;     // dS^T fp32 accumulator [j][i]
+constexpr uint32_t K1_TDSR = 128;  // dSt^T rounded [j][i]
+constexpr uint32_t K1_TDO = 256;   // dO^T rounded [j][t]
+constexpr uint32_t K1_TDU = 320;   // dU^T [j][t]
+constexpr uint32_t K1_TDR = 384;   // dR^T [j][s], then -dR^T rounded
 
-__global__ void __launch_bounds__(NTH, 1)
-    bwd_chain_kernel(const __grid_constant__ CUtensorMap tmTT, const __grid_constant__ CUtensorMap tmPT,
-                     const ChainParams p) {
+__global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant__ ChainMaps mp, const ChainParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   ChainMisc& ms = *reinterpret_cast<ChainMisc*>(sm + K1_TILES);
   const uint32_t sbase = smem_u32(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, ln = tid & 127, cg = tid >> 7;
+  const int tid = threadIdx.x, warp = tid >> 5, ln = tid & 127, cg = tid >> 7, lane = tid & 31;
   const int bh = blockIdx.x, h = bh % p.H, bb = bh / p.H, nch = p.nch;
   const bool st0 = blockIdx.x == 0;
   static_cast<void>(st0);
-  auto tok = [&](int t) -> size_t { return (((size_t)bb * p.T + t) * p.H + h) * D; };
+
+  // the copies of chunk cc, one per lane of warp 0 (lane 0 posts the byte count first):
+  // X = raw log alpha, k, q, b; Y = dO, v, w; TP = T^T, P^T
+  auto issue_x = [&](int cc) {
+    if (lane == 0) mbar_arrive_expect_tx(&ms.bar_x, 4 * R64 + 3 * 2 * R64);
+    __syncwarp();
+    if (lane == 0) tma_load_5d(sm + K1_RLA, &mp.la, &ms.bar_x, 0, C * cc, 0, h, bb);
+    else if (lane == 1) tma_load_5d(sm + K1_RK, &mp.k, &ms.bar_x, 0, C * cc, 0, h, bb);
+    else if (lane == 2) tma_load_5d(sm + K1_RQ, &mp.q, &ms.bar_x, 0, C * cc, 0, h, bb);
+    else if (lane == 3) tma_load_5d(sm + K1_RB, &mp.b, &ms.bar_x, 0, C * cc, 0, h, bb);
+  };
+  auto issue_y = [&](int cc) {
+    if (lane == 0) mbar_arrive_expect_tx(&ms.bar_y, 4 * R64 + 2 * 2 * R64);
+    __syncwarp();
+    if (lane == 0) tma_load_5d(sm + K1_DO, &mp.dO, &ms.bar_y, 0, C * cc, 0, h, bb);
+    else if (lane == 1) tma_load_5d(sm + K1_RV, &mp.v, &ms.bar_y, 0, C * cc, 0, h, bb);
+    else if (lane == 2) tma_load_5d(sm + K1_RW, &mp.w, &ms.bar_y, 0, C * cc, 0, h, bb);
+  };
+  auto issue_tp = [&](int cc) {
+    const int row = (bh * nch + cc) * C;
+    if (lane == 0) mbar_arrive_expect_tx(&ms.bar_tp, 4 * R64);
+    __syncwarp();
+    if (lane == 0) tma_load_3d(sm + K1_TP, &mp.tt, &ms.bar_tp, 0, row, 0);
+    else if (lane == 1) tma_load_3d(sm + K1_TP + 2 * R64, &mp.pt, &ms.bar_tp, 0, row, 0);
+  };
+  auto prefetch = [&](int cc) {  // every input of chunk cc into L2, one lane per tensor
+    const int row = (bh * nch + cc) * C;
+    switch (lane) {
+      case 0: tma_prefetch_l2_5d(&mp.la, 0, C * cc, 0, h, bb); break;
+      case 1: tma_prefetch_l2_5d(&mp.k, 0, C * cc, 0, h, bb); break;
+      case 2: tma_prefetch_l2_5d(&mp.q, 0, C * cc, 0, h, bb); break;
+      case 3: tma_prefetch_l2_5d(&mp.b, 0, C * cc, 0, h, bb); break;
+      case 4: tma_prefetch_l2_5d(&mp.dO, 0, C * cc, 0, h, bb); break;
+      case 5: tma_prefetch_l2_5d(&mp.v, 0, C * cc, 0, h, bb); break;
+      case 6: tma_prefetch_l2_5d(&mp.w, 0, C * cc, 0, h, bb); break;
+      case 7: tma_prefetch_l2_3d(&mp.tt, 0, row, 0); break;
+      case 8: tma_prefetch_l2_3d(&mp.pt, 0, row, 0); break;
+      default: break;
+    }
+  };
 
   if (tid == 0) {
-    mbar_init(&ms.bar_tp[0], 1);
-    mbar_init(&ms.bar_tp[1], 1);
+    mbar_init(&ms.bar_x, 1);
+    mbar_init(&ms.bar_y, 1);
+    mbar_init(&ms.bar_tp, 1);
     mbar_init(&ms.bar_mma, 1);
     mbar_init(&ms.bar_drain, 1);
     fence_mbar_init();
     ms.abort = 0;
-    tma_prefetch_desc(&tmTT);
-    tma_prefetch_desc(&tmPT);
   }
   if (warp == 0) {
     tmem_alloc(&ms.tmem_base, 512);
@@ -148,27 +187,23 @@ __global__ void __launch_bounds__(NTH, 1)
   tc_fence_after();
   const uint32_t tmem = ms.tmem_base;
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-
-  int n_tp[2] = {0, 0};  // loads issued per buffer (thread 0)
-  uint32_t ph_tp[2] = {0, 0}, ph_mma = 0;
-  auto issue_tp = [&](int cc) {  // T^T and P^T of chunk cc into buffer cc & 1
-    const int bf = cc & 1;
-    unsigned char* dst = sm + K1_TP + (uint32_t)bf * 4 * R64;
-    const int row = (bh * nch + cc) * C;
-    mbar_arrive_expect_tx(&ms.bar_tp[bf], 4 * R64);
-    tma_load_2d(dst, &tmTT, &ms.bar_tp[bf], 0, row);
-    tma_load_2d(dst + R64, &tmTT, &ms.bar_tp[bf], 32, row);
-    tma_load_2d(dst + 2 * R64, &tmPT, &ms.bar_tp[bf], 0, row);
-    tma_load_2d(dst + 3 * R64, &tmPT, &ms.bar_tp[bf], 32, row);
-    ++n_tp[bf];
-  };
-  // The products' completion: warp 0 polls the barrier (a suspended wait wakes too late for
-  // this chain of short products), the block follows through a hardware barrier; true for
-  // every thread unless the wait gave up.
-  auto wait_mma = [&]() -> bool {
+  // copies issued (warp 0): their count per barrier, for the drain after a give-up
+  int n_x = 0, n_y = 0, n_tp = 0;
+  uint32_t ph_x = 0, ph_y = 0, ph_tp = 0, ph_mma = 0;
+  if (warp == 0 && nch > 0) {
+    issue_x(nch - 1);
+    issue_y(nch - 1);
+    issue_tp(nch - 1);
+    ++n_x, ++n_y, ++n_tp;
+    if (nch > 1) prefetch(nch - 2);
+  }
+  // completion of a barrier phase: warp 0 polls (a suspended wait wakes too late for this
+  // chain of short steps), the block follows through a hardware barrier; true for every
+  // thread unless the wait gave up
+  auto wait_all = [&](uint64_t* bar, uint32_t& ph) -> bool {
     bool ok = true;
-    if (warp == 0) ok = mbar_wait_spin(&ms.bar_mma, ph_mma, &ms.abort, p.err, WAIT_LIMIT);
-    ph_mma ^= 1;
+    if (warp == 0) ok = mbar_wait_spin(bar, ph, &ms.abort, p.err, WAIT_LIMIT);
+    ph ^= 1;
     return !__syncthreads_or(!ok);
   };
   // every thread's tensor-memory and shared-memory writes visible to the next MMA; false
@@ -181,25 +216,6 @@ __global__ void __launch_bounds__(NTH, 1)
     tc_fence_after();
     return !bad;
   };
-  // the inputs of chunk cc into L2: one bulk prefetch per (tensor, token row)
-  auto prefetch = [&](int cc) {
-    const int e = tid;
-    if (e < 7 * C) {
-      const int tsr = e / C, t = C * cc + e % C;
-      if (t < p.T) {
-        const size_t x = tok(t);
-        switch (tsr) {
-          case 0: bulk_prefetch_l2(p.q + x, 2 * D); break;
-          case 1: bulk_prefetch_l2(p.k + x, 2 * D); break;
-          case 2: bulk_prefetch_l2(p.b + x, 2 * D); break;
-          case 3: bulk_prefetch_l2(p.v + x, 2 * D); break;
-          case 4: bulk_prefetch_l2(p.w + x, 2 * D); break;
-          case 5: bulk_prefetch_l2(p.la + x, 4 * D); break;
-          default: bulk_prefetch_l2(p.dO + x, 4 * D); break;
-        }
-      }
-    }
-  };
 
   // dS^T of the last chunk's end: dS_T^T (lane j, key columns [32 cg, 32 cg + 32))
   {
@@ -207,47 +223,47 @@ __global__ void __launch_bounds__(NTH, 1)
 #pragma unroll
     for (int x = 0; x < 32; ++x)
       v[x] = p.dS_T ? __ldg(p.dS_T + ((size_t)bh * D + 32 * cg + x) * D + ln) : 0.f;
-    tmem_st32(tl + K1_DS + 32 * cg, v);
+    tmem_st32(tl + K1_TDS + 32 * cg, v);
   }
-  if (tid == 0 && nch > 0) {
-    issue_tp(nch - 1);
-    if (nch > 1) issue_tp(nch - 2);
-  }
-  if (nch > 0) prefetch(nch - 1);
   bool dead = !sync_ok(true);
+  const uint32_t rb = (uint32_t)(ln >> 6) * R64 + (uint32_t)(ln & 7) * 2;  // bf16 staging: channel ln
+  const int chk = (ln & 63) >> 3;
+  auto bf_at = [&](uint32_t base, int t) -> float {
+    return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short*>(sm + base + rb + sw128_off(t, chk)))
+                           << 16);
+  };
 
   for (int c = nch - 1; c >= 0 && !dead; --c) {
     const int n = min(C, p.T - C * c);  // tokens of this chunk inside the sequence
     TC_STAMP(st0, c, 0);
-    if (c > 0) prefetch(c - 1);
-    // ===== build: thread (i = ln, cg) over the tokens [16 cg, 16 cg + 16) ===================
-    {
-      // dO^T rounded into tensor memory (lane j = ln)
-      float dv16[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const int t = 16 * cg + r;
-        const float x = __ldg(p.dO + tok(C * c + min(t, n - 1)) + ln);
-        dv16[r] = t < n ? rna(x) : 0.f;
+    if (warp == 0) {
+      // the previous chunk's stores have read their staging (over T^T, P^T and dO, v, w):
+      // this chunk's copies of those
+      if (c < nch - 1) {
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+        issue_tp(c);
+        issue_y(c);
+        ++n_tp, ++n_y;
       }
-      tmem_st16(tl + K1_DO + 16 * cg, dv16);
+      if (c >= 2) prefetch(c - 2);
     }
+    // ===== build: thread (i = ln, cg) over the tokens [16 cg, 16 cg + 16) ===================
+    if (!wait_all(&ms.bar_x, ph_x)) { dead = true; break; }
     TC_STAMP(st0, c, 1);
     float g[16], kq[16], qq[16], bq[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
       const int t = 16 * cg + r;
-      const bool val = t < n;
-      const size_t x = tok(C * c + min(t, n - 1)) + ln;
-      g[r] = val ? __ldg(p.la + x) : 0.f;
-      kq[r] = val ? bf(p.k, x) : 0.f;
-      qq[r] = val ? bf(p.q, x) : 0.f;
-      bq[r] = val ? bf(p.b, x) : 0.f;
+      g[r] = *reinterpret_cast<const float*>(sm + K1_RLA + f32_off(t, ln, R64));
+      kq[r] = bf_at(K1_RK, t);
+      qq[r] = bf_at(K1_RQ, t);
+      bq[r] = bf_at(K1_RB, t);
     }
 #pragma unroll
     for (int r = 1; r < 16; ++r) g[r] += g[r - 1];
     ms.seg[cg][ln] = g[15];
-    __syncthreads();
+    __syncthreads();  // (also: every read of the raw staging is done)
     TC_STAMP(st0, c, 2);
     float off = 0.f, tot = 0.f;
 #pragma unroll
@@ -257,6 +273,14 @@ __global__ void __launch_bounds__(NTH, 1)
       tot += sv;
     }
     if (cg == 0) ms.gC[ln] = __expf(tot);
+    if (!wait_all(&ms.bar_y, ph_y)) { dead = true; break; }
+    {
+      // dO^T rounded into tensor memory (lane j = ln); rows past the sequence read zero
+      float dv16[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) dv16[r] = rna(*reinterpret_cast<const float*>(sm + K1_DO + f32_off(16 * cg + r, ln, R64)));
+      tmem_st16(tl + K1_TDO + 16 * cg, dv16);
+    }
     {
       float qh[16], kb[16];
 #pragma unroll
@@ -276,10 +300,23 @@ __global__ void __launch_bounds__(NTH, 1)
     }
     __syncthreads();  // gC
     TC_STAMP(st0, c, 3);
+    // the first part of dU^T, dO^T P, goes as soon as the dO^T columns and P^T are in place
+    if (!sync_ok(true)) { dead = true; break; }
+    if (warp == 0) {
+      const bool ok = mbar_wait_spin(&ms.bar_tp, ph_tp, &ms.abort, p.err, WAIT_LIMIT);
+      ph_tp ^= 1;
+      if (ok && lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          umma_tf32_ts(tmem + K1_TDU, tmem + K1_TDO + 8 * ks, kdesc(sbase + K1_TP + 2 * R64, R64, ks), ID_64, ks > 0);
+      }
+      __syncwarp();
+    }
     // ===== dSn (the state gradient leaving this chunk) out; dSt^T = dS^T Diag(Gamma_C) ======
     {
       float v[32], r32[32];
-      tmem_ld32(tl + K1_DS + 32 * cg, v);
+      tmem_ld32(tl + K1_TDS + 32 * cg, v);
       tmem_ld_wait();
       float* dst = p.dsn + ((size_t)bh * nch + c) * D * D + ln;
 #pragma unroll
@@ -289,113 +326,113 @@ __global__ void __launch_bounds__(NTH, 1)
         v[x] *= ms.gC[i];
         r32[x] = rna(v[x]);
       }
-      tmem_st32(tl + K1_DS + 32 * cg, v);
-      tmem_st32(tl + K1_DSR + 32 * cg, r32);
+      tmem_st32(tl + K1_TDS + 32 * cg, v);
+      tmem_st32(tl + K1_TDSR + 32 * cg, r32);
     }
     TC_STAMP(st0, c, 4);
     if (!sync_ok(true)) { dead = true; break; }
-    // ===== dU^T = dO^T P + dSt^T Kn^T =========================================================
-    const uint32_t tp = sbase + K1_TP + (uint32_t)(c & 1) * 4 * R64;  // T^T, then P^T
+    // ===== dU^T += dSt^T Kn^T =================================================================
     if (tid == 0) {
-      const bool ok = mbar_wait_spin(&ms.bar_tp[c & 1], ph_tp[c & 1], &ms.abort, p.err, WAIT_LIMIT);
-      ph_tp[c & 1] ^= 1;
-      if (ok) {
-        tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          umma_tf32_ts(tmem + K1_DU, tmem + K1_DO + 8 * ks, kdesc(tp + 2 * R64, R64, ks), ID_64, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < 16; ++ks)
-          umma_tf32_ts(tmem + K1_DU, tmem + K1_DSR + 8 * ks, kdesc(sbase + K1_KN, R64, ks), ID_64, 1);
-        umma_commit(&ms.bar_mma);
-        TC_STAMP(st0, c, 5);
-      }
+      for (int ks = 0; ks < 16; ++ks)
+        umma_tf32_ts(tmem + K1_TDU, tmem + K1_TDSR + 8 * ks, kdesc(sbase + K1_KN, R64, ks), ID_64, 1);
+      umma_commit(&ms.bar_mma);
     }
-    // v and w of this thread's tokens (for dv, dw), in flight during the product
-    float vq[16], wq[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int t = 16 * cg + r;
-      const bool val = t < n;
-      const size_t x = tok(C * c + min(t, n - 1)) + ln;
-      vq[r] = val ? bf(p.v, x) : 0.f;
-      wq[r] = val ? bf(p.w, x) : 0.f;
-    }
-    bool ok = wait_mma();
+    TC_STAMP(st0, c, 5);
+    if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
     tc_fence_after();
     TC_STAMP(st0, c, 6);
     {
       float v[16];
-      tmem_ld16(tl + K1_DU + 16 * cg, v);
+      tmem_ld16(tl + K1_TDU + 16 * cg, v);
       tmem_ld_wait();
 #pragma unroll
       for (int r = 0; r < 16; ++r) v[r] = rna(v[r]);
-      tmem_st16(tl + K1_DU + 16 * cg, v);
+      tmem_st16(tl + K1_TDU + 16 * cg, v);
     }
-    if (!sync_ok(ok)) { dead = true; break; }
+    if (!sync_ok(true)) { dead = true; break; }
     // ===== dR^T = dU^T T =======================================================================
     if (tid == 0) {
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        umma_tf32_ts(tmem + K1_DR, tmem + K1_DU + 8 * ks, kdesc(tp, R64, ks), ID_64, ks > 0);
+        umma_tf32_ts(tmem + K1_TDR, tmem + K1_TDU + 8 * ks, kdesc(sbase + K1_TP, R64, ks), ID_64, ks > 0);
       umma_commit(&ms.bar_mma);
+      // the first part of the dS^T update, dS^T += dO^T Qh, runs behind it (tracked by the
+      // next commit)
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        umma_tf32_ts(tmem + K1_TDS, tmem + K1_TDO + 8 * ks, kdesc(sbase + K1_KQT, R128, ks), ID_128, 1);
     }
     TC_STAMP(st0, c, 7);
-    ok = wait_mma();
+    if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
     tc_fence_after();
+    TC_STAMP(st0, c, 8);
+    // ===== -dR^T rounded in place (the A operand of the update); dv = dR w, dw = dR v and -dR
+    // staged for TMA stores (v and w are read before their staging is overwritten)
     {
-      float v[16], nv[16];
-      TC_STAMP(st0, c, 8);
-      tmem_ld16(tl + K1_DR + 16 * cg, v);
+      float v[16], nv[16], wv[16], vv[16];
+      tmem_ld16(tl + K1_TDR + 16 * cg, v);
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        wv[r] = bf_at(K1_RW, 16 * cg + r);
+        vv[r] = bf_at(K1_RV, 16 * cg + r);
+      }
       tmem_ld_wait();
 #pragma unroll
       for (int r = 0; r < 16; ++r) nv[r] = rna(-v[r]);
-      tmem_st16(tl + K1_DR + 16 * cg, nv);
-      float* nr = p.nr + (((size_t)bh * nch + c) * C + 16 * cg) * D + ln;
+      tmem_st16(tl + K1_TDR + 16 * cg, nv);
+      __syncthreads();  // every read of v and w is done
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
-        const int t = 16 * cg + r;
-        nr[(size_t)r * D] = nv[r];
-        if (t < n) {
-          const size_t x = tok(C * c + t) + ln;
-          p.dv[x] = v[r] * wq[r];
-          p.dw[x] = v[r] * vq[r];
-        }
+        const uint32_t o = f32_off(16 * cg + r, ln, R64);
+        *reinterpret_cast<float*>(sm + K1_ODV + o) = v[r] * wv[r];
+        *reinterpret_cast<float*>(sm + K1_ODW + o) = v[r] * vv[r];
+        *reinterpret_cast<float*>(sm + K1_ONR + o) = nv[r];
       }
     }
-    if (!sync_ok(ok)) { dead = true; break; }
-    // ===== dS^T <- dSt^T + dO^T Qh - dR^T Kb ===================================================
+    if (!sync_ok(true)) { dead = true; break; }
+    // ===== dS^T += -dR^T Kb: the update completes ==============================================
     if (tid == 0) {
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        umma_tf32_ts(tmem + K1_DS, tmem + K1_DO + 8 * ks, kdesc(sbase + K1_KQT, R128, ks), ID_128, 1);
-#pragma unroll
       for (int ks = 8; ks < 16; ++ks)
-        umma_tf32_ts(tmem + K1_DS, tmem + K1_DR + 8 * (ks - 8), kdesc(sbase + K1_KQT, R128, ks), ID_128, 1);
+        umma_tf32_ts(tmem + K1_TDS, tmem + K1_TDR + 8 * (ks - 8), kdesc(sbase + K1_KQT, R128, ks), ID_128, 1);
       umma_commit(&ms.bar_mma);
     }
+    // the stores (rows past the sequence are clipped); the next chunk copies T^T, P^T and
+    // dO, v, w over their staging once they have read it
+    if (tid == 0) {
+      tma_store_5d(&mp.dv, sm + K1_ODV, 0, C * c, 0, h, bb);
+      tma_store_5d(&mp.dw, sm + K1_ODW, 0, C * c, 0, h, bb);
+      tma_store_3d(&mp.nr, sm + K1_ONR, 0, (bh * nch + c) * C, 0);
+      bulk_commit();
+    }
     TC_STAMP(st0, c, 9);
-    ok = wait_mma();
-    // this chunk's T^T / P^T buffer is free: chunk c - 2's
+    if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
+    // the Kn and [Qh; Kb]^T tiles are read: the next chunk's raw inputs over them
+    if (warp == 0 && c >= 1) {
+      issue_x(c - 1);
+      ++n_x;
+    }
     TC_STAMP(st0, c, 10);
-    if (tid == 0 && ok && c >= 2) issue_tp(c - 2);
-    if (!sync_ok(ok)) { dead = true; break; }
+    tc_fence_after();
   }
   // the gradient of the entering state
   if (!dead && p.dS0) {
     float v[32];
-    tmem_ld32(tl + K1_DS + 32 * cg, v);
+    tmem_ld32(tl + K1_TDS + 32 * cg, v);
     tmem_ld_wait();
 #pragma unroll
     for (int x = 0; x < 32; ++x) p.dS0[((size_t)bh * D + 32 * cg + x) * D + ln] = v[x];
   }
+  if (tid == 0) bulk_wait_all();  // the stores complete before the block exits
   // after a give-up: every MMA and copy issued lands before the block releases its memory
   if (tid == 0 && ms.abort) {
     volatile int never = 0;
     umma_commit(&ms.bar_drain);
     mbar_wait_bounded(&ms.bar_drain, 0, &never, nullptr, WAIT_LIMIT);
-    for (int bf = 0; bf < 2; ++bf)
-      if (n_tp[bf] > 0) mbar_wait_bounded(&ms.bar_tp[bf], (uint32_t)((n_tp[bf] - 1) & 1), &never, nullptr, WAIT_LIMIT);
+    if (n_x > 0) mbar_wait_bounded(&ms.bar_x, (uint32_t)((n_x - 1) & 1), &never, nullptr, WAIT_LIMIT);
+    if (n_y > 0) mbar_wait_bounded(&ms.bar_y, (uint32_t)((n_y - 1) & 1), &never, nullptr, WAIT_LIMIT);
+    if (n_tp > 0) mbar_wait_bounded(&ms.bar_tp, (uint32_t)((n_tp - 1) & 1), &never, nullptr, WAIT_LIMIT);
   }
   tc_fence_before();
   __syncthreads();
@@ -405,10 +442,8 @@ __global__ void __launch_bounds__(NTH, 1)
 
 // ============================== (3) the gradients, per chunk ==============================
 struct GradParams {
-  const __nv_bfloat16 *q, *k, *b;
   const float* S;    // [B H][chunk][d_k][d_v]: entering states
   const float* dsn;  // [B H][chunk][d_k][d_v]
-  float *dq, *dk, *db, *dla;  // [B][T][H][d_k]
   int T, H, nch, units;
   unsigned* err;
   unsigned long long* stamps;  // instrumented build only
@@ -426,6 +461,9 @@ constexpr uint32_t K2_TILES = K2_RB + 2 * R64;
 constexpr uint32_t K2_RLA = K2_PA;              // raw log alpha staging (fp32 [t][i], 4 panels of 32)
 constexpr uint32_t K2_RK = K2_PAT, K2_RQ = K2_PAT + 2 * R64;  // raw k, q staging (bf16)
 constexpr uint32_t K2_TX = 12 * R64 + 4 * R64 + 3 * 2 * R64;  // bytes of one unit's TMA loads
+// output staging of dq, dk, db, dlog alpha (fp32 [t][i], 4 panels of 32 channels each), over
+// the tiles the finished products have read
+constexpr uint32_t K2_ODQ = K2_DR, K2_ODK = K2_DR + 4 * R64, K2_ODB = K2_PA, K2_ODLA = K2_PAT;
 struct GradMisc {
   uint64_t bar_ld, bar_mma, bar_drain;
   uint32_t tmem_base;
@@ -451,12 +489,14 @@ __global__ void __launch_bounds__(NTH, 1)
     bwd_grad_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmNR,
                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmLA, const GradParams p) {
+                    const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmDQ,
+                    const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDB,
+                    const __grid_constant__ CUtensorMap tmDLA, const GradParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   GradMisc& ms = *reinterpret_cast<GradMisc*>(sm + K2_TILES);
   const uint32_t sbase = smem_u32(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, ln = tid & 127, cg = tid >> 7;
+  const int tid = threadIdx.x, warp = tid >> 5, ln = tid & 127, cg = tid >> 7, lane = tid & 31;
   const int stride = gridDim.x;
 
   // the copies of unit u, one per lane of warp 0 (lane 0 posts the byte count first): dO
@@ -495,6 +535,10 @@ __global__ void __launch_bounds__(NTH, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmLA);
+    tma_prefetch_desc(&tmDQ);
+    tma_prefetch_desc(&tmDK);
+    tma_prefetch_desc(&tmDB);
+    tma_prefetch_desc(&tmDLA);
   }
   __syncthreads();  // the barrier initialised before the copies use it
   if (warp == 0 && (int)blockIdx.x < p.units) issue(blockIdx.x);
@@ -532,7 +576,6 @@ __global__ void __launch_bounds__(NTH, 1)
     const int n = min(C, p.T - C * c);
     const int srow = it == 1 ? (int)blockIdx.x : 64;  // stamps: the second unit of the first CTAs
     static_cast<void>(srow);
-    auto tok = [&](int t) -> size_t { return (((size_t)bb * p.T + C * c + t) * p.H + h) * D; };
     TC_STAMP(true, srow, 16);
     if (u + stride < p.units) prefetch_states(u + stride);
     // S and dSn rows of this unit (L2), in flight during the wait for the copies
@@ -677,46 +720,50 @@ __global__ void __launch_bounds__(NTH, 1)
         umma_tf32_ts(tmem + K2_PX, tmem + K2_SX + 8 * ks, kdesc(sbase + K2_U, R64, ks), ID_64, ks > 0);
       umma_commit(&ms.bar_mma);
     }
-    // the raw inputs of this thread's tokens again (L2), in flight during the products
-    float kq[16], qq[16], bq[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int t = 16 * cg + r;
-      const bool val = t < n;
-      const size_t x = tok(min(t, n - 1)) + ln;
-      kq[r] = val ? bf(p.k, x) : 0.f;
-      qq[r] = val ? bf(p.q, x) : 0.f;
-      bq[r] = val ? bf(p.b, x) : 0.f;
-    }
     if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
     tc_fence_after();
     TC_STAMP(true, srow, 21);
-    // every tile is free: the next unit's copies
-    if (warp == 0 && u + stride < p.units) {
-      issue(u + stride);
-      ++n_ld;
-    }
-    float dqh[16], dkb[16], xv[16], yv[16];
-    tmem_ld16(tl + K2_QK + 16 * cg, dqh);
-    tmem_ld16(tl + K2_QK + C + 16 * cg, dkb);
-    tmem_ld16(tl + K2_PX + 16 * cg, xv);
-    tmem_ld16(tl + K2_Y + 16 * cg, yv);
-    tmem_ld_wait();
-    // per token: dg = dKb Kb + dQh Qh - dKn Kn; the in-segment suffix sums of dg
-    float dg[16], dx = 0.f;
+    // ===== the elementwise finish, in two halves of 8 tokens (the later half first, for the
+    // reverse cumsum), from on-chip copies: dQh, dKb, X, Y, Qh, Kb (tensor memory), Kn (its
+    // tile), b (its staging), Gamma (registers).  dg = dKb Kb + dQh Qh - dKn Kn per token; dq, dk,
+    // db and the in-segment suffix sums of dg go to output staging tiles over [dO; -dR] and the
+    // [dP; dA] tiles (read by the finished products), stored by TMA once complete.
+    float dx = 0.f, run = 0.f;
+    {
+      const uint32_t rbo = (uint32_t)(ln >> 6) * R64 + (uint32_t)(ln & 7) * 2;
+      const int chk = (ln & 63) >> 3;
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const float Gt = G[r], Gi = 1.f / Gt;
-      const float kn = kq[r] * Gi;
-      dx = fmaf(kn, xv[r], dx);
-      const float dkn = xv[r] + yv[r];
-      dg[r] = dkb[r] * kq[r] * bq[r] * Gt + dqh[r] * qq[r] * Gt - dkn * kn;
-      yv[r] = dkn;
-    }
+      for (int hf = 1; hf >= 0; --hf) {
+        float a8[8], b8[8], x8[8], y8[8], qh8[8], kb8[8];
+        tmem_ld8(tl + K2_QK + 16 * cg + 8 * hf, a8);
+        tmem_ld8(tl + K2_QK + C + 16 * cg + 8 * hf, b8);
+        tmem_ld8(tl + K2_PX + 16 * cg + 8 * hf, x8);
+        tmem_ld8(tl + K2_Y + 16 * cg + 8 * hf, y8);
+        tmem_ld8(tl + K2_KQ + 16 * cg + 8 * hf, qh8);
+        tmem_ld8(tl + K2_KQ + C + 16 * cg + 8 * hf, kb8);
+        const float4 kn0 = *reinterpret_cast<const float4*>(sm + K2_KNT + f32_off(ln, 16 * cg + 8 * hf, R128));
+        const float4 kn1 = *reinterpret_cast<const float4*>(sm + K2_KNT + f32_off(ln, 16 * cg + 8 * hf + 4, R128));
+        const float kn8[8] = {kn0.x, kn0.y, kn0.z, kn0.w, kn1.x, kn1.y, kn1.z, kn1.w};
+        tmem_ld_wait();
 #pragma unroll
-    for (int r = 14; r >= 0; --r) dg[r] += dg[r + 1];
+        for (int r = 7; r >= 0; --r) {
+          const int e = 8 * hf + r, t = 16 * cg + e;
+          const float Gt = G[e], Gi = 1.f / Gt, kn = kn8[r];
+          const float bt = __uint_as_float(
+              (uint32_t)(*reinterpret_cast<const unsigned short*>(sm + K2_RB + rbo + sw128_off(t, chk))) << 16);
+          const float dkn = x8[r] + y8[r];
+          dx = fmaf(kn, x8[r], dx);
+          run += b8[r] * kb8[r] + a8[r] * qh8[r] - dkn * kn;
+          const uint32_t o = f32_off(t, ln, R64);
+          *reinterpret_cast<float*>(sm + K2_ODQ + o) = a8[r] * Gt;
+          *reinterpret_cast<float*>(sm + K2_ODK + o) = b8[r] * bt * Gt + dkn * Gi;
+          *reinterpret_cast<float*>(sm + K2_ODB + o) = b8[r] * kn * Gt * Gt;
+          *reinterpret_cast<float*>(sm + K2_ODLA + o) = run;  // suffix sum within the segment
+        }
+      }
+    }
     ms.dotx[cg][ln] = dx;
-    ms.tot[cg][ln] = dg[0];
+    ms.tot[cg][ln] = run;
     __syncthreads();
     {
       const float gc = ms.gC[ln];
@@ -728,19 +775,27 @@ __global__ void __launch_bounds__(NTH, 1)
         if (s4i > cg) later += ms.tot[s4i][ln];
       }
       // dGamma_C = sum_j dSn (S + Kn^T U) = sum_j dSn S + (1 / Gamma_C) sum_s Kn (dSt U^T)
-      const float dgc = d1 + dxs / gc;
-      const float carry = dgc * gc + later;
+      const float carry = (d1 + dxs / gc) * gc + later;
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const int t = 16 * cg + r;
-        if (t < n) {
-          const size_t x = tok(t) + ln;
-          const float Gt = G[r];
-          p.dq[x] = dqh[r] * Gt;
-          p.dk[x] = dkb[r] * bq[r] * Gt + yv[r] / Gt;
-          p.db[x] = dkb[r] * kq[r] * Gt;
-          p.dla[x] = dg[r] + carry;
-        }
+      for (int r = 0; r < 16; ++r) *reinterpret_cast<float*>(sm + K2_ODLA + f32_off(16 * cg + r, ln, R64)) += carry;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    // the four outputs (rows past the sequence are clipped), then the next unit's copies once
+    // the stores have read the staging
+    if (warp == 0) {
+      if (lane == 0) {
+        tma_store_5d(&tmDQ, sm + K2_ODQ, 0, C * c, 0, h, bb);
+        tma_store_5d(&tmDK, sm + K2_ODK, 0, C * c, 0, h, bb);
+        tma_store_5d(&tmDB, sm + K2_ODB, 0, C * c, 0, h, bb);
+        tma_store_5d(&tmDLA, sm + K2_ODLA, 0, C * c, 0, h, bb);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+      __syncwarp();
+      if (u + stride < p.units) {
+        issue(u + stride);
+        ++n_ld;
       }
     }
     TC_STAMP(true, srow, 22);
@@ -749,6 +804,7 @@ __global__ void __launch_bounds__(NTH, 1)
     __syncthreads();
     tc_fence_after();
   }
+  if (tid == 0) bulk_wait_all();  // the output stores complete before the block exits
   if (tid == 0 && ms.abort) {
     volatile int never = 0;
     umma_commit(&ms.bar_drain);
@@ -859,28 +915,31 @@ cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs& a, cudaStream_t st) {
   cudaError_t e;
   ChunkArgs f{a.q, a.k, a.v, a.b, a.w, a.log_alpha, a.S0, nullptr, nullptr, a.B, a.T, a.H, D, D, true};
   if ((e = launch_chunk_states_tc(f, w.S, st, w.U, w.tt, w.pt)) != cudaSuccess) return e;
-  CUtensorMap mtt, mpt, mnr, mu, mdo, mq, mk, mb, mla;
+  CUtensorMap mnr, mu, mdo, mq, mk, mb, mla;
   const auto F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32, BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!map_rows(&mtt, w.tt, units * C, C) || !map_rows(&mpt, w.pt, units * C, C) ||
-      !map_rows(&mnr, w.nr, units * C, D) || !map_row_panels(&mu, w.U, units * C, D) ||
+  if (!map_rows(&mnr, w.nr, units * C, D) || !map_row_panels(&mu, w.U, units * C, D) ||
       !map_tokens(&mdo, a.dO, F32, 4, 32, a.B, a.T, a.H) || !map_token_panels(&mq, a.q, BF, 2, a.B, a.T, a.H) ||
       !map_token_panels(&mk, a.k, BF, 2, a.B, a.T, a.H) || !map_token_panels(&mb, a.b, BF, 2, a.B, a.T, a.H) ||
       !map_token_panels(&mla, a.log_alpha, F32, 4, a.B, a.T, a.H))
     return cudaErrorInvalidValue;
+  CUtensorMap mdq, mdk, mdb, mdla;
+  if (!map_token_panels(&mdq, a.dq, F32, 4, a.B, a.T, a.H) || !map_token_panels(&mdk, a.dk, F32, 4, a.B, a.T, a.H) ||
+      !map_token_panels(&mdb, a.db, F32, 4, a.B, a.T, a.H) ||
+      !map_token_panels(&mdla, a.dlog_alpha, F32, 4, a.B, a.T, a.H))
+    return cudaErrorInvalidValue;
+  ChainMaps cm;
+  if (!map_token_panels(&cm.q, a.q, BF, 2, a.B, a.T, a.H) || !map_token_panels(&cm.k, a.k, BF, 2, a.B, a.T, a.H) ||
+      !map_token_panels(&cm.b, a.b, BF, 2, a.B, a.T, a.H) || !map_token_panels(&cm.v, a.v, BF, 2, a.B, a.T, a.H) ||
+      !map_token_panels(&cm.w, a.w, BF, 2, a.B, a.T, a.H) ||
+      !map_token_panels(&cm.la, a.log_alpha, F32, 4, a.B, a.T, a.H) ||
+      !map_token_panels(&cm.dO, a.dO, F32, 4, a.B, a.T, a.H) || !map_row_panels(&cm.tt, w.tt, units * C, C) ||
+      !map_row_panels(&cm.pt, w.pt, units * C, C) || !map_token_panels(&cm.dv, a.dv, F32, 4, a.B, a.T, a.H) ||
+      !map_token_panels(&cm.dw, a.dw, F32, 4, a.B, a.T, a.H) || !map_row_panels(&cm.nr, w.nr, units * C, D))
+    return cudaErrorInvalidValue;
   ChainParams cp;
-  cp.q = static_cast<const __nv_bfloat16*>(a.q);
-  cp.k = static_cast<const __nv_bfloat16*>(a.k);
-  cp.b = static_cast<const __nv_bfloat16*>(a.b);
-  cp.v = static_cast<const __nv_bfloat16*>(a.v);
-  cp.w = static_cast<const __nv_bfloat16*>(a.w);
-  cp.la = a.log_alpha;
-  cp.dO = a.dO;
   cp.dS_T = a.dS_T;
   cp.dS0 = a.dS0;
-  cp.dv = a.dv;
-  cp.dw = a.dw;
   cp.dsn = w.dsn;
-  cp.nr = w.nr;
   cp.T = a.T;
   cp.H = a.H;
   cp.nch = nch;
@@ -890,18 +949,11 @@ cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs& a, cudaStream_t st) {
     static std::atomic<unsigned long long> attr_done{0};
     if ((e = smem_limit_once(bwd_chain_kernel, (int)K1_SMEM, attr_done)) != cudaSuccess) return e;
   }
-  bwd_chain_kernel<<<BH, NTH, K1_SMEM, st>>>(mtt, mpt, cp);
+  bwd_chain_kernel<<<BH, NTH, K1_SMEM, st>>>(cm, cp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   GradParams gp;
-  gp.q = cp.q;
-  gp.k = cp.k;
-  gp.b = cp.b;
   gp.S = w.S;
   gp.dsn = w.dsn;
-  gp.dq = a.dq;
-  gp.dk = a.dk;
-  gp.db = a.db;
-  gp.dla = a.dlog_alpha;
   gp.T = a.T;
   gp.H = a.H;
   gp.nch = nch;
@@ -916,7 +968,7 @@ cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs& a, cudaStream_t st) {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = (int)(units < (size_t)sms ? units : (size_t)sms);
-  bwd_grad_kernel<<<grid, NTH, K2_SMEM, st>>>(mdo, mnr, mu, mq, mk, mb, mla, gp);
+  bwd_grad_kernel<<<grid, NTH, K2_SMEM, st>>>(mdo, mnr, mu, mq, mk, mb, mla, mdq, mdk, mdb, mdla, gp);
   return cudaGetLastError();
 }
 

@@ -86,9 +86,9 @@ def main():
 
 # stamp slots of the chunk kernel (its STAMP points), by role
 STAMP_SLOTS = 32
-BWD_SLOT_NAMES = {0: "chunk start", 1: "dO^T stored", 2: "inputs loaded", 3: "operand tiles written",
+BWD_SLOT_NAMES = {0: "chunk start", 1: "copies landed", 2: "inputs read", 3: "operand tiles written",
                   4: "dSn out, dSt formed", 5: "dU issued", 6: "dU done", 7: "dU rounded, dR issued",
-                  8: "dR done", 9: "-dR, dv, dw out, dS issued", 10: "dS done"}
+                  8: "dR done", 9: "-dR staged, dS issued, stores issued", 10: "dS done"}
 GRAD_SLOT_NAMES = {16: "unit start", 17: "copies landed, S in", 18: "operands built", 19: "first products done",
                    20: "dP, dA, dSt written", 21: "second products done", 22: "gradients written"}
 SLOT_NAMES = {0: "AP issued", 1: "SP issued", 2: "U diag issued", 3: "U T21 issued", 4: "OP issued",
