@@ -87,3 +87,49 @@ def test_bwd_full_prefill_b8_h16_t4096_sampled_units():
             got = gg[n][bb:bb + 1, h:h + 1] if n == "dS0" else gg[n][bb:bb + 1, :, h:h + 1]
             err = rel_err(got.cpu().numpy(), ref[n])
             assert err <= TOL["bf16"], (bb, h, n, err)
+
+
+@pytest.mark.parametrize("T", [1, 37, 64, 129])
+def test_bwd_bf16_short_and_exact_chunks(T):
+    # a single partial chunk, exactly one chunk, one chunk and a token
+    wl = dataclasses.replace(BASE, state_std=0.05)
+    d = gi.prefill_inputs(wl, B=2, T=T, H=2)
+    do, dS = _cot(2, T, 2, 128, 128, 20 + T)
+    _check(d, do, dS, "bf16")
+
+
+def test_bwd_bf16_many_units_ragged_sampled():
+    # 2016 (batch, head, chunk) units, more than one per SM, the last chunk of every sequence
+    # partial; two (batch, head) units against the oracle
+    wl = dataclasses.replace(BASE, state_std=0.02)
+    B, T, H = 2, 4000, 16
+    d = gi.prefill_inputs(wl, B=B, T=T, H=H)
+    do, dS = _cot(B, T, H, 128, 128, 21)
+    x = {k_: (None if v_ is None else v_.cuda()) for k_, v_ in d.items()}
+    gg = g.gdn2_chunk_bwd(*(x[n] for n in NAMES), x["S0"], do.cuda(), dS.cuda())
+    torch.cuda.synchronize()
+    assert g.gdn2_device_status() == 0
+    for bb, h in [(0, 0), (1, 15)]:
+        sl = {n: gi.as_f64(d[n][bb:bb + 1, :, h:h + 1]) for n in NAMES}
+        ref = ob.backward(**sl, S0=gi.as_f64(d["S0"][bb:bb + 1, h:h + 1]),
+                          do=do[bb:bb + 1, :, h:h + 1].double().numpy(),
+                          dS_T=dS[bb:bb + 1, h:h + 1].double().numpy())
+        for n in GRADS:
+            got = gg[n][bb:bb + 1, h:h + 1] if n == "dS0" else gg[n][bb:bb + 1, :, h:h + 1]
+            err = rel_err(got.cpu().numpy(), ref[n])
+            assert err <= TOL["bf16"], (bb, h, n, err)
+
+
+def test_bwd_bf16_without_dS0():
+    # the entering-state gradient not requested (NULL): the other gradients unchanged
+    wl = dataclasses.replace(BASE, state_std=0.05)
+    d = gi.prefill_inputs(wl, B=1, T=200, H=2)
+    do, dS = _cot(1, 200, 2, 128, 128, 22)
+    x = {k_: (None if v_ is None else v_.cuda()) for k_, v_ in d.items()}
+    args = [x[n] for n in NAMES]
+    full = g.gdn2_chunk_bwd(*args, x["S0"], do.cuda(), dS.cuda())
+    part = g.gdn2_chunk_bwd(*args, x["S0"], do.cuda(), dS.cuda(), want_dS0=False)
+    torch.cuda.synchronize()
+    assert part["dS0"] is None
+    for n in GRADS[:-1]:
+        assert torch.equal(full[n], part[n]), n
