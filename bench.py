@@ -379,7 +379,7 @@ def time_raw(args, dev):
 
 def time_tiny_f32(args, dev):
     """The tiny fp32 workload (B1 H1 T256, d_k = d_v = 64, fp32 inputs: the 1e-4 parity bar)
-    through gdn2_chunk_fwd, which runs it on the fp32 kernel."""
+    through gdn2_chunk_fwd, which runs it on the split-product tensor-core kernel."""
     import torch
     import gated_delta_rule_95_b200 as g
     wl = gi.WORKLOADS["tiny_f32"]
@@ -670,8 +670,8 @@ def main():
                             for C, r in cs["sizes"].items()}},
         "tiny_f32": {"metric": "GDN-2 prefill tokens/s per layer, fp32 inputs", "value": tf["tokens"] / (tf["ms"] * 1e-3),
                      "unit": "tokens/s", "ms_per_step": tf["ms"],
-                     "workload": "tiny_f32: B=1 H=1 T=256 d_k=d_v=64, fp32 inputs (the fp32 CUDA-core kernel, "
-                                 "two CTAs of 32 value columns: latency-bound)"},
+                     "workload": "tiny_f32: B=1 H=1 T=256 d_k=d_v=64, fp32 inputs (chunk_fwd_f32_tc_kernel: split "
+                                 "tf32 products on tcgen05, one CTA: latency-bound)"},
         "conv": {"metric": "short convolution GB/s", "value": cv_gbs, "unit": "GB/s", "ms_per_step": cv["ms"],
                  "steps": args.steps,
                  "workload": f"q, k, v projections of prefill_b8_h16_t4096 side by side: [8, 4096, {cv['C']}] bf16, "

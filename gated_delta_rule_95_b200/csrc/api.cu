@@ -98,7 +98,8 @@ extern "C" gdn2_status gdn2_chunk_fwd(const void* q, const void* k, const void* 
   if (T == 0)
     e = launch_state_copy(a, st);
   else
-    e = a.bf16 ? launch_chunk_fwd_tc(a, st) : launch_chunk_fwd_f32(a, st);
+    e = a.bf16 ? launch_chunk_fwd_tc(a, st)
+               : (chunk_fwd_f32_tc_supported(a) ? launch_chunk_fwd_f32_tc(a, st) : launch_chunk_fwd_f32(a, st));
   return e == cudaSuccess ? GDN2_OK : cuda_fail(e);
 }
 

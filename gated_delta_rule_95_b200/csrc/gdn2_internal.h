@@ -106,7 +106,10 @@ cudaError_t launch_chunk_fwd_tc(const ChunkArgs& a, cudaStream_t st);
 // every chunk (the tensor-core backward's inputs).
 cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st, float* ck_u = nullptr,
                                    float* ck_tt = nullptr, float* ck_pt = nullptr);
-// fp32 inputs: fp32 CUDA-core kernel of the same chunkwise algorithm.
+// fp32 inputs, d_k = d_v = 64: tcgen05 kernel with split (3 x tf32) products.
+bool chunk_fwd_f32_tc_supported(const ChunkArgs& a);
+cudaError_t launch_chunk_fwd_f32_tc(const ChunkArgs& a, cudaStream_t st);
+// fp32 inputs of the other head sizes: fp32 CUDA-core kernel of the same chunkwise algorithm.
 cudaError_t launch_chunk_fwd_f32(const ChunkArgs& a, cudaStream_t st);
 // bf16, chunk size 32, 64 or 128: the chunk-size study kernel (warp-level tf32 MMAs);
 // shared memory per CTA, 0 for an unsupported (chunk, d_k).

@@ -75,7 +75,10 @@ typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
  * tensor-core products, the state handed across chunks) in the WY form with the
  * cumulative channel-wise decay folded into the factors of each rank-one erase
  * (snilld.dk, "Hvad betyder det for traening og inferens").  The result equals
- * the token-by-token recurrence above up to rounding.
+ * the token-by-token recurrence above up to rounding.  bf16 inputs: tcgen05 tf32
+ * products with fp32 accumulation; fp32 inputs with d_k = d_v = 64: tcgen05 split
+ * products (hi*hi + hi*lo + lo*hi of tf32 parts, fp32-accurate); fp32 inputs with a head
+ * size of 128: fp32 products on the CUDA cores.
  *
  *   q, k, b      : [B, T, H, d_k]  dt
  *   v, w         : [B, T, H, d_v]  dt
