@@ -334,9 +334,9 @@ def time_bwd(args, dev):
 
 
 def time_csize(args, dev):
-    """The prefill workload at chunk sizes 32, 64 and 128 through gdn2_chunk_fwd_csize
-    (one kernel template for the three sizes): latency, and the on-chip footprint that
-    sets how many CTAs share an SM (the call needs no device memory besides its tensors)."""
+    """The prefill workload at chunk sizes 32, 64 and 128 through gdn2_chunk_fwd_csize (32 and
+    64 on the tcgen05 kernels, 128 on the warp-MMA kernel): latency, and the on-chip footprint
+    that sets how many CTAs share an SM (the call needs no device memory besides its tensors)."""
     import torch
     import gated_delta_rule_95_b200 as g
     d = gi.prefill_inputs(PREFILL)
@@ -353,10 +353,12 @@ def time_csize(args, dev):
 
         ms = _time_loop(step, args.steps, args.warmup)
         smem = g.lib().gdn2_chunk_fwd_csize_smem_bytes(C, dk)
-        out[C] = dict(ms=ms, smem=smem, ctas_per_sm=sm_total // (smem + 1024))
+        out[C] = dict(ms=ms, smem=smem, ctas_per_sm=sm_total // (smem + 1024),
+                      kernel={32: "chunk_fwd_tc32_kernel (tcgen05)", 64: "chunk_fwd_tc_kernel (tcgen05)",
+                              128: "chunk_fwd_csize_kernel (warp-level MMA)"}[C],
+                      tmem_cols={32: 512, 64: 512, 128: 0}[C], ctas=B * H if C < 128 else B * H * (dv // 32))
     arg_bytes = sum(t.numel() * t.element_size() for t in args_t + [o, S_T])
-    return dict(sizes=out, tokens=B * T, token_heads=B * T * H, arg_bytes=arg_bytes, ctas=B * H * (dv // 32),
-                ok=g.gdn2_device_status() == 0)
+    return dict(sizes=out, tokens=B * T, token_heads=B * T * H, arg_bytes=arg_bytes, ok=g.gdn2_device_status() == 0)
 
 
 def time_raw(args, dev):
@@ -662,9 +664,10 @@ def main():
                   "workload": "prefill_b8_h16_t4096 through gdn2_chunk_fwd_csize",
                   "device_bytes": {"arguments": cs["arg_bytes"], "scratch": 0},
                   "sizes": {str(C): {"value": cs["tokens"] / (r["ms"] * 1e-3), "unit": "tokens/s",
-                                     "ms_per_step": r["ms"], "smem_bytes_per_cta": r["smem"],
+                                     "ms_per_step": r["ms"], "kernel": r["kernel"], "ctas": r["ctas"],
+                                     "smem_bytes_per_cta": r["smem"], "tmem_columns_per_cta": r["tmem_cols"],
                                      "ctas_per_sm_by_smem": r["ctas_per_sm"],
-                                     "roofline": hbm("chunk_fwd_csize_kernel",
+                                     "roofline": hbm(r["kernel"],
                                                      cs["token_heads"] * PREFILL_BYTES_PER_TOKEN_HEAD
                                                      / (r["ms"] * 1e-3) / 1e9)}
                             for C, r in cs["sizes"].items()}},

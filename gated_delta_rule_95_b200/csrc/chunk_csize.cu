@@ -499,11 +499,14 @@ cudaError_t launch_dk(const ChunkArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+// The chunk-size study's entry: C = 32 and C = 64 on the tcgen05 kernels (chunk_tc32.cu and
+// the production chunk_tc.cu), C = 128 on this warp-MMA kernel (its tiles exceed one SM's
+// shared and tensor memory on tcgen05).
 size_t chunk_fwd_csize_smem_bytes(int chunk, int dk) {
   if (dk != 64 && dk != 128) return 0;
   switch (chunk) {
-    case 32: return dk == 128 ? CsLayout<32, 128>::BYTES : CsLayout<32, 64>::BYTES;
-    case 64: return dk == 128 ? CsLayout<64, 128>::BYTES : CsLayout<64, 64>::BYTES;
+    case 32: return chunk_fwd_tc32_smem_bytes();
+    case 64: return chunk_fwd_tc_smem_bytes();
     case 128: return dk == 128 ? CsLayout<128, 128>::BYTES : CsLayout<128, 64>::BYTES;
     default: return 0;
   }
@@ -512,8 +515,8 @@ size_t chunk_fwd_csize_smem_bytes(int chunk, int dk) {
 cudaError_t launch_chunk_fwd_csize(const ChunkArgs& a, int chunk, cudaStream_t st) {
   if (a.B * a.H == 0) return cudaSuccess;
   switch (chunk) {
-    case 32: return launch_dk<32>(a, st);
-    case 64: return launch_dk<64>(a, st);
+    case 32: return launch_chunk_fwd_tc32(a, st);
+    case 64: return launch_chunk_fwd_tc(a, st);
     case 128: return launch_dk<128>(a, st);
     default: return cudaErrorInvalidValue;
   }

@@ -1248,6 +1248,8 @@ cudaError_t launch_split(const ChunkArgs& a, TcParams p, cudaStream_t st, const 
   return pass(BH * (P - 1));
 }
 
+size_t chunk_fwd_tc_smem_bytes() { return SMEM_BYTES; }
+
 // The state entering every chunk ([B H][chunk][d_k][d_v] fp32 at `states`), for the backward
 // pass: the split instantiation's checkpoint phase over whole sequences (bf16, d_k = d_v).
 cudaError_t launch_chunk_states_tc(const ChunkArgs& a, float* states, cudaStream_t st, float* ck_u, float* ck_tt,

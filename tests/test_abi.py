@@ -202,12 +202,16 @@ def test_chunk_fwd_csize_validation(kw, status):
 
 
 def test_csize_shared_memory_footprint():
-    # Kn and Kb/Qh [C][d_k], A/P [C][C], U [C][32], state [d_k][32], Gamma_C [d_k], cumsum
-    # partials [threads of the CTA: 256, or 512 at C = 128], all fp32
+    # C = 128 (the warp-MMA kernel): Kn and Kb/Qh [C][d_k], A/P [C][C], U [C][32], state
+    # [d_k][32], Gamma_C [d_k], cumsum partials [512 threads], all fp32
     L = g.lib()
-    for C in (32, 64, 128):
-        nth = 512 if C == 128 else 256
-        for dk in (64, 128):
-            assert L.gdn2_chunk_fwd_csize_smem_bytes(C, dk) == 4 * (2 * C * dk + C * C + 32 * C + 33 * dk + nth)
+    for dk in (64, 128):
+        assert L.gdn2_chunk_fwd_csize_smem_bytes(128, dk) == 4 * (2 * 128 * dk + 128 * 128 + 32 * 128 + 33 * dk + 512)
     assert L.gdn2_chunk_fwd_csize_smem_bytes(128, 128) <= 227 * 1024
+    # C = 32 and 64 (the tcgen05 kernels): one layout for both head sizes, within one block's
+    # 227 KB, the 32-token chunk's tiles the smaller
+    for C in (32, 64):
+        n = L.gdn2_chunk_fwd_csize_smem_bytes(C, 128)
+        assert 0 < n <= 227 * 1024 and L.gdn2_chunk_fwd_csize_smem_bytes(C, 64) == n
+    assert L.gdn2_chunk_fwd_csize_smem_bytes(32, 128) < L.gdn2_chunk_fwd_csize_smem_bytes(64, 128)
     assert L.gdn2_chunk_fwd_csize_smem_bytes(16, 128) == 0 and L.gdn2_chunk_fwd_csize_smem_bytes(64, 96) == 0
