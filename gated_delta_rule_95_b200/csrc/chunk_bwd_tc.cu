@@ -463,9 +463,11 @@ constexpr uint32_t K2_RK = K2_PAT, K2_RQ = K2_PAT + 2 * R64;  // raw k, q stagin
 constexpr uint32_t K2_TX = 12 * R64 + 4 * R64 + 3 * 2 * R64;  // bytes of one unit's TMA loads
 // output staging of dq, dk, db, dlog alpha (fp32 [t][i], 4 panels of 32 channels each), over
 // the tiles the finished products have read
-constexpr uint32_t K2_ODQ = K2_DR, K2_ODK = K2_DR + 4 * R64, K2_ODB = K2_PA, K2_ODLA = K2_PAT;
+constexpr uint32_t K2_ODQ = K2_U, K2_ODK = K2_KNT, K2_ODB = K2_PA, K2_ODLA = K2_PAT;
+constexpr uint32_t K2_TX_DR = 8 * R64;                  // bytes of one unit's dO and -dR copies
+constexpr uint32_t K2_TX_REST = K2_TX - K2_TX_DR;       // U and the raw inputs
 struct GradMisc {
-  uint64_t bar_ld, bar_mma, bar_drain;
+  uint64_t bar_ld, bar_dr, bar_mma, bar_drain;
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[D];
@@ -499,20 +501,27 @@ __global__ void __launch_bounds__(NTH, 1)
   const int tid = threadIdx.x, warp = tid >> 5, ln = tid & 127, cg = tid >> 7, lane = tid & 31;
   const int stride = gridDim.x;
 
-  // the copies of unit u, one per lane of warp 0 (lane 0 posts the byte count first): dO
-  // (rows past the sequence read zero) and -dR by panel into the stacked tile, U, and the raw
-  // q, k, b, log alpha as whole panel-major tiles
-  auto issue = [&](int u) {
+  // The copies of unit u, one per lane of warp 0 (lane 0 posts the byte count first), on two
+  // barriers: dO (rows past the sequence read zero) and -dR by panel into the stacked tile,
+  // issued as soon as the previous unit's first products have read that tile; U and the raw
+  // q, k, b, log alpha as whole panel-major tiles, once the previous unit's outputs have
+  // left their staging.
+  auto issue_dr = [&](int u) {
     const int c = u % p.nch, bh = u / p.nch, h = bh % p.H, bb = bh / p.H, l = tid & 31;
-    if (l == 0) mbar_arrive_expect_tx(&ms.bar_ld, K2_TX);
+    if (l == 0) mbar_arrive_expect_tx(&ms.bar_dr, K2_TX_DR);
     __syncwarp();
-    if (l < 4) tma_load_4d(sm + K2_DR + l * R128, &tmDO, &ms.bar_ld, 32 * l, h, C * c, bb);
-    else if (l < 8) tma_load_2d(sm + K2_DR + (l - 4) * R128 + R64, &tmNR, &ms.bar_ld, 32 * (l - 4), u * C);
-    else if (l == 8) tma_load_3d(sm + K2_U, &tmU, &ms.bar_ld, 0, u * C, 0);
-    else if (l == 9) tma_load_5d(sm + K2_RLA, &tmLA, &ms.bar_ld, 0, C * c, 0, h, bb);
-    else if (l == 10) tma_load_5d(sm + K2_RK, &tmK, &ms.bar_ld, 0, C * c, 0, h, bb);
-    else if (l == 11) tma_load_5d(sm + K2_RQ, &tmQ, &ms.bar_ld, 0, C * c, 0, h, bb);
-    else if (l == 12) tma_load_5d(sm + K2_RB, &tmB, &ms.bar_ld, 0, C * c, 0, h, bb);
+    if (l < 4) tma_load_4d(sm + K2_DR + l * R128, &tmDO, &ms.bar_dr, 32 * l, h, C * c, bb);
+    else if (l < 8) tma_load_2d(sm + K2_DR + (l - 4) * R128 + R64, &tmNR, &ms.bar_dr, 32 * (l - 4), u * C);
+  };
+  auto issue_rest = [&](int u) {
+    const int c = u % p.nch, bh = u / p.nch, h = bh % p.H, bb = bh / p.H, l = tid & 31;
+    if (l == 0) mbar_arrive_expect_tx(&ms.bar_ld, K2_TX_REST);
+    __syncwarp();
+    if (l == 0) tma_load_3d(sm + K2_U, &tmU, &ms.bar_ld, 0, u * C, 0);
+    else if (l == 1) tma_load_5d(sm + K2_RLA, &tmLA, &ms.bar_ld, 0, C * c, 0, h, bb);
+    else if (l == 2) tma_load_5d(sm + K2_RK, &tmK, &ms.bar_ld, 0, C * c, 0, h, bb);
+    else if (l == 3) tma_load_5d(sm + K2_RQ, &tmQ, &ms.bar_ld, 0, C * c, 0, h, bb);
+    else if (l == 4) tma_load_5d(sm + K2_RB, &tmB, &ms.bar_ld, 0, C * c, 0, h, bb);
   };
   // the entering state and state gradient of unit u into L2 (4 + 4 bulk prefetches of 16 KB)
   auto prefetch_states = [&](int u) {
@@ -524,6 +533,7 @@ __global__ void __launch_bounds__(NTH, 1)
 
   if (tid == 0) {
     mbar_init(&ms.bar_ld, 1);
+    mbar_init(&ms.bar_dr, 1);
     mbar_init(&ms.bar_mma, 1);
     mbar_init(&ms.bar_drain, 1);
     fence_mbar_init();
@@ -541,7 +551,10 @@ __global__ void __launch_bounds__(NTH, 1)
     tma_prefetch_desc(&tmDLA);
   }
   __syncthreads();  // the barrier initialised before the copies use it
-  if (warp == 0 && (int)blockIdx.x < p.units) issue(blockIdx.x);
+  if (warp == 0 && (int)blockIdx.x < p.units) {
+    issue_dr(blockIdx.x);
+    issue_rest(blockIdx.x);
+  }
   if (warp == 0) {
     tmem_alloc(&ms.tmem_base, 512);
     tmem_relinquish();
@@ -551,8 +564,9 @@ __global__ void __launch_bounds__(NTH, 1)
   tc_fence_after();
   const uint32_t tmem = ms.tmem_base;
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-  uint32_t ph_mma = 0, ph_ld = 0;
-  int n_ld = (int)blockIdx.x < p.units ? 1 : 0, n_ld_done = 0;  // copies issued / waited (thread 0)
+  uint32_t ph_mma = 0, ph_ld = 0, ph_dr = 0;
+  // copies issued / waited on each barrier (thread 0), for the drain after a give-up
+  int n_ld = (int)blockIdx.x < p.units ? 1 : 0, n_ld_done = 0, n_dr = n_ld, n_dr_done = 0;
   auto sync_ok = [&](bool ok) -> bool {
     tmem_st_wait();
     fence_proxy_async_smem();
@@ -654,7 +668,13 @@ __global__ void __launch_bounds__(NTH, 1)
     // (every raw read is done before the [dP; dA] tiles overwrite the staging: the barriers below)
     if (!sync_ok(true)) { dead = true; break; }
     // ===== [dP; dA] = [dO; -dR] U^T and [dQh^T | dKb^T] = S [dO; -dR]^T ======================
+    bool ok_dr = true;
     if (tid == 0) {
+      ok_dr = mbar_wait_spin(&ms.bar_dr, ph_dr, &ms.abort, p.err, WAIT_LIMIT);
+      ph_dr ^= 1;
+      if (ok_dr) ++n_dr_done;
+    }
+    if (tid == 0 && ok_dr) {
 #pragma unroll
       for (int ks = 0; ks < 16; ++ks)
         umma_tf32_ss(tmem + K2_PX, kdesc(sbase + K2_DR, R128, ks), kdesc(sbase + K2_U, R64, ks), ID_64, ks > 0);
@@ -672,6 +692,12 @@ __global__ void __launch_bounds__(NTH, 1)
     if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
     tc_fence_after();
     TC_STAMP(true, srow, 19);
+    // the stacked [dO; -dR] tile has been read (the second products do not use it): the next
+    // unit's dO and -dR
+    if (warp == 0 && u + stride < p.units) {
+      issue_dr(u + stride);
+      ++n_dr;
+    }
     // read-out of [dP; dA], masked (dP: s <= t, dA: s < t), to both operand tiles
     {
       float v[16];
@@ -725,9 +751,20 @@ __global__ void __launch_bounds__(NTH, 1)
     TC_STAMP(true, srow, 21);
     // ===== the elementwise finish, in two halves of 8 tokens (the later half first, for the
     // reverse cumsum), from on-chip copies: dQh, dKb, X, Y, Qh, Kb (tensor memory), Kn (its
-    // tile), b (its staging), Gamma (registers).  dg = dKb Kb + dQh Qh - dKn Kn per token; dq, dk,
-    // db and the in-segment suffix sums of dg go to output staging tiles over [dO; -dR] and the
-    // [dP; dA] tiles (read by the finished products), stored by TMA once complete.
+    // tile, read first: dk is staged over it), b (its staging), Gamma (registers).
+    // dg = dKb Kb + dQh Qh - dKn Kn per token; dq, dk, db and the in-segment suffix sums of dg
+    // go to output staging tiles over U, Kn^T and the [dP; dA] tiles (read by the finished
+    // products), stored by TMA once complete.
+    float kn16[16];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float4 k4 = *reinterpret_cast<const float4*>(sm + K2_KNT + f32_off(ln, 16 * cg + 4 * m, R128));
+      kn16[4 * m] = k4.x;
+      kn16[4 * m + 1] = k4.y;
+      kn16[4 * m + 2] = k4.z;
+      kn16[4 * m + 3] = k4.w;
+    }
+    __syncthreads();  // every read of the Kn^T tile is done
     float dx = 0.f, run = 0.f;
     {
       const uint32_t rbo = (uint32_t)(ln >> 6) * R64 + (uint32_t)(ln & 7) * 2;
@@ -741,9 +778,7 @@ __global__ void __launch_bounds__(NTH, 1)
         tmem_ld8(tl + K2_Y + 16 * cg + 8 * hf, y8);
         tmem_ld8(tl + K2_KQ + 16 * cg + 8 * hf, qh8);
         tmem_ld8(tl + K2_KQ + C + 16 * cg + 8 * hf, kb8);
-        const float4 kn0 = *reinterpret_cast<const float4*>(sm + K2_KNT + f32_off(ln, 16 * cg + 8 * hf, R128));
-        const float4 kn1 = *reinterpret_cast<const float4*>(sm + K2_KNT + f32_off(ln, 16 * cg + 8 * hf + 4, R128));
-        const float kn8[8] = {kn0.x, kn0.y, kn0.z, kn0.w, kn1.x, kn1.y, kn1.z, kn1.w};
+        const float* kn8 = kn16 + 8 * hf;
         tmem_ld_wait();
 #pragma unroll
         for (int r = 7; r >= 0; --r) {
@@ -794,7 +829,7 @@ __global__ void __launch_bounds__(NTH, 1)
       }
       __syncwarp();
       if (u + stride < p.units) {
-        issue(u + stride);
+        issue_rest(u + stride);
         ++n_ld;
       }
     }
@@ -810,6 +845,7 @@ __global__ void __launch_bounds__(NTH, 1)
     umma_commit(&ms.bar_drain);
     mbar_wait_bounded(&ms.bar_drain, 0, &never, nullptr, WAIT_LIMIT);
     if (n_ld > n_ld_done) mbar_wait_bounded(&ms.bar_ld, (uint32_t)((n_ld - 1) & 1), &never, nullptr, WAIT_LIMIT);
+    if (n_dr > n_dr_done) mbar_wait_bounded(&ms.bar_dr, (uint32_t)((n_dr - 1) & 1), &never, nullptr, WAIT_LIMIT);
   }
   tc_fence_before();
   __syncthreads();
