@@ -591,7 +591,6 @@ __global__ void __launch_bounds__(NTH, 1)
     const int srow = it == 1 ? (int)blockIdx.x : 64;  // stamps: the second unit of the first CTAs
     static_cast<void>(srow);
     TC_STAMP(true, srow, 16);
-    if (u + stride < p.units) prefetch_states(u + stride);
     // S and dSn rows of this unit (L2), in flight during the wait for the copies
     float4 s4[8], d4[8];
     {
@@ -698,6 +697,7 @@ __global__ void __launch_bounds__(NTH, 1)
       issue_dr(u + stride);
       ++n_dr;
     }
+    if (u + stride < p.units) prefetch_states(u + stride);  // (its states into L2, after this unit's loads)
     // read-out of [dP; dA], masked (dP: s <= t, dA: s < t), to both operand tiles
     {
       float v[16];
