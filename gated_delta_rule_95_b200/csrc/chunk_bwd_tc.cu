@@ -105,7 +105,7 @@ constexpr uint32_t K1_DO = K1_Y, K1_RV = K1_Y + 4 * R64, K1_RW = K1_Y + 6 * R64;
 // -dR over T^T and P^T (each read before it is overwritten)
 constexpr uint32_t K1_ODV = K1_DO, K1_ODW = K1_RV, K1_ONR = K1_TP;
 struct ChainMisc {
-  uint64_t bar_x, bar_y, bar_tp, bar_mma, bar_drain;
+  uint64_t bar_xa, bar_xq, bar_xb, bar_y, bar_tp, bar_mma, bar_dsa, bar_drain;
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[D];
@@ -131,13 +131,29 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
 
   // the copies of chunk cc, one per lane of warp 0 (lane 0 posts the byte count first):
   // X = raw log alpha, k, q, b; Y = dO, v, w; TP = T^T, P^T
-  auto issue_x = [&](int cc) {
-    if (lane == 0) mbar_arrive_expect_tx(&ms.bar_x, 4 * R64 + 3 * 2 * R64);
+  // X in three parts, each as soon as its staging is free: log alpha over the Kn tile (read
+  // by the dU product), k and q over the Qh half of [Qh; Kb]^T (read by the first part of the
+  // dS update), b over the Kb half (read by its last part)
+  auto issue_xa = [&](int cc) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&ms.bar_xa, 4 * R64);
+      tma_load_5d(sm + K1_RLA, &mp.la, &ms.bar_xa, 0, C * cc, 0, h, bb);
+    }
     __syncwarp();
-    if (lane == 0) tma_load_5d(sm + K1_RLA, &mp.la, &ms.bar_x, 0, C * cc, 0, h, bb);
-    else if (lane == 1) tma_load_5d(sm + K1_RK, &mp.k, &ms.bar_x, 0, C * cc, 0, h, bb);
-    else if (lane == 2) tma_load_5d(sm + K1_RQ, &mp.q, &ms.bar_x, 0, C * cc, 0, h, bb);
-    else if (lane == 3) tma_load_5d(sm + K1_RB, &mp.b, &ms.bar_x, 0, C * cc, 0, h, bb);
+  };
+  auto issue_xq = [&](int cc) {
+    if (lane == 0) mbar_arrive_expect_tx(&ms.bar_xq, 2 * 2 * R64);
+    __syncwarp();
+    if (lane == 0) tma_load_5d(sm + K1_RK, &mp.k, &ms.bar_xq, 0, C * cc, 0, h, bb);
+    else if (lane == 1) tma_load_5d(sm + K1_RQ, &mp.q, &ms.bar_xq, 0, C * cc, 0, h, bb);
+    __syncwarp();
+  };
+  auto issue_xb = [&](int cc) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&ms.bar_xb, 2 * R64);
+      tma_load_5d(sm + K1_RB, &mp.b, &ms.bar_xb, 0, C * cc, 0, h, bb);
+    }
+    __syncwarp();
   };
   auto issue_y = [&](int cc) {
     if (lane == 0) mbar_arrive_expect_tx(&ms.bar_y, 4 * R64 + 2 * 2 * R64);
@@ -170,7 +186,10 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
   };
 
   if (tid == 0) {
-    mbar_init(&ms.bar_x, 1);
+    mbar_init(&ms.bar_xa, 1);
+    mbar_init(&ms.bar_xq, 1);
+    mbar_init(&ms.bar_xb, 1);
+    mbar_init(&ms.bar_dsa, 1);
     mbar_init(&ms.bar_y, 1);
     mbar_init(&ms.bar_tp, 1);
     mbar_init(&ms.bar_mma, 1);
@@ -188,13 +207,15 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
   const uint32_t tmem = ms.tmem_base;
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   // copies issued (warp 0): their count per barrier, for the drain after a give-up
-  int n_x = 0, n_y = 0, n_tp = 0;
-  uint32_t ph_x = 0, ph_y = 0, ph_tp = 0, ph_mma = 0;
+  int n_xa = 0, n_xq = 0, n_xb = 0, n_y = 0, n_tp = 0;
+  uint32_t ph_xa = 0, ph_xq = 0, ph_xb = 0, ph_y = 0, ph_tp = 0, ph_mma = 0, ph_dsa = 0;
   if (warp == 0 && nch > 0) {
-    issue_x(nch - 1);
+    issue_xa(nch - 1);
+    issue_xq(nch - 1);
+    issue_xb(nch - 1);
     issue_y(nch - 1);
     issue_tp(nch - 1);
-    ++n_x, ++n_y, ++n_tp;
+    ++n_xa, ++n_xq, ++n_xb, ++n_y, ++n_tp;
     if (nch > 1) prefetch(nch - 2);
   }
   // completion of a barrier phase: warp 0 polls (a suspended wait wakes too late for this
@@ -249,7 +270,10 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
       if (c >= 2) prefetch(c - 2);
     }
     // ===== build: thread (i = ln, cg) over the tokens [16 cg, 16 cg + 16) ===================
-    if (!wait_all(&ms.bar_x, ph_x)) { dead = true; break; }
+    if (!wait_all(&ms.bar_xa, ph_xa) || !wait_all(&ms.bar_xq, ph_xq) || !wait_all(&ms.bar_xb, ph_xb)) {
+      dead = true;
+      break;
+    }
     TC_STAMP(st0, c, 1);
     float g[16], kq[16], qq[16], bq[16];
 #pragma unroll
@@ -342,6 +366,11 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
     if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
     tc_fence_after();
     TC_STAMP(st0, c, 6);
+    // the Kn tile is read: the next chunk's log alpha over it
+    if (warp == 0 && c >= 1) {
+      issue_xa(c - 1);
+      ++n_xa;
+    }
     {
       float v[16];
       tmem_ld16(tl + K1_TDU + 16 * cg, v);
@@ -362,6 +391,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         umma_tf32_ts(tmem + K1_TDS, tmem + K1_TDO + 8 * ks, kdesc(sbase + K1_KQT, R128, ks), ID_128, 1);
+      umma_commit(&ms.bar_dsa);
     }
     TC_STAMP(st0, c, 7);
     if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
@@ -391,6 +421,15 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
       }
     }
     if (!sync_ok(true)) { dead = true; break; }
+    // the first part of the update has read the Qh half of [Qh; Kb]^T: the next chunk's k, q
+    if (warp == 0) {
+      const bool ok = mbar_wait_spin(&ms.bar_dsa, ph_dsa, &ms.abort, p.err, WAIT_LIMIT);
+      ph_dsa ^= 1;
+      if (ok && c >= 1) {
+        issue_xq(c - 1);
+        ++n_xq;
+      }
+    }
     // ===== dS^T += -dR^T Kb: the update completes ==============================================
     if (tid == 0) {
 #pragma unroll
@@ -408,10 +447,10 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
     }
     TC_STAMP(st0, c, 9);
     if (!wait_all(&ms.bar_mma, ph_mma)) { dead = true; break; }
-    // the Kn and [Qh; Kb]^T tiles are read: the next chunk's raw inputs over them
+    // the Kb half of [Qh; Kb]^T is read: the next chunk's b over it
     if (warp == 0 && c >= 1) {
-      issue_x(c - 1);
-      ++n_x;
+      issue_xb(c - 1);
+      ++n_xb;
     }
     TC_STAMP(st0, c, 10);
     tc_fence_after();
@@ -430,7 +469,9 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
     volatile int never = 0;
     umma_commit(&ms.bar_drain);
     mbar_wait_bounded(&ms.bar_drain, 0, &never, nullptr, WAIT_LIMIT);
-    if (n_x > 0) mbar_wait_bounded(&ms.bar_x, (uint32_t)((n_x - 1) & 1), &never, nullptr, WAIT_LIMIT);
+    if (n_xa > 0) mbar_wait_bounded(&ms.bar_xa, (uint32_t)((n_xa - 1) & 1), &never, nullptr, WAIT_LIMIT);
+    if (n_xq > 0) mbar_wait_bounded(&ms.bar_xq, (uint32_t)((n_xq - 1) & 1), &never, nullptr, WAIT_LIMIT);
+    if (n_xb > 0) mbar_wait_bounded(&ms.bar_xb, (uint32_t)((n_xb - 1) & 1), &never, nullptr, WAIT_LIMIT);
     if (n_y > 0) mbar_wait_bounded(&ms.bar_y, (uint32_t)((n_y - 1) & 1), &never, nullptr, WAIT_LIMIT);
     if (n_tp > 0) mbar_wait_bounded(&ms.bar_tp, (uint32_t)((n_tp - 1) & 1), &never, nullptr, WAIT_LIMIT);
   }
