@@ -139,3 +139,27 @@ def test_full_long_context_b1_h16_t65536_all_units():
     g_min = float(torch.cumsum(la, dim=2).min())
     print(f"long-context workload: min in-chunk cumulative log decay = {g_min:.2f}")
     assert g_min > -80.0
+
+
+@pytest.mark.parametrize("B,T,H", [(2, 130, 3), (1, 1, 2), (3, 64, 1), (1, 200, 4)])
+def test_f32_d64_tensor_core_kernel(B, T, H):
+    # fp32 inputs with d_k = d_v = 64 run on the split-product (3 x tf32) tensor-core kernel:
+    # entering states, a single token, an exact chunk, ragged lengths, several heads
+    wl = dataclasses.replace(BASE, dk=64, dv=64, dtype="f32", state_std=0.05, seed=400 + T)
+    d = gi.prefill_inputs(wl, B=B, T=T, H=H)
+    o, S = _run(d)
+    o_ref, S_ref = _full_oracle(d)
+    assert rel_err(o.cpu().numpy(), o_ref) <= TOL["f32"]
+    assert rel_err(S.cpu().numpy(), S_ref) <= TOL["f32"]
+    assert g.gdn2_device_status() == 0
+
+
+def test_f32_d64_state_aliasing():
+    wl = dataclasses.replace(BASE, dk=64, dv=64, dtype="f32", state_std=0.05, seed=77)
+    d = gi.prefill_inputs(wl, B=2, T=100, H=2)
+    o1, S1 = _run(d)
+    x = _cuda(d)
+    S_inout = x["S0"].clone()
+    o2, S2 = g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], S_inout, S_T=S_inout)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
