@@ -24,13 +24,16 @@
 // transposed (dS^T, lanes = value channels) as an fp32 accumulator in tensor memory; per chunk
 // three products (dU^T, dR^T and the dS^T update) whose A operands (dO^T, dSt^T, dU^T, -dR^T)
 // live in tensor memory and whose B operands (P^T, Kn, T^T, [Qh; Kb]^T) are shared-memory
-// tiles; it writes dSn and -dR of every chunk and dv, dw.  (3) bwd_grad_kernel, one CTA per
-// (batch, head, chunk), all independent: [dP; dA] = [dO; -dR] U^T, then the key-side
-// gradients transposed (lanes = key channels), [dQh^T | dKb^T] = S [dO; -dR]^T +
-// Kn^T [dP; dA]^T, dKn^T = dSt U^T + [Qh; Kb]^T [dP; dA], and the elementwise finish (a
-// thread per key channel walks the chunk's tokens, so the reverse cumsum of dlog alpha needs
-// no exchange beyond four segment totals).  Operands are rounded to tf32 (nearest) except dO,
-// which the tensor core reads straight from its TMA tile; accumulation is fp32.
+// tiles; it writes dSn and -dR of every chunk and dv, dw.  Its inputs arrive by TMA as
+// panel-major tiles, each as soon as its staging is free, and its outputs leave by TMA stores.
+// (3) bwd_grad_kernel, persistent (one CTA per SM) over the (batch, head, chunk) units, all
+// independent: [dP; dA] = [dO; -dR] U^T, then the key-side gradients transposed (lanes = key
+// channels), [dQh^T | dKb^T] = S [dO; -dR]^T + Kn^T [dP; dA]^T, dKn^T = dSt U^T +
+// [Qh; Kb]^T [dP; dA], and the elementwise finish (a thread per key channel walks the chunk's
+// tokens, so the reverse cumsum of dlog alpha needs no exchange beyond four segment totals);
+// the next unit's copies are issued as their tiles free up, the gradients leave by TMA stores.
+// Operands are rounded to tf32 (nearest) except dO, which the tensor core reads straight from
+// its TMA tile; accumulation is fp32.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -129,8 +132,8 @@ __global__ void __launch_bounds__(NTH, 1) bwd_chain_kernel(const __grid_constant
   const bool st0 = blockIdx.x == 0;
   static_cast<void>(st0);
 
-  // the copies of chunk cc, one per lane of warp 0 (lane 0 posts the byte count first):
-  // X = raw log alpha, k, q, b; Y = dO, v, w; TP = T^T, P^T
+  // The copies of chunk cc, one per lane of warp 0 (lane 0 posts the byte count first):
+  // X = raw log alpha, k, q, b; Y = dO, v, w; TP = T^T, P^T.
   // X in three parts, each as soon as its staging is free: log alpha over the Kn tile (read
   // by the dU product), k and q over the Qh half of [Qh; Kb]^T (read by the first part of the
   // dS update), b over the Kb half (read by its last part)
@@ -525,9 +528,10 @@ constexpr uint32_t K2_PX = 256;  // [dP; dA] [t'][s] (lanes: stacked tokens), th
 constexpr uint32_t K2_QK = 320;  // [dQh^T | dKb^T] [i][t']
 constexpr uint32_t K2_Y = 448;   // [Qh; Kb]^T [dP; dA] [i][s]
 
-// Persistent: CTA r takes the units (batch, head, chunk) r, r + grid, ...; the copies of the
-// next unit are issued as soon as the current unit's last product is done, and its states
-// are prefetched into L2 one unit ahead.
+// Persistent: CTA r takes the units (batch, head, chunk) r, r + grid, ...; the next unit's
+// dO and -dR are copied once the current unit's first products are done, its U and raw
+// inputs once the current outputs have left their staging, and its states are prefetched
+// into L2 meanwhile.
 __global__ void __launch_bounds__(NTH, 1)
     bwd_grad_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmNR,
                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmQ,
