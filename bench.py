@@ -334,9 +334,9 @@ def time_bwd(args, dev):
 
 
 def time_csize(args, dev):
-    """The prefill workload at chunk sizes 32, 64 and 128 through gdn2_chunk_fwd_csize (32 and
-    64 on the tcgen05 kernels, 128 on the warp-MMA kernel): latency, and the on-chip footprint
-    that sets how many CTAs share an SM (the call needs no device memory besides its tensors)."""
+    """The prefill workload at chunk sizes 32, 64 and 128 through gdn2_chunk_fwd_csize (each on
+    a tcgen05 kernel): latency, and the on-chip footprint that sets how many CTAs share an SM
+    (the call needs no device memory besides its tensors)."""
     import torch
     import gated_delta_rule_95_b200 as g
     d = gi.prefill_inputs(PREFILL)
@@ -355,8 +355,8 @@ def time_csize(args, dev):
         smem = g.lib().gdn2_chunk_fwd_csize_smem_bytes(C, dk)
         out[C] = dict(ms=ms, smem=smem, ctas_per_sm=sm_total // (smem + 1024),
                       kernel={32: "chunk_fwd_tc32_kernel (tcgen05)", 64: "chunk_fwd_tc_kernel (tcgen05)",
-                              128: "chunk_fwd_csize_kernel (warp-level MMA)"}[C],
-                      tmem_cols={32: 512, 64: 512, 128: 0}[C], ctas=B * H if C < 128 else B * H * (dv // 32))
+                              128: "chunk_fwd_tc128_kernel (tcgen05, phases in sequence)"}[C],
+                      tmem_cols=512, ctas=B * H)
     arg_bytes = sum(t.numel() * t.element_size() for t in args_t + [o, S_T])
     return dict(sizes=out, tokens=B * T, token_heads=B * T * H, arg_bytes=arg_bytes, ok=g.gdn2_device_status() == 0)
 

@@ -112,11 +112,13 @@ cudaError_t launch_chunk_fwd_f32_tc(const ChunkArgs& a, cudaStream_t st);
 // fp32 inputs of the other head sizes: fp32 CUDA-core kernel of the same chunkwise algorithm.
 cudaError_t launch_chunk_fwd_f32(const ChunkArgs& a, cudaStream_t st);
 // bf16, chunk size 32 (tcgen05 kernel for 32-token chunks), 64 (the production tcgen05
-// kernel) or 128 (the warp-MMA study kernel); shared memory per CTA, 0 for an unsupported
-// (chunk, d_k).
+// kernel) or 128 (tcgen05 kernel with the phases of a chunk in sequence); shared memory per
+// CTA, 0 for an unsupported (chunk, d_k).
 size_t chunk_fwd_tc_smem_bytes();
 size_t chunk_fwd_tc32_smem_bytes();
 cudaError_t launch_chunk_fwd_tc32(const ChunkArgs& a, cudaStream_t st);
+size_t chunk_fwd_tc128_smem_bytes();
+cudaError_t launch_chunk_fwd_tc128(const ChunkArgs& a, cudaStream_t st);
 size_t chunk_fwd_csize_smem_bytes(int chunk, int dk);
 cudaError_t launch_chunk_fwd_csize(const ChunkArgs& a, int chunk, cudaStream_t st);
 // T = 0: S_T = S0 (or zeros).

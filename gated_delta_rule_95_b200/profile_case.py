@@ -6,11 +6,12 @@
     python -m gated_delta_rule_95_b200.profile_case --kind csize --chunk 128 --B 8 --H 16 --T 1024 --reps 2
     python -m gated_delta_rule_95_b200.profile_case --kind prefill --stamps
     python -m gated_delta_rule_95_b200.profile_case --kind bwd --stamps
+    python -m gated_delta_rule_95_b200.profile_case --kind csize --chunk 128 --stamps
 
 Inputs follow the recipe of the named workload (gdn2_inputs) with the given
 sizes; it exits 0 after a device synchronisation and a clean device status.
 
---stamps runs the prefill (or the backward) on the instrumented library
+--stamps runs the prefill (the backward, the chunk-size 128 forward) on the instrumented library
 (libgdn2_stamps.so, built with GDN2_STAMPS: the kernel's first CTA records clock64 at the
 points of its per-chunk schedule) and prints, per chunk, each point's cycle count relative to the
 point where the chunk's raw input tiles have landed, and the period between consecutive
@@ -91,6 +92,9 @@ BWD_SLOT_NAMES = {0: "chunk start", 1: "copies landed", 2: "inputs read", 3: "op
                   8: "dR done", 9: "-dR staged, dS issued, stores issued", 10: "dS done"}
 GRAD_SLOT_NAMES = {16: "unit start", 17: "copies landed, S in", 18: "operands built", 19: "first products done",
                    20: "dP, dA, dSt written", 21: "second products done", 22: "gradients written"}
+TC128_SLOT_NAMES = {0: "chunk start", 1: "log decay read", 2: "operands built", 3: "[-A; P] done",
+                    4: "A read out", 5: "solve done", 6: "state product done", 7: "last operands written",
+                    8: "U~ done", 9: "U~ rounded", 10: "output/state product done", 11: "o stored"}
 SLOT_NAMES = {0: "AP issued", 1: "SP issued", 2: "U diag issued", 3: "U T21 issued", 4: "OP issued",
               5: "raw landed", 6: "operands built", 7: "AP done", 8: "A/P read out", 9: "8x8 inverses",
               10: "32-level done", 11: "64-level done", 12: "U rounded", 13: "R rounded",
@@ -112,7 +116,11 @@ def stamps(a):
     wl = gi.WORKLOADS[a.workload or "prefill_b8_h16_t4096"]
     d = gi.prefill_inputs(wl, B=a.B, T=a.T, H=a.H)
     x = {k: (None if v is None else v.cuda()) for k, v in d.items()}
-    names, first = SLOT_NAMES, 5
+    names, first, csz = SLOT_NAMES, 5, 64
+    if a.kind == "csize":
+        if a.chunk != 128:
+            raise SystemExit("--stamps with --kind csize: the chunk-size 128 kernel only")
+        names, first, csz = TC128_SLOT_NAMES, 0, 128
     if a.kind == "bwd":
         B, T, H = x["q"].shape[:3]
         gen = torch.Generator(device="cuda")
@@ -123,6 +131,8 @@ def stamps(a):
     for _ in range(max(2, a.reps)):
         if a.kind == "bwd":
             g.gdn2_chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], dO, dS)
+        elif a.kind == "csize":
+            g.gdn2_chunk_fwd_csize(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], chunk=128)
         else:
             g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
     torch.cuda.synchronize()
@@ -130,7 +140,7 @@ def stamps(a):
     lib.gdn2_stamps_read.argtypes = [ctypes.c_void_p, ctypes.c_int]
     n = lib.gdn2_stamps_read(buf, 64 * STAMP_SLOTS)
     st = np.frombuffer(buf, dtype=np.uint64)[:n].astype(np.int64).reshape(-1, STAMP_SLOTS)
-    nch = min(64, (x["q"].shape[1] + 63) // 64)
+    nch = min(64, (x["q"].shape[1] + csz - 1) // csz)
     base = st[:nch, first]
     print("cycles relative to the chunk's first point (clock64 of the first CTA's SM); the "
           "backward visits the chunks in reverse")

@@ -202,15 +202,15 @@ def test_chunk_fwd_csize_validation(kw, status):
 
 
 def test_csize_shared_memory_footprint():
-    # C = 128 (the warp-MMA kernel): Kn and Kb/Qh [C][d_k], A/P [C][C], U [C][32], state
-    # [d_k][32], Gamma_C [d_k], cumsum partials [512 threads], all fp32
+    # C = 128: region X (the stacked [-Kb; Qh] tile, 256 rows x 128 fp32 channels, later
+    # [P; Kn^T]), region Y (Kn, then A solved into T: 128 x 128 fp32), the solve's 64 x 72
+    # fp32 scratch, 1 KB of alignment slack and the barrier / decay block
     L = g.lib()
-    for dk in (64, 128):
-        assert L.gdn2_chunk_fwd_csize_smem_bytes(128, dk) == 4 * (2 * 128 * dk + 128 * 128 + 32 * 128 + 33 * dk + 512)
-    assert L.gdn2_chunk_fwd_csize_smem_bytes(128, 128) <= 227 * 1024
-    # C = 32 and 64 (the tcgen05 kernels): one layout for both head sizes, within one block's
+    n128 = L.gdn2_chunk_fwd_csize_smem_bytes(128, 128)
+    assert n128 == 4 * (256 * 128 + 128 * 128 + 64 * 72) + 1024 + 2592
+    # every size on a tcgen05 kernel: one layout for both head sizes, within one block's
     # 227 KB, the 32-token chunk's tiles the smaller
-    for C in (32, 64):
+    for C in (32, 64, 128):
         n = L.gdn2_chunk_fwd_csize_smem_bytes(C, 128)
         assert 0 < n <= 227 * 1024 and L.gdn2_chunk_fwd_csize_smem_bytes(C, 64) == n
     assert L.gdn2_chunk_fwd_csize_smem_bytes(32, 128) < L.gdn2_chunk_fwd_csize_smem_bytes(64, 128)
