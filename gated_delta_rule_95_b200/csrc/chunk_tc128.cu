@@ -23,10 +23,12 @@
 // block merges T_IJ = -T_II (A_IJ T_JJ) on warp-level tf32 MMAs, in place (a merge reads only
 // the off-diagonal block it then overwrites and diagonal blocks already inverted).  One CTA
 // of 16 warps per (batch, head); inputs are read with plain coalesced loads from L2, where the
-// previous chunk prefetched them.
+// previous chunk prefetched them (tensor-map box prefetches), every load of a phase issued
+// before any is used (clamped token index, values past the sequence end zeroed).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "gdn2_internal.h"
 #include "ptx.cuh"
@@ -82,7 +84,7 @@ struct Tc128Params {
 
 #ifdef GDN2_STAMPS
 // Instrumented build (GDN2_STAMPS): clock64 at the phase boundaries of the first CTA, written
-// by thread 0 into [chunk][slot] of a 64 x 32 array (slots 0-11).
+// by thread 0 into [chunk][slot] of a 64 x 32 array (slots 0-18).
 #define TC128_STAMP(c, slot)                                                                  \
   do {                                                                                        \
     if (p.stamps && blockIdx.x == 0 && threadIdx.x == 0 && (c) < 64)                          \
@@ -197,7 +199,11 @@ __device__ __forceinline__ void solve_in_place(unsigned char* Y, float* Zs, int 
 
 // DK, DV: key and value head dimensions (64 or 128).
 template <int DK, int DV>
-__global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Params p) {
+__global__ void __launch_bounds__(NT, 1)
+    chunk_fwd_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmV,
+                           const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmLA,
+                           const Tc128Params p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Misc& ms = *reinterpret_cast<Misc*>(sm + TILES);
@@ -253,20 +259,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
     tc_fence_after();
   };
 
-  // the input rows of chunk cc into L2, one token per thread of warps 0-3 (one chunk ahead, so
-  // that the operand build and the Vw pass read from L2 rather than wait on DRAM)
+  // chunk cc's input tiles into L2 (thread 0, one box per 128-byte channel panel), one chunk
+  // ahead, so that the operand build and the Vw pass read from L2 rather than wait on DRAM
   auto prefetch_chunk = [&](int cc) {
-    const int t = cc * C + tid;
-    if (tid < C && t < len) {
-      const size_t e = tok(t);
-      bulk_prefetch_l2(p.la + e * DK, DK * 4);
-      bulk_prefetch_l2(p.q + e * DK, DK * 2);
-      bulk_prefetch_l2(p.k + e * DK, DK * 2);
-      bulk_prefetch_l2(p.b + e * DK, DK * 2);
-      bulk_prefetch_l2(p.v + e * DV, DV * 2);
-      bulk_prefetch_l2(p.w + e * DV, DV * 2);
+    if (tid != 0) return;
+    for (int pn = 0; pn < DK / 32; ++pn) tma_prefetch_l2_4d(&tmLA, 32 * pn, h, C * cc, bb);
+    for (int pn = 0; pn < DK / 64; ++pn) {
+      tma_prefetch_l2_4d(&tmQ, 64 * pn, h, C * cc, bb);
+      tma_prefetch_l2_4d(&tmK, 64 * pn, h, C * cc, bb);
+      tma_prefetch_l2_4d(&tmB, 64 * pn, h, C * cc, bb);
+    }
+    for (int pn = 0; pn < DV / 64; ++pn) {
+      tma_prefetch_l2_4d(&tmV, 64 * pn, h, C * cc, bb);
+      tma_prefetch_l2_4d(&tmW, 64 * pn, h, C * cc, bb);
     }
   };
+  if (tid == 0) {
+    tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmV); tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmLA);
+  }
   if (nch > 0) prefetch_chunk(0);
 
   if (32 * sg < DK) {  // entering state S0 -> S^T (lane j = ch, key channels [32 sg, 32 sg + 32))
@@ -284,15 +295,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
     const int t0 = c * C, n = min(C, len - t0);
     TC128_STAMP(c, 0);
     // ===== 1. cumulative decay and the folded operands: thread (key channel bi, tokens
-    // [TPP part, TPP part + TPP)); Kn is kept in registers for the Kn Gamma_C ^T rows
-    float knr[TPP];
+    // [TPP part, TPP part + TPP))
     {
+      // loads at clamped tokens, issued together; values past the sequence end are zeroed
       float g[TPP];
 #pragma unroll
       for (int r = 0; r < TPP; ++r) {
         const int t = TPP * part + r;
-        g[r] = t < n ? p.la[tok(t0 + t) * DK + bi] : 0.f;
+        g[r] = p.la[tok(t0 + min(t, n - 1)) * DK + bi];
       }
+#pragma unroll
+      for (int r = 0; r < TPP; ++r)
+        if (TPP * part + r >= n) g[r] = 0.f;
       float acc = 0.f;
 #pragma unroll
       for (int r = 0; r < TPP; ++r) {
@@ -309,28 +323,28 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
         ms.gC[bi] = ex2_approx(tot);
         if (tot < G2_MIN && p.err) atomicOr(p.err, kErrDecayRange);
       }
+      TC128_STAMP(c, 17);
 #pragma unroll
       for (int r0 = 0; r0 < TPP; r0 += 4) {  // four tokens' loads in flight at a time
         float kk[4], bg[4], qq[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int t = TPP * part + r0 + r;
-          kk[r] = bg[r] = qq[r] = 0.f;
-          if (t < n) {
-            const size_t e = tok(t0 + t) * DK + bi;
-            kk[r] = __bfloat162float(p.k[e]);
-            bg[r] = __bfloat162float(p.b[e]);
-            qq[r] = __bfloat162float(p.q[e]);
-          }
+          const size_t e = tok(t0 + min(t, n - 1)) * DK + bi;
+          kk[r] = __bfloat162float(p.k[e]);
+          bg[r] = __bfloat162float(p.b[e]);
+          qq[r] = __bfloat162float(p.q[e]);
         }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          if (TPP * part + r0 + r >= n) kk[r] = bg[r] = qq[r] = 0.f;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int t = TPP * part + r0 + r;
           const float G = ex2_approx(g[r0 + r] + off), Gi = rcp_approx(G);
-          knr[r0 + r] = kk[r] * Gi;
           *reinterpret_cast<float*>(sm + OFF_X + f32_off(t, bi, KQP)) = rna_tf32(-(kk[r] * bg[r]) * G);
           *reinterpret_cast<float*>(sm + OFF_X + f32_off(C + t, bi, KQP)) = rna_tf32(qq[r] * G);
-          *reinterpret_cast<float*>(Y + f32_off(t, bi, R128)) = rna_tf32(knr[r0 + r]);
+          *reinterpret_cast<float*>(Y + f32_off(t, bi, R128)) = rna_tf32(kk[r] * Gi);
         }
       }
     }
@@ -349,11 +363,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
     }
     if (!mma_done()) { dead = true; break; }
     TC128_STAMP(c, 3);
-    // ===== 3. A (sign restored, strictly lower) over the Kn tile the product has read
+    // ===== 3. this thread's Kn values (for the Kn Gamma_C rows), then A (sign restored,
+    // strictly lower) over the Kn tile the product has read
+    float knr[TPP];
+#pragma unroll
+    for (int r = 0; r < TPP; ++r) knr[r] = *reinterpret_cast<const float*>(Y + f32_off(TPP * part + r, bi, R128));
     {
       float v[32];
       tmem_ld32(tlane + TM_R + 32 * sg, v);
       tmem_ld_wait();
+      __syncthreads();  // every Kn read precedes the A writes
       const int t = ch;
 #pragma unroll
       for (int x = 0; x < 32; x += 4) {
@@ -381,6 +400,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
       umma_commit(&ms.bar_mma);
     }
     if (c + 1 < nch) prefetch_chunk(c + 1);
+    TC128_STAMP(c, 18);
     solve_in_place(Y, Zs, warp, lane);
     TC128_STAMP(c, 5);
     if (!mma_done()) { dead = true; break; }
@@ -400,6 +420,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
         st4_tf32(sm + OFF_X + f32_off(t, s, PKP), f);
       }
     }
+    TC128_STAMP(c, 12);
     {  // rows C + i: Kn Gamma_C, i.e. k_s Gamma_C / Gamma_s
       const float gc = ms.gC[bi];
 #pragma unroll
@@ -408,6 +429,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
         st4_tf32(sm + OFF_X + f32_off(C + bi, TPP * part + r, PKP), f);
       }
     }
+    TC128_STAMP(c, 13);
     {  // R^T <- Vw^T + R^T rounded to tf32 in place (lane j = ch, tokens [32 sg, 32 sg + 32), in
        // two halves of 16)
       const int j = ch;
@@ -417,12 +439,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
           const int t = 32 * sg + 16 * hf + r;
-          vw[r] = 0.f;
-          if (t < n && j < DV) {
-            const size_t e = tok(t0 + t) * DV + j;
-            vw[r] = __bfloat162float(p.v[e]) * __bfloat162float(p.w[e]);
-          }
+          const size_t e = tok(t0 + min(t, n - 1)) * DV + (j < DV ? j : 0);
+          vw[r] = __bfloat162float(p.v[e]) * __bfloat162float(p.w[e]);
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r)
+          if (32 * sg + 16 * hf + r >= n || j >= DV) vw[r] = 0.f;
         tmem_ld16(tlane + TM_R + 32 * sg + 16 * hf, x);
         tmem_ld_wait();
 #pragma unroll
@@ -430,6 +452,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
         tmem_st16(tlane + TM_R + 32 * sg + 16 * hf, x);
       }
     }
+    TC128_STAMP(c, 14);
     if (32 * sg < DK) {  // S^T <- S^T Diag(Gamma_C): the state product has read S^T
       float x[32];
       tmem_ld32(tlane + TM_S + 32 * sg, x);
@@ -445,11 +468,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
       tmem_st32(tlane + TM_S + 32 * sg, x);
     }
     tmem_st_wait();
+    TC128_STAMP(c, 15);
     for (int e = tid; e < C * C / 4; e += NT) {  // T rounded to tf32 in place
       float4* p4 = reinterpret_cast<float4*>(Y) + e;
       const float4 f = *p4;
       *p4 = make_float4(rna_tf32(f.x), rna_tf32(f.y), rna_tf32(f.z), rna_tf32(f.w));
     }
+    TC128_STAMP(c, 16);
     handoff();
     TC128_STAMP(c, 7);
     // ===== 6. U~^T = R^T T^T (K = t)
@@ -523,8 +548,39 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc128_kernel(const Tc128Param
   if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode128() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+// [B, T, H, D] tensor; one box = 128 bytes of channels x C tokens of one (b, h), for L2 prefetches
+bool map128(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int B, int T, int H, int D) {
+  auto fn = encode128();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * esize, (cuuint64_t)H * D * esize, (cuuint64_t)T * H * D * esize};
+  cuuint32_t box[4] = {(cuuint32_t)(128 / esize), 1, (cuuint32_t)C, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DK, int DV>
 cudaError_t launch128(const ChunkArgs& a, cudaStream_t st) {
+  CUtensorMap mq, mk, mb, mv, mw, mla;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!map128(&mq, a.q, BF, 2, a.B, a.T, a.H, DK) || !map128(&mk, a.k, BF, 2, a.B, a.T, a.H, DK) ||
+      !map128(&mb, a.b, BF, 2, a.B, a.T, a.H, DK) || !map128(&mv, a.v, BF, 2, a.B, a.T, a.H, DV) ||
+      !map128(&mw, a.w, BF, 2, a.B, a.T, a.H, DV) ||
+      !map128(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.B, a.T, a.H, DK))
+    return cudaErrorInvalidValue;
   Tc128Params p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k = static_cast<const __nv_bfloat16*>(a.k);
@@ -542,7 +598,7 @@ cudaError_t launch128(const ChunkArgs& a, cudaStream_t st) {
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = smem_limit_once(chunk_fwd_tc128_kernel<DK, DV>, (int)SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
-  chunk_fwd_tc128_kernel<DK, DV><<<a.B * a.H, NT, SMEM_BYTES, st>>>(p);
+  chunk_fwd_tc128_kernel<DK, DV><<<a.B * a.H, NT, SMEM_BYTES, st>>>(mq, mk, mb, mv, mw, mla, p);
   return cudaGetLastError();
 }
 

@@ -94,7 +94,9 @@ GRAD_SLOT_NAMES = {16: "unit start", 17: "copies landed, S in", 18: "operands bu
                    20: "dP, dA, dSt written", 21: "second products done", 22: "gradients written"}
 TC128_SLOT_NAMES = {0: "chunk start", 1: "log decay read", 2: "operands built", 3: "[-A; P] done",
                     4: "A read out", 5: "solve done", 6: "state product done", 7: "last operands written",
-                    8: "U~ done", 9: "U~ rounded", 10: "output/state product done", 11: "o stored"}
+                    8: "U~ done", 9: "U~ rounded", 10: "output/state product done", 11: "o stored",
+                    12: "P written", 13: "Kn Gamma_C written", 14: "Vw added", 15: "state decayed",
+                    16: "T rounded", 17: "offsets summed", 18: "prefetch issued"}
 SLOT_NAMES = {0: "AP issued", 1: "SP issued", 2: "U diag issued", 3: "U T21 issued", 4: "OP issued",
               5: "raw landed", 6: "operands built", 7: "AP done", 8: "A/P read out", 9: "8x8 inverses",
               10: "32-level done", 11: "64-level done", 12: "U rounded", 13: "R rounded",
