@@ -185,16 +185,17 @@ GDN2_API gdn2_status gdn2_chunk_fwd_split_static(const void* q, const void* k, c
  * snilld.dk article's proof-of-concept list asks to measure ("POC-matrix der daekker de
  * haarde hjoerner": latency, throughput and peak memory at C = 64 and also at 32 and 128).
  * Same recurrence and result as gdn2_chunk_fwd (the Gated DeltaNet-2 guide's chunkwise WY
- * form, decay folded at the chunk start); one kernel template serves the three sizes, on
- * warp-level tensor-core MMAs (tf32 operands, fp32 accumulation) rather than the tcgen05
- * kernel of gdn2_chunk_fwd, whose tensor-memory plan is built for C = 64.
+ * form, decay folded at the chunk start), each size on a tcgen05 kernel (tf32 operands,
+ * fp32 accumulation in tensor memory): C = 64 is gdn2_chunk_fwd's kernel, C = 32 the same
+ * design with 32-token chunks, C = 128 the same products with the phases of a chunk run in
+ * sequence (its tiles do not fit one SM's memory when held resident).
  *
  *   q .. S_T, B, T, H, d_k, d_v : as gdn2_chunk_fwd
  *   dt          : GDN2_BF16 (fp32 inputs return GDN2_ERR_DTYPE)
  *   chunk       : 32, 64 or 128 tokens per chunk; anything else returns GDN2_ERR_SHAPE
  * gdn2_chunk_fwd_csize_smem_bytes(chunk, d_k) is the shared memory one CTA of the kernel
- * holds (one CTA per (batch, head, 32 value columns)), or 0 for an unsupported pair; the
- * call needs no device memory besides its arguments.
+ * holds (one CTA per (batch, head)), or 0 for an unsupported pair; the call needs no device
+ * memory besides its arguments.
  */
 GDN2_API size_t gdn2_chunk_fwd_csize_smem_bytes(int chunk, int d_k);
 GDN2_API gdn2_status gdn2_chunk_fwd_csize(const void* q, const void* k, const void* v, const float* log_alpha,
