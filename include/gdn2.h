@@ -193,6 +193,8 @@ GDN2_API gdn2_status gdn2_chunk_fwd_split_static(const void* q, const void* k, c
  *   q .. S_T, B, T, H, d_k, d_v : as gdn2_chunk_fwd
  *   dt          : GDN2_BF16 (fp32 inputs return GDN2_ERR_DTYPE)
  *   chunk       : 32, 64 or 128 tokens per chunk; anything else returns GDN2_ERR_SHAPE
+ * The decay limit of the shared conventions holds per chunk of the chosen size: the
+ * cumulative log decay of a channel over 128 tokens at chunk = 128 (flagged the same way).
  * gdn2_chunk_fwd_csize_smem_bytes(chunk, d_k) is the shared memory one CTA of the kernel
  * holds (one CTA per (batch, head)), or 0 for an unsupported pair; the call needs no device
  * memory besides its arguments.
