@@ -118,3 +118,27 @@ def test_full_size_sampled(chunk, name, units):
     for (bb, h), (o_ref, S_ref) in zip(units, oracle_units(d, units)):
         assert rel_err(o_c[bb, :, h].numpy(), o_ref) <= TOL["bf16"], (bb, h)
         assert rel_err(S_c[bb, h].numpy(), S_ref) <= TOL["bf16"], (bb, h)
+
+
+GDN2_ERR_RANGE = 7
+
+
+def test_decay_bound_holds_per_chunk_of_the_chosen_size():
+    """log alpha = -1 per token: -64 over a 64-token chunk, inside the -80 bound of the chunk
+    form, but -128 over a 128-token chunk.  C = 32 and 64 run clean and match the oracle;
+    C = 128 reports the range error through the device status; a call within the bound
+    afterwards reports clean again."""
+    wl = dataclasses.replace(BASE, state_std=0.0, seed=33)
+    d = gi.prefill_inputs(wl, B=1, T=256, H=2)
+    d["log_alpha"] = torch.full_like(d["log_alpha"], -1.0)
+    x = _cuda(d)
+    o_ref, S_ref = _oracle(d)
+    for C in (32, 64):
+        o, S = _run(x, C)
+        assert g.gdn2_device_status() == 0, C
+        assert rel_err(o.cpu().numpy(), o_ref) <= TOL["bf16"], C
+        assert rel_err(S.cpu().numpy(), S_ref) <= TOL["bf16"], C
+    _run(x, 128)
+    assert g.gdn2_device_status() == GDN2_ERR_RANGE
+    _run(_cuda(gi.prefill_inputs(wl, B=1, T=256, H=2)), 128)
+    assert g.gdn2_device_status() == 0
