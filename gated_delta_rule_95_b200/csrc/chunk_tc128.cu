@@ -57,7 +57,6 @@ struct Misc {
   uint32_t tmem_base;
   int abort;
   alignas(16) float gC[128];      // Gamma at the chunk end, per key channel
-  alignas(16) float segtot[512];  // cumulative log2 decay over each token range
 };
 constexpr uint32_t SMEM_BYTES = TILES + 1024 + sizeof(Misc);
 
@@ -103,6 +102,9 @@ __device__ __forceinline__ uint32_t tfu(float x) { return __float_as_uint(rna_tf
 __device__ __forceinline__ void st4_tf32(unsigned char* p, const float* f) {
   *reinterpret_cast<float4*>(p) = make_float4(rna_tf32(f[0]), rna_tf32(f[1]), rna_tf32(f[2]), rna_tf32(f[3]));
 }
+// the low and high bf16 of a 32-bit word as fp32
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 __device__ __forceinline__ uint64_t kdesc(uint32_t base, uint32_t panel, int ks) {
   return sdesc_sw128(base + (uint32_t)(ks >> 2) * panel + (uint32_t)(ks & 3) * 32, 16, 1024);
 }
@@ -216,10 +218,12 @@ __global__ void __launch_bounds__(NT, 1)
   const int sg = tid >> 7;   // column group [32 sg, 32 sg + 32) of tensor-memory accesses
   const int unit = blockIdx.x, h = unit % p.H, bb = unit / p.H;
   const int len = p.T, nch = (len + C - 1) / C;
-  constexpr int PARTS = NT / DK, TPP = C / PARTS;     // operand build: token ranges per key channel
+  constexpr int PARTS = NT / DK, TPP = C / PARTS;     // Kn Gamma_C rows: token ranges per key channel
   constexpr uint32_t KQP = R256;                      // a panel of [-Kb; Qh]
   constexpr uint32_t PKP = (uint32_t)(C + DK) * 128;  // a panel of [P; Kn Gamma_C ^T]
-  const int bi = tid % DK, part = tid / DK;           // operand build: key channel, token range
+  const int bi = tid % DK, part = tid / DK;           // Kn Gamma_C rows: key channel, token range
+  constexpr int QPARTS = NT / (DK / 4), QTP = C / QPARTS;  // operand build: token ranges per channel quad
+  const int cq = tid % (DK / 4), qp = tid / (DK / 4);      // operand build: channel quad, token range
   auto tok = [&](int t) -> size_t { return ((size_t)bb * len + t) * p.H + h; };
 
   if (tid == 0) {
@@ -294,57 +298,76 @@ __global__ void __launch_bounds__(NT, 1)
   for (int c = 0; c < nch; ++c) {
     const int t0 = c * C, n = min(C, len - t0);
     TC128_STAMP(c, 0);
-    // ===== 1. cumulative decay and the folded operands: thread (key channel bi, tokens
-    // [TPP part, TPP part + TPP))
+    // ===== 1. cumulative decay and the folded operands: thread (key channels [4 cq, 4 cq + 4),
+    // tokens [QTP qp, QTP qp + QTP)); a warp's loads cover whole token rows (16-byte log-alpha
+    // and 8-byte bf16 groups), issued at clamped tokens before any is used, values past the
+    // sequence end zeroed
     {
-      // loads at clamped tokens, issued together; values past the sequence end are zeroed
-      float g[TPP];
+      float4 g[QTP];
 #pragma unroll
-      for (int r = 0; r < TPP; ++r) {
-        const int t = TPP * part + r;
-        g[r] = p.la[tok(t0 + min(t, n - 1)) * DK + bi];
+      for (int r = 0; r < QTP; ++r) {
+        const int t = QTP * qp + r;
+        g[r] = *reinterpret_cast<const float4*>(p.la + tok(t0 + min(t, n - 1)) * DK + 4 * cq);
       }
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int r = 0; r < TPP; ++r)
-        if (TPP * part + r >= n) g[r] = 0.f;
-      float acc = 0.f;
-#pragma unroll
-      for (int r = 0; r < TPP; ++r) {
-        acc = fmaf(g[r], LOG2E, acc);
+      for (int r = 0; r < QTP; ++r) {
+        const bool z = QTP * qp + r >= n;
+        acc.x = fmaf(z ? 0.f : g[r].x, LOG2E, acc.x);
+        acc.y = fmaf(z ? 0.f : g[r].y, LOG2E, acc.y);
+        acc.z = fmaf(z ? 0.f : g[r].z, LOG2E, acc.z);
+        acc.w = fmaf(z ? 0.f : g[r].w, LOG2E, acc.w);
         g[r] = acc;
       }
-      ms.segtot[part * DK + bi] = acc;
+      float4* segtot = reinterpret_cast<float4*>(Zs);  // [QPARTS][DK / 4]: the solve scratch, free here
+      segtot[qp * (DK / 4) + cq] = acc;
       __syncthreads();
       TC128_STAMP(c, 1);
-      float off = 0.f;
-      for (int q = 0; q < part; ++q) off += ms.segtot[q * DK + bi];
-      if (part == PARTS - 1) {
-        const float tot = off + acc;
-        ms.gC[bi] = ex2_approx(tot);
-        if (tot < G2_MIN && p.err) atomicOr(p.err, kErrDecayRange);
+      float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < qp; ++q) {
+        const float4 f = segtot[q * (DK / 4) + cq];
+        off.x += f.x;
+        off.y += f.y;
+        off.z += f.z;
+        off.w += f.w;
+      }
+      if (qp == QPARTS - 1) {
+        const float4 tot = make_float4(off.x + acc.x, off.y + acc.y, off.z + acc.z, off.w + acc.w);
+        *reinterpret_cast<float4*>(&ms.gC[4 * cq]) =
+            make_float4(ex2_approx(tot.x), ex2_approx(tot.y), ex2_approx(tot.z), ex2_approx(tot.w));
+        if (fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) < G2_MIN && p.err) atomicOr(p.err, kErrDecayRange);
       }
       TC128_STAMP(c, 17);
 #pragma unroll
-      for (int r0 = 0; r0 < TPP; r0 += 4) {  // four tokens' loads in flight at a time
-        float kk[4], bg[4], qq[4];
+      for (int r0 = 0; r0 < QTP; r0 += 2) {  // two tokens' loads in flight at a time
+        uint2 kk[2], bg[2], qq[2];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int t = TPP * part + r0 + r;
-          const size_t e = tok(t0 + min(t, n - 1)) * DK + bi;
-          kk[r] = __bfloat162float(p.k[e]);
-          bg[r] = __bfloat162float(p.b[e]);
-          qq[r] = __bfloat162float(p.q[e]);
+        for (int r = 0; r < 2; ++r) {
+          const size_t e = tok(t0 + min(QTP * qp + r0 + r, n - 1)) * DK + 4 * cq;
+          kk[r] = *reinterpret_cast<const uint2*>(p.k + e);
+          bg[r] = *reinterpret_cast<const uint2*>(p.b + e);
+          qq[r] = *reinterpret_cast<const uint2*>(p.q + e);
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-          if (TPP * part + r0 + r >= n) kk[r] = bg[r] = qq[r] = 0.f;
+        for (int r = 0; r < 2; ++r) {
+          const int t = QTP * qp + r0 + r;
+          const bool z = t >= n;
+          const float k4[4] = {bf_lo(kk[r].x), bf_hi(kk[r].x), bf_lo(kk[r].y), bf_hi(kk[r].y)};
+          const float b4[4] = {bf_lo(bg[r].x), bf_hi(bg[r].x), bf_lo(bg[r].y), bf_hi(bg[r].y)};
+          const float q4[4] = {bf_lo(qq[r].x), bf_hi(qq[r].x), bf_lo(qq[r].y), bf_hi(qq[r].y)};
+          const float gl[4] = {g[r0 + r].x + off.x, g[r0 + r].y + off.y, g[r0 + r].z + off.z, g[r0 + r].w + off.w};
+          float nkb[4], qh[4], kn[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int t = TPP * part + r0 + r;
-          const float G = ex2_approx(g[r0 + r] + off), Gi = rcp_approx(G);
-          *reinterpret_cast<float*>(sm + OFF_X + f32_off(t, bi, KQP)) = rna_tf32(-(kk[r] * bg[r]) * G);
-          *reinterpret_cast<float*>(sm + OFF_X + f32_off(C + t, bi, KQP)) = rna_tf32(qq[r] * G);
-          *reinterpret_cast<float*>(Y + f32_off(t, bi, R128)) = rna_tf32(kk[r] * Gi);
+          for (int m = 0; m < 4; ++m) {
+            const float G = ex2_approx(gl[m]), Gi = rcp_approx(G);
+            const float kv = z ? 0.f : k4[m];
+            nkb[m] = -(kv * b4[m]) * G;
+            qh[m] = (z ? 0.f : q4[m]) * G;
+            kn[m] = kv * Gi;
+          }
+          st4_tf32(sm + OFF_X + f32_off(t, 4 * cq, KQP), nkb);
+          st4_tf32(sm + OFF_X + f32_off(C + t, 4 * cq, KQP), qh);
+          st4_tf32(Y + f32_off(t, 4 * cq, R128), kn);
         }
       }
     }
