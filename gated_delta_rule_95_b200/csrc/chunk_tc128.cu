@@ -48,7 +48,8 @@ constexpr uint32_t R128 = 128 * 128;        // a panel of 128 rows
 constexpr uint32_t R256 = 256 * 128;        // a panel of 256 rows
 constexpr uint32_t OFF_X = 0;               // [-Kb; Qh] [t][i], then [P; Kn Gamma_C ^T] [t | i][s]
 constexpr uint32_t OFF_Y = OFF_X + 4 * R256;  // Kn [s][i], then A -> T [s][t]
-constexpr uint32_t OFF_Z = OFF_Y + 4 * R128;  // solve scratch: the merges' A_IJ T_JJ, 64 x LDZ fp32
+constexpr uint32_t OFF_Z = OFF_Y + 4 * R128;  // solve scratch: the merges' A_IJ T_JJ, 64 x LDZ fp32;
+                                              // in the operand build, the decay partials per range
 constexpr int LDZ = 72;
 constexpr uint32_t TILES = OFF_Z + 64 * LDZ * 4;
 
